@@ -1,0 +1,260 @@
+"""fp64 CPU oracle for 3D Deformable Slide Attention (3D-DSA).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's
+CPU-baseline leg may import this package; the product path never does.  It shares no
+code with the CUDA library.  The arithmetic lives in ``dsa_oracle.c`` (plain C, double
+precision, OpenMP over independent rows); this module compiles it with gcc, marshals
+arguments with ctypes, and scatters the per-tile results back into full tensors.
+
+Definition followed (the pages give the operator only in outline): "MegaSlide-DiT:
+Memory-Centric Adaptation and Deformable Local Attention for Efficient Video Diffusion",
+abstract (3D-DSA, a motion-adaptive local attention whose cost is linear in the sequence
+length) and "Fast Video Generation with Sliding Tile Attention", abstract (attention over
+a local spatial-temporal window, tile-granular).  The concrete window rule, softmax and
+gradients are written out in the header of ``dsa_oracle.c``.
+
+Every function here is pinned by the CPU tests in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dsa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "libdsa_oracle.so")
+_lib = None
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "heads", "d", "T", "H", "W", "tt", "th", "tw", "wt", "wh", "ww")] + [
+        ("scale", ctypes.c_double)
+    ]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into a shared library with gcc (no -ffast-math: IEEE double)."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        fp = ctypes.POINTER(ctypes.c_double)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_plan.argtypes = [ctypes.c_int32] * 6 + [i32p] * 5
+        lib.oracle_fwd.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, i32p, ctypes.c_int32, i32p, i32p, dp, dp]
+        lib.oracle_bwd_dq.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, fp, i32p, ctypes.c_int32, i32p, i32p, dp]
+        lib.oracle_bwd_dkdv.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, fp, i32p, ctypes.c_int32, i32p, i32p,
+                                        dp, dp]
+        for f in (lib.oracle_plan, lib.oracle_fwd, lib.oracle_bwd_dq, lib.oracle_bwd_dkdv):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _f64(t) -> np.ndarray:
+    """Widen a tensor (bf16, fp32 or fp64) to a contiguous float64 numpy array, exactly."""
+    if isinstance(t, torch.Tensor):
+        t = t.detach().to("cpu")
+        if t.dtype != torch.float64:
+            t = t.to(torch.float64)
+        return np.ascontiguousarray(t.numpy())
+    return np.ascontiguousarray(np.asarray(t, dtype=np.float64))
+
+
+def _i32(t) -> np.ndarray:
+    if isinstance(t, torch.Tensor):
+        t = t.detach().to("cpu").numpy()
+    return np.ascontiguousarray(np.asarray(t, dtype=np.int32))
+
+
+class Geometry:
+    """Shapes of one problem: token grid, tiles, window (all from the caller)."""
+
+    def __init__(self, B, heads, d, grid, tile, window, scale=None):
+        self.B, self.heads, self.d = int(B), int(heads), int(d)
+        self.grid = tuple(int(x) for x in grid)
+        self.tile = tuple(int(x) for x in tile)
+        self.window = tuple(int(x) for x in window)
+        self.scale = float(1.0 / np.sqrt(d)) if scale is None else float(scale)
+        for g, t in zip(self.grid, self.tile):
+            if t <= 0 or g % t:
+                raise ValueError(f"grid {self.grid} is not divisible by tile {self.tile}")
+        self.G = tuple(g // t for g, t in zip(self.grid, self.tile))
+        self.weff = tuple(min(w, g) for w, g in zip(self.window, self.G))
+        self.n_tiles = self.G[0] * self.G[1] * self.G[2]
+        self.n_window_tiles = self.weff[0] * self.weff[1] * self.weff[2]
+        self.tile_tokens = self.tile[0] * self.tile[1] * self.tile[2]
+        self.n_tokens = self.grid[0] * self.grid[1] * self.grid[2]
+
+    @classmethod
+    def of(cls, w):
+        """Geometry of a ``dsa_inputs.Workload``."""
+        return cls(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale)
+
+    def c_problem(self) -> _Problem:
+        T, H, W = self.grid
+        tt, th, tw = self.tile
+        wt, wh, ww = self.window
+        return _Problem(self.B, self.heads, self.d, T, H, W, tt, th, tw, wt, wh, ww, self.scale)
+
+    def tile_token_index(self) -> np.ndarray:
+        """[nTiles, tile_tokens] token index of each tile's tokens in raster order."""
+        T, H, W = self.grid
+        tt, th, tw = self.tile
+        idx = np.arange(self.n_tokens).reshape(T, H, W)
+        idx = idx.reshape(self.G[0], tt, self.G[1], th, self.G[2], tw).transpose(0, 2, 4, 1, 3, 5)
+        return np.ascontiguousarray(idx.reshape(self.n_tiles, self.tile_tokens))
+
+
+def plan(G, window, offsets):
+    """Window plan of the oracle: (starts[nTiles,3], kv_tiles[nTiles,Wt], row_ptr[nTiles+1], q_tiles[nnz])."""
+    lib = _load()
+    G = [int(x) for x in G]
+    window = [int(x) for x in window]
+    n = G[0] * G[1] * G[2]
+    wt = 1
+    for w, g in zip(window, G):
+        wt *= min(w, g)
+    off = _i32(offsets).reshape(n, 3)
+    starts = np.zeros((n, 3), np.int32)
+    kv = np.zeros((n, wt), np.int32)
+    row_ptr = np.zeros(n + 1, np.int32)
+    q_tiles = np.zeros(n * wt, np.int32)
+    rc = lib.oracle_plan(*G, *window, _ptr(off, ctypes.c_int32), _ptr(starts, ctypes.c_int32),
+                         _ptr(kv, ctypes.c_int32), _ptr(row_ptr, ctypes.c_int32), _ptr(q_tiles, ctypes.c_int32))
+    if rc:
+        raise ValueError(f"oracle_plan rejected G={G} window={window}")
+    return starts, kv, row_ptr, q_tiles[: row_ptr[-1]]
+
+
+def _selection(geo: Geometry, sel):
+    if sel is None:
+        bh = np.repeat(np.arange(geo.B * geo.heads, dtype=np.int32), geo.n_tiles)
+        tiles = np.tile(np.arange(geo.n_tiles, dtype=np.int32), geo.B * geo.heads)
+    else:
+        bh = _i32(sel[0]).reshape(-1)
+        tiles = _i32(sel[1]).reshape(-1)
+    return bh, tiles
+
+
+def _head_slice(t, geo: Geometry, bh: int) -> np.ndarray:
+    """float64 copy of one (b, head) slice [N, d] of a [B, heads, T, H, W, d] tensor."""
+    if isinstance(t, torch.Tensor):
+        return _f64(t.reshape(geo.B * geo.heads, geo.n_tokens, geo.d)[bh])
+    return _f64(np.asarray(t).reshape(geo.B * geo.heads, geo.n_tokens, geo.d)[bh])
+
+
+def _run_by_head(geo: Geometry, tensors, offsets, sel, n_out, call):
+    """Run ``call`` once per (b, head) present in the selection, on that head's slice
+    (heads are independent problems), so host memory holds one head in float64 at a time."""
+    bh, tiles = _selection(geo, sel)
+    off = _i32(offsets).reshape(geo.n_tiles, 3)
+    outs = [np.zeros((len(bh), geo.tile_tokens, geo.d), np.float64) for _ in range(n_out)]
+    lse = np.zeros((len(bh), geo.tile_tokens), np.float64)
+    one = Geometry(1, 1, geo.d, geo.grid, geo.tile, geo.window, geo.scale)
+    p = one.c_problem()
+    for h in np.unique(bh):
+        rows = np.nonzero(bh == h)[0]
+        sl = [_head_slice(t, geo, int(h)) for t in tensors]
+        sel_t = np.ascontiguousarray(tiles[rows])
+        sel_b = np.zeros(len(rows), np.int32)
+        part = [np.zeros((len(rows), geo.tile_tokens, geo.d), np.float64) for _ in range(n_out)]
+        part_lse = np.zeros((len(rows), geo.tile_tokens), np.float64)
+        rc = call(p, sl, off, len(rows), sel_b, sel_t, part, part_lse)
+        if rc:
+            raise RuntimeError(f"oracle call failed ({rc})")
+        for o, pt in zip(outs, part):
+            o[rows] = pt
+        lse[rows] = part_lse
+    return outs, lse
+
+
+def forward_tiles(geo: Geometry, q, k, v, offsets, sel=None):
+    """Forward on (bh, query tile) pairs.  Returns out[n_sel, tile_tokens, d] and
+    lse[n_sel, tile_tokens] (float64), rows in each tile's raster order."""
+    lib = _load()
+    D = ctypes.c_double
+
+    def call(p, sl, off, n, sb, st, part, part_lse):
+        return lib.oracle_fwd(ctypes.byref(p), _ptr(sl[0], D), _ptr(sl[1], D), _ptr(sl[2], D),
+                              _ptr(off, ctypes.c_int32), n, _ptr(sb, ctypes.c_int32), _ptr(st, ctypes.c_int32),
+                              _ptr(part[0], D), _ptr(part_lse, D))
+
+    (out,), lse = _run_by_head(geo, (q, k, v), offsets, sel, 1, call)
+    return out, lse
+
+
+def forward(geo: Geometry, q, k, v, offsets):
+    """Full forward: out[B, heads, T, H, W, d] and lse[B, heads, T, H, W] in float64."""
+    out_t, lse_t = forward_tiles(geo, q, k, v, offsets)
+    tok = geo.tile_token_index()
+    BH = geo.B * geo.heads
+    out = np.zeros((BH, geo.n_tokens, geo.d), np.float64)
+    lse = np.zeros((BH, geo.n_tokens), np.float64)
+    out_t = out_t.reshape(BH, geo.n_tiles, geo.tile_tokens, geo.d)
+    lse_t = lse_t.reshape(BH, geo.n_tiles, geo.tile_tokens)
+    out[:, tok.reshape(-1)] = out_t.reshape(BH, -1, geo.d)
+    lse[:, tok.reshape(-1)] = lse_t.reshape(BH, -1)
+    return (out.reshape((geo.B, geo.heads) + geo.grid + (geo.d,)),
+            lse.reshape((geo.B, geo.heads) + geo.grid))
+
+
+def backward_dq_tiles(geo: Geometry, q, k, v, dout, offsets, sel=None):
+    """dq on (bh, query tile) pairs: [n_sel, tile_tokens, d] float64."""
+    lib = _load()
+    D = ctypes.c_double
+
+    def call(p, sl, off, n, sb, st, part, part_lse):
+        return lib.oracle_bwd_dq(ctypes.byref(p), _ptr(sl[0], D), _ptr(sl[1], D), _ptr(sl[2], D), _ptr(sl[3], D),
+                                 _ptr(off, ctypes.c_int32), n, _ptr(sb, ctypes.c_int32), _ptr(st, ctypes.c_int32),
+                                 _ptr(part[0], D))
+
+    (dq,), _ = _run_by_head(geo, (q, k, v, dout), offsets, sel, 1, call)
+    return dq
+
+
+def backward_dkdv_tiles(geo: Geometry, q, k, v, dout, offsets, sel=None):
+    """dk, dv on (bh, key tile) pairs: each [n_sel, tile_tokens, d] float64, rows in the
+    key tile's raster order."""
+    lib = _load()
+    D = ctypes.c_double
+
+    def call(p, sl, off, n, sb, st, part, part_lse):
+        return lib.oracle_bwd_dkdv(ctypes.byref(p), _ptr(sl[0], D), _ptr(sl[1], D), _ptr(sl[2], D), _ptr(sl[3], D),
+                                   _ptr(off, ctypes.c_int32), n, _ptr(sb, ctypes.c_int32), _ptr(st, ctypes.c_int32),
+                                   _ptr(part[0], D), _ptr(part[1], D))
+
+    (dk, dv), _ = _run_by_head(geo, (q, k, v, dout), offsets, sel, 2, call)
+    return dk, dv
+
+
+def backward(geo: Geometry, q, k, v, dout, offsets):
+    """Full backward: dq, dk, dv as [B, heads, T, H, W, d] float64."""
+    dq_t = backward_dq_tiles(geo, q, k, v, dout, offsets)
+    dk_t, dv_t = backward_dkdv_tiles(geo, q, k, v, dout, offsets)
+    tok = geo.tile_token_index().reshape(-1)
+    BH = geo.B * geo.heads
+    res = []
+    for t in (dq_t, dk_t, dv_t):
+        full = np.zeros((BH, geo.n_tokens, geo.d), np.float64)
+        full[:, tok] = t.reshape(BH, -1, geo.d)
+        res.append(full.reshape((geo.B, geo.heads) + geo.grid + (geo.d,)))
+    return tuple(res)

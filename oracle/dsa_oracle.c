@@ -1,0 +1,375 @@
+/*
+ * fp64 CPU oracle for 3D Deformable Slide Attention (3D-DSA).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call this file: only the
+ * tests, the smoke check and the benchmark's CPU-baseline leg use it.  It shares no code,
+ * header, table or helper with the CUDA library.
+ *
+ * What it computes (plain definition, no blocking, fusion or reordering):
+ *
+ *   Operator: "3D Deformable Slide Attention (3D-DSA), a motion-adaptive local attention
+ *   operator" whose cost is linear in the sequence length ("MegaSlide-DiT: Memory-Centric
+ *   Adaptation and Deformable Local Attention for Efficient Video Diffusion", abstract),
+ *   in the tile-granular local 3D window form of "Fast Video Generation with Sliding Tile
+ *   Attention" (abstract: attending over a local spatial-temporal region).
+ *
+ *   Concrete form used here (the pages give only the outline above):
+ *     - the token grid T x H x W is cut into tiles tt x th x tw; tile grid G = (T/tt, H/th, W/tw);
+ *     - per axis the window length is w' = min(w, G) tiles;
+ *     - query tile i with integer offset o (tile units) gets the window start
+ *           s = clamp(i + o - floor(w'/2), 0, G - w')
+ *       per axis, and its key set K(i) is every token of the tiles j with s <= j < s + w'
+ *       on all three axes;
+ *     - for query token n in tile i:  s_nm = scale * <q_n, k_m>,  m in K(i);
+ *           lse_n = ln sum_m exp(s_nm),   o_n = sum_m exp(s_nm - lse_n) v_m;
+ *     - backward of L = sum_n <o_n, dO_n>:
+ *           P_nm = exp(s_nm - lse_n),  dP_nm = <dO_n, v_m>,
+ *           dS_nm = P_nm (dP_nm - sum_m' P_nm' dP_nm'),
+ *           dq_n = scale sum_m dS_nm k_m,  dk_m = scale sum_n dS_nm q_n,  dv_m = sum_n P_nm dO_n,
+ *       where the sums for dk_m and dv_m run over every query token n whose key set holds m.
+ *
+ * Inputs and every arithmetic step are double (bf16 and fp32 inputs widen to it exactly).  Token tensors are [B, heads, T, H, W, d] contiguous; offsets are
+ * int32 [nTiles, 3] (dt, dh, dw) in tile-raster order (t outer, w inner).
+ *
+ * Parity pins (tests, CPU only): a window covering the grid equals dense attention; a
+ * 1x1x1 window equals block-diagonal attention; softmax rows sum to one; brute-force
+ * membership by nearest window centre; backward against central finite differences.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int32_t B, heads, d;
+    int32_t T, H, W;
+    int32_t tt, th, tw;
+    int32_t wt, wh, ww;
+    double scale;
+} oracle_problem;
+
+static int32_t min_i(int32_t a, int32_t b) { return a < b ? a : b; }
+
+static int32_t clamp_i(int32_t x, int32_t lo, int32_t hi) {
+    if (x < lo) return lo;
+    if (x > hi) return hi;
+    return x;
+}
+
+/* Window start along one axis: centre = tile index + offset, start = centre - floor(w'/2),
+ * then moved so that [start, start + w') lies inside [0, G). */
+static int32_t axis_start(int32_t tile_index, int32_t offset, int32_t w_eff, int32_t G) {
+    return clamp_i(tile_index + offset - w_eff / 2, 0, G - w_eff);
+}
+
+typedef struct {
+    int32_t G[3];   /* tile grid (Gt, Gh, Gw) */
+    int32_t w[3];   /* effective window (w't, w'h, w'w) */
+    int32_t n_tiles, n_window_tiles, tile_tokens, n_tokens;
+} geometry;
+
+static int make_geometry(const oracle_problem* p, geometry* g) {
+    if (p->tt <= 0 || p->th <= 0 || p->tw <= 0) return 1;
+    if (p->T % p->tt || p->H % p->th || p->W % p->tw) return 1;
+    if (p->wt <= 0 || p->wh <= 0 || p->ww <= 0) return 1;
+    g->G[0] = p->T / p->tt;
+    g->G[1] = p->H / p->th;
+    g->G[2] = p->W / p->tw;
+    g->w[0] = min_i(p->wt, g->G[0]);
+    g->w[1] = min_i(p->wh, g->G[1]);
+    g->w[2] = min_i(p->ww, g->G[2]);
+    g->n_tiles = g->G[0] * g->G[1] * g->G[2];
+    g->n_window_tiles = g->w[0] * g->w[1] * g->w[2];
+    g->tile_tokens = p->tt * p->th * p->tw;
+    g->n_tokens = p->T * p->H * p->W;
+    return 0;
+}
+
+static void tile_coords(const geometry* g, int32_t tile, int32_t c[3]) {
+    c[2] = tile % g->G[2];
+    c[1] = (tile / g->G[2]) % g->G[1];
+    c[0] = tile / (g->G[2] * g->G[1]);
+}
+
+static void window_starts(const geometry* g, const int32_t* offsets, int32_t tile, int32_t s[3]) {
+    int32_t c[3];
+    tile_coords(g, tile, c);
+    for (int a = 0; a < 3; ++a) s[a] = axis_start(c[a], offsets[3 * tile + a], g->w[a], g->G[a]);
+}
+
+static int window_holds(const geometry* g, const int32_t s[3], int32_t key_tile) {
+    int32_t c[3];
+    tile_coords(g, key_tile, c);
+    for (int a = 0; a < 3; ++a)
+        if (c[a] < s[a] || c[a] >= s[a] + g->w[a]) return 0;
+    return 1;
+}
+
+/* Position of a key tile in the raster order (t outer, w inner) of a window box that holds it. */
+static int64_t window_position(const geometry* g, const int32_t s[3], int32_t key_tile) {
+    int32_t c[3];
+    tile_coords(g, key_tile, c);
+    return ((int64_t)(c[0] - s[0]) * g->w[1] + (c[1] - s[1])) * g->w[2] + (c[2] - s[2]);
+}
+
+/* Token index (within one (b, head) slice) of the r-th token of a tile, tokens of a tile
+ * taken in raster order (t outer, w inner). */
+static int64_t tile_token(const oracle_problem* p, const geometry* g, int32_t tile, int32_t r) {
+    int32_t c[3];
+    tile_coords(g, tile, c);
+    int32_t lw = r % p->tw, lh = (r / p->tw) % p->th, lt = r / (p->tw * p->th);
+    int64_t t = (int64_t)c[0] * p->tt + lt, h = (int64_t)c[1] * p->th + lh, w = (int64_t)c[2] * p->tw + lw;
+    return (t * p->H + h) * p->W + w;
+}
+
+/* Token indices of K(i), key tiles in raster order of the window box, tokens of each
+ * tile in raster order.  keys must hold n_window_tiles * tile_tokens entries. */
+static void key_set(const oracle_problem* p, const geometry* g, const int32_t* offsets, int32_t tile,
+                    int64_t* keys) {
+    int32_t s[3];
+    window_starts(g, offsets, tile, s);
+    int64_t n = 0;
+    for (int32_t a = s[0]; a < s[0] + g->w[0]; ++a)
+        for (int32_t b = s[1]; b < s[1] + g->w[1]; ++b)
+            for (int32_t c = s[2]; c < s[2] + g->w[2]; ++c) {
+                int32_t kt = (a * g->G[1] + b) * g->G[2] + c;
+                for (int32_t r = 0; r < g->tile_tokens; ++r) keys[n++] = tile_token(p, g, kt, r);
+            }
+}
+
+static double dot(const double* x, const double* y, int32_t d) {
+    double acc = 0.0;
+    for (int32_t c = 0; c < d; ++c) acc += x[c] * y[c];
+    return acc;
+}
+
+/* Scores of query token n over its key set, its log-sum-exp (max subtracted), and the
+ * softmax row P (written over the scores). */
+static double softmax_row(const oracle_problem* p, const double* qrow, const double* kbase, const int64_t* keys,
+                          int64_t nk, double* P) {
+    double mx = -INFINITY;
+    for (int64_t m = 0; m < nk; ++m) {
+        P[m] = p->scale * dot(qrow, kbase + keys[m] * p->d, p->d);
+        if (P[m] > mx) mx = P[m];
+    }
+    double sum = 0.0;
+    for (int64_t m = 0; m < nk; ++m) sum += exp(P[m] - mx);
+    double lse = mx + log(sum);
+    for (int64_t m = 0; m < nk; ++m) P[m] = exp(P[m] - lse);
+    return lse;
+}
+
+/* ---------------------------------------------------------------------------------- */
+
+/* Window plan: starts[nTiles,3], kv_tiles[nTiles, Wt] (key tiles of each window in
+ * ascending linear index), and the inverse map as CSR: row j lists, ascending, the query
+ * tiles whose window holds key tile j.  row_ptr / q_tiles may be NULL.  Returns 0 on
+ * success, 1 on an invalid shape. */
+int oracle_plan(int32_t Gt, int32_t Gh, int32_t Gw, int32_t wt, int32_t wh, int32_t ww, const int32_t* offsets,
+                int32_t* starts, int32_t* kv_tiles, int32_t* row_ptr, int32_t* q_tiles) {
+    if (Gt <= 0 || Gh <= 0 || Gw <= 0 || wt <= 0 || wh <= 0 || ww <= 0) return 1;
+    geometry g;
+    g.G[0] = Gt; g.G[1] = Gh; g.G[2] = Gw;
+    g.w[0] = min_i(wt, Gt); g.w[1] = min_i(wh, Gh); g.w[2] = min_i(ww, Gw);
+    g.n_tiles = Gt * Gh * Gw;
+    g.n_window_tiles = g.w[0] * g.w[1] * g.w[2];
+    for (int32_t i = 0; i < g.n_tiles; ++i) {
+        int32_t s[3];
+        window_starts(&g, offsets, i, s);
+        for (int a = 0; a < 3; ++a) starts[3 * i + a] = s[a];
+        int32_t n = 0;
+        for (int32_t a = s[0]; a < s[0] + g.w[0]; ++a)
+            for (int32_t b = s[1]; b < s[1] + g.w[1]; ++b)
+                for (int32_t c = s[2]; c < s[2] + g.w[2]; ++c)
+                    kv_tiles[(int64_t)i * g.n_window_tiles + n++] = (a * Gh + b) * Gw + c;
+    }
+    if (row_ptr && q_tiles) {
+        int32_t n = 0;
+        for (int32_t j = 0; j < g.n_tiles; ++j) {
+            row_ptr[j] = n;
+            for (int32_t i = 0; i < g.n_tiles; ++i) {
+                int32_t s[3];
+                window_starts(&g, offsets, i, s);
+                if (window_holds(&g, s, j)) q_tiles[n++] = i;
+            }
+        }
+        row_ptr[g.n_tiles] = n;
+    }
+    return 0;
+}
+
+/* Forward on selected (b*heads + head, query tile) pairs.
+ * out: [n_sel][tile_tokens][d], lse: [n_sel][tile_tokens]; rows of a selection are the
+ * tokens of its query tile in raster order. */
+int oracle_fwd(const oracle_problem* p, const double* q, const double* k, const double* v, const int32_t* offsets,
+               int32_t n_sel, const int32_t* sel_bh, const int32_t* sel_tile, double* out, double* lse) {
+    geometry g;
+    if (make_geometry(p, &g)) return 1;
+    const int64_t nk = (int64_t)g.n_window_tiles * g.tile_tokens;
+    const int64_t slice = (int64_t)g.n_tokens * p->d;
+    int status = 0;
+#pragma omp parallel
+    {
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * nk);
+        double* P = (double*)malloc(sizeof(double) * nk);
+        if (!keys || !P) {
+#pragma omp atomic write
+            status = 2;
+        }
+#pragma omp for schedule(dynamic)
+        for (int64_t job = 0; job < (int64_t)n_sel * g.tile_tokens; ++job) {
+            if (!keys || !P) continue;
+            int32_t s = (int32_t)(job / g.tile_tokens), r = (int32_t)(job % g.tile_tokens);
+            const double* qb = q + sel_bh[s] * slice;
+            const double* kb = k + sel_bh[s] * slice;
+            const double* vb = v + sel_bh[s] * slice;
+            key_set(p, &g, offsets, sel_tile[s], keys);
+            int64_t n = tile_token(p, &g, sel_tile[s], r);
+            double l = softmax_row(p, qb + n * p->d, kb, keys, nk, P);
+            double* o = out + ((int64_t)s * g.tile_tokens + r) * p->d;
+            for (int32_t c = 0; c < p->d; ++c) o[c] = 0.0;
+            for (int64_t m = 0; m < nk; ++m) {
+                const double* vm = vb + keys[m] * p->d;
+                for (int32_t c = 0; c < p->d; ++c) o[c] += P[m] * vm[c];
+            }
+            lse[(int64_t)s * g.tile_tokens + r] = l;
+        }
+        free(keys);
+        free(P);
+    }
+    return status;
+}
+
+/* Backward for dq on selected (bh, query tile) pairs.  dq: [n_sel][tile_tokens][d]. */
+int oracle_bwd_dq(const oracle_problem* p, const double* q, const double* k, const double* v, const double* dout,
+                  const int32_t* offsets, int32_t n_sel, const int32_t* sel_bh, const int32_t* sel_tile, double* dq) {
+    geometry g;
+    if (make_geometry(p, &g)) return 1;
+    const int64_t nk = (int64_t)g.n_window_tiles * g.tile_tokens;
+    const int64_t slice = (int64_t)g.n_tokens * p->d;
+    int status = 0;
+#pragma omp parallel
+    {
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * nk);
+        double* P = (double*)malloc(sizeof(double) * nk);
+        double* dP = (double*)malloc(sizeof(double) * nk);
+        if (!keys || !P || !dP) {
+#pragma omp atomic write
+            status = 2;
+        }
+#pragma omp for schedule(dynamic)
+        for (int64_t job = 0; job < (int64_t)n_sel * g.tile_tokens; ++job) {
+            if (!keys || !P || !dP) continue;
+            int32_t s = (int32_t)(job / g.tile_tokens), r = (int32_t)(job % g.tile_tokens);
+            const double* qb = q + sel_bh[s] * slice;
+            const double* kb = k + sel_bh[s] * slice;
+            const double* vb = v + sel_bh[s] * slice;
+            const double* dob = dout + sel_bh[s] * slice;
+            key_set(p, &g, offsets, sel_tile[s], keys);
+            int64_t n = tile_token(p, &g, sel_tile[s], r);
+            softmax_row(p, qb + n * p->d, kb, keys, nk, P);
+            double D = 0.0;
+            for (int64_t m = 0; m < nk; ++m) {
+                dP[m] = dot(dob + n * p->d, vb + keys[m] * p->d, p->d);
+                D += P[m] * dP[m];
+            }
+            double* o = dq + ((int64_t)s * g.tile_tokens + r) * p->d;
+            for (int32_t c = 0; c < p->d; ++c) o[c] = 0.0;
+            for (int64_t m = 0; m < nk; ++m) {
+                double dS = P[m] * (dP[m] - D);
+                const double* km = kb + keys[m] * p->d;
+                for (int32_t c = 0; c < p->d; ++c) o[c] += p->scale * dS * km[c];
+            }
+        }
+        free(keys);
+        free(P);
+        free(dP);
+    }
+    return status;
+}
+
+/* Backward for dk and dv on selected (bh, key tile) pairs.  For each selected key tile j,
+ * every query token whose window holds j contributes.  dk, dv: [n_sel][tile_tokens][d],
+ * rows in the key tile's raster order. */
+int oracle_bwd_dkdv(const oracle_problem* p, const double* q, const double* k, const double* v, const double* dout,
+                    const int32_t* offsets, int32_t n_sel, const int32_t* sel_bh, const int32_t* sel_tile,
+                    double* dk, double* dv) {
+    geometry g;
+    if (make_geometry(p, &g)) return 1;
+    const int64_t nk = (int64_t)g.n_window_tiles * g.tile_tokens;
+    const int64_t slice = (int64_t)g.n_tokens * p->d;
+    const int64_t tile_elems = (int64_t)g.tile_tokens * p->d;
+    int32_t* q_list = (int32_t*)malloc(sizeof(int32_t) * g.n_tiles);
+    if (!q_list) return 2;
+    int status = 0;
+    memset(dk, 0, sizeof(double) * n_sel * tile_elems);
+    memset(dv, 0, sizeof(double) * n_sel * tile_elems);
+    for (int32_t s = 0; s < n_sel; ++s) {
+        const int32_t j = sel_tile[s];
+        int32_t nq = 0;
+        for (int32_t i = 0; i < g.n_tiles; ++i) {
+            int32_t st[3];
+            window_starts(&g, offsets, i, st);
+            if (window_holds(&g, st, j)) q_list[nq++] = i;
+        }
+        const double* qb = q + sel_bh[s] * slice;
+        const double* kb = k + sel_bh[s] * slice;
+        const double* vb = v + sel_bh[s] * slice;
+        const double* dob = dout + sel_bh[s] * slice;
+        double* dks = dk + s * tile_elems;
+        double* dvs = dv + s * tile_elems;
+#pragma omp parallel
+        {
+            int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * nk);
+            double* P = (double*)malloc(sizeof(double) * nk);
+            double* dP = (double*)malloc(sizeof(double) * nk);
+            double* dk_local = (double*)calloc(tile_elems, sizeof(double));
+            double* dv_local = (double*)calloc(tile_elems, sizeof(double));
+            int ok = keys && P && dP && dk_local && dv_local;
+            if (!ok) {
+#pragma omp atomic write
+                status = 2;
+            }
+#pragma omp for schedule(dynamic)
+            for (int64_t job = 0; job < (int64_t)nq * g.tile_tokens; ++job) {
+                if (!ok) continue;
+                int32_t i = q_list[job / g.tile_tokens], r = (int32_t)(job % g.tile_tokens);
+                key_set(p, &g, offsets, i, keys);
+                int64_t n = tile_token(p, &g, i, r);
+                softmax_row(p, qb + n * p->d, kb, keys, nk, P);
+                double D = 0.0;
+                for (int64_t m = 0; m < nk; ++m) {
+                    dP[m] = dot(dob + n * p->d, vb + keys[m] * p->d, p->d);
+                    D += P[m] * dP[m];
+                }
+                /* key tile j sits at position pos of the window's tile list, so its r-th
+                 * token is entry pos * tile_tokens + r of the key set */
+                int32_t st[3];
+                window_starts(&g, offsets, i, st);
+                int64_t pos = window_position(&g, st, j);
+                for (int32_t rk = 0; rk < g.tile_tokens; ++rk) {
+                    int64_t m = pos * g.tile_tokens + rk;
+                    double dS = P[m] * (dP[m] - D);
+                    for (int32_t c = 0; c < p->d; ++c) {
+                        dk_local[(int64_t)rk * p->d + c] += p->scale * dS * qb[n * p->d + c];
+                        dv_local[(int64_t)rk * p->d + c] += P[m] * dob[n * p->d + c];
+                    }
+                }
+            }
+            if (ok) {
+#pragma omp critical
+                for (int64_t e = 0; e < tile_elems; ++e) {
+                    dks[e] += dk_local[e];
+                    dvs[e] += dv_local[e];
+                }
+            }
+            free(keys);
+            free(P);
+            free(dP);
+            free(dk_local);
+            free(dv_local);
+        }
+    }
+    free(q_list);
+    return status;
+}

@@ -1,0 +1,352 @@
+"""Pins for the fp64 oracle: facts the definition fixes, checked without the oracle's own code.
+
+The operator is 3D Deformable Slide Attention ("MegaSlide-DiT: Memory-Centric Adaptation
+and Deformable Local Attention for Efficient Video Diffusion", abstract) in the
+tile-granular sliding-window form of "Fast Video Generation with Sliding Tile Attention"
+(abstract).  The pages print no worked example, so the oracle is pinned by:
+
+* hand-worked plans (tests/golden/plan_hand.txt);
+* an independent characterisation of the window start (the in-grid start whose centre is
+  nearest the shifted centre), by brute force over all tiny grids;
+* a window covering the grid = dense attention (a separately written numpy formula and
+  torch's scaled_dot_product_attention in float64);
+* a 1x1x1 window = block-diagonal attention;
+* softmax rows sum to one (V = 1 gives O = 1; V = identity exposes P), and the LSE
+  normalises each row;
+* masked dense attention with the brute-force mask = the windowed oracle;
+* backward = central finite differences of L = sum(O * dO) in float64;
+* dv = P^T dO with P read off the forward (V = identity).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dsa_inputs import WORKLOADS, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------------------------
+# independent helpers (written from the definition, sharing nothing with the oracle)
+
+def nearest_start(centre: int, w_eff: int, G: int) -> int:
+    """Among in-grid starts s in [0, G - w'], the one whose window centre s + floor(w'/2)
+    is nearest the shifted centre (the distance is V-shaped in s, so the minimiser is unique)."""
+    cands = list(range(0, G - w_eff + 1))
+    dist = [abs(s + w_eff // 2 - centre) for s in cands]
+    best = min(dist)
+    assert dist.count(best) == 1
+    return cands[dist.index(best)]
+
+
+def brute_mask(grid, tile, window, offsets):
+    """[N, N] boolean: key token m is in the window of query token n."""
+    T, H, W = grid
+    tt, th, tw = tile
+    G = (T // tt, H // th, W // tw)
+    weff = [min(w, g) for w, g in zip(window, G)]
+    off = np.asarray(offsets).reshape(-1, 3)
+    coords = np.array([(t, h, w) for t in range(T) for h in range(H) for w in range(W)])
+    tcoord = coords // np.array(tile)
+    lin = (tcoord[:, 0] * G[1] + tcoord[:, 1]) * G[2] + tcoord[:, 2]
+    N = len(coords)
+    mask = np.zeros((N, N), bool)
+    for n in range(N):
+        i = tcoord[n]
+        o = off[lin[n]]
+        s = [nearest_start(int(i[a] + o[a]), weff[a], G[a]) for a in range(3)]
+        inside = np.ones(N, bool)
+        for a in range(3):
+            inside &= (tcoord[:, a] >= s[a]) & (tcoord[:, a] < s[a] + weff[a])
+        mask[n] = inside
+    return mask
+
+
+def dense_attention_np(q, k, v, scale, mask=None):
+    """Plain softmax attention in float64 over [BH, N, d] arrays, optional [N, N] mask."""
+    s = np.einsum("bnc,bmc->bnm", q, k) * scale
+    if mask is not None:
+        s = np.where(mask[None], s, -np.inf)
+    mx = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - mx)
+    z = e.sum(axis=-1, keepdims=True)
+    return np.einsum("bnm,bmc->bnc", e / z, v), (mx + np.log(z))[..., 0]
+
+
+def flat(x, geo):
+    return np.asarray(x, dtype=np.float64).reshape(geo.B * geo.heads, geo.n_tokens, geo.d)
+
+
+def rand_inputs(geo, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    shape = (geo.B, geo.heads) + geo.grid + (geo.d,)
+    return [torch.randn(shape, generator=g, dtype=torch.float64) * scale for _ in range(4)]
+
+
+def rand_offsets(geo, lo, hi, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(lo, hi + 1, (geo.n_tiles, 3), generator=g).to(torch.int32)
+
+
+# ------------------------------------------------------------------------------------
+# plan
+
+def _golden_cases():
+    cases = []
+    with open(os.path.join(GOLDEN, "plan_hand.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = [list(map(int, p.split())) for p in line.split("|")]
+            cases.append(parts)
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_cases())
+def test_plan_hand_worked(case):
+    G, window, tile, off, start, keys = case
+    n = G[0] * G[1] * G[2]
+    offsets = np.zeros((n, 3), np.int32)
+    i = (tile[0] * G[1] + tile[1]) * G[2] + tile[2]
+    offsets[i] = off
+    starts, kv, _, _ = oracle.plan(G, window, offsets)
+    assert list(starts[i]) == start
+    assert list(kv[i]) == keys
+
+
+def test_plan_nearest_centre_brute_force():
+    """Every 1D grid G <= 6, window <= 7, offset in [-G, G]: start = nearest in-grid start."""
+    for G in range(1, 7):
+        for w in range(1, 8):
+            for axis in range(3):
+                for o in range(-G, G + 1):
+                    Gs = [1, 1, 1]
+                    Gs[axis] = G
+                    ws = [1, 1, 1]
+                    ws[axis] = w
+                    offsets = np.zeros((G, 3), np.int32)
+                    offsets[:, axis] = o
+                    starts, kv, _, _ = oracle.plan(Gs, ws, offsets)
+                    weff = min(w, G)
+                    for i in range(G):
+                        assert starts[i, axis] == nearest_start(i + o, weff, G)
+                        assert list(kv[i]) == list(range(starts[i, axis], starts[i, axis] + weff))
+
+
+def test_plan_inverse_is_transpose():
+    rng = np.random.default_rng(0)
+    for trial in range(40):
+        G = list(rng.integers(1, 6, size=3))
+        window = list(rng.integers(1, 7, size=3))
+        n = int(np.prod(G))
+        offsets = rng.integers(-4, 5, size=(n, 3)).astype(np.int32)
+        starts, kv, row_ptr, q_tiles = oracle.plan(G, window, offsets)
+        wt = int(np.prod([min(w, g) for w, g in zip(window, G)]))
+        assert kv.shape == (n, wt)
+        assert row_ptr[-1] == n * wt
+        pairs_fwd = {(int(i), int(j)) for i in range(n) for j in kv[i]}
+        pairs_inv = set()
+        for j in range(n):
+            row = q_tiles[row_ptr[j]:row_ptr[j + 1]]
+            assert list(row) == sorted(row)
+            pairs_inv |= {(int(i), j) for i in row}
+        assert pairs_fwd == pairs_inv
+        for i in range(n):
+            assert list(kv[i]) == sorted(kv[i])
+            assert len(set(kv[i])) == wt
+
+
+# ------------------------------------------------------------------------------------
+# forward
+
+def test_full_window_equals_dense_attention():
+    """A window at least as large as the tile grid covers every key: dense attention."""
+    geo = oracle.Geometry(2, 2, 16, (4, 4, 6), (2, 2, 3), (3, 2, 5))
+    q, k, v, _ = rand_inputs(geo, 1)
+    off = rand_offsets(geo, -3, 3, 2)
+    out, lse = oracle.forward(geo, q, k, v, off)
+    ref_np, lse_np = dense_attention_np(flat(q, geo), flat(k, geo), flat(v, geo), geo.scale)
+    np.testing.assert_allclose(flat(out, geo), ref_np, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(lse_np.shape), lse_np, rtol=0, atol=1e-12)
+    sdpa = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(flat(q, geo)), torch.from_numpy(flat(k, geo)), torch.from_numpy(flat(v, geo)),
+        scale=geo.scale)
+    np.testing.assert_allclose(flat(out, geo), sdpa.numpy(), rtol=0, atol=1e-12)
+
+
+def test_peaky_scores_full_window():
+    """Large scores exercise the max subtraction: still equal to dense attention."""
+    geo = oracle.Geometry(1, 2, 8, (2, 4, 4), (1, 2, 2), (4, 4, 4))
+    q, k, v, _ = rand_inputs(geo, 3, scale=6.0)
+    off = torch.zeros((geo.n_tiles, 3), dtype=torch.int32)
+    out, lse = oracle.forward(geo, q, k, v, off)
+    sdpa = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(flat(q, geo)), torch.from_numpy(flat(k, geo)), torch.from_numpy(flat(v, geo)),
+        scale=geo.scale)
+    assert np.isfinite(lse).all()
+    np.testing.assert_allclose(flat(out, geo), sdpa.numpy(), rtol=0, atol=1e-10)
+
+
+def test_unit_window_equals_block_diagonal():
+    geo = oracle.Geometry(1, 3, 8, (2, 4, 6), (1, 2, 3), (1, 1, 1))
+    q, k, v, _ = rand_inputs(geo, 4)
+    off = torch.zeros((geo.n_tiles, 3), dtype=torch.int32)
+    out, _ = oracle.forward(geo, q, k, v, off)
+    tok = geo.tile_token_index()
+    qf, kf, vf, of = flat(q, geo), flat(k, geo), flat(v, geo), flat(out, geo)
+    for t in range(geo.n_tiles):
+        idx = tok[t]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(qf[:, idx]), torch.from_numpy(kf[:, idx]), torch.from_numpy(vf[:, idx]),
+            scale=geo.scale)
+        np.testing.assert_allclose(of[:, idx], ref.numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("window,lo,hi", [((2, 1, 3), -2, 2), ((3, 3, 3), -1, 1), ((1, 2, 2), -3, 3),
+                                          ((2, 2, 1), 0, 0)])
+def test_masked_dense_brute_force(window, lo, hi):
+    geo = oracle.Geometry(1, 2, 8, (3, 4, 6), (1, 2, 2), window)
+    q, k, v, _ = rand_inputs(geo, 5)
+    off = rand_offsets(geo, lo, hi, 6)
+    out, lse = oracle.forward(geo, q, k, v, off)
+    mask = brute_mask(geo.grid, geo.tile, geo.window, off.numpy())
+    assert (mask.sum(1) == geo.n_window_tiles * geo.tile_tokens).all()
+    ref, ref_lse = dense_attention_np(flat(q, geo), flat(k, geo), flat(v, geo), geo.scale, mask)
+    np.testing.assert_allclose(flat(out, geo), ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(ref_lse.shape), ref_lse, rtol=0, atol=1e-12)
+    sdpa = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(flat(q, geo)), torch.from_numpy(flat(k, geo)), torch.from_numpy(flat(v, geo)),
+        attn_mask=torch.from_numpy(mask), scale=geo.scale)
+    np.testing.assert_allclose(flat(out, geo), sdpa.numpy(), rtol=0, atol=1e-12)
+
+
+def test_rows_sum_to_one_and_lse_normalises():
+    geo = oracle.Geometry(1, 1, 48, (2, 4, 6), (1, 2, 3), (2, 1, 1))
+    q, k, _, _ = rand_inputs(geo, 7)
+    off = rand_offsets(geo, -1, 1, 8)
+    # V = 1 gives O = 1
+    ones = torch.ones_like(q)
+    out1, _ = oracle.forward(geo, q, k, ones, off)
+    np.testing.assert_allclose(out1, 1.0, rtol=0, atol=1e-13)
+    # V = identity (d = N) exposes the softmax rows
+    eye = torch.eye(geo.n_tokens, dtype=torch.float64).reshape((1, 1) + geo.grid + (geo.n_tokens,))
+    out, lse = oracle.forward(geo, q, k, eye, off)
+    P = flat(out, geo)[0]
+    mask = brute_mask(geo.grid, geo.tile, geo.window, off.numpy())
+    np.testing.assert_allclose(P.sum(1), 1.0, rtol=0, atol=1e-13)
+    assert (P[~mask] == 0).all()
+    assert (P[mask] > 0).all()
+    s = flat(q, geo)[0] @ flat(k, geo)[0].T * geo.scale
+    lse = lse.reshape(-1)
+    z = np.where(mask, np.exp(s - lse[:, None]), 0.0).sum(1)
+    np.testing.assert_allclose(z, 1.0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(P[mask], np.exp(s - lse[:, None])[mask], rtol=1e-12, atol=0)
+
+
+def test_oracle_selection_matches_full():
+    """Sampled (bh, tile) calls give the rows of the full call."""
+    geo = oracle.Geometry(2, 3, 16, (4, 4, 4), (2, 2, 2), (1, 2, 2))
+    q, k, v, _ = rand_inputs(geo, 9)
+    off = rand_offsets(geo, -1, 1, 10)
+    out, lse = oracle.forward(geo, q, k, v, off)
+    sel_bh = np.array([5, 0, 3], np.int32)
+    sel_t = np.array([7, 2, 0], np.int32)
+    o_t, l_t = oracle.forward_tiles(geo, q, k, v, off, (sel_bh, sel_t))
+    tok = geo.tile_token_index()
+    of, lf = flat(out, geo), lse.reshape(geo.B * geo.heads, -1)
+    for s in range(3):
+        np.testing.assert_array_equal(o_t[s], of[sel_bh[s], tok[sel_t[s]]])
+        np.testing.assert_array_equal(l_t[s], lf[sel_bh[s], tok[sel_t[s]]])
+
+
+# ------------------------------------------------------------------------------------
+# backward
+
+def _loss(geo, q, k, v, dout, off):
+    out, _ = oracle.forward(geo, q, k, v, off)
+    return float((out * dout.numpy()).sum())
+
+
+@pytest.mark.parametrize("window", [(2, 1, 1), (1, 1, 2), (3, 2, 2)])
+def test_backward_finite_differences(window):
+    geo = oracle.Geometry(1, 1, 3, (3, 2, 4), (1, 2, 2), window)
+    q, k, v, dout = rand_inputs(geo, 11)
+    off = rand_offsets(geo, -1, 1, 12)
+    dq, dk, dv = oracle.backward(geo, q, k, v, dout, off)
+    h = 1e-5
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros(x.numel())
+        xf = x.reshape(-1)
+        for e in range(x.numel()):
+            old = float(xf[e])
+            xf[e] = old + h
+            lp = _loss(geo, q, k, v, dout, off)
+            xf[e] = old - h
+            lm = _loss(geo, q, k, v, dout, off)
+            xf[e] = old
+            fd[e] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g.reshape(-1), fd, rtol=0, atol=2e-9, err_msg=name)
+
+
+def test_dv_is_pt_dout():
+    """dv = P^T dO, with P read off the forward by V = identity."""
+    geo = oracle.Geometry(1, 1, 24, (2, 2, 6), (1, 2, 2), (2, 1, 2))
+    q, k, v, _ = rand_inputs(geo, 13)
+    off = rand_offsets(geo, -1, 1, 14)
+    eye = torch.eye(geo.n_tokens, dtype=torch.float64).reshape((1, 1) + geo.grid + (geo.n_tokens,))
+    P = flat(oracle.forward(geo, q, k, eye, off)[0], geo)[0]
+    g = torch.Generator().manual_seed(15)
+    dout = torch.randn(q.shape, generator=g, dtype=torch.float64)
+    _, _, dv = oracle.backward(geo, q, k, v, dout, off)
+    np.testing.assert_allclose(flat(dv, geo)[0], P.T @ flat(dout, geo)[0], rtol=0, atol=1e-12)
+
+
+def test_backward_selection_matches_full():
+    geo = oracle.Geometry(2, 1, 8, (2, 4, 4), (1, 2, 2), (2, 1, 2))
+    q, k, v, dout = rand_inputs(geo, 16)
+    off = rand_offsets(geo, -1, 1, 17)
+    dq, dk, dv = oracle.backward(geo, q, k, v, dout, off)
+    sel = (np.array([1, 0], np.int32), np.array([3, 6], np.int32))
+    dq_t = oracle.backward_dq_tiles(geo, q, k, v, dout, off, sel)
+    dk_t, dv_t = oracle.backward_dkdv_tiles(geo, q, k, v, dout, off, sel)
+    tok = geo.tile_token_index()
+    for s in range(2):
+        bh, t = sel[0][s], sel[1][s]
+        # dk/dv sum per-thread partials in a thread-dependent order: equal up to rounding
+        np.testing.assert_allclose(dq_t[s], flat(dq, geo)[bh, tok[t]], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(dk_t[s], flat(dk, geo)[bh, tok[t]], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(dv_t[s], flat(dv, geo)[bh, tok[t]], rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------------------------------
+# workloads
+
+def test_workload_sizes():
+    """Derived sizes of the five workloads (effective window, keys per query, FLOP)."""
+    expect = {
+        "tiny_f32": (16, 12, 192, 2.52e7),
+        "bf16_16x32x32": (64, 27, 6912, 1.392e12),
+        "bf16_480p": (140, 45, 11520, 2.537e12),
+        "bf16_720p": (300, 27, 10368, 1.4677e13),
+        "adapt_480p_b2": (140, 45, 11520, 5.073e12),
+    }
+    for name, (nt, wt, kpq, flops) in expect.items():
+        w = WORKLOADS[name]
+        assert w.n_tiles == nt and w.window_tiles == wt and w.keys_per_query == kpq
+        assert abs(w.fwd_flops() / flops - 1) < 2e-3  # the table rounds to 4 digits
+
+
+def test_tiny_workload_inputs_are_seeded():
+    w = WORKLOADS["tiny_f32"]
+    a = make_inputs(w)
+    b = make_inputs(w)
+    assert torch.equal(a.q, b.q) and torch.equal(a.offsets, b.offsets)
+    assert a.q.dtype == torch.float32 and (a.offsets == 0).all()
+    w2 = WORKLOADS["bf16_16x32x32"].replace(heads=1, grid=(4, 8, 8))
+    c = make_inputs(w2)
+    assert c.q.dtype == torch.bfloat16
+    assert int(c.offsets.min()) >= -1 and int(c.offsets.max()) <= 1
