@@ -1,0 +1,361 @@
+"""Benchmark of 3D Deformable Slide Attention on B200: effective TFLOP/s and the fraction of
+the dense bf16 tensor peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dsa|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input: the window
+planner and the forward kernel (dsa_fwd), plus the backward (dsa_bwd) for workloads with
+a backward.  Effective FLOP per step = 4 * B * heads * N * keys_per_query * d forward,
+2.5x that backward.  Inputs (2.1 GB for the 720p-shaped workload) are larger than the
+126 MB L2, so no flush is needed between steps.  Multi-GPU (torchrun, one rank per GPU):
+every rank solves its own independent problem of the same shape (weak scaling, no
+data-path collective); the step time is the max over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle instead, on a
+bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dsa_inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+METRIC = "3D-DSA fwd/bwd effective TFLOP/s and % of B200 dense BF16 peak"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- inputs
+def device_inputs(w: Workload, device, seed_offset: int = 0):
+    """Seeded synthetic inputs drawn on the device (same distributions as dsa_inputs, which
+    draws on the CPU for the parity tests)."""
+    g = torch.Generator(device=device).manual_seed(1000 + w.seed + seed_offset)
+    shape = (w.B, w.heads) + tuple(w.grid) + (w.d,)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt)
+    k = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt)
+    v = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt)
+    dout = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt) if w.backward else None
+    gc = torch.Generator().manual_seed(w.seed + seed_offset)
+    lo, hi = w.offset_range
+    off = torch.randint(lo, hi + 1, (w.n_tiles, 3), generator=gc).to(torch.int32).to(device)
+    return q, k, v, dout, off
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def time_steps(step, steps: int, warmup: int, stream):
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps  # ms per step
+
+
+def run_workload(dsa, w: Workload, device, steps: int, warmup: int, seed_offset: int = 0, with_e2e: bool = False):
+    stream = torch.cuda.current_stream(device)
+    q, k, v, dout, off = device_inputs(w, device, seed_offset)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:5], dtype=torch.float32, device=device)
+    p = dsa.make_problem(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale,
+                         dsa.DSA_BF16 if w.dtype == "bf16" else dsa.DSA_F32)
+    ws_f = dsa.workspace(p, device)
+    res = {}
+
+    def fwd():
+        dsa.forward(q, k, v, off, w.tile, w.window, w.scale, out=out, lse=lse, ws=ws_f, stream=stream)
+
+    fwd()
+    res["fwd_ms"] = time_steps(fwd, steps, warmup, stream)
+    res["fwd_tflops"] = w.fwd_flops() / (res["fwd_ms"] * 1e-3) / 1e12
+    launches = 2  # planner + forward
+    step_ms = res["fwd_ms"]
+    step_flops = w.fwd_flops()
+    if w.backward:
+        ws_b = dsa.workspace(p, device, backward=True)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+
+        def bwd():
+            dsa.backward(q, k, v, out, lse, dout, off, w.tile, w.window, w.scale, dq=dq, dk=dk, dv=dv, ws=ws_b,
+                         stream=stream)
+
+        bwd()
+        res["bwd_ms"] = time_steps(bwd, steps, warmup, stream)
+        res["bwd_tflops"] = w.bwd_flops() / (res["bwd_ms"] * 1e-3) / 1e12
+        step_ms += res["bwd_ms"]
+        step_flops += w.bwd_flops()
+        launches += res.get("bwd_launches", 5)
+    res["step_ms"] = step_ms
+    res["step_flops"] = step_flops
+    res["launches_per_step"] = launches
+    st = dsa.device_status(stream)
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st} after {w.name}")
+    if with_e2e:
+        res["e2e"] = run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream)
+    return res
+
+
+def run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream):
+    """Same forward through the host-buffer entry point: H2D of q, k, v, offsets from pinned
+    memory, planner + forward, D2H of out and lse, all inside the timed region."""
+    qh, kh, vh = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+    oh_ = off.cpu().pin_memory()
+    outh = torch.empty_like(qh).pin_memory()
+    lseh = torch.empty(qh.shape[:5], dtype=torch.float32).pin_memory()
+    dev = torch.empty(dsa.forward_host_bytes(p), dtype=torch.uint8, device=device)
+
+    def step():
+        dsa.forward_host(p, qh, kh, vh, oh_, outh, lseh, dev, stream=stream)
+
+    ms = time_steps(step, max(1, steps // 2), max(1, warmup // 2), stream)
+    h2d = 3 * qh.numel() * qh.element_size() + oh_.numel() * 4
+    d2h = outh.numel() * outh.element_size() + lseh.numel() * 4
+    return {"value": w.fwd_flops() / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_sample_rate(w: Workload, target_s: float, max_tiles: int = 4096):
+    """Time the fp64 oracle (as it stands) on a growing sample of query tiles of head 0
+    until one run takes about target_s.  Returns (TFLOP/s, sample description, threads)."""
+    import oracle
+
+    inp_w = w.replace(B=1, heads=1)
+    g = torch.Generator().manual_seed(w.seed)
+    shape = (1, 1) + tuple(w.grid) + (w.d,)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q, k, v = (torch.randn(shape, generator=g).to(dt) for _ in range(3))
+    lo, hi = w.offset_range
+    off = torch.randint(lo, hi + 1, (w.n_tiles, 3), generator=g).to(torch.int32)
+    geo = oracle.Geometry.of(inp_w)
+    per_tile = 4.0 * w.tile_tokens * w.keys_per_query * w.d
+    n = 1
+    rng = np.random.default_rng(0)
+    while True:
+        tiles = rng.integers(0, geo.n_tiles, n).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.forward_tiles(geo, q, k, v, off, (np.zeros(n, np.int32), tiles))
+        dt_s = time.perf_counter() - t0
+        if dt_s >= target_s or n >= max_tiles:
+            break
+        n = min(max_tiles, max(n + 1, int(n * min(8.0, 1.2 * target_s / max(dt_s, 1e-3)))))
+    threads = len(os.sched_getaffinity(0))
+    return per_tile * n / dt_s / 1e12, f"{n} query tiles of one head ({n * w.tile_tokens} query rows), forward", \
+        threads, dt_s
+
+
+def reference_arm(args, w: Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    rates = []
+    desc, threads = "", 0
+    for i in range(args.warmup + args.steps):
+        r, desc, threads, _ = oracle_sample_rate(w, per_step)
+        if i >= args.warmup:
+            rates.append(r)
+    value = statistics.median(rates)
+    flops = w.fwd_flops() + (w.bwd_flops() if w.backward else 0)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops / (value * 1e12) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": list(w.grid),
+                       "tile": list(w.tile), "window": list(w.window), "pass": "fwd"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+def aggregate(per_rank_ms, flops_per_rank):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    t = max(per_rank_ms)
+    return len(per_rank_ms) * flops_per_rank / (t * 1e-3) / 1e12, t
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="bf16_720p", choices=[k for k, w in WORKLOADS.items() if w.dtype == "bf16"])
+    ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the per-workload table")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, w)
+        return
+
+    import video_dit_sparse_dsa_b200 as dsa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    dsa.load_library()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier()
+    if sampler:
+        sampler.start()
+    res = run_workload(dsa, w, device, args.steps, args.warmup, seed_offset=rank, with_e2e=(rank == 0))
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    step_ms = res["step_ms"]
+    if dist is not None:
+        t = torch.tensor([step_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+    value, _ = aggregate([step_ms] * world, res["step_flops"])
+
+    e2e = None
+    extra = {}
+    if rank == 0:
+        e2e = dict(res["e2e"])
+        e2e["value"] = res["e2e"]["value"] * world  # every rank runs the same host-buffer path
+    if rank == 0 and not args.no_extra:
+        for name, ow in WORKLOADS.items():
+            if ow.dtype != "bf16" or name == w.name:
+                continue
+            try:
+                r = run_workload(dsa, ow, device, max(3, args.steps // 2), 3)
+                extra[name] = {k2: round(v2, 4) for k2, v2 in r.items()
+                               if k2.endswith("_ms") or k2.endswith("_tflops")}
+            except Exception as e:  # report, do not hide: the line carries the error
+                extra[name] = {"error": str(e)}
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        rate, desc, threads, secs = oracle_sample_rate(w, 12.0)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc + f", {secs:.1f} s"}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    burst, sustained, src = peaks()
+    fwd_tflops = res["fwd_tflops"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": list(w.grid),
+                   "tile": list(w.tile), "window": list(w.window), "offsets": list(w.offset_range),
+                   "keys_per_query": w.keys_per_query, "pass": "fwd+bwd" if w.backward else "fwd",
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"independent problem per rank x{world}"},
+        "pct_of_peak": {"nominal_2250": 100 * fwd_tflops / NOMINAL_BF16_TFLOPS,
+                        f"{src}_{burst:g}": 100 * fwd_tflops / burst},
+        "roofline": {"bound": "tensor", "kernel": "fwd_bf16_kernel (timed with the planner, one dsa_fwd call)",
+                     "achieved": fwd_tflops, "peak": burst, "peak_kind": f"{src} burst bf16", "unit": "TFLOP/s",
+                     "frac": fwd_tflops / burst, "traffic": None},
+        "e2e": e2e, "gpu_launches": res["launches_per_step"] * args.steps, "clocks": clocks,
+        "cpu_baseline": cpu, "workloads": extra,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

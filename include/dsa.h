@@ -1,0 +1,134 @@
+/*
+ * dsa.h - C ABI of a B200 (sm_100a) library for 3D Deformable Slide Attention (3D-DSA).
+ *
+ * The operator.  3D-DSA is the motion-adaptive local attention of "MegaSlide-DiT:
+ * Memory-Centric Adaptation and Deformable Local Attention for Efficient Video Diffusion"
+ * (abstract), which makes attention cost linear in the sequence length; its window is
+ * tile-granular in the manner of "Fast Video Generation with Sliding Tile Attention"
+ * (abstract: attention over a local spatial-temporal region).  The pages give the operator
+ * in outline only; this library fixes the following concrete form.
+ *
+ *   - Tokens form a T x H x W grid, cut into tiles of tt x th x tw tokens; the tile grid is
+ *     G = (T/tt, H/th, W/tw).  Per axis the window is w' = min(w, G) tiles long.
+ *   - Query tile i carries an integer offset o (tile units).  Per axis its window starts at
+ *         s = clamp(i + o - floor(w'/2), 0, G - w'),
+ *     i.e. it is centred on i + o and then moved to lie fully inside the tile grid.
+ *   - Every query token n of tile i attends to exactly the tokens K(i) of the tiles in that
+ *     window:  O_n = sum_m softmax_m(scale * <q_n, k_m>) v_m,  LSE_n = ln sum_m exp(scale * <q_n, k_m>).
+ *
+ * Layouts (all contiguous, row-major):
+ *   q, k, v, out, dout, dq, dk, dv : [B, heads, T, H, W, d]  (token n = (t*H + h)*W + w)
+ *   lse                            : [B, heads, T, H, W] fp32, natural log
+ *   tile_offsets                   : int32 [nTiles, 3] = (dt, dh, dw) per query tile, tiles in
+ *                                    raster order (t outer, w inner); shared by all B and heads
+ *   starts                         : int32 [nTiles, 3] window start per axis (tile units)
+ *   kv_tiles                       : int32 [nTiles, Wt] key tiles of each window, ascending
+ *   inv_row_ptr, inv_q_tiles       : CSR of the inverse map: row j lists, ascending, the query
+ *                                    tiles whose window holds key tile j (nnz = nTiles * Wt)
+ *
+ * Ownership and execution.  Every pointer argument except `p` (and the host buffers of
+ * dsa_fwd_host) is DEVICE memory owned by the caller.  The library allocates no memory:
+ * scratch lives in the caller's workspace (dsa_workspace_size).  All work is enqueued on
+ * `stream` (a cudaStream_t; NULL = the legacy default stream) and returns without waiting.
+ * The library holds no per-call state and may be called from several threads.
+ *
+ * Errors.  Argument errors are returned synchronously and nothing is launched.  A launch
+ * error returns DSA_ERR_CUDA.  Kernels never trap: a device-side failure (a bounded wait
+ * that ran out, an index outside its buffer) is recorded in a device status word that
+ * dsa_device_status() reads.
+ *
+ * Supported: bf16 with d = 128 on the tensor-core path, where a 128-token chunk of a tile
+ * must be a whole number of (h, w) planes (th*tw divides 128 and 128/(th*tw) divides tt);
+ * fp32 with d in {64, 128} on the exact-fp32 path (any tile shape).  Pointers of the bf16
+ * path must be 16-byte aligned.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1, /* a size, pointer, alignment or shape is invalid */
+  DSA_ERR_UNSUPPORTED = 2, /* valid, but outside what the kernels implement */
+  DSA_ERR_CUDA = 3,        /* a CUDA call or launch failed */
+  DSA_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out */
+  DSA_ERR_WORKSPACE = 5,   /* workspace missing or smaller than dsa_workspace_size() */
+  DSA_ERR_DEVICE = 6       /* a device-side bounds check failed */
+} dsa_status_t;
+
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1 } dsa_dtype_t;
+
+typedef struct {
+  int32_t B, heads, d;  /* batch, heads, head dimension */
+  int32_t T, H, W;      /* token grid */
+  int32_t tile[3];      /* tt, th, tw: tokens per tile along T, H, W */
+  int32_t window[3];    /* wt, wh, ww: window length in tiles (limited to the tile grid) */
+  float scale;          /* softmax scale, > 0 (usually 1/sqrt(d)) */
+  int32_t dtype;        /* dsa_dtype_t of q, k, v, out, dout, dq, dk, dv */
+} dsa_problem_t;
+
+/* Which call a workspace is sized for. */
+typedef enum { DSA_WS_FWD = 0, DSA_WS_BWD = 1 } dsa_ws_kind_t;
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t dsa_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* dsa_status_string(dsa_status_t s);
+
+/* Plan sizes of a problem: *n_tiles = nTiles, *window_tiles = Wt (per-axis min(w, G)
+ * multiplied).  Host only; validates the shape (not the dtype-specific limits). */
+dsa_status_t dsa_plan_shape(const dsa_problem_t* p, int32_t* n_tiles, int32_t* window_tiles);
+
+/* Bytes of device workspace dsa_fwd (kind = DSA_WS_FWD) or dsa_bwd (DSA_WS_BWD) needs;
+ * 0 if the problem is invalid. */
+size_t dsa_workspace_size(const dsa_problem_t* p, int32_t kind);
+
+/* Window planner (the window rule above).  Writes starts[nTiles,3] and kv_tiles[nTiles,Wt];
+ * if both inv_row_ptr[nTiles+1] and inv_q_tiles[nTiles*Wt] are non-NULL also the inverse
+ * CSR.  All pointers are device memory. */
+dsa_status_t dsa_plan(const dsa_problem_t* p, const int32_t* tile_offsets, int32_t* starts, int32_t* kv_tiles,
+                      int32_t* inv_row_ptr, int32_t* inv_q_tiles, void* stream);
+
+/* Forward: plans the windows of tile_offsets, then writes out (dtype of p) and lse (fp32).
+ * workspace: device memory of at least dsa_workspace_size(p, DSA_WS_FWD) bytes, 256-byte
+ * aligned; its contents on entry do not matter. */
+dsa_status_t dsa_fwd(const dsa_problem_t* p, const void* q, const void* k, const void* v,
+                     const int32_t* tile_offsets, void* out, float* lse, void* workspace, size_t ws_bytes,
+                     void* stream);
+
+/* Forward from and to HOST memory (pinned, for asynchronous copies): copies q, k, v and
+ * tile_offsets into the caller's device buffer `dev`, runs dsa_fwd there, and copies out and
+ * lse back, all on `stream`.  dev: at least dsa_fwd_host_bytes(p) bytes of device memory,
+ * 256-byte aligned.  The host buffers must stay valid until the stream reaches the end of
+ * the call. */
+size_t dsa_fwd_host_bytes(const dsa_problem_t* p);
+dsa_status_t dsa_fwd_host(const dsa_problem_t* p, const void* q_host, const void* k_host, const void* v_host,
+                          const int32_t* tile_offsets_host, void* out_host, float* lse_host, void* dev,
+                          size_t dev_bytes, void* stream);
+
+/* Backward of L = sum(out * dout) (gradients of the forward above with respect to q, k, v;
+ * the integer offsets have none).  out and lse are the forward's outputs for the same
+ * inputs.  Writes dq, dk, dv (dtype of p).  workspace: at least
+ * dsa_workspace_size(p, DSA_WS_BWD) bytes; its contents on entry do not matter.
+ * bf16 only. */
+dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,
+                     const float* lse, const void* dout, const int32_t* tile_offsets, void* dq, void* dk, void* dv,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Waits for `stream`, then reads and clears the device status word of the current device.
+ * Returns DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE (or DSA_ERR_CUDA if the read failed);
+ * site / block (either may be NULL) receive where the first failure was raised. */
+dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

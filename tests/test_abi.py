@@ -1,0 +1,114 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol, and rejects
+bad arguments synchronously (no GPU is touched on these paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import video_dit_sparse_dsa_b200 as dsa
+from video_dit_sparse_dsa_b200 import build as dsa_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dsa_build.build()
+    return dsa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names, "no declarations found"
+    for n in names:
+        assert hasattr(lib, n), f"{n} missing from the library"
+    assert set(names) == set(dsa.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dsa_version() >= 100
+    for code in range(7):
+        assert lib.dsa_status_string(code)
+
+
+def _prob(**kw):
+    args = dict(B=1, heads=2, d=128, grid=(16, 32, 32), tile=(4, 8, 8), window=(3, 3, 3), dtype=dsa.DSA_BF16)
+    args.update(kw)
+    return dsa.make_problem(args["B"], args["heads"], args["d"], args["grid"], args["tile"], args["window"],
+                            dtype=args["dtype"])
+
+
+def test_plan_shape(lib):
+    assert dsa.plan_shape(_prob()) == (64, 27)
+    assert dsa.plan_shape(_prob(grid=(4, 8, 8), tile=(1, 4, 4), d=64, dtype=dsa.DSA_F32)) == (16, 12)
+    assert dsa.plan_shape(_prob(grid=(30, 48, 80), tile=(6, 8, 8))) == (300, 27)
+
+
+def test_workspace_sizes(lib):
+    p = _prob()
+    assert dsa.workspace_size(p) >= 4 * (64 * 3 + 64 * 27)
+    assert dsa.workspace_size(p, backward=True) > dsa.workspace_size(p)
+    bad = _prob(grid=(15, 32, 32))
+    assert dsa.workspace_size(bad) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # 256-byte aligned, never dereferenced on these paths
+
+
+def _fwd(lib, p, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, off=FAKE, out=FAKE, lse=FAKE, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    return lib.dsa_fwd(ctypes.byref(p), a["q"], a["k"], a["v"], a["off"], a["out"], a["lse"], a["ws"],
+                       a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(grid=(15, 32, 32)), 1),            # T not divisible by tt
+    (dict(window=(0, 3, 3)), 1),             # empty window
+    (dict(B=0), 1),                          # empty batch
+    (dict(d=64), 2),                         # bf16 needs d = 128
+    (dict(tile=(4, 3, 8), grid=(16, 30, 32)), 2),  # a 128-token chunk is not whole (h, w) planes
+    (dict(tile=(1, 8, 8), grid=(16, 32, 32)), 2),  # 64-token tile: no whole 128-token chunk
+    (dict(d=96, dtype=dsa.DSA_F32), 2),      # fp32 path: d in {64, 128}
+])
+def test_fwd_rejects_bad_problems(lib, kw, status):
+    assert _fwd(lib, _prob(**kw)) == status
+
+
+def test_fwd_rejects_bad_pointers_and_workspace(lib):
+    p = _prob()
+    assert _fwd(lib, p, q=None) == 1
+    assert _fwd(lib, p, out=ctypes.c_void_p((1 << 20) + 8)) == 1   # misaligned for TMA
+    assert _fwd(lib, p, ws=None) == 5
+    assert _fwd(lib, p, ws_bytes=16) == 5
+    assert _fwd(lib, p, ws=ctypes.c_void_p((1 << 20) + 64)) == 5   # workspace not 256-aligned
+    assert lib.dsa_fwd(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == 1
+    p.scale = -1.0
+    assert _fwd(lib, p) == 1
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    p = _prob()
+    f = FAKE
+    assert lib.dsa_bwd(ctypes.byref(p), f, f, f, f, f, f, f, f, f, None, f, 1 << 30, None) == 1
+    p32 = _prob(d=64, dtype=dsa.DSA_F32, grid=(4, 8, 8), tile=(1, 4, 4))
+    assert lib.dsa_bwd(ctypes.byref(p32), f, f, f, f, f, f, f, f, f, f, f, 1 << 30, None) == 2
+    assert lib.dsa_bwd(ctypes.byref(p), f, f, f, f, f, f, f, f, f, f, f, 16, None) == 5
+
+
+def test_plan_rejects_half_inverse(lib):
+    p = _prob()
+    assert lib.dsa_plan(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.dsa_plan(ctypes.byref(p), None, FAKE, FAKE, None, None, None) == 1
+
+
+def test_product_path_has_no_cpu_fallback(tmp_path):
+    with pytest.raises(RuntimeError):
+        dsa.load_library(str(tmp_path / "missing.so"))

@@ -1,0 +1,131 @@
+"""GPU forward (C ABI through the Python binding) against the fp64 oracle.
+
+Small problems are compared element by element in full; the full-size workloads are
+compared on sampled query tiles (every row of each sampled tile, including the first and
+last tile of the grid), in the same launch configuration the benchmark times."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import video_dit_sparse_dsa_b200 as dsa
+from dsa_inputs import WORKLOADS, Workload, make_inputs
+from tests._parity import assert_close, assert_lse_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(w: Workload, inp):
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    off = inp.offsets.cuda()
+    out, lse = dsa.forward(q, k, v, off, w.tile, w.window, w.scale)
+    st, site, block = dsa.device_status()
+    assert st == 0, f"device status {st} at site {site} block {block}"
+    return out, lse
+
+
+def compare_full(w: Workload, inp, out, lse):
+    geo = oracle.Geometry.of(w)
+    ref, ref_lse = oracle.forward(geo, inp.q, inp.k, inp.v, inp.offsets)
+    assert_close(out.float().cpu().numpy(), ref, w.dtype, "out")
+    assert_lse_close(lse.cpu().numpy(), ref_lse, w.dtype)
+
+
+def compare_sampled(w: Workload, inp, out, lse, n_samples=6, seed=0):
+    geo = oracle.Geometry.of(w)
+    rng = np.random.default_rng(seed)
+    BH = w.B * w.heads
+    bh = np.concatenate([[0, BH - 1], rng.integers(0, BH, n_samples)]).astype(np.int32)
+    tiles = np.concatenate([[0, geo.n_tiles - 1], rng.integers(0, geo.n_tiles, n_samples)]).astype(np.int32)
+    ref, ref_lse = oracle.forward_tiles(geo, inp.q, inp.k, inp.v, inp.offsets, (bh, tiles))
+    tok = geo.tile_token_index()
+    o = out.reshape(BH, geo.n_tokens, w.d)
+    l = lse.reshape(BH, geo.n_tokens)
+    idx_b = torch.as_tensor(np.repeat(bh, geo.tile_tokens), device=out.device, dtype=torch.long)
+    idx_t = torch.as_tensor(tok[tiles].reshape(-1), device=out.device, dtype=torch.long)
+    got = o[idx_b, idx_t].float().cpu().numpy().reshape(ref.shape)
+    got_lse = l[idx_b, idx_t].cpu().numpy().reshape(ref_lse.shape)
+    assert_close(got, ref, w.dtype, "out")
+    assert_lse_close(got_lse, ref_lse, w.dtype)
+
+
+def test_tiny_f32_full():
+    w = WORKLOADS["tiny_f32"]
+    inp = make_inputs(w)
+    out, lse = run_gpu(w, inp)
+    compare_full(w, inp, out, lse)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_f32_ragged_tiles_full(d):
+    """fp32 path with a tile of 3x2x5 tokens (not a power of two) and clamped windows."""
+    w = Workload("f32_odd", 2, 2, d, (6, 4, 10), (3, 2, 5), (3, 1, 2), (-2, 2), "f32", 11)
+    inp = make_inputs(w)
+    out, lse = run_gpu(w, inp)
+    compare_full(w, inp, out, lse)
+
+
+SMALL_BF16 = [
+    # several tiles, clamped windows at every edge, random offsets
+    Workload("bf16_small_a", 1, 3, 128, (8, 16, 24), (4, 8, 8), (3, 3, 3), (-2, 2), "bf16", 21),
+    # 384-token tiles (three 128-row chunks), window wider than the tile grid on one axis
+    Workload("bf16_small_b", 2, 1, 128, (12, 16, 16), (6, 8, 8), (5, 3, 1), (-1, 1), "bf16", 22),
+    # 128-token tiles of 2x8x8 and of 8x4x4 (one chunk = 4 h-planes ... whole planes)
+    Workload("bf16_small_c", 1, 2, 128, (8, 16, 16), (2, 8, 8), (3, 2, 2), (-3, 3), "bf16", 23),
+    Workload("bf16_small_d", 1, 2, 128, (16, 8, 8), (8, 4, 4), (1, 3, 3), (-1, 1), "bf16", 24),
+    # window covering the whole grid: dense attention
+    Workload("bf16_small_dense", 1, 2, 128, (8, 8, 16), (4, 8, 8), (9, 9, 9), (0, 0), "bf16", 25),
+    # 1x1x1 window: block-diagonal
+    Workload("bf16_small_diag", 1, 2, 128, (8, 16, 16), (4, 8, 8), (1, 1, 1), (0, 0), "bf16", 26),
+]
+
+
+@pytest.mark.parametrize("w", SMALL_BF16, ids=lambda w: w.name)
+def test_bf16_small_full(w):
+    inp = make_inputs(w)
+    out, lse = run_gpu(w, inp)
+    compare_full(w, inp, out, lse)
+
+
+def test_bf16_peaky_scores():
+    """Q and K scaled by 4: large score spread exercises the running-max rescale."""
+    w = Workload("bf16_peaky", 1, 2, 128, (8, 16, 16), (4, 8, 8), (3, 3, 3), (-1, 1), "bf16", 27)
+    inp = make_inputs(w)
+    inp.q = (inp.q.float() * 4).to(torch.bfloat16)
+    inp.k = (inp.k.float() * 4).to(torch.bfloat16)
+    out, lse = run_gpu(w, inp)
+    compare_full(w, inp, out, lse)
+
+
+def test_bf16_every_output_written():
+    """Outputs prefilled with NaN: every element must be overwritten."""
+    w = SMALL_BF16[1]
+    inp = make_inputs(w)
+    q, k, v, off = inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.offsets.cuda()
+    out = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:5], float("nan"), device=q.device)
+    dsa.forward(q, k, v, off, w.tile, w.window, w.scale, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("name", ["bf16_16x32x32", "bf16_480p", "bf16_720p", "adapt_480p_b2"])
+def test_bf16_workload_sampled(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    out, lse = run_gpu(w, inp)
+    compare_sampled(w, inp, out, lse)
+
+
+def test_forward_host_matches_device():
+    w = SMALL_BF16[0]
+    inp = make_inputs(w)
+    out, lse = run_gpu(w, inp)
+    p = dsa.make_problem(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale, dsa.DSA_BF16)
+    dev = torch.empty(dsa.forward_host_bytes(p), dtype=torch.uint8, device="cuda")
+    qh, kh, vh = inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(qh.shape[:5], dtype=torch.float32).pin_memory()
+    dsa.forward_host(p, qh, kh, vh, inp.offsets.contiguous(), oh, lh, dev)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, out.cpu()) and torch.equal(lh, lse.cpu())

@@ -1,0 +1,242 @@
+"""3D Deformable Slide Attention (3D-DSA) on NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/dsa.h`` (argument marshalling only: every
+step of the computation runs in the library's CUDA kernels).  PyTorch provides device
+memory and streams.  The library is built in-tree by ``video_dit_sparse_dsa_b200.build``;
+if it is missing, every entry point raises: there is no CPU fallback.
+
+Operator ("MegaSlide-DiT: Memory-Centric Adaptation and Deformable Local Attention for
+Efficient Video Diffusion", abstract; tile-granular window as in "Fast Video Generation
+with Sliding Tile Attention", abstract): for query tile i with integer offset o, the
+window of w' = min(w, G) tiles per axis starts at clamp(i + o - floor(w'/2), 0, G - w');
+each query token attends with softmax(scale q K^T) V to exactly the tokens of those tiles.
+
+Tensors: q, k, v, out, dout, dq, dk, dv are ``[B, heads, T, H, W, d]`` contiguous CUDA
+tensors (bf16 with d = 128, or fp32 with d in {64, 128} for the forward); lse is
+``[B, heads, T, H, W]`` fp32; tile offsets are int32 ``[nTiles, 3]`` in tile units.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libdsa_b200.so")
+
+DSA_F32, DSA_BF16 = 0, 1
+DSA_WS_FWD, DSA_WS_BWD = 0, 1
+_STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_CUDA",
+           4: "DSA_ERR_TIMEOUT", 5: "DSA_ERR_WORKSPACE", 6: "DSA_ERR_DEVICE"}
+
+# every symbol include/dsa.h declares
+EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_size", "dsa_plan", "dsa_fwd",
+           "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status")
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_STATUS.get(status, status)}")
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("heads", ctypes.c_int32), ("d", ctypes.c_int32), ("T", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("W", ctypes.c_int32), ("tile", ctypes.c_int32 * 3),
+                ("window", ctypes.c_int32 * 3), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: Optional[str] = None):
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"3D-DSA CUDA library not built ({p}); run python -m video_dit_sparse_dsa_b200.build")
+    lib = ctypes.CDLL(p)
+    vp, sz, i32, i32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)
+    pp = ctypes.POINTER(Problem)
+    lib.dsa_version.restype = i32
+    lib.dsa_version.argtypes = []
+    lib.dsa_status_string.restype = ctypes.c_char_p
+    lib.dsa_status_string.argtypes = [ctypes.c_int]
+    lib.dsa_plan_shape.argtypes = [pp, i32p, i32p]
+    lib.dsa_workspace_size.restype = sz
+    lib.dsa_workspace_size.argtypes = [pp, i32]
+    lib.dsa_plan.argtypes = [pp, vp, vp, vp, vp, vp, vp]
+    lib.dsa_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_fwd_host_bytes.restype = sz
+    lib.dsa_fwd_host_bytes.argtypes = [pp]
+    lib.dsa_fwd_host.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_device_status.argtypes = [vp, i32p, i32p]
+    for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status"):
+        getattr(lib, name).restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def make_problem(B, heads, d, grid, tile, window, scale=None, dtype=DSA_BF16) -> Problem:
+    p = Problem()
+    p.B, p.heads, p.d = int(B), int(heads), int(d)
+    p.T, p.H, p.W = (int(x) for x in grid)
+    for a in range(3):
+        p.tile[a] = int(tile[a])
+        p.window[a] = int(window[a])
+    p.scale = float(1.0 / math.sqrt(d)) if scale is None else float(scale)
+    p.dtype = int(dtype)
+    return p
+
+
+def _problem_of(q: torch.Tensor, tile, window, scale) -> Problem:
+    if q.dim() != 6:
+        raise ValueError("q must be [B, heads, T, H, W, d]")
+    if q.dtype == torch.bfloat16:
+        dt = DSA_BF16
+    elif q.dtype == torch.float32:
+        dt = DSA_F32
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    B, heads, T, H, W, d = q.shape
+    return make_problem(B, heads, d, (T, H, W), tile, window, scale, dt)
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise DsaError(st, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, like: torch.Tensor, dtype=None):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, q on {like.device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def plan_shape(problem: Problem):
+    lib = load_library()
+    n, wt = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib.dsa_plan_shape(ctypes.byref(problem), ctypes.byref(n), ctypes.byref(wt)), "dsa_plan_shape")
+    return n.value, wt.value
+
+
+def workspace_size(problem: Problem, backward: bool = False) -> int:
+    return int(load_library().dsa_workspace_size(ctypes.byref(problem), DSA_WS_BWD if backward else DSA_WS_FWD))
+
+
+def workspace(problem: Problem, device, backward: bool = False) -> torch.Tensor:
+    """A device workspace of the right size (torch's caching allocator returns 512-byte
+    aligned blocks)."""
+    return torch.empty(max(workspace_size(problem, backward), 256), dtype=torch.uint8, device=device)
+
+
+def plan(problem: Problem, offsets: torch.Tensor, inverse: bool = True, stream=None):
+    """Run the window planner.  Returns (starts, kv_tiles[, row_ptr, q_tiles]) on the device."""
+    lib = load_library()
+    n, wt = plan_shape(problem)
+    dev = offsets.device
+    if not offsets.is_cuda or offsets.dtype != torch.int32 or not offsets.is_contiguous() or offsets.numel() != 3 * n:
+        raise ValueError("offsets must be a contiguous int32 CUDA tensor [nTiles, 3]")
+    starts = torch.empty((n, 3), dtype=torch.int32, device=dev)
+    kv = torch.empty((n, wt), dtype=torch.int32, device=dev)
+    row_ptr = torch.empty(n + 1, dtype=torch.int32, device=dev) if inverse else None
+    q_tiles = torch.empty(n * wt, dtype=torch.int32, device=dev) if inverse else None
+    _check(lib.dsa_plan(ctypes.byref(problem), _ptr(offsets), _ptr(starts), _ptr(kv), _ptr(row_ptr), _ptr(q_tiles),
+                        ctypes.c_void_p(_stream(stream))), "dsa_plan")
+    return (starts, kv, row_ptr, q_tiles) if inverse else (starts, kv)
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, tile: Sequence[int],
+            window: Sequence[int], scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+            lse: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """3D-DSA forward.  Returns (out, lse)."""
+    lib = load_library()
+    p = _problem_of(q, tile, window, scale)
+    for t, name in ((k, "k"), (v, "v")):
+        _need(t, name, q, q.dtype)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
+    _need(q, "q", q)
+    _need(offsets, "offsets", q, torch.int32)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:5], dtype=torch.float32, device=q.device)
+    _need(out, "out", q, q.dtype)
+    _need(lse, "lse", q, torch.float32)
+    if ws is None:
+        ws = workspace(p, q.device)
+    _check(lib.dsa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(offsets), _ptr(out), _ptr(lse), _ptr(ws),
+                       ws.numel(), ctypes.c_void_p(_stream(stream))), "dsa_fwd")
+    return out, lse
+
+
+def forward_host_bytes(problem: Problem) -> int:
+    return int(load_library().dsa_fwd_host_bytes(ctypes.byref(problem)))
+
+
+def forward_host(problem: Problem, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+                 offsets_host: torch.Tensor, out_host: torch.Tensor, lse_host: torch.Tensor, dev: torch.Tensor,
+                 stream=None):
+    """3D-DSA forward from pinned host tensors through the caller's device buffer ``dev``
+    (uint8, at least forward_host_bytes(problem) bytes); asynchronous on ``stream``."""
+    lib = load_library()
+    for t in (q_host, k_host, v_host, offsets_host, out_host, lse_host):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host tensors must be contiguous CPU tensors")
+    _check(lib.dsa_fwd_host(ctypes.byref(problem), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(offsets_host),
+                            _ptr(out_host), _ptr(lse_host), _ptr(dev), dev.numel(), ctypes.c_void_p(_stream(stream))),
+           "dsa_fwd_host")
+
+
+def backward(q, k, v, out, lse, dout, offsets, tile, window, scale=None, dq=None, dk=None, dv=None, ws=None,
+             stream=None):
+    """3D-DSA backward of sum(out * dout).  Returns (dq, dk, dv)."""
+    lib = load_library()
+    p = _problem_of(q, tile, window, scale)
+    for t, name in ((k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, name, q, q.dtype)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
+    _need(q, "q", q)
+    _need(lse, "lse", q, torch.float32)
+    _need(offsets, "offsets", q, torch.int32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, name, q, q.dtype)
+    if ws is None:
+        ws = workspace(p, q.device, backward=True)
+    _check(lib.dsa_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(offsets),
+                       _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream))),
+           "dsa_bwd")
+    return dq, dk, dv
+
+
+def device_status(stream=None):
+    """Synchronise ``stream`` and read/clear the device status word: (status, site, block)."""
+    lib = load_library()
+    site, block = ctypes.c_int32(), ctypes.c_int32()
+    st = lib.dsa_device_status(ctypes.c_void_p(_stream(stream)), ctypes.byref(site), ctypes.byref(block))
+    return st, site.value, block.value

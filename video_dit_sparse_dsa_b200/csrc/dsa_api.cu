@@ -1,0 +1,381 @@
+// C ABI of the 3D-DSA library (declared in include/dsa.h): argument validation, workspace
+// layout, TMA tensor maps and kernel launches.  The whole library is this one translation
+// unit (the kernels are header-only), so the device status word is unique per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "../../include/dsa.h"
+#include "dsa_bwd_bf16.cuh"
+#include "dsa_device_status.cuh"
+#include "dsa_fwd_bf16.cuh"
+#include "dsa_fwd_f32.cuh"
+#include "dsa_plan.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Geom {
+  int G[3], w[3];
+  int n_tiles, Wt, tile_tokens;
+  int64_t N, BH;
+};
+
+dsa_status_t check_shape(const dsa_problem_t* p, Geom* g) {
+  if (p == nullptr) return DSA_ERR_INVALID_ARG;
+  if (p->B <= 0 || p->heads <= 0 || p->d <= 0 || p->T <= 0 || p->H <= 0 || p->W <= 0) return DSA_ERR_INVALID_ARG;
+  const int dims[3] = {p->T, p->H, p->W};
+  for (int a = 0; a < 3; ++a) {
+    if (p->tile[a] <= 0 || p->window[a] <= 0) return DSA_ERR_INVALID_ARG;
+    if (dims[a] % p->tile[a] != 0) return DSA_ERR_INVALID_ARG;
+    g->G[a] = dims[a] / p->tile[a];
+    g->w[a] = p->window[a] < g->G[a] ? p->window[a] : g->G[a];
+  }
+  if (!(p->scale > 0.f) || !std::isfinite(p->scale)) return DSA_ERR_INVALID_ARG;
+  if (p->dtype != DSA_F32 && p->dtype != DSA_BF16) return DSA_ERR_INVALID_ARG;
+  const int64_t n_tiles = static_cast<int64_t>(g->G[0]) * g->G[1] * g->G[2];
+  const int64_t N = static_cast<int64_t>(p->T) * p->H * p->W;
+  const int64_t BH = static_cast<int64_t>(p->B) * p->heads;
+  const int64_t tile_tokens = static_cast<int64_t>(p->tile[0]) * p->tile[1] * p->tile[2];
+  // the kernels index a (b, head) slice with 32-bit token counts and tile lists with int32
+  if (n_tiles * static_cast<int64_t>(g->w[0]) * g->w[1] * g->w[2] > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (N > INT32_MAX / 2 || BH > INT32_MAX / 2 || BH * N > (int64_t(1) << 40)) return DSA_ERR_UNSUPPORTED;
+  g->n_tiles = static_cast<int>(n_tiles);
+  g->Wt = g->w[0] * g->w[1] * g->w[2];
+  g->tile_tokens = static_cast<int>(tile_tokens);
+  g->N = N;
+  g->BH = BH;
+  return DSA_OK;
+}
+
+dsa_status_t check_kernel_limits(const dsa_problem_t* p, const Geom& g, bool backward) {
+  if (p->dtype == DSA_F32) {
+    if (backward) return DSA_ERR_UNSUPPORTED;
+    if (p->d != 64 && p->d != 128) return DSA_ERR_UNSUPPORTED;
+    if (g.n_tiles > 65535 * 64 || g.BH > 65535) return DSA_ERR_UNSUPPORTED;
+    return DSA_OK;
+  }
+  if (p->d != 128) return DSA_ERR_UNSUPPORTED;
+  const int plane = p->tile[1] * p->tile[2];
+  if (plane > 128 || 128 % plane != 0) return DSA_ERR_UNSUPPORTED;
+  if (p->tile[0] % (128 / plane) != 0) return DSA_ERR_UNSUPPORTED;
+  if (g.BH * g.n_tiles * (g.tile_tokens / 128) > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+struct FwdWorkspace {
+  int32_t* starts;
+  int32_t* kv_tiles;
+  size_t bytes;
+};
+
+FwdWorkspace fwd_workspace(const Geom& g, void* base) {
+  FwdWorkspace w;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  w.starts = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * 3 * g.n_tiles, kAlign);
+  w.kv_tiles = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * static_cast<size_t>(g.n_tiles) * g.Wt, kAlign);
+  w.bytes = off;
+  return w;
+}
+
+struct BwdWorkspace {
+  int32_t* starts;
+  int32_t* kv_tiles;
+  int32_t* row_ptr;
+  int32_t* q_tiles;
+  float* delta;  // D = rowsum(dO * O), [BH, N]
+  float* dq_acc; // fp32 dq accumulator, [BH, N, d]
+  size_t bytes;
+};
+
+BwdWorkspace bwd_workspace(const Geom& g, int d, void* base) {
+  BwdWorkspace w;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  w.starts = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * 3 * g.n_tiles, kAlign);
+  w.kv_tiles = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * static_cast<size_t>(g.n_tiles) * g.Wt, kAlign);
+  w.row_ptr = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * (g.n_tiles + 1), kAlign);
+  w.q_tiles = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * static_cast<size_t>(g.n_tiles) * g.Wt, kAlign);
+  w.delta = reinterpret_cast<float*>(b + off);
+  off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N), kAlign);
+  w.dq_acc = reinterpret_cast<float*>(b + off);
+  off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N) * d, kAlign);
+  w.bytes = off;
+  return w;
+}
+
+dsa::PlanGeom plan_geom(const Geom& g) {
+  dsa::PlanGeom pg;
+  for (int a = 0; a < 3; ++a) {
+    pg.G[a] = g.G[a];
+    pg.w[a] = g.w[a];
+  }
+  pg.n_tiles = g.n_tiles;
+  pg.n_window_tiles = g.Wt;
+  return pg;
+}
+
+dsa_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---- TMA tensor maps (driver entry point fetched through the runtime; no libcuda link)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// A [BH, T, H, W, 128] bf16 tensor seen as 5-D (d, W, H, T, BH); one box is a 128-token
+// chunk of a tile (tw x th x tcs tokens) times 64 channels, 128-byte swizzled.
+bool make_token_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, const Geom& g) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const int tcs = 128 / (p->tile[1] * p->tile[2]);
+  cuuint64_t dims[5] = {128, static_cast<cuuint64_t>(p->W), static_cast<cuuint64_t>(p->H),
+                        static_cast<cuuint64_t>(p->T), static_cast<cuuint64_t>(g.BH)};
+  cuuint64_t strides[4] = {128 * 2, static_cast<cuuint64_t>(p->W) * 128 * 2,
+                           static_cast<cuuint64_t>(p->H) * p->W * 128 * 2,
+                           static_cast<cuuint64_t>(p->T) * p->H * p->W * 128 * 2};
+  cuuint32_t box[5] = {64, static_cast<cuuint32_t>(p->tile[2]), static_cast<cuuint32_t>(p->tile[1]),
+                       static_cast<cuuint32_t>(tcs), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+dsa_status_t launch_plan(const Geom& g, const int32_t* offsets, int32_t* starts, int32_t* kv_tiles,
+                         int32_t* row_ptr, int32_t* q_tiles, cudaStream_t s) {
+  dsa::plan_kernel<<<1, 1024, 0, s>>>(plan_geom(g), offsets, starts, kv_tiles, row_ptr, q_tiles);
+  return launch_status();
+}
+
+dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
+                        const int32_t* kv_tiles, void* out, float* lse, cudaStream_t s) {
+  if (p->dtype == DSA_F32) {
+    dsa::FwdF32Params fp;
+    fp.q = static_cast<const float*>(q);
+    fp.k = static_cast<const float*>(k);
+    fp.v = static_cast<const float*>(v);
+    fp.kv_tiles = kv_tiles;
+    fp.out = static_cast<float*>(out);
+    fp.lse = lse;
+    fp.T = p->T;
+    fp.H = p->H;
+    fp.W = p->W;
+    fp.N = static_cast<int>(g.N);
+    fp.tt = p->tile[0];
+    fp.th = p->tile[1];
+    fp.tw = p->tile[2];
+    fp.tile_tokens = g.tile_tokens;
+    fp.G1 = g.G[1];
+    fp.G2 = g.G[2];
+    fp.Wt = g.Wt;
+    fp.scale = p->scale;
+    const int rows_per_block = dsa::kF32Threads / (p->d / 64);
+    dim3 grid(g.n_tiles, static_cast<unsigned>(g.BH), (g.tile_tokens + rows_per_block - 1) / rows_per_block);
+    if (p->d == 64)
+      dsa::fwd_f32_kernel<64><<<grid, dsa::kF32Threads, 0, s>>>(fp);
+    else
+      dsa::fwd_f32_kernel<128><<<grid, dsa::kF32Threads, 0, s>>>(fp);
+    return launch_status();
+  }
+  CUtensorMap tq, tk, tv;
+  if (!make_token_map(&tq, q, p, g) || !make_token_map(&tk, k, p, g) || !make_token_map(&tv, v, p, g))
+    return DSA_ERR_CUDA;
+  dsa::FwdBf16Params bp;
+  bp.kv_tiles = kv_tiles;
+  bp.out = static_cast<__nv_bfloat16*>(out);
+  bp.lse = lse;
+  bp.n_tiles = g.n_tiles;
+  bp.Wt = g.Wt;
+  bp.S = g.tile_tokens / 128;
+  bp.G1 = g.G[1];
+  bp.G2 = g.G[2];
+  bp.tt = p->tile[0];
+  bp.th = p->tile[1];
+  bp.tw = p->tile[2];
+  bp.tcs = 128 / (p->tile[1] * p->tile[2]);
+  bp.T = p->T;
+  bp.H = p->H;
+  bp.W = p->W;
+  bp.N = static_cast<int>(g.N);
+  bp.scale_log2 = p->scale * 1.4426950408889634f;
+  if (cudaFuncSetAttribute(dsa::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dsa::fwd1::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const unsigned n_units = static_cast<unsigned>(g.BH * g.n_tiles * bp.S);
+  dsa::fwd_bf16_kernel<<<n_units, dsa::fwd1::kThreads, dsa::fwd1::kSmemBytes, s>>>(tq, tk, tv, bp);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t dsa_version(void) { return 100; }
+
+const char* dsa_status_string(dsa_status_t s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported problem";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_WORKSPACE: return "workspace too small";
+    case DSA_ERR_DEVICE: return "device bounds check failed";
+  }
+  return "unknown status";
+}
+
+dsa_status_t dsa_plan_shape(const dsa_problem_t* p, int32_t* n_tiles, int32_t* window_tiles) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (n_tiles) *n_tiles = g.n_tiles;
+  if (window_tiles) *window_tiles = g.Wt;
+  return DSA_OK;
+}
+
+size_t dsa_workspace_size(const dsa_problem_t* p, int32_t kind) {
+  Geom g;
+  if (check_shape(p, &g) != DSA_OK) return 0;
+  if (kind == DSA_WS_FWD) return fwd_workspace(g, nullptr).bytes;
+  if (kind == DSA_WS_BWD) return bwd_workspace(g, p->d, nullptr).bytes;
+  return 0;
+}
+
+dsa_status_t dsa_plan(const dsa_problem_t* p, const int32_t* tile_offsets, int32_t* starts, int32_t* kv_tiles,
+                      int32_t* inv_row_ptr, int32_t* inv_q_tiles, void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!tile_offsets || !starts || !kv_tiles) return DSA_ERR_INVALID_ARG;
+  if ((inv_row_ptr == nullptr) != (inv_q_tiles == nullptr)) return DSA_ERR_INVALID_ARG;
+  return launch_plan(g, tile_offsets, starts, kv_tiles, inv_row_ptr, inv_q_tiles, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_fwd(const dsa_problem_t* p, const void* q, const void* k, const void* v,
+                     const int32_t* tile_offsets, void* out, float* lse, void* workspace, size_t ws_bytes,
+                     void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !tile_offsets || !out || !lse) return DSA_ERR_INVALID_ARG;
+  st = check_kernel_limits(p, g, false);
+  if (st != DSA_OK) return st;
+  const size_t elem_align = p->dtype == DSA_BF16 ? 16 : 4;
+  if (!aligned(q, elem_align) || !aligned(k, elem_align) || !aligned(v, elem_align) || !aligned(out, elem_align) ||
+      !aligned(lse, 4) || !aligned(tile_offsets, 4))
+    return DSA_ERR_INVALID_ARG;
+  FwdWorkspace ws = fwd_workspace(g, workspace);
+  if (workspace == nullptr || ws_bytes < ws.bytes || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_plan(g, tile_offsets, ws.starts, ws.kv_tiles, nullptr, nullptr, s);
+  if (st != DSA_OK) return st;
+  return launch_fwd(p, g, q, k, v, ws.kv_tiles, out, lse, s);
+}
+
+size_t dsa_fwd_host_bytes(const dsa_problem_t* p) {
+  Geom g;
+  if (check_shape(p, &g) != DSA_OK) return 0;
+  const size_t elem = p->dtype == DSA_BF16 ? 2 : 4;
+  const size_t tok = static_cast<size_t>(g.BH * g.N) * p->d * elem;
+  return 4 * round_up(tok, kAlign) + round_up(sizeof(float) * g.BH * g.N, kAlign) +
+         round_up(sizeof(int32_t) * 3 * g.n_tiles, kAlign) + fwd_workspace(g, nullptr).bytes;
+}
+
+dsa_status_t dsa_fwd_host(const dsa_problem_t* p, const void* q_host, const void* k_host, const void* v_host,
+                          const int32_t* tile_offsets_host, void* out_host, float* lse_host, void* dev,
+                          size_t dev_bytes, void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q_host || !k_host || !v_host || !tile_offsets_host || !out_host || !lse_host) return DSA_ERR_INVALID_ARG;
+  st = check_kernel_limits(p, g, false);
+  if (st != DSA_OK) return st;
+  if (dev == nullptr || dev_bytes < dsa_fwd_host_bytes(p) || !aligned(dev, kAlign)) return DSA_ERR_WORKSPACE;
+  const size_t elem = p->dtype == DSA_BF16 ? 2 : 4;
+  const size_t tok = static_cast<size_t>(g.BH * g.N) * p->d * elem;
+  const size_t lse_bytes = sizeof(float) * g.BH * g.N, off_bytes = sizeof(int32_t) * 3 * g.n_tiles;
+  uint8_t* b = static_cast<uint8_t*>(dev);
+  void* dq = b;
+  void* dk = b + round_up(tok, kAlign);
+  void* dv = b + 2 * round_up(tok, kAlign);
+  void* dout = b + 3 * round_up(tok, kAlign);
+  float* dlse = reinterpret_cast<float*>(b + 4 * round_up(tok, kAlign));
+  int32_t* doff = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(dlse) + round_up(lse_bytes, kAlign));
+  uint8_t* ws = reinterpret_cast<uint8_t*>(doff) + round_up(off_bytes, kAlign);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(dq, q_host, tok, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k_host, tok, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v_host, tok, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(doff, tile_offsets_host, off_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  st = dsa_fwd(p, dq, dk, dv, doff, dout, dlse, ws, fwd_workspace(g, nullptr).bytes, stream);
+  if (st != DSA_OK) return st;
+  if (cudaMemcpyAsync(out_host, dout, tok, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(lse_host, dlse, lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,
+                     const float* lse, const void* dout, const int32_t* tile_offsets, void* dq, void* dk, void* dv,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !out || !lse || !dout || !tile_offsets || !dq || !dk || !dv) return DSA_ERR_INVALID_ARG;
+  st = check_kernel_limits(p, g, true);
+  if (st != DSA_OK) return st;
+  const void* ptrs[] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned(ptr, 16)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4) || !aligned(tile_offsets, 4)) return DSA_ERR_INVALID_ARG;
+  BwdWorkspace ws = bwd_workspace(g, p->d, workspace);
+  if (workspace == nullptr || ws_bytes < ws.bytes || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
+  return DSA_ERR_UNSUPPORTED;
+}
+
+dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h[4] = {0, 0, 0, 0};
+  const int zero[4] = {0, 0, 0, 0};
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(h, dsa::g_status, sizeof(h)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(dsa::g_status, zero, sizeof(zero)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (site) *site = h[1];
+  if (block) *block = h[2];
+  if (h[0] == dsa::DSA_DEV_TIMEOUT) return DSA_ERR_TIMEOUT;
+  if (h[0] == dsa::DSA_DEV_BOUNDS) return DSA_ERR_DEVICE;
+  return DSA_OK;
+}
+
+}  // extern "C"
