@@ -361,7 +361,51 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
   if (!aligned(lse, 4) || !aligned(tile_offsets, 4)) return DSA_ERR_INVALID_ARG;
   BwdWorkspace ws = bwd_workspace(g, p->d, workspace);
   if (workspace == nullptr || ws_bytes < ws.bytes || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
-  return DSA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_plan(g, tile_offsets, ws.starts, ws.kv_tiles, ws.row_ptr, ws.q_tiles, s);
+  if (st != DSA_OK) return st;
+  const int64_t rows = g.BH * g.N;
+  dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), ws.delta, ws.dq_acc, rows);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_token_map(&tq, q, p, g) || !make_token_map(&tk, k, p, g) || !make_token_map(&tv, v, p, g) ||
+      !make_token_map(&tdo, dout, p, g))
+    return DSA_ERR_CUDA;
+  dsa::BwdBf16Params bp;
+  bp.row_ptr = ws.row_ptr;
+  bp.q_tiles = ws.q_tiles;
+  bp.lse = lse;
+  bp.delta = ws.delta;
+  bp.dq_acc = ws.dq_acc;
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.n_tiles = g.n_tiles;
+  bp.S = g.tile_tokens / 128;
+  bp.G1 = g.G[1];
+  bp.G2 = g.G[2];
+  bp.tt = p->tile[0];
+  bp.th = p->tile[1];
+  bp.tw = p->tile[2];
+  bp.tcs = 128 / (p->tile[1] * p->tile[2]);
+  bp.T = p->T;
+  bp.H = p->H;
+  bp.W = p->W;
+  bp.N = static_cast<int>(g.N);
+  bp.scale = p->scale;
+  bp.scale_log2 = p->scale * 1.4426950408889634f;
+  if (cudaFuncSetAttribute(dsa::bwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dsa::bwd1::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const unsigned n_units = static_cast<unsigned>(g.BH * g.n_tiles * bp.S);
+  dsa::bwd_bf16_kernel<<<n_units, dsa::bwd1::kThreads, dsa::bwd1::kSmemBytes, s>>>(tq, tk, tv, tdo, bp);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  const int64_t n8 = rows * p->d / 8;
+  dsa::bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
+      ws.dq_acc, static_cast<__nv_bfloat16*>(dq), p->scale, n8);
+  return launch_status();
 }
 
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {
