@@ -169,7 +169,7 @@ def run_workload(dsa, w: Workload, device, steps: int, warmup: int, seed_offset:
         res["bwd_tflops"] = w.bwd_flops() / (res["bwd_ms"] * 1e-3) / 1e12
         step_ms += res["bwd_ms"]
         step_flops += w.bwd_flops()
-        launches += res.get("bwd_launches", 5)
+        launches += 4  # planner (with inverse map), D preprocess, backward, dQ convert
     res["step_ms"] = step_ms
     res["step_flops"] = step_flops
     res["launches_per_step"] = launches
