@@ -260,6 +260,16 @@ def aggregate(per_rank_ms, flops_per_rank):
     return len(per_rank_ms) * flops_per_rank / (t * 1e-3) / 1e12, t
 
 
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """Max of a per-rank scalar over all ranks (every rank gets it); identity without a
+    process group."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -304,11 +314,7 @@ def main():
     res = run_workload(dsa, w, device, args.steps, args.warmup, seed_offset=rank, with_e2e=(rank == 0))
     barrier()
     clocks = sampler.stop() if sampler else None
-    step_ms = res["step_ms"]
-    if dist is not None:
-        t = torch.tensor([step_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = max_over_ranks(res["step_ms"], dist, device)
     value, _ = aggregate([step_ms] * world, res["step_flops"])
 
     e2e = None
