@@ -122,6 +122,20 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
                      const float* lse, const void* dout, const int32_t* tile_offsets, void* dq, void* dk, void* dv,
                      void* workspace, size_t ws_bytes, void* stream);
 
+/* Forward that allocates nothing and takes no workspace, for callers that cannot
+ * allocate device memory (a plugin whose host engine owns all device memory, a loop that
+ * must not call cudaMalloc because it can synchronize the device, a process with a memory
+ * budget fixed at start-up).  It computes exactly what dsa_fwd computes; the paper has no
+ * counterpart of this entry point.  The planner's scratch is a fixed 256 KB device array
+ * inside the library, held by every GPU that loads it until the process exits, so a
+ * problem must satisfy  roundup(3 * nTiles, 64) + nTiles * Wt <= 65536;  larger ones
+ * return DSA_ERR_UNSUPPORTED before anything is launched.  The first call on each device
+ * looks up the array's device address (make that first call before any stream capture).
+ * All calls on a device share the array: calls whose work overlaps on the GPU (other
+ * streams, other threads) race and must be serialized by the caller. */
+dsa_status_t dsa_fwd_noalloc(const dsa_problem_t* p, const void* q, const void* k, const void* v,
+                             const int32_t* tile_offsets, void* out, float* lse, void* stream);
+
 /* Waits for `stream`, then reads and clears the device status word of the current device.
  * Returns DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE (or DSA_ERR_CUDA if the read failed);
  * site / block (either may be NULL) receive where the first failure was raised. */

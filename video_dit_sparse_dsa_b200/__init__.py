@@ -34,7 +34,7 @@ _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "
 
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_size", "dsa_plan", "dsa_fwd",
-           "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status")
+           "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status", "dsa_fwd_noalloc")
 
 
 class DsaError(RuntimeError):
@@ -77,7 +77,9 @@ def load_library(path: Optional[str] = None):
     lib.dsa_fwd_host.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_device_status.argtypes = [vp, i32p, i32p]
-    for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status"):
+    lib.dsa_fwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp]
+    for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status",
+                 "dsa_fwd_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib

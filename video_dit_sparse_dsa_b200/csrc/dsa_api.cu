@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/dsa.h"
 #include "dsa_bwd_bf16.cuh"
@@ -423,3 +424,67 @@ dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Forward for callers that cannot allocate device memory.
+//
+// Some callers have no way to give this library a workspace: a plugin hosted by an
+// inference engine that owns every byte of device memory and hands its plugins none, a
+// latency-critical loop that must not call cudaMalloc because it can synchronize the
+// whole device, or a process whose memory budget is fixed when it starts.  For them the
+// planner's scratch (window starts and key-tile lists) lives in the fixed array below,
+// which every GPU that loads this library holds until the process exits.
+namespace {
+
+constexpr int kNoAllocPlanInts = 65536;  // 256 KB: 3 starts + Wt key tiles per query tile
+static __device__ __align__(256) int32_t g_noalloc_plan[kNoAllocPlanInts];
+
+constexpr int kNoAllocMaxDevices = 128;
+int32_t* g_noalloc_addr[kNoAllocMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Device address of g_noalloc_plan on the current device.  In host code the array's name
+// is only a host-side stand-in, so the address is looked up once per device, with that
+// device current, and cached.
+dsa_status_t noalloc_plan_address(int32_t** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return DSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_plan) != cudaSuccess || ptr == nullptr) return DSA_ERR_CUDA;
+    g_noalloc_addr[dev] = static_cast<int32_t*>(ptr);
+  }
+  *addr = g_noalloc_addr[dev];
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" dsa_status_t dsa_fwd_noalloc(const dsa_problem_t* p, const void* q, const void* k, const void* v,
+                                        const int32_t* tile_offsets, void* out, float* lse, void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !tile_offsets || !out || !lse) return DSA_ERR_INVALID_ARG;
+  st = check_kernel_limits(p, g, false);
+  if (st != DSA_OK) return st;
+  const size_t elem_align = p->dtype == DSA_BF16 ? 16 : 4;
+  if (!aligned(q, elem_align) || !aligned(k, elem_align) || !aligned(v, elem_align) || !aligned(out, elem_align) ||
+      !aligned(lse, 4) || !aligned(tile_offsets, 4))
+    return DSA_ERR_INVALID_ARG;
+  // starts first, then the key-tile lists on a 256-byte boundary
+  const int64_t starts_ints = (3 * static_cast<int64_t>(g.n_tiles) + 63) / 64 * 64;
+  const int64_t need = starts_ints + static_cast<int64_t>(g.n_tiles) * g.Wt;
+  if (need > kNoAllocPlanInts) return DSA_ERR_UNSUPPORTED;
+  int32_t* plan = nullptr;
+  st = noalloc_plan_address(&plan);
+  if (st != DSA_OK) return st;
+  // The planner writes every entry the forward reads, so nothing left from an earlier
+  // call needs clearing.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_plan(g, tile_offsets, plan, plan + starts_ints, nullptr, nullptr, s);
+  if (st != DSA_OK) return st;
+  return launch_fwd(p, g, q, k, v, plan + starts_ints, out, lse, s);
+}
