@@ -130,6 +130,14 @@ dsa::PlanGeom plan_geom(const Geom& g) {
   return pg;
 }
 
+// Number of SMs of the current device (persistent kernels launch one CTA per SM).
+dsa_status_t sm_count(int* n) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *n <= 0) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
 dsa_status_t launch_status() {
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
@@ -228,11 +236,15 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.W = p->W;
   bp.N = static_cast<int>(g.N);
   bp.scale_log2 = p->scale * 1.4426950408889634f;
+  bp.n_pass = (bp.S + 1) / 2;
+  bp.n_units = static_cast<int>(g.BH * bp.n_pass * g.n_tiles);
   if (cudaFuncSetAttribute(dsa::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dsa::fwd1::kSmemBytes) != cudaSuccess)
+                           dsa::fwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
-  const unsigned n_units = static_cast<unsigned>(g.BH * g.n_tiles * bp.S);
-  dsa::fwd_bf16_kernel<<<n_units, dsa::fwd1::kThreads, dsa::fwd1::kSmemBytes, s>>>(tq, tk, tv, bp);
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
+  dsa::fwd_bf16_kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, bp);
   return launch_status();
 }
 

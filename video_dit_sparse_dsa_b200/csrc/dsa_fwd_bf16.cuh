@@ -6,17 +6,23 @@
 // Video Diffusion", abstract, 3D-DSA; tile-granular window form from "Fast Video
 // Generation with Sliding Tile Attention", abstract).
 //
-// One CTA per 128-row query sub-tile (a box of tw x th x 128/(tw*th) tokens of one query
-// tile), 128 threads, thread r owning query row r (TMEM lane r).  For every 128-token
-// chunk of every key tile in the window:
-//   TMA: K and V chunk boxes -> shared memory (128-byte swizzle, two 64-column halves)
-//   tcgen05.mma: S = Q K^T into TMEM (fp32), 8 k-steps of 16
-//   softmax: each thread reads its S row from TMEM, updates its running max / sum
-//            (base-2 domain), writes P = exp2(S * scale * log2 e - m) as bf16 into shared
-//            memory in the operand layout of the next MMA
-//   tcgen05.mma: O_chunk = P V into TMEM; each thread folds it into its register
-//            accumulator with the running rescale factor.
-// The epilogue writes O / l as bf16 and LSE = (m + log2 l) * ln 2.
+// Persistent, warp-specialised kernel, one CTA per SM.  A work unit is a pair of 128-row
+// query chunks ("slots") of one query tile of one (batch, head); both slots share every
+// K/V chunk of the tile's window.  Roles:
+//   warp 8      TMA producer: Q of both slots, then K and V chunks through a 4-stage ring;
+//   warp 9      MMA issuer: S_i = Q_i K^T into TMEM, then O_i += P_i V with P_i read from
+//               TMEM (the scores' own columns), order S0 S1 | PV0 S0' PV1 S1' | ...;
+//   warps 0-3   softmax of slot 0, warps 4-7 softmax of slot 1: one thread per query row
+//               reads its S row from TMEM, keeps a running max m and sum l (base 2), writes
+//               P = exp2(S * scale * log2 e - m) as bf16 back into TMEM, and at the end of a
+//               unit normalises its O row and writes O and LSE.
+// The running max is only moved when it grows by more than 8 (a factor 256): P stays
+// <= 256, which bf16 and the fp32 accumulators hold exactly as well, and the O rescale
+// (a TMEM read-modify-write of the row) happens a few times per row instead of per chunk.
+// The result is exact: O = sum P V / sum P with the same reference max in both sums.
+//
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// Shared memory: Q0, Q1 (32 KB each), 4 K/V stages (32 KB each), barriers.
 #pragma once
 
 #include <stdint.h>
@@ -31,56 +37,92 @@ struct FwdBf16Params {
   float* lse;               // [B*heads, N]
   int n_tiles, Wt;
   int S;                    // 128-row chunks per tile
+  int n_pass;               // slot pairs per tile, ceil(S / 2)
+  int n_units;              // B*heads * n_pass * n_tiles
   int G1, G2;               // Gh, Gw
   int tt, th, tw, tcs;      // tile shape; t-extent of one 128-token chunk
   int T, H, W, N;
   float scale_log2;         // scale * log2(e)
 };
 
-namespace fwd1 {
-constexpr int kThreads = 128;
-constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 operand
-constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 128 x 64 swizzled half
-constexpr uint32_t kOffQ = 0, kOffK = kTileBytes, kOffV = 2 * kTileBytes, kOffP = 3 * kTileBytes;
-constexpr uint32_t kOffBar = 4 * kTileBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;  // + alignment slack
-constexpr uint32_t kTmemCols = 256;                    // S: [0,128), O: [128,256)
-constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
-constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, 0, 1);
-}  // namespace fwd1
+namespace fwd {
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kStages = 4;
+constexpr uint32_t kTileBytes = 128 * 128 * 2;
+constexpr uint32_t kHalfBytes = kTileBytes / 2;
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffKV + kStages * kTileBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // Q, K both K-major (smem)
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P from TMEM, V MN-major (smem)
+constexpr float kRescaleThreshold = 8.0f;                      // log2 units
 
-__global__ void __launch_bounds__(fwd1::kThreads, 1)
+struct Unit {
+  int bh, tile, sub0;
+  bool has1;
+};
+
+__device__ __forceinline__ Unit decode(const FwdBf16Params& p, int u) {
+  Unit x;
+  const int per_bh = p.n_pass * p.n_tiles;
+  x.bh = u / per_bh;
+  const int rem = u % per_bh;
+  const int pass = rem / p.n_tiles;
+  x.tile = rem % p.n_tiles;
+  x.sub0 = 2 * pass;
+  x.has1 = x.sub0 + 1 < p.S;
+  return x;
+}
+}  // namespace fwd
+
+__global__ void __launch_bounds__(fwd::kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, FwdBf16Params p) {
-  using namespace fwd1;
+  using namespace fwd;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw + pad;
-  uint64_t* load_bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* mma_bar = load_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(load_bar + 2);
-  volatile int* abort = reinterpret_cast<volatile int*>(load_bar + 3);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;   // [kStages]
+  uint64_t* kv_empty = bars + 6;  // [kStages]
+  uint64_t* s_full = bars + 10;   // [2]
+  uint64_t* p_full = bars + 12;   // [2]
+  uint64_t* o_done = bars + 14;   // [2]
+  uint64_t* o_free = bars + 16;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + 19);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int u = blockIdx.x;
-  const int sub = u % p.S;
-  const int tile = (u / p.S) % p.n_tiles;
-  const int bh = u / (p.S * p.n_tiles);
-  const int qt = tile / (p.G1 * p.G2), qh = (tile / p.G2) % p.G1, qw = tile % p.G2;
-  const int q_t0 = qt * p.tt + sub * p.tcs, q_h0 = qh * p.th, q_w0 = qw * p.tw;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_chunks = p.Wt * p.S;
 
   if (tid == 0) {
     tma_prefetch_map(&tmQ);
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
-    mbar_init(load_bar, 1);
-    mbar_init(mma_bar, 1);
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, 128);
+      mbar_init(o_done + i, 1);
+      mbar_init(o_free + i, 128);
+    }
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -88,136 +130,223 @@ __global__ void __launch_bounds__(fwd1::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
 
-  float acc[128];
-#pragma unroll
-  for (int c = 0; c < 128; ++c) acc[c] = 0.f;
-  float m = -INFINITY, l = 0.f;
-  uint32_t load_phase = 0, mma_phase = 0;
-  bool ok = true;
-
-  const int n_chunks = p.Wt * p.S;
-  for (int c = 0; c < n_chunks && ok; ++c) {
-    if (tid == 0) {
-      const int kt = p.kv_tiles[static_cast<int64_t>(tile) * p.Wt + c / p.S];
-      const int ks = c % p.S;
-      const int kt_t = kt / (p.G1 * p.G2), kt_h = (kt / p.G2) % p.G1, kt_w = kt % p.G2;
-      const int t0 = kt_t * p.tt + ks * p.tcs, h0 = kt_h * p.th, w0 = kt_w * p.tw;
-      mbar_arrive_expect_tx(load_bar, (c == 0 ? 3u : 2u) * kTileBytes);
-      if (c == 0) {
-        tma_load_5d(smem + kOffQ, &tmQ, load_bar, 0, q_w0, q_h0, q_t0, bh);
-        tma_load_5d(smem + kOffQ + kHalfBytes, &tmQ, load_bar, 64, q_w0, q_h0, q_t0, bh);
-      }
-      tma_load_5d(smem + kOffK, &tmK, load_bar, 0, w0, h0, t0, bh);
-      tma_load_5d(smem + kOffK + kHalfBytes, &tmK, load_bar, 64, w0, h0, t0, bh);
-      tma_load_5d(smem + kOffV, &tmV, load_bar, 0, w0, h0, t0, bh);
-      tma_load_5d(smem + kOffV + kHalfBytes, &tmV, load_bar, 64, w0, h0, t0, bh);
-    }
-    ok = mbar_wait(load_bar, load_phase, abort, 1);
-    load_phase ^= 1;
-    if (!__syncthreads_and(ok)) break;
-
-    // S = Q K^T
-    tc_fence_after();
-    if (tid == 0) {
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        mma_ss(tS, smem_desc_sw128(sbase + kOffQ + koff, 16, 1024), smem_desc_sw128(sbase + kOffK + koff, 16, 1024),
-               kIdescS, kk > 0);
-      }
-      mma_commit(mma_bar);
-    }
-    ok = mbar_wait(mma_bar, mma_phase, abort, 2);
-    mma_phase ^= 1;
-    if (!__syncthreads_and(ok)) break;
-    tc_fence_after();
-
-    // online softmax on this thread's row
-    uint32_t r[32];
-    float cmax = -INFINITY;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      tmem_ld32_wait(tS + lane_off + g * 32, r);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) cmax = fmaxf(cmax, __uint_as_float(r[j]));
-    }
-    const float m_new = fmaxf(m, cmax * p.scale_log2);
-    const float alpha = ex2_approx(m - m_new);
-    m = m_new;
-    float psum = 0.f;
-    const int rr = tid & 7;
-    const uint32_t prow = sbase + kOffP + (tid >> 3) * 1024 + rr * 128;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      tmem_ld32_wait(tS + lane_off + g * 32, r);
-      uint32_t pk[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * j]), p.scale_log2, -m_new));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * j + 1]), p.scale_log2, -m_new));
-        psum += p0 + p1;
-        pk[j] = pack_bf16x2(p0, p1);
-      }
-      // keys 32g .. 32g+31 live in half g/2, 16-byte chunks (g%2)*4 .. +3 of the row
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const int chunk = (g & 1) * 4 + q4;
-        st_shared_v4(prow + (g >> 1) * kHalfBytes + ((chunk ^ rr) << 4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2],
-                     pk[4 * q4 + 3]);
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int kv_load = 0, uc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+        const Unit x = decode(p, u);
+        const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
+        ok = mbar_wait(q_empty, (uc & 1) ^ 1, abort, 20);
+        if (!ok) break;
+        mbar_arrive_expect_tx(q_full, (x.has1 ? 2u : 1u) * kTileBytes);
+        for (int i = 0; i < (x.has1 ? 2 : 1); ++i) {
+          const int t0 = qt * p.tt + (x.sub0 + i) * p.tcs;
+          uint8_t* dst = smem + kOffQ + i * kTileBytes;
+          tma_load_5d(dst, &tmQ, q_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
+          tma_load_5d(dst + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
+        }
+        const int32_t* kv = p.kv_tiles + static_cast<int64_t>(x.tile) * p.Wt;
+        for (int j = 0; j < n_chunks && ok; ++j) {
+          const int kt = kv[j / p.S], ks = j % p.S;
+          const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
+          const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
+          for (int which = 0; which < 2; ++which, ++kv_load) {
+            const int st = kv_load % kStages;
+            ok = mbar_wait(kv_empty + st, ((kv_load / kStages) & 1) ^ 1, abort, 21);
+            if (!ok) break;
+            mbar_arrive_expect_tx(kv_full + st, kTileBytes);
+            uint8_t* dst = smem + kOffKV + st * kTileBytes;
+            const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+            tma_load_5d(dst, map, kv_full + st, 0, w0, h0, t0, x.bh);
+            tma_load_5d(dst + kHalfBytes, map, kv_full + st, 64, w0, h0, t0, x.bh);
+          }
+        }
       }
     }
-    l = l * alpha + psum;
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // O_chunk = P V
-    if (tid == 0) {
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int kv_use = 0, uc = 0;
+      int pc[2] = {0, 0}, uslot[2] = {0, 0};
+      bool ok = true;
+      auto issue_s = [&](int i, int stage) {
+        const uint32_t qa = sbase + kOffQ + i * kTileBytes, ka = sbase + kOffKV + stage * kTileBytes;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t poff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        mma_ss(tO, smem_desc_sw128(sbase + kOffP + poff, 16, 1024),
-               smem_desc_sw128(sbase + kOffV + kk * 2048, kHalfBytes, 1024), kIdescO, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          mma_ss(tmem + i * 128, smem_desc_sw128(qa + koff, 16, 1024), smem_desc_sw128(ka + koff, 16, 1024), kIdescS,
+                 kk > 0);
+        }
+        mma_commit(s_full + i);
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+        const Unit x = decode(p, u);
+        const int ns = x.has1 ? 2 : 1;
+        ok = mbar_wait(q_full, uc & 1, abort, 30);
+        if (!ok) break;
+        int k_idx = kv_use++;
+        ok = mbar_wait(kv_full + k_idx % kStages, (k_idx / kStages) & 1, abort, 31);
+        if (!ok) break;
+        tc_fence_after();
+        for (int i = 0; i < ns; ++i) issue_s(i, k_idx % kStages);
+        mma_commit(kv_empty + k_idx % kStages);
+        if (n_chunks == 1) mma_commit(q_empty);
+        for (int j = 0; j < n_chunks && ok; ++j) {
+          const int v_idx = kv_use++;
+          ok = mbar_wait(kv_full + v_idx % kStages, (v_idx / kStages) & 1, abort, 32);
+          if (!ok) break;
+          k_idx = (j + 1 < n_chunks) ? kv_use++ : -1;
+          for (int i = 0; i < ns && ok; ++i) {
+            ok = mbar_wait(p_full + i, pc[i] & 1, abort, 33);
+            ++pc[i];
+            if (ok && j == 0) ok = mbar_wait(o_free + i, (uslot[i] & 1) ^ 1, abort, 34);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t va = sbase + kOffKV + (v_idx % kStages) * kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024),
+                     kIdescPV, (j > 0) || (kk > 0));
+            mma_commit(o_done + i);
+            if (k_idx >= 0) {
+              if (i == 0) {
+                ok = mbar_wait(kv_full + k_idx % kStages, (k_idx / kStages) & 1, abort, 35);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              issue_s(i, k_idx % kStages);
+            }
+          }
+          if (!ok) break;
+          mma_commit(kv_empty + v_idx % kStages);
+          if (k_idx >= 0) mma_commit(kv_empty + k_idx % kStages);
+          if (j + 2 == n_chunks) mma_commit(q_empty);
+        }
+        for (int i = 0; i < ns; ++i) ++uslot[i];
       }
-      mma_commit(mma_bar);
     }
-    ok = mbar_wait(mma_bar, mma_phase, abort, 3);
-    mma_phase ^= 1;
-    if (!__syncthreads_and(ok)) break;
-    tc_fence_after();
+  } else {
+    // ------------------------------------------------------------------ softmax (slot i)
+    const int i = warp >> 2;
+    const int r = tid & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + i * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + i * 128 + lane_off;
+    int sc = 0, pv_base = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const Unit x = decode(p, u);
+      if (i == 1 && !x.has1) continue;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_chunks; ++j) {
+        ok = mbar_wait(s_full + i, sc & 1, abort, 40);
+        ++sc;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t s[128];
+        tmem_ld128_wait(tS, s);
+        float mxs[8];
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      tmem_ld32_wait(tO + lane_off + g * 32, r);
+        for (int e = 0; e < 8; ++e) mxs[e] = __uint_as_float(s[e]);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) acc[g * 32 + j] = fmaf(acc[g * 32 + j], alpha, __uint_as_float(r[j]));
+        for (int c = 8; c < 128; ++c) mxs[c & 7] = fmaxf(mxs[c & 7], __uint_as_float(s[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                               fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
+        const float m_new = fmaxf(m_used, mx * p.scale_log2);
+        const bool need = m_new > m_used + kRescaleThreshold;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2_approx(m_used - m_new);
+          m_used = m_new;
+        }
+        l *= alpha;
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(s[16 * g + 2 * e]), p.scale_log2, -m_used));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(s[16 * g + 2 * e + 1]), p.scale_log2, -m_used));
+            ps[e] += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          s[8 * g + 0] = pk[0];  // pack in place: P pairs of columns 16g..16g+15 -> word 8g..8g+7
+          s[8 * g + 1] = pk[1];
+          s[8 * g + 2] = pk[2];
+          s[8 * g + 3] = pk[3];
+          s[8 * g + 4] = pk[4];
+          s[8 * g + 5] = pk[5];
+          s[8 * g + 6] = pk[6];
+          s[8 * g + 7] = pk[7];
+        }
+        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = s[16 * g + e];
+          tmem_st16(tS + 16 * g, w);
+        }
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O_i holds sum P V up to chunk j-1 with the old reference max: rescale it
+          ok = mbar_wait(o_done + i, (pv_base + j - 1) & 1, abort, 41);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int g = 0; g < 4; ++g) {
+            uint32_t o[32];
+            tmem_ld32_wait(tO + 32 * g, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32 * g, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + i);
+      }
+      if (!ok) break;
+      // epilogue: O / l as bf16, LSE = (m + log2 l) ln 2
+      ok = mbar_wait(o_done + i, (pv_base + n_chunks - 1) & 1, abort, 42);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      pv_base += n_chunks;
+      const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
+      const int t0 = qt * p.tt + (x.sub0 + i) * p.tcs;
+      const int lw = r % p.tw, lh = (r / p.tw) % p.th, lt = r / (p.tw * p.th);
+      const int64_t tok = (static_cast<int64_t>(t0 + lt) * p.H + (qh * p.th + lh)) * p.W + (qw * p.tw + lw);
+      const float inv = 1.f / l;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * p.N + tok) * 128);
+#pragma unroll 1
+      for (int g = 0; g < 4; ++g) {
+        uint32_t o[32];
+        tmem_ld32_wait(tO + 32 * g, o);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
+          dst[4 * g + c] = v;
+        }
+      }
+      p.lse[static_cast<int64_t>(x.bh) * p.N + tok] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      tc_fence_before();
+      mbar_arrive(o_free + i);
     }
-    tc_fence_before();
-    __syncthreads();
   }
 
-  if (ok) {
-    const int lw = tid % p.tw, lh = (tid / p.tw) % p.th, lt = tid / (p.tw * p.th);
-    const int64_t tok = (static_cast<int64_t>(q_t0 + lt) * p.H + (q_h0 + lh)) * p.W + (q_w0 + lw);
-    const float inv = 1.f / l;
-    uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(bh) * p.N + tok) * 128);
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      uint4 v;
-      v.x = pack_bf16x2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
-      v.y = pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
-      v.z = pack_bf16x2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
-      v.w = pack_bf16x2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
-      dst[c] = v;
-    }
-    p.lse[static_cast<int64_t>(bh) * p.N + tok] = (m + __log2f(l)) * 0.69314718055994531f;
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace dsa
