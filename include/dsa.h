@@ -37,8 +37,9 @@
  * that ran out, an index outside its buffer) is recorded in a device status word that
  * dsa_device_status() reads.
  *
- * Supported: bf16 with d = 128 on the tensor-core path, where a 128-token chunk of a tile
- * must be a whole number of (h, w) planes (th*tw divides 128 and 128/(th*tw) divides tt);
+ * Supported: bf16 with d = 128 on the tensor-core path, where 64-token key chunks and
+ * 128-token query chunks of a tile must be whole (h, w) planes (th*tw divides 64 and
+ * 128/(th*tw) divides tt);
  * fp32 with d in {64, 128} on the exact-fp32 path (any tile shape).  Pointers of the bf16
  * path must be 16-byte aligned.
  */

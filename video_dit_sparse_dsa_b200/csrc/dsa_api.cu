@@ -62,8 +62,9 @@ dsa_status_t check_kernel_limits(const dsa_problem_t* p, const Geom& g, bool bac
     return DSA_OK;
   }
   if (p->d != 128) return DSA_ERR_UNSUPPORTED;
+  // a 128-token query chunk and a 64-token key chunk must both be whole (h, w) planes
   const int plane = p->tile[1] * p->tile[2];
-  if (plane > 128 || 128 % plane != 0) return DSA_ERR_UNSUPPORTED;
+  if (plane > 64 || 64 % plane != 0) return DSA_ERR_UNSUPPORTED;
   if (p->tile[0] % (128 / plane) != 0) return DSA_ERR_UNSUPPORTED;
   if (g.BH * g.n_tiles * (g.tile_tokens / 128) > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
@@ -159,12 +160,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// A [BH, T, H, W, 128] bf16 tensor seen as 5-D (d, W, H, T, BH); one box is a 128-token
-// chunk of a tile (tw x th x tcs tokens) times 64 channels, 128-byte swizzled.
-bool make_token_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, const Geom& g) {
+// A [BH, T, H, W, 128] bf16 tensor seen as 5-D (d, W, H, T, BH); one box is a chunk of
+// box_tokens tokens of a tile (tw x th x box_tokens/(tw*th)) times 64 channels, 128-byte
+// swizzled.
+bool make_token_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, const Geom& g, int box_tokens = 128) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
-  const int tcs = 128 / (p->tile[1] * p->tile[2]);
+  const int tcs = box_tokens / (p->tile[1] * p->tile[2]);
   cuuint64_t dims[5] = {128, static_cast<cuuint64_t>(p->W), static_cast<cuuint64_t>(p->H),
                         static_cast<cuuint64_t>(p->T), static_cast<cuuint64_t>(g.BH)};
   cuuint64_t strides[4] = {128 * 2, static_cast<cuuint64_t>(p->W) * 128 * 2,
@@ -175,6 +177,25 @@ bool make_token_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, c
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A [BH, T, H, W] fp32 per-token vector (LSE, D) seen as 4-D (W, H, T, BH); one box is
+// the box_tokens tokens of a tile chunk (tw x th x box_tokens/(tw*th)), no swizzle.
+bool make_row_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, const Geom& g, int box_tokens) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const int tcs = box_tokens / (p->tile[1] * p->tile[2]);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(p->W), static_cast<cuuint64_t>(p->H), static_cast<cuuint64_t>(p->T),
+                        static_cast<cuuint64_t>(g.BH)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(p->W) * 4, static_cast<cuuint64_t>(p->H) * p->W * 4,
+                           static_cast<cuuint64_t>(p->T) * p->H * p->W * 4};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(p->tile[2]), static_cast<cuuint32_t>(p->tile[1]),
+                       static_cast<cuuint32_t>(tcs), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -216,7 +237,7 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
     return launch_status();
   }
   CUtensorMap tq, tk, tv;
-  if (!make_token_map(&tq, q, p, g) || !make_token_map(&tk, k, p, g) || !make_token_map(&tv, v, p, g))
+  if (!make_token_map(&tq, q, p, g, 128) || !make_token_map(&tk, k, p, g, 128) || !make_token_map(&tv, v, p, g, 128))
     return DSA_ERR_CUDA;
   dsa::FwdBf16Params bp;
   bp.kv_tiles = kv_tiles;
@@ -236,8 +257,8 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.W = p->W;
   bp.N = static_cast<int>(g.N);
   bp.scale_log2 = p->scale * 1.4426950408889634f;
-  bp.n_pass = (bp.S + 1) / 2;
-  bp.n_units = static_cast<int>(g.BH * bp.n_pass * g.n_tiles);
+  bp.n_sub = static_cast<int>(g.BH * g.n_tiles * bp.S);
+  bp.n_units = (bp.n_sub + 1) / 2;
   if (cudaFuncSetAttribute(dsa::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            dsa::fwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
@@ -382,26 +403,28 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
       static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), ws.delta, ws.dq_acc, rows);
   st = launch_status();
   if (st != DSA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_token_map(&tq, q, p, g) || !make_token_map(&tk, k, p, g) || !make_token_map(&tv, v, p, g) ||
-      !make_token_map(&tdo, dout, p, g))
+  CUtensorMap tq, tk, tv, tdo, tlse, tdel;
+  if (!make_token_map(&tq, q, p, g, 64) || !make_token_map(&tk, k, p, g, 128) ||
+      !make_token_map(&tv, v, p, g, 128) || !make_token_map(&tdo, dout, p, g, 64) ||
+      !make_row_map(&tlse, lse, p, g, 64) || !make_row_map(&tdel, ws.delta, p, g, 64))
     return DSA_ERR_CUDA;
   dsa::BwdBf16Params bp;
   bp.row_ptr = ws.row_ptr;
   bp.q_tiles = ws.q_tiles;
-  bp.lse = lse;
-  bp.delta = ws.delta;
   bp.dq_acc = ws.dq_acc;
   bp.dk = static_cast<__nv_bfloat16*>(dk);
   bp.dv = static_cast<__nv_bfloat16*>(dv);
   bp.n_tiles = g.n_tiles;
-  bp.S = g.tile_tokens / 128;
+  bp.KU = g.tile_tokens / 128;
+  bp.QS = g.tile_tokens / 64;
+  bp.n_units = static_cast<int>(g.BH * g.n_tiles * bp.KU);
   bp.G1 = g.G[1];
   bp.G2 = g.G[2];
   bp.tt = p->tile[0];
   bp.th = p->tile[1];
   bp.tw = p->tile[2];
-  bp.tcs = 128 / (p->tile[1] * p->tile[2]);
+  bp.kcs = 128 / (p->tile[1] * p->tile[2]);
+  bp.qcs = 64 / (p->tile[1] * p->tile[2]);
   bp.T = p->T;
   bp.H = p->H;
   bp.W = p->W;
@@ -409,10 +432,12 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
   bp.scale = p->scale;
   bp.scale_log2 = p->scale * 1.4426950408889634f;
   if (cudaFuncSetAttribute(dsa::bwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dsa::bwd1::kSmemBytes) != cudaSuccess)
+                           dsa::bwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
-  const unsigned n_units = static_cast<unsigned>(g.BH * g.n_tiles * bp.S);
-  dsa::bwd_bf16_kernel<<<n_units, dsa::bwd1::kThreads, dsa::bwd1::kSmemBytes, s>>>(tq, tk, tv, tdo, bp);
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
+  dsa::bwd_bf16_kernel<<<grid, dsa::bwd::kThreads, dsa::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tlse, tdel, bp);
   st = launch_status();
   if (st != DSA_OK) return st;
   const int64_t n8 = rows * p->d / 8;

@@ -10,13 +10,7 @@
 //
 // Three kernels:
 //   bwd_preprocess : D = rowsum(dO * O) (fp32) and zeroes the fp32 dQ accumulator;
-//   bwd_bf16_kernel: key-major; one CTA per 128-key chunk of a key tile, walking the query
-//                    tiles of the inverse plan (CSR row of the key tile).  Per 128-query
-//                    chunk: S^T = K Q^T and dP^T = V dO^T on tcgen05 into TMEM; each thread
-//                    (one key row) forms P^T and dS^T in registers and stores them as bf16
-//                    operands; then dV += P^T dO and dK += dS^T Q accumulate in TMEM and
-//                    dQ_chunk = dS K lands in TMEM, from where each thread (one query row)
-//                    adds it to the fp32 accumulator in global memory;
+//   bwd_bf16_kernel: key-major and persistent (described above the kernel);
 //   bwd_dq_convert : dQ = scale * accumulator, as bf16.
 #pragma once
 
@@ -29,33 +23,43 @@ namespace dsa {
 struct BwdBf16Params {
   const int32_t* row_ptr;  // [n_tiles + 1] inverse plan
   const int32_t* q_tiles;  // [n_tiles * Wt]
-  const float* lse;        // [BH, N]
-  const float* delta;      // [BH, N]
-  float* dq_acc;           // [BH, N, 128]
+  float* dq_acc;           // [BH, N, 128] fp32, zeroed by bwd_preprocess
   __nv_bfloat16* dk;       // [BH, N, 128]
   __nv_bfloat16* dv;
-  int n_tiles, S;
+  int n_tiles;
+  int KU;                  // 128-key units per tile
+  int QS;                  // 64-query chunks per tile
+  int n_units;             // B*heads * n_tiles * KU
   int G1, G2;
-  int tt, th, tw, tcs;
+  int tt, th, tw;
+  int kcs;                 // t-extent of a 128-token key chunk
+  int qcs;                 // t-extent of a 64-token query chunk
   int T, H, W, N;
   float scale, scale_log2;
 };
 
-namespace bwd1 {
-constexpr int kThreads = 128;
-constexpr uint32_t kTileBytes = 128 * 128 * 2;
-constexpr uint32_t kHalfBytes = kTileBytes / 2;
-constexpr uint32_t kOffK = 0, kOffV = kTileBytes, kOffQ = 2 * kTileBytes, kOffDO = 3 * kTileBytes;
-constexpr uint32_t kOffP = 4 * kTileBytes, kOffDS = 5 * kTileBytes;
-constexpr uint32_t kOffLse = 6 * kTileBytes;      // 128 floats (base-2 LSE)
-constexpr uint32_t kOffD = kOffLse + 512;         // 128 floats
-constexpr uint32_t kOffBar = kOffD + 512;
-constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;
-constexpr uint32_t kTmemCols = 512;  // S^T / dQ, dP^T, dV, dK
-constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, 0, 0);   // both operands K-major
-constexpr uint32_t kIdescKM = idesc_bf16_f32(128, 128, 0, 1);   // B MN-major
-constexpr uint32_t kIdescMM = idesc_bf16_f32(128, 128, 1, 1);   // A and B MN-major
-}  // namespace bwd1
+namespace bwd {
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kStages = 3;
+constexpr uint32_t kKBytes = 128 * 128 * 2;  // K or V of a 128-key unit
+constexpr uint32_t kKHalf = kKBytes / 2;
+constexpr uint32_t kQBytes = 64 * 128 * 2;   // Q or dO of a 64-query chunk
+constexpr uint32_t kQHalf = kQBytes / 2;
+constexpr uint32_t kStageBytes = 2 * kQBytes + 1024;  // Q, dO, LSE (at +0) and D (at +512) vectors
+constexpr uint32_t kOffK = 0, kOffV = kKBytes;
+constexpr uint32_t kOffStage = 2 * kKBytes;
+constexpr uint32_t kOffDS = kOffStage + kStages * kStageBytes;  // 2 buffers of 128 x 64 bf16
+constexpr uint32_t kDSBytes = 128 * 64 * 2;
+constexpr uint32_t kOffRel = kOffDS + 2 * kDSBytes;  // 64 int32 token offsets within a query chunk
+constexpr uint32_t kOffBar = kOffRel + 256;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+constexpr uint32_t kTmemCols = 512;  // dV [0,128), dK [128,256), S^T buffers [256,384), dP^T / dQ^T [384,512)
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // K Q^T and V dO^T
+constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 128, 0, 1);  // P^T dO, dS^T Q
+constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, 64, 1, 1);    // K^T dS^T
+}  // namespace bwd
 
 __device__ __forceinline__ int64_t chunk_row_token(int r, int t0, int h0, int w0, int th, int tw, int H, int W) {
   const int lw = r % tw, lh = (r / tw) % th, lt = r / (tw * th);
@@ -105,45 +109,81 @@ __global__ void __launch_bounds__(256) bwd_dq_convert(const float* __restrict__ 
   reinterpret_cast<uint4*>(dq)[i] = v;
 }
 
-__global__ void __launch_bounds__(bwd1::kThreads, 1)
+// Persistent, warp-specialised backward; one CTA per SM, one 128-key chunk of a key tile
+// per work unit.  The unit walks the 64-query chunks of every query tile whose window
+// holds its key tile (the CSR row of the inverse plan).  Roles:
+//   warp 8      TMA producer: K and V of the unit, then per query chunk Q, dO, LSE and D
+//               through a 3-stage ring;
+//   warp 9      MMA issuer, per chunk c (buffer b = c % 2):
+//                 S^T_b = K Q_c^T, dP^T_b = V dO_c^T                 (TMEM, 64 columns each)
+//                 dV += P^T dO_c (P^T read from TMEM), dK += dS^T Q_c (dS^T from smem)
+//                 dQ^T_c = K^T dS^T into the dP^T_b columns
+//               so the scores of chunk c+1 are ready while chunk c's softmax runs;
+//   warps 0-3   one thread per key row: P^T = exp2(S^T * scale * log2 e - LSE_n * log2 e),
+//               dS^T = P^T (dP^T - D_n); P^T goes back into TMEM as bf16, dS^T into smem;
+//   warps 4-7   one thread per channel d: reads dQ^T_c and adds it to the fp32 dQ
+//               accumulator (a warp covers 32 consecutive channels of one query row); at
+//               the end of a unit, one thread per key row writes dV and scale * dK as bf16.
+// Barriers advance at most one phase ahead of their waiters (each refill of a buffer waits
+// for the previous consumer), so waiting by phase parity is unambiguous.
+__global__ void __launch_bounds__(bwd::kThreads, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const __grid_constant__ CUtensorMap tmLse, const __grid_constant__ CUtensorMap tmD,
                     BwdBf16Params p) {
-  using namespace bwd1;
+  using namespace bwd;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw + pad;
-  float* s_lse = reinterpret_cast<float*>(smem + kOffLse);
-  float* s_d = reinterpret_cast<float*>(smem + kOffD);
-  uint64_t* load_bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* mma_bar = load_bar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(load_bar + 2);
-  volatile int* abort = reinterpret_cast<volatile int*>(load_bar + 3);
+  int32_t* rel = reinterpret_cast<int32_t*>(smem + kOffRel);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_free = bars + 1;
+  uint64_t* ld_full = bars + 2;               // [kStages]
+  uint64_t* ld_empty = bars + 2 + kStages;    // [kStages]
+  uint64_t* s_full = bars + 2 + 2 * kStages;  // [2]
+  uint64_t* p_full = s_full + 2;              // [2]
+  uint64_t* dq_full = s_full + 4;             // [2]
+  uint64_t* dq_free = s_full + 6;             // [2]
+  uint64_t* dkv_full = s_full + 8;
+  uint64_t* dkv_free = s_full + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
+  volatile int* abort = reinterpret_cast<volatile int*>(s_full + 11);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int u = blockIdx.x;
-  const int ks = u % p.S;
-  const int kt = (u / p.S) % p.n_tiles;
-  const int bh = u / (p.S * p.n_tiles);
-  const int k_t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
-  const int k_h0 = ((kt / p.G2) % p.G1) * p.th;
-  const int k_w0 = (kt % p.G2) * p.tw;
-  const int row0 = p.row_ptr[kt], row1 = p.row_ptr[kt + 1];
-  const int n_chunks = (row1 - row0) * p.S;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     tma_prefetch_map(&tmQ);
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
     tma_prefetch_map(&tmDO);
-    mbar_init(load_bar, 1);
-    mbar_init(mma_bar, 1);
+    tma_prefetch_map(&tmLse);
+    tma_prefetch_map(&tmD);
+    mbar_init(kv_full, 1);
+    mbar_init(kv_free, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(ld_full + s, 1);
+      mbar_init(ld_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(p_full + b, 4);
+      mbar_init(dq_full + b, 1);
+      mbar_init(dq_free + b, 4);
+    }
+    mbar_init(dkv_full, 1);
+    mbar_init(dkv_free, 4);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (tid < 64) {
+    // token offset of row n of a 64-query chunk box, relative to the box origin
+    const int lw = tid % p.tw, lh = (tid / p.tw) % p.th, lt = tid / (p.tw * p.th);
+    rel[tid] = (lt * p.H + lh) * p.W + lw;
+  }
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -151,169 +191,261 @@ __global__ void __launch_bounds__(bwd1::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const int64_t slice = static_cast<int64_t>(bh) * p.N;
+  const uint32_t tDV = tmem, tDK = tmem + 128, tS = tmem + 256, tDP = tmem + 384;
 
-  uint32_t load_phase = 0, mma_phase = 0;
-  bool ok = true;
-  for (int c = 0; c < n_chunks && ok; ++c) {
-    const int qi = p.q_tiles[row0 + c / p.S];
-    const int qs = c % p.S;
-    const int q_t0 = (qi / (p.G1 * p.G2)) * p.tt + qs * p.tcs;
-    const int q_h0 = ((qi / p.G2) % p.G1) * p.th;
-    const int q_w0 = (qi % p.G2) * p.tw;
-    if (tid == 0) {
-      mbar_arrive_expect_tx(load_bar, (c == 0 ? 4u : 2u) * kTileBytes);
-      if (c == 0) {
-        tma_load_5d(smem + kOffK, &tmK, load_bar, 0, k_w0, k_h0, k_t0, bh);
-        tma_load_5d(smem + kOffK + kHalfBytes, &tmK, load_bar, 64, k_w0, k_h0, k_t0, bh);
-        tma_load_5d(smem + kOffV, &tmV, load_bar, 0, k_w0, k_h0, k_t0, bh);
-        tma_load_5d(smem + kOffV + kHalfBytes, &tmV, load_bar, 64, k_w0, k_h0, k_t0, bh);
+  // unit u -> (bh, key tile, 128-key chunk); its query chunks come from CSR row kt
+  auto unit_of = [&](int u, int& bh, int& kt, int& ku) {
+    ku = u % p.KU;
+    kt = (u / p.KU) % p.n_tiles;
+    bh = u / (p.KU * p.n_tiles);
+  };
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int ld = 0, uc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        int bh, kt, ku;
+        unit_of(u, bh, kt, ku);
+        const int row0 = p.row_ptr[kt], n = (p.row_ptr[kt + 1] - row0) * p.QS;
+        if (n == 0) continue;
+        ok = mbar_wait(kv_free, (uc & 1) ^ 1, abort, 50);
+        if (!ok) break;
+        ++uc;
+        const int k_t0 = (kt / (p.G1 * p.G2)) * p.tt + ku * p.kcs;
+        const int k_h0 = ((kt / p.G2) % p.G1) * p.th, k_w0 = (kt % p.G2) * p.tw;
+        mbar_arrive_expect_tx(kv_full, 2 * kKBytes);
+        tma_load_5d(smem + kOffK, &tmK, kv_full, 0, k_w0, k_h0, k_t0, bh);
+        tma_load_5d(smem + kOffK + kKHalf, &tmK, kv_full, 64, k_w0, k_h0, k_t0, bh);
+        tma_load_5d(smem + kOffV, &tmV, kv_full, 0, k_w0, k_h0, k_t0, bh);
+        tma_load_5d(smem + kOffV + kKHalf, &tmV, kv_full, 64, k_w0, k_h0, k_t0, bh);
+        for (int c = 0; c < n && ok; ++c, ++ld) {
+          const int qi = p.q_tiles[row0 + c / p.QS], qs = c % p.QS;
+          const int q_t0 = (qi / (p.G1 * p.G2)) * p.tt + qs * p.qcs;
+          const int q_h0 = ((qi / p.G2) % p.G1) * p.th, q_w0 = (qi % p.G2) * p.tw;
+          const int st = ld % kStages;
+          ok = mbar_wait(ld_empty + st, ((ld / kStages) & 1) ^ 1, abort, 51);
+          if (!ok) break;
+          uint8_t* dst = smem + kOffStage + st * kStageBytes;
+          mbar_arrive_expect_tx(ld_full + st, 2 * kQBytes + 512);
+          tma_load_5d(dst, &tmQ, ld_full + st, 0, q_w0, q_h0, q_t0, bh);
+          tma_load_5d(dst + kQHalf, &tmQ, ld_full + st, 64, q_w0, q_h0, q_t0, bh);
+          tma_load_5d(dst + kQBytes, &tmDO, ld_full + st, 0, q_w0, q_h0, q_t0, bh);
+          tma_load_5d(dst + kQBytes + kQHalf, &tmDO, ld_full + st, 64, q_w0, q_h0, q_t0, bh);
+          tma_load_4d(dst + 2 * kQBytes, &tmLse, ld_full + st, q_w0, q_h0, q_t0, bh);
+          tma_load_4d(dst + 2 * kQBytes + 512, &tmD, ld_full + st, q_w0, q_h0, q_t0, bh);
+        }
       }
-      tma_load_5d(smem + kOffQ, &tmQ, load_bar, 0, q_w0, q_h0, q_t0, bh);
-      tma_load_5d(smem + kOffQ + kHalfBytes, &tmQ, load_bar, 64, q_w0, q_h0, q_t0, bh);
-      tma_load_5d(smem + kOffDO, &tmDO, load_bar, 0, q_w0, q_h0, q_t0, bh);
-      tma_load_5d(smem + kOffDO + kHalfBytes, &tmDO, load_bar, 64, q_w0, q_h0, q_t0, bh);
     }
-    // per-query-row LSE (to base 2) and D of this chunk; thread r = query row r
-    const int64_t qtok = chunk_row_token(tid, q_t0, q_h0, q_w0, p.th, p.tw, p.H, p.W);
-    s_lse[tid] = p.lse[slice + qtok] * 1.4426950408889634f;
-    s_d[tid] = p.delta[slice + qtok];
-    ok = mbar_wait(load_bar, load_phase, abort, 11);
-    load_phase ^= 1;
-    if (!__syncthreads_and(ok)) break;
-
-    // S^T = K Q^T, dP^T = V dO^T
-    tc_fence_after();
-    if (tid == 0) {
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int ld = 0, uc = 0, sc = 0, pc = 0;
+      bool ok = true;
+      auto stage_addr = [&](int l) { return sbase + kOffStage + (l % kStages) * kStageBytes; };
+      // S^T and dP^T of the chunk in ring entry l into buffer sc % 2
+      auto issue_sdp = [&](int l) -> bool {
+        const int b = sc & 1;
+        if (!mbar_wait(ld_full + l % kStages, (l / kStages) & 1, abort, 61)) return false;
+        tc_fence_after();
+        const uint32_t qa = stage_addr(l), da = qa + kQBytes;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        mma_ss(tS, smem_desc_sw128(sbase + kOffK + koff, 16, 1024), smem_desc_sw128(sbase + kOffQ + koff, 16, 1024),
-               kIdescKK, kk > 0);
-      }
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
+          mma_ss(tS + b * 64, smem_desc_sw128(sbase + kOffK + ko, 16, 1024), smem_desc_sw128(qa + qo, 16, 1024),
+                 kIdescS, kk > 0);
+        }
+        // dP^T overwrites the dQ^T of chunk sc - 2: wait until it has been read out
+        if (sc >= 2 && !mbar_wait(dq_free + b, ((sc >> 1) - 1) & 1, abort, 62)) return false;
+        tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        mma_ss(tDP, smem_desc_sw128(sbase + kOffV + koff, 16, 1024),
-               smem_desc_sw128(sbase + kOffDO + koff, 16, 1024), kIdescKK, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
+          mma_ss(tDP + b * 64, smem_desc_sw128(sbase + kOffV + ko, 16, 1024), smem_desc_sw128(da + qo, 16, 1024),
+                 kIdescS, kk > 0);
+        }
+        mma_commit(s_full + b);
+        ++sc;
+        return true;
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        int bh, kt, ku;
+        unit_of(u, bh, kt, ku);
+        const int n = (p.row_ptr[kt + 1] - p.row_ptr[kt]) * p.QS;
+        if (n == 0) continue;
+        ok = mbar_wait(kv_full, uc & 1, abort, 60);
+        if (!ok) break;
+        const int ld0 = ld;
+        ld += n;
+        ok = issue_sdp(ld0);
+        if (ok && n > 1) ok = issue_sdp(ld0 + 1);
+        for (int c = 0; c < n && ok; ++c) {
+          const int b = pc & 1;
+          ok = mbar_wait(p_full + b, (pc >> 1) & 1, abort, 63);
+          ++pc;
+          if (ok && c == 0) ok = mbar_wait(dkv_free, (uc & 1) ^ 1, abort, 64);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qa = stage_addr(ld0 + c), da = qa + kQBytes;
+          const uint32_t dsa = sbase + kOffDS + b * kDSBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
+            mma_ts(tDV, tS + b * 64 + kk * 8, smem_desc_sw128(da + kk * 2048, kQHalf, 1024), kIdescAcc,
+                   (c > 0) || (kk > 0));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
+            mma_ss(tDK, smem_desc_sw128(dsa + kk * 32, 16, 1024), smem_desc_sw128(qa + kk * 2048, kQHalf, 1024),
+                   kIdescAcc, (c > 0) || (kk > 0));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
+            mma_ss(tDP + b * 64, smem_desc_sw128(sbase + kOffK + kk * 2048, kKHalf, 1024),
+                   smem_desc_sw128(dsa + kk * 2048, kKHalf, 1024), kIdescDQ, kk > 0);
+          mma_commit(dq_full + b);
+          mma_commit(ld_empty + (ld0 + c) % kStages);
+          if (c + 2 < n) ok = issue_sdp(ld0 + c + 2);
+        }
+        if (!ok) break;
+        mma_commit(dkv_full);
+        mma_commit(kv_free);
+        ++uc;
       }
-      mma_commit(mma_bar);
     }
-    ok = mbar_wait(mma_bar, mma_phase, abort, 12);
-    mma_phase ^= 1;
-    if (!__syncthreads_and(ok)) break;
-    tc_fence_after();
-
-    // thread = key row m: P^T and dS^T over the chunk's 128 query columns
-    const int rr = tid & 7;
-    const uint32_t prow = sbase + kOffP + (tid >> 3) * 1024 + rr * 128;
-    const uint32_t dsrow = sbase + kOffDS + (tid >> 3) * 1024 + rr * 128;
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------ P^T, dS^T (key rows)
+    const int m = tid;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    int cc = 0, ld = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      int bh, kt, ku;
+      unit_of(u, bh, kt, ku);
+      const int n = (p.row_ptr[kt + 1] - p.row_ptr[kt]) * p.QS;
+      for (int c = 0; c < n; ++c, ++cc, ++ld) {
+        const int b = cc & 1;
+        ok = mbar_wait(s_full + b, (cc >> 1) & 1, abort, 70);
+        if (ok) ok = mbar_wait(ld_full + ld % kStages, (ld / kStages) & 1, abort, 71);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float* lse = reinterpret_cast<const float*>(smem + kOffStage + (ld % kStages) * kStageBytes + 2 * kQBytes);
+        const float* dd = lse + 128;
+        uint32_t sr[64], dr[64];
+        tmem_ld64_wait(tS + lane_off + b * 64, sr);
+        tmem_ld64_wait(tDP + lane_off + b * 64, dr);
+        const uint32_t dsrow = sbase + kOffDS + b * kDSBytes + (m >> 3) * 1024 + (m & 7) * 128;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {  // query columns 8g..8g+7 form one 16-byte chunk
+          uint32_t pk[4], dk2[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int n0 = 8 * g + 2 * e;
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[n0]), p.scale_log2, -lse[n0] * 1.4426950408889634f));
+            const float p1 =
+                ex2_approx(fmaf(__uint_as_float(sr[n0 + 1]), p.scale_log2, -lse[n0 + 1] * 1.4426950408889634f));
+            pk[e] = pack_bf16x2(p0, p1);
+            dk2[e] = pack_bf16x2(p0 * (__uint_as_float(dr[n0]) - dd[n0]), p1 * (__uint_as_float(dr[n0 + 1]) - dd[n0 + 1]));
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sr[4 * g + e] = pk[e];  // packed P^T of columns 8g..8g+7
+          st_shared_v4(dsrow + ((g ^ (m & 7)) << 4), dk2[0], dk2[1], dk2[2], dk2[3]);
+        }
+        {
+          uint32_t w[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w[e] = sr[e];
+          tmem_st32(tS + lane_off + b * 64, w);
+        }
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + b);
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------------------------------ dQ out, dK/dV epilogue
+    const int t = tid - 128;  // channel d for dQ^T, key row for dK / dV
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int cc = 0, uc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      int bh, kt, ku;
+      unit_of(u, bh, kt, ku);
+      const int row0 = p.row_ptr[kt], n = (p.row_ptr[kt + 1] - row0) * p.QS;
+      const int64_t slice = static_cast<int64_t>(bh) * p.N;
+      for (int c = 0; c < n; ++c, ++cc) {
+        const int b = cc & 1;
+        ok = mbar_wait(dq_full + b, (cc >> 1) & 1, abort, 80);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld64_wait(tDP + lane_off + b * 64, r);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free + b);
+        const int qi = p.q_tiles[row0 + c / p.QS], qs = c % p.QS;
+        const int q_t0 = (qi / (p.G1 * p.G2)) * p.tt + qs * p.qcs;
+        const int q_h0 = ((qi / p.G2) % p.G1) * p.th, q_w0 = (qi % p.G2) * p.tw;
+        float* base = p.dq_acc + (slice + (static_cast<int64_t>(q_t0) * p.H + q_h0) * p.W + q_w0) * 128 + t;
+#pragma unroll
+        for (int nn = 0; nn < 64; ++nn) atomicAdd(base + static_cast<int64_t>(rel[nn]) * 128, __uint_as_float(r[nn]));
+      }
+      if (!ok) break;
+      // dV and scale * dK of the unit's 128 keys; zeros for a key tile no window holds
+      const int k_t0 = (kt / (p.G1 * p.G2)) * p.tt + ku * p.kcs;
+      const int k_h0 = ((kt / p.G2) % p.G1) * p.th, k_w0 = (kt % p.G2) * p.tw;
+      const int64_t ktok = chunk_row_token(t, k_t0, k_h0, k_w0, p.th, p.tw, p.H, p.W);
+      uint4* dv_dst = reinterpret_cast<uint4*>(p.dv + (slice + ktok) * 128);
+      uint4* dk_dst = reinterpret_cast<uint4*>(p.dk + (slice + ktok) * 128);
+      if (n > 0) {
+        ok = mbar_wait(dkv_full, uc & 1, abort, 81);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+      }
 #pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
-      uint32_t sr[32], dr[32];
-      tmem_ld32_wait(tS + lane_off + g * 32, sr);
-      tmem_ld32_wait(tDP + lane_off + g * 32, dr);
-      uint32_t pk[16], dk2[16];
+      for (int g = 0; g < 4; ++g) {
+        uint32_t a[32], bb[32];
+        if (n > 0) {
+          tmem_ld32_wait(tDV + lane_off + g * 32, a);
+          tmem_ld32_wait(tDK + lane_off + g * 32, bb);
+        } else {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int n0 = g * 32 + 2 * j;
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * j]), p.scale_log2, -s_lse[n0]));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * j + 1]), p.scale_log2, -s_lse[n0 + 1]));
-        const float d0 = p0 * (__uint_as_float(dr[2 * j]) - s_d[n0]);
-        const float d1 = p1 * (__uint_as_float(dr[2 * j + 1]) - s_d[n0 + 1]);
-        pk[j] = pack_bf16x2(p0, p1);
-        dk2[j] = pack_bf16x2(d0, d1);
+          for (int j = 0; j < 32; ++j) a[j] = bb[j] = 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 x, y;
+          x.x = pack_bf16x2(__uint_as_float(a[8 * j + 0]), __uint_as_float(a[8 * j + 1]));
+          x.y = pack_bf16x2(__uint_as_float(a[8 * j + 2]), __uint_as_float(a[8 * j + 3]));
+          x.z = pack_bf16x2(__uint_as_float(a[8 * j + 4]), __uint_as_float(a[8 * j + 5]));
+          x.w = pack_bf16x2(__uint_as_float(a[8 * j + 6]), __uint_as_float(a[8 * j + 7]));
+          y.x = pack_bf16x2(__uint_as_float(bb[8 * j + 0]) * p.scale, __uint_as_float(bb[8 * j + 1]) * p.scale);
+          y.y = pack_bf16x2(__uint_as_float(bb[8 * j + 2]) * p.scale, __uint_as_float(bb[8 * j + 3]) * p.scale);
+          y.z = pack_bf16x2(__uint_as_float(bb[8 * j + 4]) * p.scale, __uint_as_float(bb[8 * j + 5]) * p.scale);
+          y.w = pack_bf16x2(__uint_as_float(bb[8 * j + 6]) * p.scale, __uint_as_float(bb[8 * j + 7]) * p.scale);
+          dv_dst[g * 4 + j] = x;
+          dk_dst[g * 4 + j] = y;
+        }
       }
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const uint32_t off = (g >> 1) * kHalfBytes + ((((g & 1) * 4 + q4) ^ rr) << 4);
-        st_shared_v4(prow + off, pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        st_shared_v4(dsrow + off, dk2[4 * q4], dk2[4 * q4 + 1], dk2[4 * q4 + 2], dk2[4 * q4 + 3]);
+      if (n > 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dkv_free);
+        ++uc;
       }
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // dV += P^T dO, dK += dS^T Q, dQ_chunk = dS K
-    if (tid == 0) {
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t aoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        mma_ss(tDV, smem_desc_sw128(sbase + kOffP + aoff, 16, 1024),
-               smem_desc_sw128(sbase + kOffDO + kk * 2048, kHalfBytes, 1024), kIdescKM, (c > 0) || (kk > 0));
-      }
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t aoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        mma_ss(tDK, smem_desc_sw128(sbase + kOffDS + aoff, 16, 1024),
-               smem_desc_sw128(sbase + kOffQ + kk * 2048, kHalfBytes, 1024), kIdescKM, (c > 0) || (kk > 0));
-      }
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        mma_ss(tS, smem_desc_sw128(sbase + kOffDS + kk * 2048, kHalfBytes, 1024),
-               smem_desc_sw128(sbase + kOffK + kk * 2048, kHalfBytes, 1024), kIdescMM, kk > 0);
-      }
-      mma_commit(mma_bar);
-    }
-    ok = mbar_wait(mma_bar, mma_phase, abort, 13);
-    mma_phase ^= 1;
-    if (!__syncthreads_and(ok)) break;
-    tc_fence_after();
-
-    // thread = query row n: add its dQ row to the fp32 accumulator
-    float4* dst = reinterpret_cast<float4*>(p.dq_acc + (slice + qtok) * 128);
-#pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
-      uint32_t r[32];
-      tmem_ld32_wait(tS + lane_off + g * 32, r);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        atomicAdd(dst + g * 8 + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                               __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
-    }
-    tc_fence_before();
-    __syncthreads();
   }
 
-  if (ok) {
-    // thread = key row m: dV and scale * dK as bf16 (zeros for a key tile no window holds)
-    const int64_t ktok = chunk_row_token(tid, k_t0, k_h0, k_w0, p.th, p.tw, p.H, p.W);
-    uint4* dv_dst = reinterpret_cast<uint4*>(p.dv + (slice + ktok) * 128);
-    uint4* dk_dst = reinterpret_cast<uint4*>(p.dk + (slice + ktok) * 128);
-    tc_fence_after();
-#pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
-      uint32_t a[32], b[32];
-      if (n_chunks > 0) {
-        tmem_ld32_wait(tDV + lane_off + g * 32, a);
-        tmem_ld32_wait(tDK + lane_off + g * 32, b);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) a[j] = b[j] = 0u;
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint4 x, y;
-        x.x = pack_bf16x2(__uint_as_float(a[8 * j + 0]), __uint_as_float(a[8 * j + 1]));
-        x.y = pack_bf16x2(__uint_as_float(a[8 * j + 2]), __uint_as_float(a[8 * j + 3]));
-        x.z = pack_bf16x2(__uint_as_float(a[8 * j + 4]), __uint_as_float(a[8 * j + 5]));
-        x.w = pack_bf16x2(__uint_as_float(a[8 * j + 6]), __uint_as_float(a[8 * j + 7]));
-        y.x = pack_bf16x2(__uint_as_float(b[8 * j + 0]) * p.scale, __uint_as_float(b[8 * j + 1]) * p.scale);
-        y.y = pack_bf16x2(__uint_as_float(b[8 * j + 2]) * p.scale, __uint_as_float(b[8 * j + 3]) * p.scale);
-        y.z = pack_bf16x2(__uint_as_float(b[8 * j + 4]) * p.scale, __uint_as_float(b[8 * j + 5]) * p.scale);
-        y.w = pack_bf16x2(__uint_as_float(b[8 * j + 6]) * p.scale, __uint_as_float(b[8 * j + 7]) * p.scale);
-        dv_dst[g * 4 + j] = x;
-        dk_dst[g * 4 + j] = y;
-      }
-    }
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
 }
 
 }  // namespace dsa

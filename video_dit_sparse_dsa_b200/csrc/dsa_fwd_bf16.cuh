@@ -6,10 +6,13 @@
 // Video Diffusion", abstract, 3D-DSA; tile-granular window form from "Fast Video
 // Generation with Sliding Tile Attention", abstract).
 //
-// Persistent, warp-specialised kernel, one CTA per SM.  A work unit is a pair of 128-row
-// query chunks ("slots") of one query tile of one (batch, head); both slots share every
-// K/V chunk of the tile's window.  Roles:
-//   warp 8      TMA producer: Q of both slots, then K and V chunks through a 4-stage ring;
+// Persistent, warp-specialised kernel, one CTA per SM.  A work unit is two 128-row query
+// chunks ("slots"): consecutive chunks in (batch*head, query tile, chunk) order, so both
+// slots usually belong to the same query tile and share every K/V chunk of its window;
+// when a tile has an odd number of chunks, a unit may pair the last chunk of one tile with
+// the first of the next, and then each slot streams its own window's K/V.  Roles:
+//   warp 8      TMA producer: Q of both slots, then per step the K chunk(s) and V chunk(s)
+//               through a 5-stage shared-memory ring;
 //   warp 9      MMA issuer: S_i = Q_i K^T into TMEM, then O_i += P_i V with P_i read from
 //               TMEM (the scores' own columns), order S0 S1 | PV0 S0' PV1 S1' | ...;
 //   warps 0-3   softmax of slot 0, warps 4-7 softmax of slot 1: one thread per query row
@@ -22,7 +25,7 @@
 // The result is exact: O = sum P V / sum P with the same reference max in both sums.
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
-// Shared memory: Q0, Q1 (32 KB each), 4 K/V stages (32 KB each), barriers.
+// Shared memory: Q0, Q1 (32 KB each), 5 K/V stages (32 KB each), barriers.
 #pragma once
 
 #include <stdint.h>
@@ -37,8 +40,8 @@ struct FwdBf16Params {
   float* lse;               // [B*heads, N]
   int n_tiles, Wt;
   int S;                    // 128-row chunks per tile
-  int n_pass;               // slot pairs per tile, ceil(S / 2)
-  int n_units;              // B*heads * n_pass * n_tiles
+  int n_sub;                // B*heads * n_tiles * S query chunks in all
+  int n_units;              // ceil(n_sub / 2)
   int G1, G2;               // Gh, Gw
   int tt, th, tw, tcs;      // tile shape; t-extent of one 128-token chunk
   int T, H, W, N;
@@ -49,7 +52,7 @@ namespace fwd {
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 constexpr uint32_t kOffQ = 0;
@@ -60,21 +63,32 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // Q, K both K-major (smem)
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P from TMEM, V MN-major (smem)
 constexpr float kRescaleThreshold = 8.0f;                      // log2 units
+constexpr int kPolyEvery = 4;  // one 16-column group in 4 takes 2^x from the FMA-pipe polynomial
+
+struct Slot {
+  int bh, tile, sub;
+};
 
 struct Unit {
-  int bh, tile, sub0;
-  bool has1;
+  Slot s[2];
+  int ns;       // slots in use (1 only for the last unit of an odd total)
+  int streams;  // K/V streams: 1 when the slots share a window, else ns
 };
+
+__device__ __forceinline__ Slot slot_of(const FwdBf16Params& p, int f) {
+  Slot x;
+  x.sub = f % p.S;
+  x.tile = (f / p.S) % p.n_tiles;
+  x.bh = f / (p.S * p.n_tiles);
+  return x;
+}
 
 __device__ __forceinline__ Unit decode(const FwdBf16Params& p, int u) {
   Unit x;
-  const int per_bh = p.n_pass * p.n_tiles;
-  x.bh = u / per_bh;
-  const int rem = u % per_bh;
-  const int pass = rem / p.n_tiles;
-  x.tile = rem % p.n_tiles;
-  x.sub0 = 2 * pass;
-  x.has1 = x.sub0 + 1 < p.S;
+  x.s[0] = slot_of(p, 2 * u);
+  x.ns = (2 * u + 1 < p.n_sub) ? 2 : 1;
+  x.s[1] = x.ns == 2 ? slot_of(p, 2 * u + 1) : x.s[0];
+  x.streams = (x.ns == 2 && (x.s[1].tile != x.s[0].tile || x.s[1].bh != x.s[0].bh)) ? 2 : 1;
   return x;
 }
 }  // namespace fwd
@@ -91,14 +105,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;   // [kStages]
-  uint64_t* kv_empty = bars + 6;  // [kStages]
-  uint64_t* s_full = bars + 10;   // [2]
-  uint64_t* p_full = bars + 12;   // [2]
-  uint64_t* o_done = bars + 14;   // [2]
-  uint64_t* o_free = bars + 16;   // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
-  volatile int* abort = reinterpret_cast<volatile int*>(bars + 19);
+  uint64_t* kv_full = bars + 2;              // [kStages]
+  uint64_t* kv_empty = bars + 2 + kStages;   // [kStages]
+  uint64_t* s_full = bars + 2 + 2 * kStages; // [2]
+  uint64_t* p_full = s_full + 2;             // [2]
+  uint64_t* o_done = s_full + 4;             // [2]
+  uint64_t* o_free = s_full + 6;             // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
+  volatile int* abort = reinterpret_cast<volatile int*>(s_full + 9);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_chunks = p.Wt * p.S;
@@ -115,9 +129,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 128);
+      mbar_init(p_full + i, 4);  // one arrival per softmax warp
       mbar_init(o_done + i, 1);
-      mbar_init(o_free + i, 128);
+      mbar_init(o_free + i, 4);
     }
     *abort = 0;
     fence_mbar_init();
@@ -138,30 +152,33 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
         const Unit x = decode(p, u);
-        const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
         ok = mbar_wait(q_empty, (uc & 1) ^ 1, abort, 20);
         if (!ok) break;
-        mbar_arrive_expect_tx(q_full, (x.has1 ? 2u : 1u) * kTileBytes);
-        for (int i = 0; i < (x.has1 ? 2 : 1); ++i) {
-          const int t0 = qt * p.tt + (x.sub0 + i) * p.tcs;
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(x.ns) * kTileBytes);
+        for (int i = 0; i < x.ns; ++i) {
+          const Slot& q = x.s[i];
+          const int qt = q.tile / (p.G1 * p.G2), qh = (q.tile / p.G2) % p.G1, qw = q.tile % p.G2;
+          const int t0 = qt * p.tt + q.sub * p.tcs;
           uint8_t* dst = smem + kOffQ + i * kTileBytes;
-          tma_load_5d(dst, &tmQ, q_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
-          tma_load_5d(dst + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
+          tma_load_5d(dst, &tmQ, q_full, 0, qw * p.tw, qh * p.th, t0, q.bh);
+          tma_load_5d(dst + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, t0, q.bh);
         }
-        const int32_t* kv = p.kv_tiles + static_cast<int64_t>(x.tile) * p.Wt;
         for (int j = 0; j < n_chunks && ok; ++j) {
-          const int kt = kv[j / p.S], ks = j % p.S;
-          const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
-          const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
-          for (int which = 0; which < 2; ++which, ++kv_load) {
-            const int st = kv_load % kStages;
-            ok = mbar_wait(kv_empty + st, ((kv_load / kStages) & 1) ^ 1, abort, 21);
-            if (!ok) break;
-            mbar_arrive_expect_tx(kv_full + st, kTileBytes);
-            uint8_t* dst = smem + kOffKV + st * kTileBytes;
-            const CUtensorMap* map = which == 0 ? &tmK : &tmV;
-            tma_load_5d(dst, map, kv_full + st, 0, w0, h0, t0, x.bh);
-            tma_load_5d(dst + kHalfBytes, map, kv_full + st, 64, w0, h0, t0, x.bh);
+          for (int which = 0; which < 2 && ok; ++which) {
+            for (int st_i = 0; st_i < x.streams; ++st_i, ++kv_load) {
+              const Slot& q = x.s[st_i];
+              const int kt = p.kv_tiles[static_cast<int64_t>(q.tile) * p.Wt + j / p.S], ks = j % p.S;
+              const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
+              const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
+              const int st = kv_load % kStages;
+              ok = mbar_wait(kv_empty + st, ((kv_load / kStages) & 1) ^ 1, abort, 21);
+              if (!ok) break;
+              mbar_arrive_expect_tx(kv_full + st, kTileBytes);
+              uint8_t* dst = smem + kOffKV + st * kTileBytes;
+              const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+              tma_load_5d(dst, map, kv_full + st, 0, w0, h0, t0, q.bh);
+              tma_load_5d(dst + kHalfBytes, map, kv_full + st, 64, w0, h0, t0, q.bh);
+            }
           }
         }
       }
@@ -182,47 +199,63 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
         mma_commit(s_full + i);
       };
+      // K/V ring indices of one step: `streams` consecutive loads, slot i uses entry i (or 0)
+      auto wait_loads = [&](int base, int streams, int site) {
+        bool good = true;
+        for (int t = 0; t < streams && good; ++t)
+          good = mbar_wait(kv_full + (base + t) % kStages, ((base + t) / kStages) & 1, abort, site);
+        return good;
+      };
+      auto release_loads = [&](int base, int streams) {
+        for (int t = 0; t < streams; ++t) mma_commit(kv_empty + (base + t) % kStages);
+      };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
         const Unit x = decode(p, u);
-        const int ns = x.has1 ? 2 : 1;
+        const int ns = x.ns, nst = x.streams;
         ok = mbar_wait(q_full, uc & 1, abort, 30);
         if (!ok) break;
-        int k_idx = kv_use++;
-        ok = mbar_wait(kv_full + k_idx % kStages, (k_idx / kStages) & 1, abort, 31);
+        int k_base = kv_use;
+        kv_use += nst;
+        ok = wait_loads(k_base, nst, 31);
         if (!ok) break;
         tc_fence_after();
-        for (int i = 0; i < ns; ++i) issue_s(i, k_idx % kStages);
-        mma_commit(kv_empty + k_idx % kStages);
+        for (int i = 0; i < ns; ++i) issue_s(i, (k_base + (nst == 2 ? i : 0)) % kStages);
+        release_loads(k_base, nst);
         if (n_chunks == 1) mma_commit(q_empty);
         for (int j = 0; j < n_chunks && ok; ++j) {
-          const int v_idx = kv_use++;
-          ok = mbar_wait(kv_full + v_idx % kStages, (v_idx / kStages) & 1, abort, 32);
+          const int v_base = kv_use;
+          kv_use += nst;
+          ok = wait_loads(v_base, nst, 32);
           if (!ok) break;
-          k_idx = (j + 1 < n_chunks) ? kv_use++ : -1;
+          k_base = -1;
+          if (j + 1 < n_chunks) {
+            k_base = kv_use;
+            kv_use += nst;
+          }
           for (int i = 0; i < ns && ok; ++i) {
             ok = mbar_wait(p_full + i, pc[i] & 1, abort, 33);
             ++pc[i];
             if (ok && j == 0) ok = mbar_wait(o_free + i, (uslot[i] & 1) ^ 1, abort, 34);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t va = sbase + kOffKV + (v_idx % kStages) * kTileBytes;
+            const uint32_t va = sbase + kOffKV + ((v_base + (nst == 2 ? i : 0)) % kStages) * kTileBytes;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024),
                      kIdescPV, (j > 0) || (kk > 0));
             mma_commit(o_done + i);
-            if (k_idx >= 0) {
+            if (k_base >= 0) {
               if (i == 0) {
-                ok = mbar_wait(kv_full + k_idx % kStages, (k_idx / kStages) & 1, abort, 35);
+                ok = wait_loads(k_base, nst, 35);
                 if (!ok) break;
                 tc_fence_after();
               }
-              issue_s(i, k_idx % kStages);
+              issue_s(i, (k_base + (nst == 2 ? i : 0)) % kStages);
             }
           }
           if (!ok) break;
-          mma_commit(kv_empty + v_idx % kStages);
-          if (k_idx >= 0) mma_commit(kv_empty + k_idx % kStages);
+          release_loads(v_base, nst);
+          if (k_base >= 0) release_loads(k_base, nst);
           if (j + 2 == n_chunks) mma_commit(q_empty);
         }
         for (int i = 0; i < ns; ++i) ++uslot[i];
@@ -239,7 +272,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit x = decode(p, u);
-      if (i == 1 && !x.has1) continue;
+      if (i >= x.ns) continue;
+      const Slot& q = x.s[i];
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n_chunks; ++j) {
         ok = mbar_wait(s_full + i, sc & 1, abort, 40);
@@ -249,13 +283,16 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         tc_fence_after();
         uint32_t s[128];
         tmem_ld128_wait(tS, s);
+        // row max: 8 independent chains of 3-input max
         float mxs[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mxs[e] = __uint_as_float(s[e]);
+        for (int e = 0; e < 8; ++e) {
+          mxs[e] = __uint_as_float(s[e]);
 #pragma unroll
-        for (int c = 8; c < 128; ++c) mxs[c & 7] = fmaxf(mxs[c & 7], __uint_as_float(s[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
-                               fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
+          for (int c = 8 + e; c < 128; c += 16)
+            mxs[e] = max3f(mxs[e], __uint_as_float(s[c]), __uint_as_float(s[c + 8]));
+        }
+        const float mx = max3f(max3f(mxs[0], mxs[1], mxs[2]), max3f(mxs[3], mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7]));
         const float m_new = fmaxf(m_used, mx * p.scale_log2);
         const bool need = m_new > m_used + kRescaleThreshold;
         float alpha = 1.f;
@@ -264,27 +301,31 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           m_used = m_new;
         }
         l *= alpha;
-        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float neg_m = -m_used;
+        // P = 2^(s * scale * log2 e - m): paired fp32 arithmetic; one column group in
+        // kPolyEvery goes to the FMA-pipe polynomial to unload the MUFU unit
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
           uint32_t pk[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(s[16 * g + 2 * e]), p.scale_log2, -m_used));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(s[16 * g + 2 * e + 1]), p.scale_log2, -m_used));
-            ps[e] += p0 + p1;
+            float x0, x1, p0, p1;
+            ffma2(x0, x1, __uint_as_float(s[16 * g + 2 * e]), __uint_as_float(s[16 * g + 2 * e + 1]), p.scale_log2,
+                  p.scale_log2, neg_m, neg_m);
+            if (kPolyEvery > 0 && (g % kPolyEvery) == kPolyEvery - 1) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            fadd2(sa[e & 3], sb[e & 3], sa[e & 3], sb[e & 3], p0, p1);
             pk[e] = pack_bf16x2(p0, p1);
           }
-          s[8 * g + 0] = pk[0];  // pack in place: P pairs of columns 16g..16g+15 -> word 8g..8g+7
-          s[8 * g + 1] = pk[1];
-          s[8 * g + 2] = pk[2];
-          s[8 * g + 3] = pk[3];
-          s[8 * g + 4] = pk[4];
-          s[8 * g + 5] = pk[5];
-          s[8 * g + 6] = pk[6];
-          s[8 * g + 7] = pk[7];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s[8 * g + e] = pk[e];  // packed P of columns 16g..16g+15
         }
-        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        l += ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           uint32_t w[16];
@@ -309,7 +350,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full + i);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + i);
       }
       if (!ok) break;
       // epilogue: O / l as bf16, LSE = (m + log2 l) ln 2
@@ -318,12 +360,12 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       pv_base += n_chunks;
-      const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
-      const int t0 = qt * p.tt + (x.sub0 + i) * p.tcs;
+      const int qt = q.tile / (p.G1 * p.G2), qh = (q.tile / p.G2) % p.G1, qw = q.tile % p.G2;
+      const int t0 = qt * p.tt + q.sub * p.tcs;
       const int lw = r % p.tw, lh = (r / p.tw) % p.th, lt = r / (p.tw * p.th);
       const int64_t tok = (static_cast<int64_t>(t0 + lt) * p.H + (qh * p.th + lh)) * p.W + (qw * p.tw + lw);
       const float inv = 1.f / l;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * p.N + tok) * 128);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(q.bh) * p.N + tok) * 128);
 #pragma unroll 1
       for (int g = 0; g < 4; ++g) {
         uint32_t o[32];
@@ -338,15 +380,19 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           dst[4 * g + c] = v;
         }
       }
-      p.lse[static_cast<int64_t>(x.bh) * p.N + tok] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      p.lse[static_cast<int64_t>(q.bh) * p.N + tok] = (m_used + __log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(o_free + i);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free + i);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
 }
 
 }  // namespace dsa
