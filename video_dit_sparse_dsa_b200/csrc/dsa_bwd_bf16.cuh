@@ -59,6 +59,8 @@ constexpr uint32_t kTmemCols = 512;  // dV [0,128), dK [128,256), S^T buffers [2
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // K Q^T and V dO^T
 constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 128, 0, 1);  // P^T dO, dS^T Q
 constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, 64, 1, 1);    // K^T dS^T
+// A byte offset added to a shared-memory descriptor's address field (16-byte units).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
 }  // namespace bwd
 
 __device__ __forceinline__ int64_t chunk_row_token(int r, int t0, int h0, int w0, int th, int tw, int H, int W) {
@@ -239,75 +241,80 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------------ MMA issuer (whole warp)
+    {
+      const uint64_t dK = smem_desc_sw128(sbase + kOffK, 16, 1024);            // K, K-major
+      const uint64_t dV = smem_desc_sw128(sbase + kOffV, 16, 1024);            // V, K-major
+      const uint64_t dKt = smem_desc_sw128(sbase + kOffK, kKHalf, 1024);       // K^T, MN-major
+      const uint64_t dQk = smem_desc_sw128(sbase + kOffStage, 16, 1024);       // stage 0 Q, K-major
+      const uint64_t dQm = smem_desc_sw128(sbase + kOffStage, kQHalf, 1024);   // stage 0 Q, MN-major
+      const uint64_t dSk = smem_desc_sw128(sbase + kOffDS, 16, 1024);          // dS^T buffer 0, K-major
+      const uint64_t dSm = smem_desc_sw128(sbase + kOffDS, kKHalf, 1024);      // dS^T buffer 0, MN-major
       int ld = 0, uc = 0, sc = 0, pc = 0;
       bool ok = true;
-      auto stage_addr = [&](int l) { return sbase + kOffStage + (l % kStages) * kStageBytes; };
-      // S^T and dP^T of the chunk in ring entry l into buffer sc % 2
-      auto issue_sdp = [&](int l) -> bool {
-        const int b = sc & 1;
-        if (!mbar_wait(ld_full + l % kStages, (l / kStages) & 1, abort, 61)) return false;
-        tc_fence_after();
-        const uint32_t qa = stage_addr(l), da = qa + kQBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          mma_ss(tS + b * 64, smem_desc_sw128(sbase + kOffK + ko, 16, 1024), smem_desc_sw128(qa + qo, 16, 1024),
-                 kIdescS, kk > 0);
-        }
-        // dP^T overwrites the dQ^T of chunk sc - 2: wait until it has been read out
-        if (sc >= 2 && !mbar_wait(dq_free + b, ((sc >> 1) - 1) & 1, abort, 62)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          mma_ss(tDP + b * 64, smem_desc_sw128(sbase + kOffV + ko, 16, 1024), smem_desc_sw128(da + qo, 16, 1024),
-                 kIdescS, kk > 0);
-        }
-        mma_commit(s_full + b);
-        ++sc;
-        return true;
-      };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         int bh, kt, ku;
         unit_of(u, bh, kt, ku);
         const int n = (p.row_ptr[kt + 1] - p.row_ptr[kt]) * p.QS;
         if (n == 0) continue;
-        ok = mbar_wait(kv_full, uc & 1, abort, 60);
+        ok = __all_sync(0xffffffffu, mbar_wait(kv_full, uc & 1, abort, 60));
         if (!ok) break;
         const int ld0 = ld;
         ld += n;
-        ok = issue_sdp(ld0);
-        if (ok && n > 1) ok = issue_sdp(ld0 + 1);
-        for (int c = 0; c < n && ok; ++c) {
-          const int b = pc & 1;
-          ok = mbar_wait(p_full + b, (pc >> 1) & 1, abort, 63);
-          ++pc;
-          if (ok && c == 0) ok = mbar_wait(dkv_free, (uc & 1) ^ 1, abort, 64);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t qa = stage_addr(ld0 + c), da = qa + kQBytes;
-          const uint32_t dsa = sbase + kOffDS + b * kDSBytes;
+        // S^T and dP^T of chunk c (ring entry ld0 + c) into buffer sc % 2; the first two
+        // chunks here, chunk c + 2 after chunk c's gradient products
+        for (int c = 0; c < n + 2 && ok; ++c) {
+          if (c >= 2) {
+            const int cc = c - 2;  // gradient products of chunk cc
+            const int b = pc & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(p_full + b, (pc >> 1) & 1, abort, 63));
+            ++pc;
+            if (ok && cc == 0) ok = __all_sync(0xffffffffu, mbar_wait(dkv_free, (uc & 1) ^ 1, abort, 64));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t so = ((ld0 + cc) % kStages) * kStageBytes;
+            const uint64_t q_m = desc_add(dQm, so), do_m = desc_add(dQm, so + kQBytes);
+            const uint64_t ds_k = desc_add(dSk, b * kDSBytes), ds_m = desc_add(dSm, b * kDSBytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
-            mma_ts(tDV, tS + b * 64 + kk * 8, smem_desc_sw128(da + kk * 2048, kQHalf, 1024), kIdescAcc,
-                   (c > 0) || (kk > 0));
+            for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
+              mma_ts_warp(tDV, tS + b * 64 + kk * 8, desc_add(do_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-            mma_ss(tDK, smem_desc_sw128(dsa + kk * 32, 16, 1024), smem_desc_sw128(qa + kk * 2048, kQHalf, 1024),
-                   kIdescAcc, (c > 0) || (kk > 0));
+            for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
+              mma_ss_warp(tDK, desc_add(ds_k, kk * 32), desc_add(q_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
-            mma_ss(tDP + b * 64, smem_desc_sw128(sbase + kOffK + kk * 2048, kKHalf, 1024),
-                   smem_desc_sw128(dsa + kk * 2048, kKHalf, 1024), kIdescDQ, kk > 0);
-          mma_commit(dq_full + b);
-          mma_commit(ld_empty + (ld0 + c) % kStages);
-          if (c + 2 < n) ok = issue_sdp(ld0 + c + 2);
+            for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
+              mma_ss_warp(tDP + b * 64, desc_add(dKt, kk * 2048), desc_add(ds_m, kk * 2048), kIdescDQ, kk > 0);
+            mma_commit_warp(dq_full + b);
+            mma_commit_warp(ld_empty + (ld0 + cc) % kStages);
+          }
+          if (c < n) {
+            const int l = ld0 + c, b = sc & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(ld_full + l % kStages, (l / kStages) & 1, abort, 61));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t so = (l % kStages) * kStageBytes;
+            const uint64_t q_k = desc_add(dQk, so), do_k = desc_add(dQk, so + kQBytes);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
+              mma_ss_warp(tS + b * 64, desc_add(dK, ko), desc_add(q_k, qo), kIdescS, kk > 0);
+            }
+            // dP^T overwrites the dQ^T of chunk sc - 2: wait until it has been read out
+            if (sc >= 2) ok = __all_sync(0xffffffffu, mbar_wait(dq_free + b, ((sc >> 1) - 1) & 1, abort, 62));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
+              mma_ss_warp(tDP + b * 64, desc_add(dV, ko), desc_add(do_k, qo), kIdescS, kk > 0);
+            }
+            mma_commit_warp(s_full + b);
+            ++sc;
+          }
         }
         if (!ok) break;
-        mma_commit(dkv_full);
-        mma_commit(kv_free);
+        mma_commit_warp(dkv_full);
+        mma_commit_warp(kv_free);
         ++uc;
       }
     }

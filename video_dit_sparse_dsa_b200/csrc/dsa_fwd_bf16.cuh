@@ -91,6 +91,42 @@ __device__ __forceinline__ Unit decode(const FwdBf16Params& p, int u) {
   x.streams = (x.ns == 2 && (x.s[1].tile != x.s[0].tile || x.s[1].bh != x.s[0].bh)) ? 2 : 1;
   return x;
 }
+// Shared-memory descriptors are built once; a byte offset is added in 16-byte units to
+// the address field (all addresses stay below 256 KB, so the 14-bit field cannot carry).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
+// S = Q K^T over the 128 channels: 8 k-steps of 16 within the two 64-channel halves.
+__device__ __forceinline__ void issue_scores(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    mma_ss_warp(d_tmem, desc_add(q_desc, off), desc_add(k_desc, off), kIdescS, kk > 0);
+  }
+}
+
+// O (+)= P V over 128 keys: P from TMEM (8 columns of packed bf16 per 16 keys), V
+// MN-major with 16 keys = two 8-row groups = 2048 bytes per k-step.
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts_warp(d_tmem, p_tmem + kk * 8, desc_add(v_desc, kk * 2048), kIdescPV, accumulate || kk > 0);
+}
+
+// Waits (whole warp) for `count` consecutive ring entries from `base` to be full.
+__device__ __forceinline__ bool wait_entries(uint64_t* full, int base, int count, volatile int* abort, int site) {
+  bool ok = true;
+  for (int t = 0; t < count && ok; ++t) ok = mbar_wait(full + (base + t) % kStages, ((base + t) / kStages) & 1, abort, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void release_entries(uint64_t* empty, int base, int count) {
+  for (int t = 0; t < count; ++t) mma_commit_warp(empty + (base + t) % kStages);
+}
+
+// Barrier wait by a whole warp, with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, site));
+}
 }  // namespace fwd
 
 __global__ void __launch_bounds__(fwd::kThreads, 1)
@@ -155,19 +191,24 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         ok = mbar_wait(q_empty, (uc & 1) ^ 1, abort, 20);
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(x.ns) * kTileBytes);
-        for (int i = 0; i < x.ns; ++i) {
-          const Slot& q = x.s[i];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (i >= x.ns) break;
+          const Slot q = i == 0 ? x.s[0] : x.s[1];
           const int qt = q.tile / (p.G1 * p.G2), qh = (q.tile / p.G2) % p.G1, qw = q.tile % p.G2;
           const int t0 = qt * p.tt + q.sub * p.tcs;
           uint8_t* dst = smem + kOffQ + i * kTileBytes;
           tma_load_5d(dst, &tmQ, q_full, 0, qw * p.tw, qh * p.th, t0, q.bh);
           tma_load_5d(dst + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, t0, q.bh);
         }
+        const int32_t* kv0 = p.kv_tiles + static_cast<int64_t>(x.s[0].tile) * p.Wt;
+        const int32_t* kv1 = p.kv_tiles + static_cast<int64_t>(x.s[1].tile) * p.Wt;
+        const int bh0 = x.s[0].bh, bh1 = x.s[1].bh;
         for (int j = 0; j < n_chunks && ok; ++j) {
+          const int ks = j % p.S;
           for (int which = 0; which < 2 && ok; ++which) {
             for (int st_i = 0; st_i < x.streams; ++st_i, ++kv_load) {
-              const Slot& q = x.s[st_i];
-              const int kt = p.kv_tiles[static_cast<int64_t>(q.tile) * p.Wt + j / p.S], ks = j % p.S;
+              const int kt = (st_i == 0 ? kv0 : kv1)[j / p.S];
               const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
               const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
               const int st = kv_load % kStages;
@@ -176,89 +217,86 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
               mbar_arrive_expect_tx(kv_full + st, kTileBytes);
               uint8_t* dst = smem + kOffKV + st * kTileBytes;
               const CUtensorMap* map = which == 0 ? &tmK : &tmV;
-              tma_load_5d(dst, map, kv_full + st, 0, w0, h0, t0, q.bh);
-              tma_load_5d(dst + kHalfBytes, map, kv_full + st, 64, w0, h0, t0, q.bh);
+              const int bh = st_i == 0 ? bh0 : bh1;
+              tma_load_5d(dst, map, kv_full + st, 0, w0, h0, t0, bh);
+              tma_load_5d(dst + kHalfBytes, map, kv_full + st, 64, w0, h0, t0, bh);
             }
           }
         }
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int kv_use = 0, uc = 0;
-      int pc[2] = {0, 0}, uslot[2] = {0, 0};
+    // ------------------------------------------------------------------ MMA issuer (whole warp)
+    {
+      const uint64_t dQ0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
+      const uint64_t dQ1 = desc_add(dQ0, kTileBytes);
+      const uint64_t dK = smem_desc_sw128(sbase + kOffKV, 16, 1024);          // stage 0, K-major
+      const uint64_t dV = smem_desc_sw128(sbase + kOffKV, kHalfBytes, 1024);  // stage 0, MN-major
+      int kv_use = 0, uc = 0, pc0 = 0, pc1 = 0, us0 = 0, us1 = 0;
       bool ok = true;
-      auto issue_s = [&](int i, int stage) {
-        const uint32_t qa = sbase + kOffQ + i * kTileBytes, ka = sbase + kOffKV + stage * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(tmem + i * 128, smem_desc_sw128(qa + koff, 16, 1024), smem_desc_sw128(ka + koff, 16, 1024), kIdescS,
-                 kk > 0);
-        }
-        mma_commit(s_full + i);
-      };
-      // K/V ring indices of one step: `streams` consecutive loads, slot i uses entry i (or 0)
-      auto wait_loads = [&](int base, int streams, int site) {
-        bool good = true;
-        for (int t = 0; t < streams && good; ++t)
-          good = mbar_wait(kv_full + (base + t) % kStages, ((base + t) / kStages) & 1, abort, site);
-        return good;
-      };
-      auto release_loads = [&](int base, int streams) {
-        for (int t = 0; t < streams; ++t) mma_commit(kv_empty + (base + t) % kStages);
-      };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
         const Unit x = decode(p, u);
-        const int ns = x.ns, nst = x.streams;
-        ok = mbar_wait(q_full, uc & 1, abort, 30);
+        const bool two = x.ns == 2;
+        const int nst = x.streams, e1 = nst == 2 ? 1 : 0;  // ring entry offset of slot 1
+        ok = warp_wait(q_full, uc & 1, abort, 30);
         if (!ok) break;
         int k_base = kv_use;
         kv_use += nst;
-        ok = wait_loads(k_base, nst, 31);
+        ok = wait_entries(kv_full, k_base, nst, abort, 31);
         if (!ok) break;
         tc_fence_after();
-        for (int i = 0; i < ns; ++i) issue_s(i, (k_base + (nst == 2 ? i : 0)) % kStages);
-        release_loads(k_base, nst);
-        if (n_chunks == 1) mma_commit(q_empty);
+        issue_scores(tmem, dQ0, desc_add(dK, (k_base % kStages) * kTileBytes));
+        mma_commit_warp(s_full);
+        if (two) {
+          issue_scores(tmem + 128, dQ1, desc_add(dK, ((k_base + e1) % kStages) * kTileBytes));
+          mma_commit_warp(s_full + 1);
+        }
+        release_entries(kv_empty, k_base, nst);
+        if (n_chunks == 1) mma_commit_warp(q_empty);
         for (int j = 0; j < n_chunks && ok; ++j) {
           const int v_base = kv_use;
           kv_use += nst;
-          ok = wait_loads(v_base, nst, 32);
+          ok = wait_entries(kv_full, v_base, nst, abort, 32);
           if (!ok) break;
           k_base = -1;
           if (j + 1 < n_chunks) {
             k_base = kv_use;
             kv_use += nst;
           }
-          for (int i = 0; i < ns && ok; ++i) {
-            ok = mbar_wait(p_full + i, pc[i] & 1, abort, 33);
-            ++pc[i];
-            if (ok && j == 0) ok = mbar_wait(o_free + i, (uslot[i] & 1) ^ 1, abort, 34);
+          // slot 0: O0 += P0 V, then the next scores S0 = Q0 K'
+          ok = warp_wait(p_full, pc0 & 1, abort, 33);
+          ++pc0;
+          if (ok && j == 0) ok = warp_wait(o_free, (us0 & 1) ^ 1, abort, 34);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(tmem + 256, tmem, desc_add(dV, (v_base % kStages) * kTileBytes), j > 0);
+          mma_commit_warp(o_done);
+          if (k_base >= 0) {
+            ok = wait_entries(kv_full, k_base, nst, abort, 35);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t va = sbase + kOffKV + ((v_base + (nst == 2 ? i : 0)) % kStages) * kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024),
-                     kIdescPV, (j > 0) || (kk > 0));
-            mma_commit(o_done + i);
+            issue_scores(tmem, dQ0, desc_add(dK, (k_base % kStages) * kTileBytes));
+            mma_commit_warp(s_full);
+          }
+          if (two) {
+            ok = warp_wait(p_full + 1, pc1 & 1, abort, 33);
+            ++pc1;
+            if (ok && j == 0) ok = warp_wait(o_free + 1, (us1 & 1) ^ 1, abort, 34);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(tmem + 384, tmem + 128, desc_add(dV, ((v_base + e1) % kStages) * kTileBytes), j > 0);
+            mma_commit_warp(o_done + 1);
             if (k_base >= 0) {
-              if (i == 0) {
-                ok = wait_loads(k_base, nst, 35);
-                if (!ok) break;
-                tc_fence_after();
-              }
-              issue_s(i, (k_base + (nst == 2 ? i : 0)) % kStages);
+              issue_scores(tmem + 128, dQ1, desc_add(dK, ((k_base + e1) % kStages) * kTileBytes));
+              mma_commit_warp(s_full + 1);
             }
           }
-          if (!ok) break;
-          release_loads(v_base, nst);
-          if (k_base >= 0) release_loads(k_base, nst);
-          if (j + 2 == n_chunks) mma_commit(q_empty);
+          release_entries(kv_empty, v_base, nst);
+          if (k_base >= 0) release_entries(kv_empty, k_base, nst);
+          if (j + 2 == n_chunks) mma_commit_warp(q_empty);
         }
-        for (int i = 0; i < ns; ++i) ++uslot[i];
+        ++us0;
+        if (two) ++us1;
       }
     }
   } else {
@@ -273,7 +311,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit x = decode(p, u);
       if (i >= x.ns) continue;
-      const Slot& q = x.s[i];
+      const Slot q = i == 0 ? x.s[0] : x.s[1];
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n_chunks; ++j) {
         ok = mbar_wait(s_full + i, sc & 1, abort, 40);
