@@ -257,8 +257,8 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.W = p->W;
   bp.N = static_cast<int>(g.N);
   bp.scale_log2 = p->scale * 1.4426950408889634f;
-  bp.n_sub = static_cast<int>(g.BH * g.n_tiles * bp.S);
-  bp.n_units = (bp.n_sub + 1) / 2;
+  bp.n_pass = (bp.S + 1) / 2;
+  bp.n_units = static_cast<int>(g.BH * bp.n_pass * g.n_tiles);
   if (cudaFuncSetAttribute(dsa::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            dsa::fwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;

@@ -6,25 +6,30 @@
 // Video Diffusion", abstract, 3D-DSA; tile-granular window form from "Fast Video
 // Generation with Sliding Tile Attention", abstract).
 //
-// Persistent, warp-specialised kernel, one CTA per SM.  A work unit is two 128-row query
-// chunks ("slots"): consecutive chunks in (batch*head, query tile, chunk) order, so both
-// slots usually belong to the same query tile and share every K/V chunk of its window;
-// when a tile has an odd number of chunks, a unit may pair the last chunk of one tile with
-// the first of the next, and then each slot streams its own window's K/V.  Roles:
-//   warp 8      TMA producer: Q of both slots, then per step the K chunk(s) and V chunk(s)
-//               through a 5-stage shared-memory ring;
-//   warp 9      MMA issuer: S_i = Q_i K^T into TMEM, then O_i += P_i V with P_i read from
-//               TMEM (the scores' own columns), order S0 S1 | PV0 S0' PV1 S1' | ...;
-//   warps 0-3   softmax of slot 0, warps 4-7 softmax of slot 1: one thread per query row
-//               reads its S row from TMEM, keeps a running max m and sum l (base 2), writes
-//               P = exp2(S * scale * log2 e - m) as bf16 back into TMEM, and at the end of a
-//               unit normalises its O row and writes O and LSE.
+// Persistent, warp-specialised kernel, one CTA per SM.  A work unit takes 128-row query
+// chunks of one query tile of one (batch, head): two chunks ("slots") that share every
+// K/V chunk of the tile's window, or, for the last chunk of a tile with an odd number of
+// chunks, one chunk alone.  Roles:
+//   warp 8      TMA producer: Q of the unit, then K and V chunks through a 5-stage ring;
+//   warp 9      MMA issuer (a converged warp; one elected lane issues):
+//                 two slots: S_i = Q_i K^T into score buffer i, O_i += P_i V with P_i read
+//                 from TMEM (the scores' own columns), order S0 S1 | PV0 S0' PV1 S1' | ...;
+//                 one slot:  S(j) into buffer j % 2, so S(j+1) is computed while the
+//                 softmax of S(j) runs; O_0 += P(j) V;
+//   warps 0-3   softmax of slot 0 (and of single-slot units), warps 4-7 softmax of slot 1:
+//               one thread per query row reads its S row from TMEM, keeps a running max m
+//               and sum l (base 2), writes P = exp2(S * scale * log2 e - m) as bf16 back
+//               into TMEM, and at the end of a unit normalises its O row and writes O, LSE.
 // The running max is only moved when it grows by more than 8 (a factor 256): P stays
 // <= 256, which bf16 and the fp32 accumulators hold exactly as well, and the O rescale
 // (a TMEM read-modify-write of the row) happens a few times per row instead of per chunk.
 // The result is exact: O = sum P V / sum P with the same reference max in both sums.
 //
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// Units are ordered (batch*head, pass, tile): pass p takes chunks 2p and 2p+1 of every
+// tile, so consecutive units work on neighbouring tiles of one head (their windows
+// overlap in L2), and the persistent CTAs' strided walk mixes paired and single units.
+//
+// TMEM (512 columns): score buffers 0 [0,128) and 1 [128,256), O0 [256,384), O1 [384,512).
 // Shared memory: Q0, Q1 (32 KB each), 5 K/V stages (32 KB each), barriers.
 #pragma once
 
@@ -40,8 +45,8 @@ struct FwdBf16Params {
   float* lse;               // [B*heads, N]
   int n_tiles, Wt;
   int S;                    // 128-row chunks per tile
-  int n_sub;                // B*heads * n_tiles * S query chunks in all
-  int n_units;              // ceil(n_sub / 2)
+  int n_pass;               // units per tile, ceil(S / 2)
+  int n_units;              // B*heads * n_pass * n_tiles
   int G1, G2;               // Gh, Gw
   int tt, th, tw, tcs;      // tile shape; t-extent of one 128-token chunk
   int T, H, W, N;
@@ -65,32 +70,22 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P from TMEM, V
 constexpr float kRescaleThreshold = 8.0f;                      // log2 units
 constexpr int kPolyEvery = 4;  // one 16-column group in 4 takes 2^x from the FMA-pipe polynomial
 
-struct Slot {
-  int bh, tile, sub;
-};
-
 struct Unit {
-  Slot s[2];
-  int ns;       // slots in use (1 only for the last unit of an odd total)
-  int streams;  // K/V streams: 1 when the slots share a window, else ns
+  int bh, tile, sub0;
+  bool two;  // two slots (chunks sub0, sub0 + 1) or one
 };
-
-__device__ __forceinline__ Slot slot_of(const FwdBf16Params& p, int f) {
-  Slot x;
-  x.sub = f % p.S;
-  x.tile = (f / p.S) % p.n_tiles;
-  x.bh = f / (p.S * p.n_tiles);
-  return x;
-}
 
 __device__ __forceinline__ Unit decode(const FwdBf16Params& p, int u) {
   Unit x;
-  x.s[0] = slot_of(p, 2 * u);
-  x.ns = (2 * u + 1 < p.n_sub) ? 2 : 1;
-  x.s[1] = x.ns == 2 ? slot_of(p, 2 * u + 1) : x.s[0];
-  x.streams = (x.ns == 2 && (x.s[1].tile != x.s[0].tile || x.s[1].bh != x.s[0].bh)) ? 2 : 1;
+  const int per_bh = p.n_pass * p.n_tiles;
+  x.bh = u / per_bh;
+  const int rem = u % per_bh;
+  x.sub0 = 2 * (rem / p.n_tiles);
+  x.tile = rem % p.n_tiles;
+  x.two = x.sub0 + 1 < p.S;
   return x;
 }
+
 // Shared-memory descriptors are built once; a byte offset is added in 16-byte units to
 // the address field (all addresses stay below 256 KB, so the 14-bit field cannot carry).
 __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
@@ -143,12 +138,16 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   uint64_t* q_empty = bars + 1;
   uint64_t* kv_full = bars + 2;              // [kStages]
   uint64_t* kv_empty = bars + 2 + kStages;   // [kStages]
-  uint64_t* s_full = bars + 2 + 2 * kStages; // [2]
-  uint64_t* p_full = s_full + 2;             // [2]
-  uint64_t* o_done = s_full + 4;             // [2]
-  uint64_t* o_free = s_full + 6;             // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
-  volatile int* abort = reinterpret_cast<volatile int*>(s_full + 9);
+  // scores ready / P ready, indexed 0: buffer 0, 1: buffer 1 of a two-slot unit, 2: buffer 1
+  // of a single-slot unit (warpgroup 0's odd chunks) -- a separate barrier, so that the
+  // phases warpgroup 1 waits for are its own chunks only
+  uint64_t* s_full = bars + 2 + 2 * kStages; // [3]
+  uint64_t* p_full = s_full + 3;             // [3]
+  uint64_t* o_done = s_full + 6;             // [2]
+  uint64_t* o_free = s_full + 8;             // [2]
+  uint64_t* o_final = s_full + 10;           // [2] every product of a unit into O_i done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 12);
+  volatile int* abort = reinterpret_cast<volatile int*>(s_full + 13);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_chunks = p.Wt * p.S;
@@ -163,11 +162,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(p_full + i, 4);  // one arrival per softmax warp
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(o_done + i, 1);
       mbar_init(o_free + i, 4);
+      mbar_init(o_final + i, 1);
     }
     *abort = 0;
     fence_mbar_init();
@@ -188,115 +190,140 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
         const Unit x = decode(p, u);
+        const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
         ok = mbar_wait(q_empty, (uc & 1) ^ 1, abort, 20);
         if (!ok) break;
-        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(x.ns) * kTileBytes);
+        mbar_arrive_expect_tx(q_full, (x.two ? 2u : 1u) * kTileBytes);
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          if (i >= x.ns) break;
-          const Slot q = i == 0 ? x.s[0] : x.s[1];
-          const int qt = q.tile / (p.G1 * p.G2), qh = (q.tile / p.G2) % p.G1, qw = q.tile % p.G2;
-          const int t0 = qt * p.tt + q.sub * p.tcs;
+          if (i == 1 && !x.two) break;
+          const int t0 = qt * p.tt + (x.sub0 + i) * p.tcs;
           uint8_t* dst = smem + kOffQ + i * kTileBytes;
-          tma_load_5d(dst, &tmQ, q_full, 0, qw * p.tw, qh * p.th, t0, q.bh);
-          tma_load_5d(dst + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, t0, q.bh);
+          tma_load_5d(dst, &tmQ, q_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
+          tma_load_5d(dst + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
         }
-        const int32_t* kv0 = p.kv_tiles + static_cast<int64_t>(x.s[0].tile) * p.Wt;
-        const int32_t* kv1 = p.kv_tiles + static_cast<int64_t>(x.s[1].tile) * p.Wt;
-        const int bh0 = x.s[0].bh, bh1 = x.s[1].bh;
+        const int32_t* kv = p.kv_tiles + static_cast<int64_t>(x.tile) * p.Wt;
         for (int j = 0; j < n_chunks && ok; ++j) {
-          const int ks = j % p.S;
-          for (int which = 0; which < 2 && ok; ++which) {
-            for (int st_i = 0; st_i < x.streams; ++st_i, ++kv_load) {
-              const int kt = (st_i == 0 ? kv0 : kv1)[j / p.S];
-              const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
-              const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
-              const int st = kv_load % kStages;
-              ok = mbar_wait(kv_empty + st, ((kv_load / kStages) & 1) ^ 1, abort, 21);
-              if (!ok) break;
-              mbar_arrive_expect_tx(kv_full + st, kTileBytes);
-              uint8_t* dst = smem + kOffKV + st * kTileBytes;
-              const CUtensorMap* map = which == 0 ? &tmK : &tmV;
-              const int bh = st_i == 0 ? bh0 : bh1;
-              tma_load_5d(dst, map, kv_full + st, 0, w0, h0, t0, bh);
-              tma_load_5d(dst + kHalfBytes, map, kv_full + st, 64, w0, h0, t0, bh);
-            }
+          const int kt = kv[j / p.S], ks = j % p.S;
+          const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
+          const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
+          for (int which = 0; which < 2; ++which, ++kv_load) {
+            const int st = kv_load % kStages;
+            ok = mbar_wait(kv_empty + st, ((kv_load / kStages) & 1) ^ 1, abort, 21);
+            if (!ok) break;
+            mbar_arrive_expect_tx(kv_full + st, kTileBytes);
+            uint8_t* dst = smem + kOffKV + st * kTileBytes;
+            const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+            tma_load_5d(dst, map, kv_full + st, 0, w0, h0, t0, x.bh);
+            tma_load_5d(dst + kHalfBytes, map, kv_full + st, 64, w0, h0, t0, x.bh);
           }
         }
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer (whole warp)
-    {
-      const uint64_t dQ0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
-      const uint64_t dQ1 = desc_add(dQ0, kTileBytes);
-      const uint64_t dK = smem_desc_sw128(sbase + kOffKV, 16, 1024);          // stage 0, K-major
-      const uint64_t dV = smem_desc_sw128(sbase + kOffKV, kHalfBytes, 1024);  // stage 0, MN-major
-      int kv_use = 0, uc = 0, pc0 = 0, pc1 = 0, us0 = 0, us1 = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
-        const Unit x = decode(p, u);
-        const bool two = x.ns == 2;
-        const int nst = x.streams, e1 = nst == 2 ? 1 : 0;  // ring entry offset of slot 1
-        ok = warp_wait(q_full, uc & 1, abort, 30);
-        if (!ok) break;
-        int k_base = kv_use;
-        kv_use += nst;
-        ok = wait_entries(kv_full, k_base, nst, abort, 31);
+    const uint64_t dQ0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
+    const uint64_t dQ1 = desc_add(dQ0, kTileBytes);
+    const uint64_t dK = smem_desc_sw128(sbase + kOffKV, 16, 1024);          // stage 0, K-major
+    const uint64_t dV = smem_desc_sw128(sbase + kOffKV, kHalfBytes, 1024);  // stage 0, MN-major
+    int kv_use = 0, uc = 0;
+    int pb0 = 0, pb1 = 0, pb2 = 0;  // P consumed per ready-barrier
+    int us0 = 0, us1 = 0;  // units that used O0 / O1
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+      const Unit x = decode(p, u);
+      ok = warp_wait(q_full, uc & 1, abort, 30);
+      if (!ok) break;
+      // K(j) is ring entry base + 2j, V(j) is base + 2j + 1
+      const int base = kv_use;
+      kv_use += 2 * n_chunks;
+      if (x.two) {
+        ok = wait_entries(kv_full, base, 1, abort, 31);
         if (!ok) break;
         tc_fence_after();
-        issue_scores(tmem, dQ0, desc_add(dK, (k_base % kStages) * kTileBytes));
+        issue_scores(tmem, dQ0, desc_add(dK, (base % kStages) * kTileBytes));
         mma_commit_warp(s_full);
-        if (two) {
-          issue_scores(tmem + 128, dQ1, desc_add(dK, ((k_base + e1) % kStages) * kTileBytes));
-          mma_commit_warp(s_full + 1);
-        }
-        release_entries(kv_empty, k_base, nst);
+        issue_scores(tmem + 128, dQ1, desc_add(dK, (base % kStages) * kTileBytes));
+        mma_commit_warp(s_full + 1);
+        release_entries(kv_empty, base, 1);
         if (n_chunks == 1) mma_commit_warp(q_empty);
         for (int j = 0; j < n_chunks && ok; ++j) {
-          const int v_base = kv_use;
-          kv_use += nst;
-          ok = wait_entries(kv_full, v_base, nst, abort, 32);
+          const int v_idx = base + 2 * j + 1, k_idx = base + 2 * j + 2;
+          const bool more = j + 1 < n_chunks;
+          ok = wait_entries(kv_full, v_idx, 1, abort, 32);
           if (!ok) break;
-          k_base = -1;
-          if (j + 1 < n_chunks) {
-            k_base = kv_use;
-            kv_use += nst;
-          }
-          // slot 0: O0 += P0 V, then the next scores S0 = Q0 K'
-          ok = warp_wait(p_full, pc0 & 1, abort, 33);
-          ++pc0;
+          // slot 0: O0 += P0 V, then S0 = Q0 K'
+          ok = warp_wait(p_full, pb0++ & 1, abort, 33);
           if (ok && j == 0) ok = warp_wait(o_free, (us0 & 1) ^ 1, abort, 34);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(tmem + 256, tmem, desc_add(dV, (v_base % kStages) * kTileBytes), j > 0);
+          issue_pv(tmem + 256, tmem, desc_add(dV, (v_idx % kStages) * kTileBytes), j > 0);
           mma_commit_warp(o_done);
-          if (k_base >= 0) {
-            ok = wait_entries(kv_full, k_base, nst, abort, 35);
+          if (more) {
+            ok = wait_entries(kv_full, k_idx, 1, abort, 35);
             if (!ok) break;
             tc_fence_after();
-            issue_scores(tmem, dQ0, desc_add(dK, (k_base % kStages) * kTileBytes));
+            issue_scores(tmem, dQ0, desc_add(dK, (k_idx % kStages) * kTileBytes));
             mma_commit_warp(s_full);
           }
-          if (two) {
-            ok = warp_wait(p_full + 1, pc1 & 1, abort, 33);
-            ++pc1;
-            if (ok && j == 0) ok = warp_wait(o_free + 1, (us1 & 1) ^ 1, abort, 34);
+          // slot 1
+          ok = warp_wait(p_full + 1, pb1++ & 1, abort, 33);
+          if (ok && j == 0) ok = warp_wait(o_free + 1, (us1 & 1) ^ 1, abort, 34);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(tmem + 384, tmem + 128, desc_add(dV, (v_idx % kStages) * kTileBytes), j > 0);
+          mma_commit_warp(o_done + 1);
+          if (more) {
+            issue_scores(tmem + 128, dQ1, desc_add(dK, (k_idx % kStages) * kTileBytes));
+            mma_commit_warp(s_full + 1);
+            release_entries(kv_empty, k_idx, 1);
+          }
+          release_entries(kv_empty, v_idx, 1);
+          if (j + 2 == n_chunks) mma_commit_warp(q_empty);  // every score of this unit issued
+        }
+        if (!ok) break;
+        mma_commit_warp(o_final);
+        mma_commit_warp(o_final + 1);
+        ++us0;
+        ++us1;
+      } else {
+        // one slot: scores alternate between the two buffers, O0 accumulates
+        const int pre = n_chunks < 2 ? n_chunks : 2;
+        for (int j = 0; j < pre && ok; ++j) {
+          ok = wait_entries(kv_full, base + 2 * j, 1, abort, 31);
+          if (!ok) break;
+          tc_fence_after();
+          const int b = j;  // buffer of chunk j
+          issue_scores(tmem + b * 128, dQ0, desc_add(dK, ((base + 2 * j) % kStages) * kTileBytes));
+          mma_commit_warp(s_full + 2 * b);
+          release_entries(kv_empty, base + 2 * j, 1);
+        }
+        if (ok && n_chunks <= 2) mma_commit_warp(q_empty);
+        for (int j = 0; j < n_chunks && ok; ++j) {
+          const int b = j & 1;
+          const int v_idx = base + 2 * j + 1, k_idx = base + 2 * j + 4;
+          ok = wait_entries(kv_full, v_idx, 1, abort, 32);
+          if (ok) ok = warp_wait(p_full + 2 * b, (b == 0 ? pb0++ : pb2++) & 1, abort, 33);
+          if (ok && j == 0) ok = warp_wait(o_free, (us0 & 1) ^ 1, abort, 34);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(tmem + 256, tmem + b * 128, desc_add(dV, (v_idx % kStages) * kTileBytes), j > 0);
+          mma_commit_warp(o_done);
+          if (j + 2 < n_chunks) {
+            // S(j+2) reuses buffer b; in issue order it follows the product that reads P(j)
+            ok = wait_entries(kv_full, k_idx, 1, abort, 35);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(tmem + 384, tmem + 128, desc_add(dV, ((v_base + e1) % kStages) * kTileBytes), j > 0);
-            mma_commit_warp(o_done + 1);
-            if (k_base >= 0) {
-              issue_scores(tmem + 128, dQ1, desc_add(dK, ((k_base + e1) % kStages) * kTileBytes));
-              mma_commit_warp(s_full + 1);
-            }
+            issue_scores(tmem + b * 128, dQ0, desc_add(dK, (k_idx % kStages) * kTileBytes));
+            mma_commit_warp(s_full + 2 * b);
+            release_entries(kv_empty, k_idx, 1);
           }
-          release_entries(kv_empty, v_base, nst);
-          if (k_base >= 0) release_entries(kv_empty, k_base, nst);
-          if (j + 2 == n_chunks) mma_commit_warp(q_empty);
+          release_entries(kv_empty, v_idx, 1);
+          if (j + 3 == n_chunks) mma_commit_warp(q_empty);
         }
+        if (!ok) break;
+        mma_commit_warp(o_final);
         ++us0;
-        if (two) ++us1;
       }
     }
   } else {
@@ -304,18 +331,20 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const int i = warp >> 2;
     const int r = tid & 127;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + i * 128 + lane_off;
     const uint32_t tO = tmem + 256 + i * 128 + lane_off;
-    int sc = 0, pv_base = 0;
+    int sc0 = 0, sc1 = 0, sc2 = 0;  // phases waited per ready-barrier
+    int pv_base = 0, uf = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit x = decode(p, u);
-      if (i >= x.ns) continue;
-      const Slot q = i == 0 ? x.s[0] : x.s[1];
+      if (!x.two && i == 1) continue;
+      const int sub = x.sub0 + i;
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n_chunks; ++j) {
-        ok = mbar_wait(s_full + i, sc & 1, abort, 40);
-        ++sc;
+        const int b = x.two ? i : (j & 1);                   // score buffer of this chunk
+        const int rb = x.two ? i : 2 * (j & 1);              // its ready-barrier index
+        const uint32_t tS = tmem + b * 128 + lane_off;
+        ok = mbar_wait(s_full + rb, (rb == 0 ? sc0++ : (rb == 1 ? sc1++ : sc2++)) & 1, abort, 40);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
@@ -389,21 +418,23 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + i);
+        if (lane == 0) mbar_arrive(p_full + rb);
       }
       if (!ok) break;
-      // epilogue: O / l as bf16, LSE = (m + log2 l) ln 2
-      ok = mbar_wait(o_done + i, (pv_base + n_chunks - 1) & 1, abort, 42);
+      // epilogue: O / l as bf16, LSE = (m + log2 l) ln 2.  o_final completes once per unit
+      // (after the unit's last product into O_i), so its parity is never ambiguous.
+      ok = mbar_wait(o_final + i, uf & 1, abort, 42);
+      ++uf;
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       pv_base += n_chunks;
-      const int qt = q.tile / (p.G1 * p.G2), qh = (q.tile / p.G2) % p.G1, qw = q.tile % p.G2;
-      const int t0 = qt * p.tt + q.sub * p.tcs;
+      const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
+      const int t0 = qt * p.tt + sub * p.tcs;
       const int lw = r % p.tw, lh = (r / p.tw) % p.th, lt = r / (p.tw * p.th);
       const int64_t tok = (static_cast<int64_t>(t0 + lt) * p.H + (qh * p.th + lh)) * p.W + (qw * p.tw + lw);
       const float inv = 1.f / l;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(q.bh) * p.N + tok) * 128);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * p.N + tok) * 128);
 #pragma unroll 1
       for (int g = 0; g < 4; ++g) {
         uint32_t o[32];
@@ -418,7 +449,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           dst[4 * g + c] = v;
         }
       }
-      p.lse[static_cast<int64_t>(q.bh) * p.N + tok] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      p.lse[static_cast<int64_t>(x.bh) * p.N + tok] = (m_used + __log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_free + i);
