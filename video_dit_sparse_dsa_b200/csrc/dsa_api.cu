@@ -257,11 +257,14 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.W = p->W;
   bp.N = static_cast<int>(g.N);
   bp.scale_log2 = p->scale * 1.4426950408889634f;
-  bp.n_pass = (bp.S + 1) / 2;
-  bp.n_units = static_cast<int>(g.BH * bp.n_pass * g.n_tiles);
+  bp.n_units = static_cast<int>(g.BH * bp.S * g.n_tiles);
   if (cudaFuncSetAttribute(dsa::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            dsa::fwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
+  // the kernel's setmaxnreg split needs exactly the registers it was compiled for at launch
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, dsa::fwd_bf16_kernel) != cudaSuccess) return DSA_ERR_CUDA;
+  if (fa.numRegs < dsa::fwd::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
   int sms = 0;
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
