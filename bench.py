@@ -17,6 +17,7 @@ bounded sample of the same workload, on the host cores.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -48,11 +49,42 @@ def peaks():
         return FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+# ----------------------------------------------------------------------------- DRAM traffic
+# DRAM bytes (read + write) of one fwd_bf16_kernel launch per workload, from the
+# single-pass ncu capture summarised in profiles/fwd_bf16_kernel__bf16_720p_dram.md.  The
+# figure holds only for the kernel sources it was taken on, identified by a hash of them;
+# with any other sources the line reports null.
+FWD_TRAFFIC = {"bf16_720p": (4.99e9, "619b1a789b3ad6c1")}
+FWD_SOURCES = ("dsa_fwd_bf16.cuh", "sm100.cuh")
+
+
+def fwd_source_hash() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in FWD_SOURCES:
+        with open(os.path.join(ROOT, "video_dit_sparse_dsa_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def fwd_traffic(workload: str):
+    entry = FWD_TRAFFIC.get(workload)
+    if entry is None:
+        return None
+    try:
+        return entry[0] if fwd_source_hash() == entry[1] else None
+    except OSError:
+        return None
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+    """Samples SM clocks, power and throttle reasons with nvidia-smi every 20 ms; stop()
+    keeps only the samples taken inside the timed regions (TIMED_WINDOWS, host wall-clock
+    intervals around each CUDA-event-timed loop)."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
@@ -66,7 +98,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
@@ -77,7 +109,29 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
+    @staticmethod
+    def parse(lines):
+        """-> list of (epoch seconds, sm MHz, max sm MHz, power W, set of active reasons)."""
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        out = []
+        for line in lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                t = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, smax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            try:
+                pw = float(parts[3])
+            except ValueError:
+                pw = None
+            reasons = {n for n, v in zip(names, parts[4:8]) if v.lower().startswith("active")}
+            out.append((t, sm, smax, pw, reasons))
+        return out
+
+    def stop(self, windows):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -87,22 +141,19 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        rows = self.parse(self.lines)
+        inside = [r for r in rows if any(a <= r[0] <= b for a, b in windows)]
+        use = inside if inside else rows
+        power = [r[3] for r in use if r[3] is not None]
+        return {"sm_mhz": statistics.median(r[1] for r in use) if use else None,
+                "sm_max_mhz": max(r[2] for r in use) if use else None,
+                "power_w": statistics.median(power) if power else None,
+                "samples": len(use), "in_timed_region": bool(inside),
+                "reasons": sorted(set().union(*[r[4] for r in use])) if use else []}
+
+
+# host wall-clock intervals of the CUDA-event-timed loops of the headline workload
+TIMED_WINDOWS = []
 
 
 # ----------------------------------------------------------------------------- inputs
@@ -123,17 +174,20 @@ def device_inputs(w: Workload, device, seed_offset: int = 0):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def time_steps(step, steps: int, warmup: int, stream):
+def time_steps(step, steps: int, warmup: int, stream, record: bool = True):
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
     start.record(stream)
     for _ in range(steps):
         step()
     end.record(stream)
     torch.cuda.synchronize()
+    if record:
+        TIMED_WINDOWS.append((t0, time.time()))
     return start.elapsed_time(end) / steps  # ms per step
 
 
@@ -193,7 +247,7 @@ def run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream):
     def step():
         dsa.forward_host(p, qh, kh, vh, oh_, outh, lseh, dev, stream=stream)
 
-    ms = time_steps(step, max(1, steps // 2), max(1, warmup // 2), stream)
+    ms = time_steps(step, max(1, steps // 2), max(1, warmup // 2), stream, record=False)
     h2d = 3 * qh.numel() * qh.element_size() + oh_.numel() * 4
     d2h = outh.numel() * outh.element_size() + lseh.numel() * 4
     return {"value": w.fwd_flops() / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
@@ -295,8 +349,6 @@ def main():
     torch.cuda.set_device(device)
     dist = None
     if world > 1:
-        import datetime
-
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
@@ -313,7 +365,8 @@ def main():
         sampler.start()
     res = run_workload(dsa, w, device, args.steps, args.warmup, seed_offset=rank, with_e2e=(rank == 0))
     barrier()
-    clocks = sampler.stop() if sampler else None
+    timed = list(TIMED_WINDOWS)
+    clocks = sampler.stop(timed) if sampler else None
     step_ms = max_over_ranks(res["step_ms"], dist, device)
     value, _ = aggregate([step_ms] * world, res["step_flops"])
 
@@ -356,7 +409,7 @@ def main():
                         f"{src}_{burst:g}": 100 * fwd_tflops / burst},
         "roofline": {"bound": "tensor", "kernel": "fwd_bf16_kernel (timed with the planner, one dsa_fwd call)",
                      "achieved": fwd_tflops, "peak": burst, "peak_kind": f"{src} burst bf16", "unit": "TFLOP/s",
-                     "frac": fwd_tflops / burst, "traffic": None},
+                     "frac": fwd_tflops / burst, "traffic": fwd_traffic(w.name), "traffic_unit": "bytes per launch"},
         "e2e": e2e, "gpu_launches": res["launches_per_step"] * args.steps, "clocks": clocks,
         "cpu_baseline": cpu, "workloads": extra,
     }

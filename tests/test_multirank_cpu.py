@@ -52,3 +52,42 @@ def test_aggregate_single_rank():
     v, t = bench.aggregate([20.0], 1e12)
     assert t == 20.0 and v == pytest.approx(50.0)
     assert bench.max_over_ranks(3.0) == 3.0
+
+
+def test_clock_samples_are_kept_only_inside_timed_windows():
+    """The benchmark's clock summary uses only nvidia-smi samples taken while a timed loop ran."""
+    import datetime
+
+    def line(t, sm, pw, cap):
+        ts = datetime.datetime.fromtimestamp(t).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, {sm}, 1965, {pw}, Not Active, Not Active, Not Active, {'Active' if cap else 'Not Active'}"
+
+    base = 1_800_000_000.0
+    lines = [line(base + 0.0, 1965, 200.0, False), line(base + 1.0, 1400, 990.0, True),
+             line(base + 1.1, 1420, 995.0, True), line(base + 2.0, 1965, 210.0, False), "garbage"]
+    rows = bench.ClockSampler.parse(lines)
+    assert len(rows) == 4 and rows[1][4] == {"sw_power_cap"}
+    s = bench.ClockSampler(0)
+    s.proc = None
+    assert s.stop([(base + 0.5, base + 1.5)])["sm_mhz"] is None  # no sampler process: reported as unavailable
+
+    class Done:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            pass
+
+    s.proc, s.lines = Done(), lines
+    got = s.stop([(base + 0.5, base + 1.5)])
+    assert got["samples"] == 2 and got["in_timed_region"]
+    assert got["sm_mhz"] == 1410 and got["reasons"] == ["sw_power_cap"] and got["power_w"] == 992.5
+
+
+def test_traffic_is_reported_only_for_the_profiled_kernel_sources(monkeypatch):
+    """The roofline's DRAM traffic is tied to the kernel sources it was measured on."""
+    h = bench.fwd_source_hash()
+    monkeypatch.setattr(bench, "FWD_TRAFFIC", {"w": (123.0, h), "stale": (5.0, "0" * 16)})
+    assert bench.fwd_traffic("w") == 123.0
+    assert bench.fwd_traffic("stale") is None
+    assert bench.fwd_traffic("unknown") is None

@@ -96,7 +96,10 @@ constexpr uint32_t kIdescS256 = idesc_bf16_f32(128, 256, 0, 0);  // Q, K both K-
 constexpr uint32_t kIdescS128 = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);    // P from TMEM, V MN-major (smem)
 constexpr float kRescaleThreshold = 8.0f;                        // log2 units
-constexpr int kPolyEvery = 4;  // one 16-column group in 4 takes 2^x from the FMA-pipe polynomial
+// 16-column groups (bit g of a step's 8 groups; a half step uses the low 4) whose 2^x is
+// taken from the FMA-pipe polynomial instead of the MUFU unit, which takes 16 per clock per
+// SM and would otherwise bound the softmax
+constexpr uint32_t kPolyMask = 0x88u;
 
 // TMEM columns of the scores and of P for a step of parity e.
 __device__ __forceinline__ uint32_t col_s(int e) { return e ? 128u : 0u; }
@@ -210,8 +213,8 @@ __device__ __forceinline__ bool softmax_step(bool ok, uint32_t tS, uint32_t tP, 
   }
   l *= alpha;
   const float neg_m = -m_used;
-  // P = 2^(s * scale * log2 e - m): paired fp32 arithmetic; one column group in
-  // kPolyEvery goes to the FMA-pipe polynomial to unload the MUFU unit
+  // P = 2^(s * scale * log2 e - m): paired fp32 arithmetic; the kPolyMask column groups
+  // go to the FMA-pipe polynomial to unload the MUFU unit
   float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int g = 0; g < NC / 16; ++g) {
@@ -221,7 +224,7 @@ __device__ __forceinline__ bool softmax_step(bool ok, uint32_t tS, uint32_t tP, 
       float x0, x1, p0, p1;
       ffma2(x0, x1, __uint_as_float(s[16 * g + 2 * e]), __uint_as_float(s[16 * g + 2 * e + 1]), scale_log2,
             scale_log2, neg_m, neg_m);
-      if (kPolyEvery > 0 && (g % kPolyEvery) == kPolyEvery - 1) {
+      if ((kPolyMask >> g) & 1u) {
         exp2_poly2(x0, x1, p0, p1);
       } else {
         p0 = ex2_approx(x0);
