@@ -13,6 +13,11 @@ length) and "Fast Video Generation with Sliding Tile Attention", abstract (atten
 a local spatial-temporal window, tile-granular).  The concrete window rule, softmax and
 gradients are written out in the header of ``dsa_oracle.c``.
 
+The key-tile-list functions (``forward_list``, ``backward_list``) take a CSR of key tiles
+per query tile instead of window offsets: the block-sparse generalisation of the window
+(the MOD-DiT page, Method section, Stage 2 "Online Block Masking", attends over selected
+blocks of keys).
+
 Every function here is pinned by the CPU tests in ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
@@ -59,7 +64,14 @@ def _load():
         lib.oracle_bwd_dq.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, fp, i32p, ctypes.c_int32, i32p, i32p, dp]
         lib.oracle_bwd_dkdv.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, fp, i32p, ctypes.c_int32, i32p, i32p,
                                         dp, dp]
-        for f in (lib.oracle_plan, lib.oracle_fwd, lib.oracle_bwd_dq, lib.oracle_bwd_dkdv):
+        lib.oracle_fwd_list.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, i32p, i32p, ctypes.c_int32, i32p, i32p,
+                                        dp, dp]
+        lib.oracle_bwd_dq_list.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, fp, i32p, i32p, ctypes.c_int32, i32p,
+                                           i32p, dp]
+        lib.oracle_bwd_dkdv_list.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, fp, i32p, i32p, ctypes.c_int32,
+                                             i32p, i32p, dp, dp]
+        for f in (lib.oracle_plan, lib.oracle_fwd, lib.oracle_bwd_dq, lib.oracle_bwd_dkdv, lib.oracle_fwd_list,
+                  lib.oracle_bwd_dq_list, lib.oracle_bwd_dkdv_list):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -258,3 +270,90 @@ def backward(geo: Geometry, q, k, v, dout, offsets):
         full[:, tok] = t.reshape(BH, -1, geo.d)
         res.append(full.reshape((geo.B, geo.heads) + geo.grid + (geo.d,)))
     return tuple(res)
+
+
+# ------------------------------------------------------------------------------------------
+# Key-tile lists (block-sparse form): query tile i attends to the key tiles
+# kv_list[row_ptr[i]:row_ptr[i+1]] instead of its window box; see dsa_oracle.c.
+
+
+def _lists(geo: Geometry, row_ptr, kv_list):
+    rp = _i32(row_ptr).reshape(-1)
+    kl = _i32(kv_list).reshape(-1)
+    if rp.shape[0] != geo.n_tiles + 1:
+        raise ValueError("row_ptr must have nTiles + 1 entries")
+    if kl.shape[0] == 0:
+        kl = np.zeros(1, np.int32)  # a valid pointer for an all-empty list
+    return rp, kl
+
+
+def _run_by_head_lists(geo: Geometry, tensors, row_ptr, kv_list, sel, n_out, call):
+    """As _run_by_head, with key-tile lists instead of window offsets."""
+    bh, tiles = _selection(geo, sel)
+    rp, kl = _lists(geo, row_ptr, kv_list)
+    outs = [np.zeros((len(bh), geo.tile_tokens, geo.d), np.float64) for _ in range(n_out)]
+    lse = np.zeros((len(bh), geo.tile_tokens), np.float64)
+    one = Geometry(1, 1, geo.d, geo.grid, geo.tile, (1, 1, 1), geo.scale)
+    p = one.c_problem()
+    for h in np.unique(bh):
+        rows = np.nonzero(bh == h)[0]
+        sl = [_head_slice(t, geo, int(h)) for t in tensors]
+        sel_t = np.ascontiguousarray(tiles[rows])
+        sel_b = np.zeros(len(rows), np.int32)
+        part = [np.zeros((len(rows), geo.tile_tokens, geo.d), np.float64) for _ in range(n_out)]
+        part_lse = np.zeros((len(rows), geo.tile_tokens), np.float64)
+        rc = call(p, sl, rp, kl, len(rows), sel_b, sel_t, part, part_lse)
+        if rc:
+            raise RuntimeError(f"oracle list call failed ({rc})")
+        for o, pt in zip(outs, part):
+            o[rows] = pt
+        lse[rows] = part_lse
+    return outs, lse
+
+
+def _scatter(geo: Geometry, tiles_major):
+    """[BH * nTiles, tile_tokens, ...] in (bh, tile) order -> [B, heads, T, H, W, ...]."""
+    tok = geo.tile_token_index().reshape(-1)
+    BH = geo.B * geo.heads
+    rest = tiles_major.shape[2:]
+    full = np.zeros((BH, geo.n_tokens) + rest, np.float64)
+    full[:, tok] = tiles_major.reshape((BH, -1) + rest)
+    return full.reshape((geo.B, geo.heads) + geo.grid + rest)
+
+
+def forward_list(geo: Geometry, q, k, v, row_ptr, kv_list, sel=None):
+    """Forward over key-tile lists.  With sel=None: out[B, heads, T, H, W, d] and
+    lse[B, heads, T, H, W] (float64); with sel: per (bh, query tile) rows as forward_tiles."""
+    lib = _load()
+    D = ctypes.c_double
+    I = ctypes.c_int32
+
+    def call(p, sl, rp, kl, n, sb, st, part, part_lse):
+        return lib.oracle_fwd_list(ctypes.byref(p), _ptr(sl[0], D), _ptr(sl[1], D), _ptr(sl[2], D), _ptr(rp, I),
+                                   _ptr(kl, I), n, _ptr(sb, I), _ptr(st, I), _ptr(part[0], D), _ptr(part_lse, D))
+
+    (out,), lse = _run_by_head_lists(geo, (q, k, v), row_ptr, kv_list, sel, 1, call)
+    if sel is not None:
+        return out, lse
+    return _scatter(geo, out), _scatter(geo, lse)
+
+
+def backward_list(geo: Geometry, q, k, v, dout, row_ptr, kv_list):
+    """Backward over key-tile lists: dq, dk, dv as [B, heads, T, H, W, d] float64."""
+    lib = _load()
+    D = ctypes.c_double
+    I = ctypes.c_int32
+
+    def call_dq(p, sl, rp, kl, n, sb, st, part, part_lse):
+        return lib.oracle_bwd_dq_list(ctypes.byref(p), _ptr(sl[0], D), _ptr(sl[1], D), _ptr(sl[2], D),
+                                      _ptr(sl[3], D), _ptr(rp, I), _ptr(kl, I), n, _ptr(sb, I), _ptr(st, I),
+                                      _ptr(part[0], D))
+
+    def call_dkdv(p, sl, rp, kl, n, sb, st, part, part_lse):
+        return lib.oracle_bwd_dkdv_list(ctypes.byref(p), _ptr(sl[0], D), _ptr(sl[1], D), _ptr(sl[2], D),
+                                        _ptr(sl[3], D), _ptr(rp, I), _ptr(kl, I), n, _ptr(sb, I), _ptr(st, I),
+                                        _ptr(part[0], D), _ptr(part[1], D))
+
+    (dq,), _ = _run_by_head_lists(geo, (q, k, v, dout), row_ptr, kv_list, None, 1, call_dq)
+    (dk, dv), _ = _run_by_head_lists(geo, (q, k, v, dout), row_ptr, kv_list, None, 2, call_dkdv)
+    return _scatter(geo, dq), _scatter(geo, dk), _scatter(geo, dv)

@@ -31,9 +31,17 @@
  * Inputs and every arithmetic step are double (bf16 and fp32 inputs widen to it exactly).  Token tensors are [B, heads, T, H, W, d] contiguous; offsets are
  * int32 [nTiles, 3] (dt, dh, dw) in tile-raster order (t outer, w inner).
  *
+ *   Key-tile-list form (block-sparse attention, the generalisation of the box to an
+ *   arbitrary per-query-tile list of key tiles, as in the MOD-DiT page's Method section,
+ *   Stage 2, online block masking):
+ *   K(i) is every token of the tiles listed for i in a CSR (row_ptr, list); a tile listed
+ *   twice counts twice; an empty list gives o = 0 and lse = -inf.  Functions *_list.
+ *
  * Parity pins (tests, CPU only): a window covering the grid equals dense attention; a
  * 1x1x1 window equals block-diagonal attention; softmax rows sum to one; brute-force
- * membership by nearest window centre; backward against central finite differences.
+ * membership by nearest window centre; backward against central finite differences;
+ * lists: multiset-weighted dense attention and its autograd backward, doubled lists
+ * (same o, lse + ln 2), lists of the window plan equal the window form.
  */
 #include <math.h>
 #include <stdint.h>
@@ -353,6 +361,219 @@ int oracle_bwd_dkdv(const oracle_problem* p, const double* q, const double* k, c
                     for (int32_t c = 0; c < p->d; ++c) {
                         dk_local[(int64_t)rk * p->d + c] += p->scale * dS * qb[n * p->d + c];
                         dv_local[(int64_t)rk * p->d + c] += P[m] * dob[n * p->d + c];
+                    }
+                }
+            }
+            if (ok) {
+#pragma omp critical
+                for (int64_t e = 0; e < tile_elems; ++e) {
+                    dks[e] += dk_local[e];
+                    dvs[e] += dv_local[e];
+                }
+            }
+            free(keys);
+            free(P);
+            free(dP);
+            free(dk_local);
+            free(dv_local);
+        }
+    }
+    free(q_list);
+    return status;
+}
+
+/* ---------------------------------------------------------------------------------- */
+/* Key-tile lists (the block-sparse form: a per-query-tile list of key tiles in place of
+ * the window box).  Query tile i attends to every token of the key tiles
+ * list[row_ptr[i]] .. list[row_ptr[i+1] - 1], in list order, tokens of a tile in raster
+ * order.  A tile listed twice counts twice (the softmax runs over the multiset).  An empty
+ * list gives o = 0 and lse = -inf (the log of an empty sum).  Returns 1 for a list that is
+ * not a CSR over valid tiles (row_ptr[0] = 0, non-decreasing, entries in [0, nTiles)). */
+
+static int check_lists(const geometry* g, const int32_t* row_ptr, const int32_t* list) {
+    if (row_ptr[0] != 0) return 1;
+    for (int32_t i = 0; i < g->n_tiles; ++i) {
+        if (row_ptr[i + 1] < row_ptr[i]) return 1;
+        for (int32_t e = row_ptr[i]; e < row_ptr[i + 1]; ++e)
+            if (list[e] < 0 || list[e] >= g->n_tiles) return 1;
+    }
+    return 0;
+}
+
+static int64_t longest_list(const geometry* g, const int32_t* row_ptr) {
+    int64_t m = 0;
+    for (int32_t i = 0; i < g->n_tiles; ++i)
+        if (row_ptr[i + 1] - row_ptr[i] > m) m = row_ptr[i + 1] - row_ptr[i];
+    return m;
+}
+
+static int64_t list_key_set(const oracle_problem* p, const geometry* g, const int32_t* row_ptr, const int32_t* list,
+                            int32_t tile, int64_t* keys) {
+    int64_t n = 0;
+    for (int32_t e = row_ptr[tile]; e < row_ptr[tile + 1]; ++e)
+        for (int32_t r = 0; r < g->tile_tokens; ++r) keys[n++] = tile_token(p, g, list[e], r);
+    return n;
+}
+
+/* Forward on selected (bh, query tile) pairs over key-tile lists; layouts as oracle_fwd. */
+int oracle_fwd_list(const oracle_problem* p, const double* q, const double* k, const double* v,
+                    const int32_t* row_ptr, const int32_t* list, int32_t n_sel, const int32_t* sel_bh,
+                    const int32_t* sel_tile, double* out, double* lse) {
+    geometry g;
+    if (make_geometry(p, &g) || check_lists(&g, row_ptr, list)) return 1;
+    const int64_t nk_max = longest_list(&g, row_ptr) * g.tile_tokens + 1;
+    const int64_t slice = (int64_t)g.n_tokens * p->d;
+    int status = 0;
+#pragma omp parallel
+    {
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * nk_max);
+        double* P = (double*)malloc(sizeof(double) * nk_max);
+        if (!keys || !P) {
+#pragma omp atomic write
+            status = 2;
+        }
+#pragma omp for schedule(dynamic)
+        for (int64_t job = 0; job < (int64_t)n_sel * g.tile_tokens; ++job) {
+            if (!keys || !P) continue;
+            int32_t s = (int32_t)(job / g.tile_tokens), r = (int32_t)(job % g.tile_tokens);
+            const double* qb = q + sel_bh[s] * slice;
+            const double* kb = k + sel_bh[s] * slice;
+            const double* vb = v + sel_bh[s] * slice;
+            int64_t nk = list_key_set(p, &g, row_ptr, list, sel_tile[s], keys);
+            int64_t n = tile_token(p, &g, sel_tile[s], r);
+            double* o = out + ((int64_t)s * g.tile_tokens + r) * p->d;
+            for (int32_t c = 0; c < p->d; ++c) o[c] = 0.0;
+            if (nk == 0) {
+                lse[(int64_t)s * g.tile_tokens + r] = -INFINITY;
+                continue;
+            }
+            double l = softmax_row(p, qb + n * p->d, kb, keys, nk, P);
+            for (int64_t m = 0; m < nk; ++m) {
+                const double* vm = vb + keys[m] * p->d;
+                for (int32_t c = 0; c < p->d; ++c) o[c] += P[m] * vm[c];
+            }
+            lse[(int64_t)s * g.tile_tokens + r] = l;
+        }
+        free(keys);
+        free(P);
+    }
+    return status;
+}
+
+/* dq on selected (bh, query tile) pairs over key-tile lists; zero for an empty list. */
+int oracle_bwd_dq_list(const oracle_problem* p, const double* q, const double* k, const double* v, const double* dout,
+                       const int32_t* row_ptr, const int32_t* list, int32_t n_sel, const int32_t* sel_bh,
+                       const int32_t* sel_tile, double* dq) {
+    geometry g;
+    if (make_geometry(p, &g) || check_lists(&g, row_ptr, list)) return 1;
+    const int64_t nk_max = longest_list(&g, row_ptr) * g.tile_tokens + 1;
+    const int64_t slice = (int64_t)g.n_tokens * p->d;
+    int status = 0;
+#pragma omp parallel
+    {
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * nk_max);
+        double* P = (double*)malloc(sizeof(double) * nk_max);
+        double* dP = (double*)malloc(sizeof(double) * nk_max);
+        if (!keys || !P || !dP) {
+#pragma omp atomic write
+            status = 2;
+        }
+#pragma omp for schedule(dynamic)
+        for (int64_t job = 0; job < (int64_t)n_sel * g.tile_tokens; ++job) {
+            if (!keys || !P || !dP) continue;
+            int32_t s = (int32_t)(job / g.tile_tokens), r = (int32_t)(job % g.tile_tokens);
+            const double* qb = q + sel_bh[s] * slice;
+            const double* kb = k + sel_bh[s] * slice;
+            const double* vb = v + sel_bh[s] * slice;
+            const double* dob = dout + sel_bh[s] * slice;
+            int64_t nk = list_key_set(p, &g, row_ptr, list, sel_tile[s], keys);
+            int64_t n = tile_token(p, &g, sel_tile[s], r);
+            double* o = dq + ((int64_t)s * g.tile_tokens + r) * p->d;
+            for (int32_t c = 0; c < p->d; ++c) o[c] = 0.0;
+            if (nk == 0) continue;
+            softmax_row(p, qb + n * p->d, kb, keys, nk, P);
+            double D = 0.0;
+            for (int64_t m = 0; m < nk; ++m) {
+                dP[m] = dot(dob + n * p->d, vb + keys[m] * p->d, p->d);
+                D += P[m] * dP[m];
+            }
+            for (int64_t m = 0; m < nk; ++m) {
+                double dS = P[m] * (dP[m] - D);
+                const double* km = kb + keys[m] * p->d;
+                for (int32_t c = 0; c < p->d; ++c) o[c] += p->scale * dS * km[c];
+            }
+        }
+        free(keys);
+        free(P);
+        free(dP);
+    }
+    return status;
+}
+
+/* dk, dv on selected (bh, key tile) pairs over key-tile lists: every occurrence of key
+ * tile j in the list of query tile i contributes for every query token of i. */
+int oracle_bwd_dkdv_list(const oracle_problem* p, const double* q, const double* k, const double* v,
+                         const double* dout, const int32_t* row_ptr, const int32_t* list, int32_t n_sel,
+                         const int32_t* sel_bh, const int32_t* sel_tile, double* dk, double* dv) {
+    geometry g;
+    if (make_geometry(p, &g) || check_lists(&g, row_ptr, list)) return 1;
+    const int64_t nk_max = longest_list(&g, row_ptr) * g.tile_tokens + 1;
+    const int64_t slice = (int64_t)g.n_tokens * p->d;
+    const int64_t tile_elems = (int64_t)g.tile_tokens * p->d;
+    int32_t* q_list = (int32_t*)malloc(sizeof(int32_t) * (g.n_tiles + 1));
+    if (!q_list) return 2;
+    int status = 0;
+    memset(dk, 0, sizeof(double) * n_sel * tile_elems);
+    memset(dv, 0, sizeof(double) * n_sel * tile_elems);
+    for (int32_t s = 0; s < n_sel; ++s) {
+        const int32_t j = sel_tile[s];
+        int32_t nq = 0;  /* query tiles whose list holds j at least once */
+        for (int32_t i = 0; i < g.n_tiles; ++i)
+            for (int32_t e = row_ptr[i]; e < row_ptr[i + 1]; ++e)
+                if (list[e] == j) {
+                    q_list[nq++] = i;
+                    break;
+                }
+        const double* qb = q + sel_bh[s] * slice;
+        const double* kb = k + sel_bh[s] * slice;
+        const double* vb = v + sel_bh[s] * slice;
+        const double* dob = dout + sel_bh[s] * slice;
+        double* dks = dk + s * tile_elems;
+        double* dvs = dv + s * tile_elems;
+#pragma omp parallel
+        {
+            int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * nk_max);
+            double* P = (double*)malloc(sizeof(double) * nk_max);
+            double* dP = (double*)malloc(sizeof(double) * nk_max);
+            double* dk_local = (double*)calloc(tile_elems, sizeof(double));
+            double* dv_local = (double*)calloc(tile_elems, sizeof(double));
+            int ok = keys && P && dP && dk_local && dv_local;
+            if (!ok) {
+#pragma omp atomic write
+                status = 2;
+            }
+#pragma omp for schedule(dynamic)
+            for (int64_t job = 0; job < (int64_t)nq * g.tile_tokens; ++job) {
+                if (!ok) continue;
+                int32_t i = q_list[job / g.tile_tokens], r = (int32_t)(job % g.tile_tokens);
+                int64_t nk = list_key_set(p, &g, row_ptr, list, i, keys);
+                int64_t n = tile_token(p, &g, i, r);
+                softmax_row(p, qb + n * p->d, kb, keys, nk, P);
+                double D = 0.0;
+                for (int64_t m = 0; m < nk; ++m) {
+                    dP[m] = dot(dob + n * p->d, vb + keys[m] * p->d, p->d);
+                    D += P[m] * dP[m];
+                }
+                for (int32_t e = row_ptr[i]; e < row_ptr[i + 1]; ++e) {
+                    if (list[e] != j) continue;
+                    const int64_t pos = e - row_ptr[i];  /* j's tokens are entries pos * tile_tokens + rk */
+                    for (int32_t rk = 0; rk < g.tile_tokens; ++rk) {
+                        int64_t m = pos * g.tile_tokens + rk;
+                        double dS = P[m] * (dP[m] - D);
+                        for (int32_t c = 0; c < p->d; ++c) {
+                            dk_local[(int64_t)rk * p->d + c] += p->scale * dS * qb[n * p->d + c];
+                            dv_local[(int64_t)rk * p->d + c] += P[m] * dob[n * p->d + c];
+                        }
                     }
                 }
             }

@@ -350,3 +350,133 @@ def test_tiny_workload_inputs_are_seeded():
     c = make_inputs(w2)
     assert c.q.dtype == torch.bfloat16
     assert int(c.offsets.min()) >= -1 and int(c.offsets.max()) <= 1
+
+
+# ------------------------------------------------------------------------------------
+# key-tile lists (block-sparse form): pinned against multiset-weighted dense attention
+# written here with torch (autograd gives the backward), sharing nothing with the oracle
+
+def tile_of_token(geo):
+    """[N] linear tile index of every token of the raster grid."""
+    T, H, W = geo.grid
+    tt, th, tw = geo.tile
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    return (((t // tt) * geo.G[1] + h // th) * geo.G[2] + w // tw).reshape(-1)
+
+
+def list_counts(geo, row_ptr, kv_list):
+    """[nTiles, nTiles] how often query tile i lists key tile j."""
+    c = np.zeros((geo.n_tiles, geo.n_tiles), np.int64)
+    for i in range(geo.n_tiles):
+        for e in range(row_ptr[i], row_ptr[i + 1]):
+            c[i, kv_list[e]] += 1
+    return c
+
+
+def multiset_attention(geo, q, k, v, row_ptr, kv_list):
+    """Dense fp64 attention with each key weighted by how often its tile is listed:
+    o_n = sum_m c_nm e^{s_nm} v_m / sum_m c_nm e^{s_nm}, lse_n = ln sum_m c_nm e^{s_nm};
+    rows with no key: o = 0, lse = -inf.  Differentiable in q, k, v."""
+    tot = tile_of_token(geo)
+    cnt = torch.tensor(list_counts(geo, row_ptr, kv_list)[tot][:, tot], dtype=torch.float64)  # [N, N]
+    BH = geo.B * geo.heads
+    qf, kf, vf = (t.reshape(BH, geo.n_tokens, geo.d) for t in (q, k, v))
+    s = torch.einsum("hnd,hmd->hnm", qf, kf) * geo.scale
+    logw = torch.where(cnt > 0, torch.log(cnt.clamp(min=1)), torch.full_like(cnt, -torch.inf))
+    has = (cnt > 0).any(dim=-1)  # [N] rows with at least one key
+    # rows without keys get a finite stand-in row (no NaN in autograd) and are zeroed
+    z = torch.where(has[:, None], s + logw, torch.zeros_like(s))
+    lse = torch.logsumexp(z, dim=-1)
+    p = torch.exp(z - lse[..., None]) * has[:, None]
+    o = p @ vf
+    lse = torch.where(has, lse, torch.full_like(lse, -torch.inf))
+    return o.reshape(q.shape), lse.reshape(q.shape[:-1])
+
+
+def random_lists(geo, seed, max_len, allow_empty=True, allow_dup=True):
+    rng = np.random.default_rng(seed)
+    rows = []
+    for i in range(geo.n_tiles):
+        n = int(rng.integers(0 if allow_empty else 1, max_len + 1))
+        if allow_empty and i == geo.n_tiles // 2:
+            n = 0  # every such case holds an empty list
+        if allow_dup:
+            rows.append(rng.integers(0, geo.n_tiles, n))
+        else:
+            rows.append(rng.permutation(geo.n_tiles)[:n])
+    row_ptr = np.zeros(geo.n_tiles + 1, np.int32)
+    row_ptr[1:] = np.cumsum([len(r) for r in rows])
+    kv_list = np.concatenate(rows).astype(np.int32) if row_ptr[-1] else np.zeros(0, np.int32)
+    return row_ptr, kv_list
+
+
+def small_inputs(geo, seed):
+    g = torch.Generator().manual_seed(seed)
+    shape = (geo.B, geo.heads) + geo.grid + (geo.d,)
+    return [torch.randn(shape, generator=g, dtype=torch.float64) for _ in range(4)]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_lists_forward_equal_multiset_attention(seed):
+    """Random lists (empty rows, repeated tiles, any order) = weighted dense attention."""
+    geo = oracle.Geometry(1, 2, 16, (2, 4, 6), (1, 2, 2), (1, 1, 1))
+    q, k, v, _ = small_inputs(geo, seed)
+    row_ptr, kv_list = random_lists(geo, seed, 5)
+    assert (np.diff(row_ptr) == 0).any(), "the case must hold an empty list"
+    out, lse = oracle.forward_list(geo, q, k, v, row_ptr, kv_list)
+    ref_o, ref_lse = multiset_attention(geo, q, k, v, row_ptr, kv_list)
+    np.testing.assert_allclose(out, ref_o.numpy(), rtol=0, atol=1e-12)
+    finite = np.isfinite(ref_lse.numpy())
+    assert np.array_equal(np.isfinite(lse), finite)
+    np.testing.assert_allclose(lse[finite], ref_lse.numpy()[finite], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_lists_backward_equal_autograd_of_multiset_attention(seed):
+    geo = oracle.Geometry(1, 2, 8, (2, 4, 4), (1, 2, 2), (1, 1, 1))
+    q, k, v, do = small_inputs(geo, 10 + seed)
+    row_ptr, kv_list = random_lists(geo, 10 + seed, 4)
+    dq, dk, dv = oracle.backward_list(geo, q, k, v, do, row_ptr, kv_list)
+    qr, kr, vr = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o, _ = multiset_attention(geo, qr, kr, vr, row_ptr, kv_list)
+    (o * do).sum().backward()
+    for got, ref in ((dq, qr.grad), (dk, kr.grad), (dv, vr.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-11)
+
+
+def test_lists_repeated_tiles_closed_form():
+    """Listing every tile of a list twice leaves O unchanged and adds ln 2 to the LSE."""
+    geo = oracle.Geometry(1, 1, 16, (2, 4, 4), (1, 2, 2), (1, 1, 1))
+    q, k, v, _ = small_inputs(geo, 5)
+    row_ptr, kv_list = random_lists(geo, 5, 4, allow_empty=False, allow_dup=False)
+    doubled = np.concatenate([np.concatenate([kv_list[row_ptr[i]:row_ptr[i + 1]]] * 2)
+                              for i in range(geo.n_tiles)]).astype(np.int32)
+    o1, l1 = oracle.forward_list(geo, q, k, v, row_ptr, kv_list)
+    o2, l2 = oracle.forward_list(geo, q, k, v, 2 * row_ptr, doubled)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l2, l1 + np.log(2.0), rtol=0, atol=1e-13)
+
+
+def test_lists_of_the_window_plan_equal_the_windowed_oracle():
+    geo = oracle.Geometry(1, 2, 16, (4, 4, 6), (1, 2, 2), (3, 1, 3))
+    q, k, v, do = small_inputs(geo, 7)
+    off = torch.randint(-1, 2, (geo.n_tiles, 3), generator=torch.Generator().manual_seed(7)).to(torch.int32)
+    _, kv, _, _ = oracle.plan(geo.G, geo.window, off)
+    row_ptr = (np.arange(geo.n_tiles + 1) * kv.shape[1]).astype(np.int32)
+    o_box, l_box = oracle.forward(geo, q, k, v, off)
+    o_list, l_list = oracle.forward_list(geo, q, k, v, row_ptr, kv.reshape(-1))
+    np.testing.assert_allclose(o_list, o_box, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l_list, l_box, rtol=0, atol=1e-13)
+    for a, b in zip(oracle.backward_list(geo, q, k, v, do, row_ptr, kv.reshape(-1)), oracle.backward(geo, q, k, v, do, off)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_lists_reject_invalid_csr():
+    geo = oracle.Geometry(1, 1, 8, (1, 2, 2), (1, 1, 1), (1, 1, 1))
+    q, k, v, _ = small_inputs(geo, 0)
+    bad = [(np.array([0, 1, 1, 1, 2], np.int32), np.array([0, 4], np.int32)),   # tile out of range
+           (np.array([0, 2, 1, 2, 2], np.int32), np.array([0, 1], np.int32)),   # decreasing row_ptr
+           (np.array([1, 1, 1, 1, 2], np.int32), np.array([0, 1], np.int32))]   # row_ptr[0] != 0
+    for rp, kl in bad:
+        with pytest.raises(RuntimeError):
+            oracle.forward_list(geo, q, k, v, rp, kl)
