@@ -103,6 +103,32 @@ def test_bwd_rejects_bad_arguments(lib):
     assert lib.dsa_bwd(ctypes.byref(p), f, f, f, f, f, f, f, f, f, f, f, 16, None) == 5
 
 
+def test_list_entry_points_reject_bad_arguments(lib):
+    p = _prob()
+    f = FAKE
+    # forward: (p, q, k, v, row_ptr, list, nnz, out, lse, stream)
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, None, f, 4, f, f, None) == 1      # no row_ptr
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, None, 4, f, f, None) == 1      # nnz > 0 without a list
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, f, -1, f, f, None) == 1        # negative nnz
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, f, 4, ctypes.c_void_p((1 << 20) + 8), f, None) == 1
+    p32 = _prob(d=64, dtype=dsa.DSA_F32, grid=(4, 8, 8), tile=(1, 4, 4))
+    assert lib.dsa_fwd_list(ctypes.byref(p32), f, f, f, f, f, 4, f, f, None) == 2       # bf16 only
+    assert lib.dsa_fwd_list(ctypes.byref(_prob(d=64)), f, f, f, f, f, 4, f, f, None) == 2
+    # backward: (p, q, k, v, out, lse, dout, row_ptr, list, nnz, dq, dk, dv, ws, ws_bytes, stream)
+    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, None, f, 4, f, f, f, f, 1 << 30, None) == 1
+    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, f, f, 4, f, f, f, f, 16, None) == 5
+    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, f, f, 4, f, f, f, None, 1 << 30, None) == 5
+
+
+def test_list_workspace_sizes(lib):
+    p = _prob()
+    assert lib.dsa_list_workspace_size(ctypes.byref(p), 100, dsa.DSA_WS_FWD) == 0  # the forward needs none
+    small = lib.dsa_list_workspace_size(ctypes.byref(p), 10, dsa.DSA_WS_BWD)
+    big = lib.dsa_list_workspace_size(ctypes.byref(p), 10000, dsa.DSA_WS_BWD)
+    assert big > small > 4 * (2 * 16 * 32 * 32 * 129)  # at least D and the fp32 dQ accumulator
+    assert lib.dsa_list_workspace_size(ctypes.byref(p), -1, dsa.DSA_WS_BWD) == 0
+
+
 def test_plan_rejects_half_inverse(lib):
     p = _prob()
     assert lib.dsa_plan(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None) == 1

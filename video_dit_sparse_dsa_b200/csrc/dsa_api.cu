@@ -13,6 +13,7 @@
 #include "dsa_device_status.cuh"
 #include "dsa_fwd_bf16.cuh"
 #include "dsa_fwd_f32.cuh"
+#include "dsa_lists.cuh"
 #include "dsa_plan.cuh"
 
 namespace {
@@ -120,6 +121,35 @@ BwdWorkspace bwd_workspace(const Geom& g, int d, void* base) {
   return w;
 }
 
+// Backward over a caller's key-tile lists: the inverse CSR built on the device, then the
+// same D and dQ accumulator scratch as dsa_bwd.
+struct ListBwdWorkspace {
+  int32_t* counts;   // [n_tiles] scratch of the inversion
+  int32_t* row_ptr;  // [n_tiles + 1] inverse CSR
+  int32_t* q_tiles;  // [nnz]
+  float* delta;      // [BH, N]
+  float* dq_acc;     // [BH, N, d]
+  size_t bytes;
+};
+
+ListBwdWorkspace list_bwd_workspace(const Geom& g, int d, int nnz, void* base) {
+  ListBwdWorkspace w;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  w.counts = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * g.n_tiles, kAlign);
+  w.row_ptr = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * (g.n_tiles + 1), kAlign);
+  w.q_tiles = reinterpret_cast<int32_t*>(b + off);
+  off += round_up(sizeof(int32_t) * static_cast<size_t>(nnz > 0 ? nnz : 1), kAlign);
+  w.delta = reinterpret_cast<float*>(b + off);
+  off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N), kAlign);
+  w.dq_acc = reinterpret_cast<float*>(b + off);
+  off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N) * d, kAlign);
+  w.bytes = off;
+  return w;
+}
+
 dsa::PlanGeom plan_geom(const Geom& g) {
   dsa::PlanGeom pg;
   for (int a = 0; a < 3; ++a) {
@@ -200,14 +230,27 @@ bool make_row_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, con
   return r == CUDA_SUCCESS;
 }
 
+// Validation of a caller's CSR on the device (records DSA_DEV_BOUNDS; never faults).
+dsa_status_t launch_list_check(const Geom& g, const int32_t* row_ptr, const int32_t* list, int nnz, cudaStream_t s) {
+  const int64_t work = g.n_tiles > nnz ? g.n_tiles : nnz;
+  int64_t blocks = (work + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 1024) blocks = 1024;
+  dsa::list_check_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(row_ptr, list, g.n_tiles, nnz);
+  return launch_status();
+}
+
 dsa_status_t launch_plan(const Geom& g, const int32_t* offsets, int32_t* starts, int32_t* kv_tiles,
                          int32_t* row_ptr, int32_t* q_tiles, cudaStream_t s) {
   dsa::plan_kernel<<<1, 1024, 0, s>>>(plan_geom(g), offsets, starts, kv_tiles, row_ptr, q_tiles);
   return launch_status();
 }
 
+// kv_tiles: the plan's [n_tiles, Wt] key tiles (row_ptr null) or a caller's key-tile list
+// with its CSR offsets row_ptr [n_tiles + 1] and nnz entries (bf16 only).
 dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
-                        const int32_t* kv_tiles, void* out, float* lse, cudaStream_t s) {
+                        const int32_t* kv_tiles, void* out, float* lse, cudaStream_t s,
+                        const int32_t* row_ptr = nullptr, int nnz = 0) {
   if (p->dtype == DSA_F32) {
     dsa::FwdF32Params fp;
     fp.q = static_cast<const float*>(q);
@@ -241,6 +284,8 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
     return DSA_ERR_CUDA;
   dsa::FwdBf16Params bp;
   bp.kv_tiles = kv_tiles;
+  bp.row_ptr = row_ptr;
+  bp.nnz = nnz;
   bp.out = static_cast<__nv_bfloat16*>(out);
   bp.lse = lse;
   bp.n_tiles = g.n_tiles;
@@ -269,6 +314,61 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
   dsa::fwd_bf16_kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, bp);
+  return launch_status();
+}
+
+// The backward after planning: D preprocess (and zeroing of the dQ accumulator), the
+// key-major kernel over the inverse CSR (row_ptr, q_tiles), and the dQ conversion.
+dsa_status_t launch_bwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
+                        const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
+                        const int32_t* q_tiles, float* delta, float* dq_acc, void* dq, void* dk, void* dv,
+                        cudaStream_t s) {
+  dsa_status_t st;
+  const int64_t rows = g.BH * g.N;
+  dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta, dq_acc, rows);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo, tlse, tdel;
+  if (!make_token_map(&tq, q, p, g, 64) || !make_token_map(&tk, k, p, g, 128) ||
+      !make_token_map(&tv, v, p, g, 128) || !make_token_map(&tdo, dout, p, g, 64) ||
+      !make_row_map(&tlse, lse, p, g, 64) || !make_row_map(&tdel, delta, p, g, 64))
+    return DSA_ERR_CUDA;
+  dsa::BwdBf16Params bp;
+  bp.row_ptr = row_ptr;
+  bp.q_tiles = q_tiles;
+  bp.dq_acc = dq_acc;
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.n_tiles = g.n_tiles;
+  bp.KU = g.tile_tokens / 128;
+  bp.QS = g.tile_tokens / 64;
+  bp.n_units = static_cast<int>(g.BH * g.n_tiles * bp.KU);
+  bp.G1 = g.G[1];
+  bp.G2 = g.G[2];
+  bp.tt = p->tile[0];
+  bp.th = p->tile[1];
+  bp.tw = p->tile[2];
+  bp.kcs = 128 / (p->tile[1] * p->tile[2]);
+  bp.qcs = 64 / (p->tile[1] * p->tile[2]);
+  bp.T = p->T;
+  bp.H = p->H;
+  bp.W = p->W;
+  bp.N = static_cast<int>(g.N);
+  bp.scale = p->scale;
+  bp.scale_log2 = p->scale * 1.4426950408889634f;
+  if (cudaFuncSetAttribute(dsa::bwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dsa::bwd::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
+  dsa::bwd_bf16_kernel<<<grid, dsa::bwd::kThreads, dsa::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tlse, tdel, bp);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  const int64_t n8 = rows * p->d / 8;
+  dsa::bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
+      dq_acc, static_cast<__nv_bfloat16*>(dq), p->scale, n8);
   return launch_status();
 }
 
@@ -401,52 +501,61 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_plan(g, tile_offsets, ws.starts, ws.kv_tiles, ws.row_ptr, ws.q_tiles, s);
   if (st != DSA_OK) return st;
-  const int64_t rows = g.BH * g.N;
-  dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), ws.delta, ws.dq_acc, rows);
+  return launch_bwd(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, ws.delta, ws.dq_acc, dq, dk, dv, s);
+}
+
+size_t dsa_list_workspace_size(const dsa_problem_t* p, int32_t nnz, int32_t kind) {
+  Geom g;
+  if (check_shape(p, &g) != DSA_OK || nnz < 0) return 0;
+  if (kind == DSA_WS_FWD) return 0;
+  if (kind == DSA_WS_BWD) return list_bwd_workspace(g, p->d, nnz, nullptr).bytes;
+  return 0;
+}
+
+dsa_status_t dsa_fwd_list(const dsa_problem_t* p, const void* q, const void* k, const void* v,
+                          const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, void* out, float* lse,
+                          void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !kv_row_ptr || !out || !lse || nnz < 0 || (nnz > 0 && !kv_list)) return DSA_ERR_INVALID_ARG;
+  if (p->dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  st = check_kernel_limits(p, g, false);
+  if (st != DSA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+      !aligned(kv_row_ptr, 4) || (kv_list && !aligned(kv_list, 4)))
+    return DSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_list_check(g, kv_row_ptr, kv_list, nnz, s);
+  if (st != DSA_OK) return st;
+  return launch_fwd(p, g, q, k, v, kv_list, out, lse, s, kv_row_ptr, nnz);
+}
+
+dsa_status_t dsa_bwd_list(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,
+                          const float* lse, const void* dout, const int32_t* kv_row_ptr, const int32_t* kv_list,
+                          int32_t nnz, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !out || !lse || !dout || !kv_row_ptr || !dq || !dk || !dv || nnz < 0 ||
+      (nnz > 0 && !kv_list))
+    return DSA_ERR_INVALID_ARG;
+  st = check_kernel_limits(p, g, true);
+  if (st != DSA_OK) return st;
+  const void* ptrs[] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned(ptr, 16)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4) || !aligned(kv_row_ptr, 4) || (kv_list && !aligned(kv_list, 4))) return DSA_ERR_INVALID_ARG;
+  ListBwdWorkspace ws = list_bwd_workspace(g, p->d, nnz, workspace);
+  if (workspace == nullptr || ws_bytes < ws.bytes || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_list_check(g, kv_row_ptr, kv_list, nnz, s);
+  if (st != DSA_OK) return st;
+  dsa::invert_lists_kernel<<<1, 1024, 0, s>>>(kv_row_ptr, kv_list, g.n_tiles, nnz, ws.counts, ws.row_ptr,
+                                              ws.q_tiles);
   st = launch_status();
   if (st != DSA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo, tlse, tdel;
-  if (!make_token_map(&tq, q, p, g, 64) || !make_token_map(&tk, k, p, g, 128) ||
-      !make_token_map(&tv, v, p, g, 128) || !make_token_map(&tdo, dout, p, g, 64) ||
-      !make_row_map(&tlse, lse, p, g, 64) || !make_row_map(&tdel, ws.delta, p, g, 64))
-    return DSA_ERR_CUDA;
-  dsa::BwdBf16Params bp;
-  bp.row_ptr = ws.row_ptr;
-  bp.q_tiles = ws.q_tiles;
-  bp.dq_acc = ws.dq_acc;
-  bp.dk = static_cast<__nv_bfloat16*>(dk);
-  bp.dv = static_cast<__nv_bfloat16*>(dv);
-  bp.n_tiles = g.n_tiles;
-  bp.KU = g.tile_tokens / 128;
-  bp.QS = g.tile_tokens / 64;
-  bp.n_units = static_cast<int>(g.BH * g.n_tiles * bp.KU);
-  bp.G1 = g.G[1];
-  bp.G2 = g.G[2];
-  bp.tt = p->tile[0];
-  bp.th = p->tile[1];
-  bp.tw = p->tile[2];
-  bp.kcs = 128 / (p->tile[1] * p->tile[2]);
-  bp.qcs = 64 / (p->tile[1] * p->tile[2]);
-  bp.T = p->T;
-  bp.H = p->H;
-  bp.W = p->W;
-  bp.N = static_cast<int>(g.N);
-  bp.scale = p->scale;
-  bp.scale_log2 = p->scale * 1.4426950408889634f;
-  if (cudaFuncSetAttribute(dsa::bwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dsa::bwd::kSmemBytes) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  int sms = 0;
-  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
-  dsa::bwd_bf16_kernel<<<grid, dsa::bwd::kThreads, dsa::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tlse, tdel, bp);
-  st = launch_status();
-  if (st != DSA_OK) return st;
-  const int64_t n8 = rows * p->d / 8;
-  dsa::bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
-      ws.dq_acc, static_cast<__nv_bfloat16*>(dq), p->scale, n8);
-  return launch_status();
+  return launch_bwd(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, ws.delta, ws.dq_acc, dq, dk, dv, s);
 }
 
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {

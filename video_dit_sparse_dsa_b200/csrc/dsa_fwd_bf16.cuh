@@ -52,7 +52,9 @@
 namespace dsa {
 
 struct FwdBf16Params {
-  const int32_t* kv_tiles;  // [n_tiles, Wt]
+  const int32_t* kv_tiles;  // window form: [n_tiles, Wt]; list form: the caller's list [nnz]
+  const int32_t* row_ptr;   // list form: [n_tiles + 1] CSR offsets into kv_tiles; null: window form
+  int nnz;                  // list form: entries of the list
   __nv_bfloat16* out;       // [B*heads, N, 128]
   float* lse;               // [B*heads, N]
   int n_tiles, Wt;
@@ -108,6 +110,19 @@ __device__ __forceinline__ uint32_t col_p(int e) { return e ? 256u : 0u; }
 struct Unit {
   int bh, tile, sub;
 };
+
+// Key tiles of query tile `tile` and their count: the window's Wt tiles, or the tile's
+// row of the caller's list with every index clamped into the list (an invalid list gives
+// wrong numbers and a device error from the list check, never an access outside it).
+__device__ __forceinline__ const int32_t* unit_keys(const FwdBf16Params& p, int tile, int& n_list) {
+  if (p.row_ptr == nullptr) {
+    n_list = p.Wt;
+    return p.kv_tiles + static_cast<int64_t>(tile) * p.Wt;
+  }
+  const int a = min(max(p.row_ptr[tile], 0), p.nnz), b = min(max(p.row_ptr[tile + 1], a), p.nnz);
+  n_list = b - a;
+  return p.kv_tiles + a;
+}
 
 __device__ __forceinline__ Unit decode(const FwdBf16Params& p, int u) {
   Unit x;
@@ -317,8 +332,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   float* xbuf = reinterpret_cast<float*>(smem + kOffX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_chunks = p.Wt * p.S;        // 128-key chunks per unit
-  const int n_steps = (n_chunks + 1) / 2;  // 256-key steps per unit
 
   if (tid == 0) {
     tma_prefetch_map(&tmQ);
@@ -360,10 +373,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       // ------------------------------------------------------------------ TMA producers
       if (lane == 0) {
         const bool is_k = warp == kProducerWarp;
-        int ld = 0, uc = 0;  // ring entries loaded, units
+        int ld = 0, uc = 0;  // ring entries loaded, units with keys
         bool ok = true;
-        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
           const Unit x = decode(p, u);
+          int n_list;
+          const int32_t* kv = unit_keys(p, x.tile, n_list);
+          const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
+          if (n_chunks == 0) continue;  // nothing to load: the softmax warps write O = 0
           if (is_k) {
             const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
             ok = mbar_wait(q_empty, (uc & 1) ^ 1, abort, 20);
@@ -373,7 +390,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             tma_load_5d(smem + kOffQ, &tmQ, q_full, 0, qw * p.tw, qh * p.th, tq0, x.bh);
             tma_load_5d(smem + kOffQ + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, tq0, x.bh);
           }
-          const int32_t* kv = p.kv_tiles + static_cast<int64_t>(x.tile) * p.Wt;
+          ++uc;
           // K: one stage per step, chunk b's channel half h at h * 32 KB + b * 16 KB;
           // V: one entry per chunk
           const int n_loads = is_k ? n_steps : n_chunks;
@@ -387,7 +404,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             mbar_arrive_expect_tx(full, nb * kTileBytes);
             for (int b = 0; b < nb; ++b) {
               const int c = is_k ? 2 * j + b : j;
-              const int kt = kv[c / p.S], ks = c % p.S;
+              const int kt = min(max(kv[c / p.S], 0), p.n_tiles - 1), ks = c % p.S;
               const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
               const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
               if (is_k) {
@@ -412,7 +429,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       int uc = 0, g = 0;              // units and steps so far
       int pc0 = 0, pc1 = 0;           // phases of p_full[0 / 1] and s_read[0 / 1] consumed
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uc) {
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        int n_list;
+        unit_keys(p, decode(p, u).tile, n_list);
+        const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
+        if (n_chunks == 0) continue;
         ok = warp_wait(q_full, uc & 1, abort, 30);
         if (ok) ok = warp_wait(k_full + ks % kKStages, (ks / kKStages) & 1, abort, 31);
         if (!ok) break;
@@ -454,6 +475,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (!ok) break;
         mma_commit_warp(o_final);
         g += n_steps;
+        ++uc;
       }
     }
   } else {
@@ -472,11 +494,24 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const uint32_t tO = tmem + kColO + 64 * i + lane_off;  // this warpgroup's 64 channels of O
     int sc0 = 0, sc1 = 0;  // phases of s_full[0 / 1] waited
     int g = 0;             // steps before the current unit (products into O, step parity)
-    int uc = 0;            // units before the current one
+    int uc = 0;            // units with keys before the current one
     int xe = 0;            // pair exchanges so far
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++uc) {
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
       const Unit x = decode(p, u);
+      int n_list;
+      unit_keys(p, x.tile, n_list);
+      const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
+      if (n_chunks == 0) {
+        // no keys: O = 0 and LSE = ln 0 = -inf (the softmax of an empty set has no value;
+        // this is the limit the oracle and the list form define)
+        const int64_t tok = chunk_token(p, x.tile, x.sub, r);
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * p.N + tok) * 128) + 8 * i;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (i == 0) p.lse[static_cast<int64_t>(x.bh) * p.N + tok] = -INFINITY;
+        continue;
+      }
       float m_used = -INFINITY, l = 0.f;
       for (int t = 0; t < n_steps; ++t) {
         const int e = (g + t) & 1;
@@ -520,6 +555,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (lane == 0) mbar_arrive(o_free);
       }
       g += n_steps;
+      ++uc;
     }
   }
 
