@@ -143,25 +143,39 @@ dsa_status_t dsa_fwd_noalloc(const dsa_problem_t* p, const void* q, const void* 
  * generalisation MOD-DiT's online block masking uses (the MOD-DiT page, Method section,
  * Stage 2 "Online Block Masking": attention over selected key blocks); the window form is
  * the case kv_row_ptr[i] = i * Wt with the plan's key tiles.
- *   kv_row_ptr: device int32 [nTiles + 1], kv_row_ptr[0] = 0, non-decreasing,
- *               kv_row_ptr[nTiles] = nnz;  kv_list: device int32 [nnz] (may be NULL when
- *               nnz = 0), entries in [0, nTiles).  A tile listed twice in a row counts twice
- *               (the softmax runs over the multiset); an empty row gives out = 0 and
- *               lse = -inf.  p->window is not used (any positive values).
+ *   per_head = 0: one list for every (batch, head): kv_row_ptr is device int32 [nTiles + 1];
+ *   per_head = 1: a list per (batch, head) (head-adaptive sparsity, or per-head offsets via
+ *                 dsa_plan_heads): kv_row_ptr is [B * heads, nTiles + 1], row i of head h at
+ *                 kv_row_ptr[h * (nTiles + 1) + i], with absolute positions in kv_list;
+ *   in both cases kv_row_ptr, read as one sequence, starts at 0, never decreases and ends at
+ *   nnz (so each head's rows follow the previous head's); kv_list: device int32 [nnz] (may
+ *   be NULL when nnz = 0), entries in [0, nTiles).  A tile listed twice in a row counts
+ *   twice (the softmax runs over the multiset); an empty row gives out = 0 and lse = -inf.
+ *   p->window is not used (any positive values).
  * The lists are checked on the device: a violation is recorded in the status word
  * (DSA_ERR_DEVICE from dsa_device_status) and the results are then unspecified; every
  * index the kernels take from the lists is clamped, so an invalid list never makes them
  * read or write outside the buffers.  bf16 with d = 128, tile limits as dsa_fwd.
  * The forward needs no workspace; the backward builds the inverse lists in its workspace
- * of at least dsa_list_workspace_size(p, nnz, DSA_WS_BWD) bytes (256-byte aligned, contents
- * on entry do not matter). */
-size_t dsa_list_workspace_size(const dsa_problem_t* p, int32_t nnz, int32_t kind);
+ * of at least dsa_list_workspace_size(p, nnz, per_head, DSA_WS_BWD) bytes (256-byte
+ * aligned, contents on entry do not matter). */
+size_t dsa_list_workspace_size(const dsa_problem_t* p, int32_t nnz, int32_t per_head, int32_t kind);
 dsa_status_t dsa_fwd_list(const dsa_problem_t* p, const void* q, const void* k, const void* v,
-                          const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, void* out, float* lse,
-                          void* stream);
+                          const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, int32_t per_head, void* out,
+                          float* lse, void* stream);
 dsa_status_t dsa_bwd_list(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,
                           const float* lse, const void* dout, const int32_t* kv_row_ptr, const int32_t* kv_list,
-                          int32_t nnz, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream);
+                          int32_t nnz, int32_t per_head, void* dq, void* dk, void* dv, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* Per-(batch, head) window offsets as per-head key-tile lists: head h = b * heads + j
+ * plans its own offsets tile_offsets[h][i][3] (device int32 [B * heads, nTiles, 3], the
+ * window rule of dsa_plan) into kv_list[(h * nTiles + i) * Wt ...] (device int32
+ * [B * heads * nTiles * Wt]) with kv_row_ptr[h][i] = (h * nTiles + i) * Wt (device int32
+ * [B * heads, nTiles + 1]), ready for dsa_fwd_list / dsa_bwd_list with per_head = 1 and
+ * nnz = B * heads * nTiles * Wt. */
+dsa_status_t dsa_plan_heads(const dsa_problem_t* p, const int32_t* tile_offsets, int32_t* kv_row_ptr, int32_t* kv_list,
+                            void* stream);
 
 /* Waits for `stream`, then reads and clears the device status word of the current device.
  * Returns DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE (or DSA_ERR_CUDA if the read failed);

@@ -277,26 +277,39 @@ def backward(geo: Geometry, q, k, v, dout, offsets):
 # kv_list[row_ptr[i]:row_ptr[i+1]] instead of its window box; see dsa_oracle.c.
 
 
-def _lists(geo: Geometry, row_ptr, kv_list):
-    rp = _i32(row_ptr).reshape(-1)
+def _head_lists(geo: Geometry, row_ptr, kv_list, h: int):
+    """CSR of (b, head) h: row_ptr is [nTiles + 1] (one list for every head) or
+    [B * heads, nTiles + 1] with absolute positions in kv_list (a list per head)."""
+    rp = _i32(row_ptr)
     kl = _i32(kv_list).reshape(-1)
+    if rp.ndim == 2:
+        if rp.shape != (geo.B * geo.heads, geo.n_tiles + 1):
+            raise ValueError("per-head row_ptr must be [B * heads, nTiles + 1]")
+        rp = rp[h]
+        lo, hi = int(rp[0]), int(rp[-1])
+        if not 0 <= lo <= hi <= kl.shape[0]:
+            raise RuntimeError("per-head row_ptr outside the list")
+        rp, kl = rp - lo, kl[lo:hi]
+    rp = np.ascontiguousarray(rp.reshape(-1), dtype=np.int32)
     if rp.shape[0] != geo.n_tiles + 1:
         raise ValueError("row_ptr must have nTiles + 1 entries")
+    kl = np.ascontiguousarray(kl, dtype=np.int32)
     if kl.shape[0] == 0:
         kl = np.zeros(1, np.int32)  # a valid pointer for an all-empty list
     return rp, kl
 
 
 def _run_by_head_lists(geo: Geometry, tensors, row_ptr, kv_list, sel, n_out, call):
-    """As _run_by_head, with key-tile lists instead of window offsets."""
+    """As _run_by_head, with key-tile lists (shared by every head, or one per head)
+    instead of window offsets."""
     bh, tiles = _selection(geo, sel)
-    rp, kl = _lists(geo, row_ptr, kv_list)
     outs = [np.zeros((len(bh), geo.tile_tokens, geo.d), np.float64) for _ in range(n_out)]
     lse = np.zeros((len(bh), geo.tile_tokens), np.float64)
     one = Geometry(1, 1, geo.d, geo.grid, geo.tile, (1, 1, 1), geo.scale)
     p = one.c_problem()
     for h in np.unique(bh):
         rows = np.nonzero(bh == h)[0]
+        rp, kl = _head_lists(geo, row_ptr, kv_list, int(h))
         sl = [_head_slice(t, geo, int(h)) for t in tensors]
         sel_t = np.ascontiguousarray(tiles[rows])
         sel_b = np.zeros(len(rows), np.int32)
@@ -322,7 +335,8 @@ def _scatter(geo: Geometry, tiles_major):
 
 
 def forward_list(geo: Geometry, q, k, v, row_ptr, kv_list, sel=None):
-    """Forward over key-tile lists.  With sel=None: out[B, heads, T, H, W, d] and
+    """Forward over key-tile lists (row_ptr [nTiles + 1] for every head, or
+    [B * heads, nTiles + 1] per head).  With sel=None: out[B, heads, T, H, W, d] and
     lse[B, heads, T, H, W] (float64); with sel: per (bh, query tile) rows as forward_tiles."""
     lib = _load()
     D = ctypes.c_double

@@ -106,27 +106,33 @@ def test_bwd_rejects_bad_arguments(lib):
 def test_list_entry_points_reject_bad_arguments(lib):
     p = _prob()
     f = FAKE
-    # forward: (p, q, k, v, row_ptr, list, nnz, out, lse, stream)
-    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, None, f, 4, f, f, None) == 1      # no row_ptr
-    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, None, 4, f, f, None) == 1      # nnz > 0 without a list
-    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, f, -1, f, f, None) == 1        # negative nnz
-    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, f, 4, ctypes.c_void_p((1 << 20) + 8), f, None) == 1
+    # forward: (p, q, k, v, row_ptr, list, nnz, per_head, out, lse, stream)
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, None, f, 4, 0, f, f, None) == 1      # no row_ptr
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, None, 4, 0, f, f, None) == 1      # nnz > 0 without a list
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, f, -1, 0, f, f, None) == 1        # negative nnz
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, f, 4, 2, f, f, None) == 1         # per_head not 0 / 1
+    assert lib.dsa_fwd_list(ctypes.byref(p), f, f, f, f, f, 4, 0, ctypes.c_void_p((1 << 20) + 8), f, None) == 1
     p32 = _prob(d=64, dtype=dsa.DSA_F32, grid=(4, 8, 8), tile=(1, 4, 4))
-    assert lib.dsa_fwd_list(ctypes.byref(p32), f, f, f, f, f, 4, f, f, None) == 2       # bf16 only
-    assert lib.dsa_fwd_list(ctypes.byref(_prob(d=64)), f, f, f, f, f, 4, f, f, None) == 2
-    # backward: (p, q, k, v, out, lse, dout, row_ptr, list, nnz, dq, dk, dv, ws, ws_bytes, stream)
-    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, None, f, 4, f, f, f, f, 1 << 30, None) == 1
-    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, f, f, 4, f, f, f, f, 16, None) == 5
-    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, f, f, 4, f, f, f, None, 1 << 30, None) == 5
+    assert lib.dsa_fwd_list(ctypes.byref(p32), f, f, f, f, f, 4, 0, f, f, None) == 2       # bf16 only
+    assert lib.dsa_fwd_list(ctypes.byref(_prob(d=64)), f, f, f, f, f, 4, 1, f, f, None) == 2
+    # backward: (p, q, k, v, out, lse, dout, row_ptr, list, nnz, per_head, dq, dk, dv, ws, ws_bytes, stream)
+    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, None, f, 4, 0, f, f, f, f, 1 << 30, None) == 1
+    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, f, f, 4, 0, f, f, f, f, 16, None) == 5
+    assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, f, f, 4, 1, f, f, f, None, 1 << 30, None) == 5
+    # per-head planner: (p, offsets, row_ptr, list, stream)
+    assert lib.dsa_plan_heads(ctypes.byref(p), None, f, f, None) == 1
+    assert lib.dsa_plan_heads(ctypes.byref(_prob(window=(0, 1, 1))), f, f, f, None) == 1
 
 
 def test_list_workspace_sizes(lib):
     p = _prob()
-    assert lib.dsa_list_workspace_size(ctypes.byref(p), 100, dsa.DSA_WS_FWD) == 0  # the forward needs none
-    small = lib.dsa_list_workspace_size(ctypes.byref(p), 10, dsa.DSA_WS_BWD)
-    big = lib.dsa_list_workspace_size(ctypes.byref(p), 10000, dsa.DSA_WS_BWD)
+    assert lib.dsa_list_workspace_size(ctypes.byref(p), 100, 0, dsa.DSA_WS_FWD) == 0  # the forward needs none
+    small = lib.dsa_list_workspace_size(ctypes.byref(p), 10, 0, dsa.DSA_WS_BWD)
+    big = lib.dsa_list_workspace_size(ctypes.byref(p), 10000, 0, dsa.DSA_WS_BWD)
+    heads = lib.dsa_list_workspace_size(ctypes.byref(p), 10, 1, dsa.DSA_WS_BWD)
     assert big > small > 4 * (2 * 16 * 32 * 32 * 129)  # at least D and the fp32 dQ accumulator
-    assert lib.dsa_list_workspace_size(ctypes.byref(p), -1, dsa.DSA_WS_BWD) == 0
+    assert heads > small  # an inverse map per head
+    assert lib.dsa_list_workspace_size(ctypes.byref(p), -1, 0, dsa.DSA_WS_BWD) == 0
 
 
 def test_plan_rejects_half_inverse(lib):

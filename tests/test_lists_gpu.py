@@ -154,3 +154,63 @@ def test_block_sparse_lists_at_480p_sampled():
         idx = torch.as_tensor(tok[tiles[s]], device="cuda", dtype=torch.long)
         assert_close(flat_o[int(bh[s])][idx].float().cpu().numpy(), ref_o[s], "bf16", f"out sample {s}")
         assert_lse_close(flat_l[int(bh[s])][idx].cpu().numpy(), ref_l[s], "bf16")
+
+
+def per_head_lists(geo, B, heads, seed, max_len):
+    rps, lists, base = [], [], 0
+    for h in range(B * heads):
+        rp, kl = random_lists(geo.n_tiles, seed + h, max_len)
+        rps.append(rp + base)
+        lists.append(kl)
+        base += len(kl)
+    return np.stack(rps).astype(np.int32), np.concatenate(lists).astype(np.int32)
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_per_head_lists_against_oracle(w):
+    """Head-adaptive sparsity: a different key-tile list for every (batch, head)."""
+    inp = make_inputs(w)
+    geo = oracle.Geometry.of(w)
+    row_ptr, kv_list = per_head_lists(geo, w.B, w.heads, w.seed + 200, 6)
+    q, k, v, dout = inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.dout.cuda()
+    rp, kl = torch.from_numpy(row_ptr).cuda(), torch.from_numpy(kv_list).cuda()
+    out, lse = dsa.forward_list(q, k, v, rp, kl, w.tile, w.scale)
+    dq, dk, dv = dsa.backward_list(q, k, v, out, lse, dout, rp, kl, w.tile, w.scale)
+    st, site, _ = dsa.device_status()
+    assert st == 0, f"device status {st} at site {site}"
+    ref_o, ref_l = oracle.forward_list(geo, inp.q, inp.k, inp.v, row_ptr, kv_list)
+    got_o, got_l = out.float().cpu().numpy(), lse.cpu().numpy()
+    fin = np.isfinite(ref_l)
+    assert not fin.all() and np.all(np.isneginf(got_l[~fin])) and np.all(got_o[~fin] == 0.0)
+    assert_close(got_o[fin], ref_o[fin], "bf16", "out")
+    assert_lse_close(got_l[fin], ref_l[fin], "bf16")
+    rq, rk, rv = oracle.backward_list(geo, inp.q, inp.k, inp.v, inp.dout, row_ptr, kv_list)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        assert_close(got.float().cpu().numpy(), ref, "bf16", name)
+
+
+def test_per_head_offsets_against_the_windowed_oracle():
+    """Per-(batch, head) window offsets, planned on the device into per-head lists, against
+    the oracle's window form run head by head with that head's offsets."""
+    w = Workload("heads_offsets", 2, 2, 128, (8, 16, 24), (4, 8, 8), (3, 1, 3), (-2, 2), "bf16", 45, backward=True)
+    inp = make_inputs(w)
+    geo = oracle.Geometry.of(w)
+    BH = w.B * w.heads
+    g = torch.Generator().manual_seed(99)
+    offs = torch.randint(-2, 3, (BH, geo.n_tiles, 3), generator=g).to(torch.int32)
+    p = dsa.make_problem(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale)
+    rp, kl = dsa.plan_heads(p, offs.cuda())
+    q, k, v, dout = inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.dout.cuda()
+    out, lse = dsa.forward_list(q, k, v, rp, kl, w.tile, w.scale)
+    dq, dk, dv = dsa.backward_list(q, k, v, out, lse, dout, rp, kl, w.tile, w.scale)
+    assert dsa.device_status()[0] == 0
+    one = oracle.Geometry(1, 1, w.d, w.grid, w.tile, w.window, w.scale)
+    for h in range(BH):
+        b, j = divmod(h, w.heads)
+        sl = [t[b:b + 1, j:j + 1] for t in (inp.q, inp.k, inp.v, inp.dout)]
+        ref_o, ref_l = oracle.forward(one, sl[0], sl[1], sl[2], offs[h])
+        assert_close(out[b, j].float().cpu().numpy(), ref_o[0, 0], "bf16", f"out head {h}")
+        assert_lse_close(lse[b, j].cpu().numpy(), ref_l[0, 0], "bf16")
+        rq, rk, rv = oracle.backward(one, *sl, offs[h])
+        for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            assert_close(got[b, j].float().cpu().numpy(), ref[0, 0], "bf16", f"{name} head {h}")

@@ -480,3 +480,34 @@ def test_lists_reject_invalid_csr():
     for rp, kl in bad:
         with pytest.raises(RuntimeError):
             oracle.forward_list(geo, q, k, v, rp, kl)
+
+
+def test_lists_per_head_equal_multiset_attention_per_head():
+    """A list per (batch, head): each head's rows against its own weighted dense attention."""
+    geo = oracle.Geometry(2, 2, 16, (2, 4, 4), (1, 2, 2), (1, 1, 1))
+    q, k, v, do = small_inputs(geo, 21)
+    BH = geo.B * geo.heads
+    rps, lists, base = [], [], 0
+    for h in range(BH):
+        rp, kl = random_lists(geo, 30 + h, 4)
+        rps.append(rp + base)
+        lists.append(kl)
+        base += len(kl)
+    row_ptr = np.stack(rps).astype(np.int32)
+    kv_list = np.concatenate(lists).astype(np.int32)
+    out, lse = oracle.forward_list(geo, q, k, v, row_ptr, kv_list)
+    dq, dk, dv = oracle.backward_list(geo, q, k, v, do, row_ptr, kv_list)
+    one = oracle.Geometry(1, 1, 16, geo.grid, geo.tile, (1, 1, 1))
+    for h in range(BH):
+        b, j = divmod(h, geo.heads)
+        sl = [t[b:b + 1, j:j + 1] for t in (q, k, v, do)]
+        rp = rps[h] - rps[h][0]
+        ref_o, ref_l = multiset_attention(one, sl[0], sl[1], sl[2], rp, lists[h])
+        np.testing.assert_allclose(out[b, j], ref_o.numpy()[0, 0], rtol=0, atol=1e-12)
+        fin = np.isfinite(ref_l.numpy()[0, 0])
+        np.testing.assert_allclose(lse[b, j][fin], ref_l.numpy()[0, 0][fin], rtol=0, atol=1e-12)
+        qr, kr, vr = (t.clone().requires_grad_(True) for t in sl[:3])
+        o, _ = multiset_attention(one, qr, kr, vr, rp, lists[h])
+        (o * sl[3]).sum().backward()
+        for got, ref in ((dq, qr.grad), (dk, kr.grad), (dv, vr.grad)):
+            np.testing.assert_allclose(got[b, j], ref.numpy()[0, 0], rtol=0, atol=1e-11)

@@ -35,7 +35,7 @@ _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_size", "dsa_plan", "dsa_fwd",
            "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status", "dsa_fwd_noalloc",
-           "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list")
+           "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads")
 
 
 class DsaError(RuntimeError):
@@ -80,11 +80,12 @@ def load_library(path: Optional[str] = None):
     lib.dsa_device_status.argtypes = [vp, i32p, i32p]
     lib.dsa_fwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp]
     lib.dsa_list_workspace_size.restype = sz
-    lib.dsa_list_workspace_size.argtypes = [pp, i32, i32]
-    lib.dsa_fwd_list.argtypes = [pp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
-    lib.dsa_bwd_list.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+    lib.dsa_list_workspace_size.argtypes = [pp, i32, i32, i32]
+    lib.dsa_fwd_list.argtypes = [pp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp]
+    lib.dsa_bwd_list.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]
+    lib.dsa_plan_heads.argtypes = [pp, vp, vp, vp, vp]
     for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status",
-                 "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list"):
+                 "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -242,13 +243,20 @@ def backward(q, k, v, out, lse, dout, offsets, tile, window, scale=None, dq=None
 
 
 def _list_args(q: torch.Tensor, row_ptr: torch.Tensor, kv_list: torch.Tensor, n_tiles: int):
+    """-> (list pointer, nnz, per_head): row_ptr [nTiles + 1] is one list for every head,
+    [B * heads, nTiles + 1] one list per (batch, head)."""
     _need(row_ptr, "row_ptr", q, torch.int32)
-    if row_ptr.numel() != n_tiles + 1:
-        raise ValueError(f"row_ptr must have nTiles + 1 = {n_tiles + 1} entries")
+    BH = q.shape[0] * q.shape[1]
+    if row_ptr.numel() == n_tiles + 1 and row_ptr.dim() == 1:
+        per_head = 0
+    elif tuple(row_ptr.shape) == (BH, n_tiles + 1):
+        per_head = 1
+    else:
+        raise ValueError(f"row_ptr must be [nTiles + 1] or [B * heads, nTiles + 1], got {tuple(row_ptr.shape)}")
     if kv_list is not None and kv_list.numel() > 0:
         _need(kv_list, "kv_list", q, torch.int32)
-        return _ptr(kv_list), int(kv_list.numel())
-    return None, 0
+        return _ptr(kv_list), int(kv_list.numel()), per_head
+    return None, 0, per_head
 
 
 def forward_list(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: torch.Tensor, kv_list: torch.Tensor,
@@ -256,7 +264,9 @@ def forward_list(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: tor
                  lse: Optional[torch.Tensor] = None, stream=None):
     """Block-sparse forward over key-tile lists: query tile i attends to the key tiles
     kv_list[row_ptr[i]:row_ptr[i+1]] (int32 CUDA tensors; tiles in raster order of the tile
-    grid).  Returns (out, lse); an empty row gives out = 0 and lse = -inf."""
+    grid); row_ptr [nTiles + 1] is one list for every head, [B * heads, nTiles + 1] one per
+    (batch, head) with absolute positions in kv_list.  Returns (out, lse); an empty row
+    gives out = 0 and lse = -inf."""
     lib = load_library()
     p = _problem_of(q, tile, (1, 1, 1), scale)
     for t, name in ((k, "k"), (v, "v")):
@@ -265,15 +275,15 @@ def forward_list(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, row_ptr: tor
             raise ValueError(f"{name} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
     _need(q, "q", q)
     n_tiles, _ = plan_shape(p)
-    lst, nnz = _list_args(q, row_ptr, kv_list, n_tiles)
+    lst, nnz, per_head = _list_args(q, row_ptr, kv_list, n_tiles)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty(q.shape[:5], dtype=torch.float32, device=q.device)
     _need(out, "out", q, q.dtype)
     _need(lse, "lse", q, torch.float32)
-    _check(lib.dsa_fwd_list(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), lst, nnz, _ptr(out), _ptr(lse),
-                            ctypes.c_void_p(_stream(stream))), "dsa_fwd_list")
+    _check(lib.dsa_fwd_list(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), lst, nnz, per_head, _ptr(out),
+                            _ptr(lse), ctypes.c_void_p(_stream(stream))), "dsa_fwd_list")
     return out, lse
 
 
@@ -289,19 +299,36 @@ def backward_list(q, k, v, out, lse, dout, row_ptr, kv_list, tile, scale=None, d
     _need(q, "q", q)
     _need(lse, "lse", q, torch.float32)
     n_tiles, _ = plan_shape(p)
-    lst, nnz = _list_args(q, row_ptr, kv_list, n_tiles)
+    lst, nnz, per_head = _list_args(q, row_ptr, kv_list, n_tiles)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
         _need(t, name, q, q.dtype)
     if ws is None:
-        size = int(lib.dsa_list_workspace_size(ctypes.byref(p), nnz, DSA_WS_BWD))
+        size = int(lib.dsa_list_workspace_size(ctypes.byref(p), nnz, per_head, DSA_WS_BWD))
         ws = torch.empty(max(size, 256), dtype=torch.uint8, device=q.device)
     _check(lib.dsa_bwd_list(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
-                            _ptr(row_ptr), lst, nnz, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                            _ptr(row_ptr), lst, nnz, per_head, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
                             ctypes.c_void_p(_stream(stream))), "dsa_bwd_list")
     return dq, dk, dv
+
+
+def plan_heads(problem: Problem, offsets: torch.Tensor, stream=None):
+    """Per-(batch, head) window offsets [B * heads, nTiles, 3] (int32 CUDA) as per-head
+    key-tile lists: returns (row_ptr [B * heads, nTiles + 1], kv_list) for forward_list /
+    backward_list."""
+    lib = load_library()
+    n, wt = plan_shape(problem)
+    BH = problem.B * problem.heads
+    if not offsets.is_cuda or offsets.dtype != torch.int32 or not offsets.is_contiguous() or \
+            offsets.numel() != BH * n * 3:
+        raise ValueError("offsets must be a contiguous int32 CUDA tensor [B * heads, nTiles, 3]")
+    row_ptr = torch.empty((BH, n + 1), dtype=torch.int32, device=offsets.device)
+    kv_list = torch.empty(BH * n * wt, dtype=torch.int32, device=offsets.device)
+    _check(lib.dsa_plan_heads(ctypes.byref(problem), _ptr(offsets), _ptr(row_ptr), _ptr(kv_list),
+                              ctypes.c_void_p(_stream(stream))), "dsa_plan_heads")
+    return row_ptr, kv_list
 
 
 def device_status(stream=None):

@@ -124,22 +124,22 @@ BwdWorkspace bwd_workspace(const Geom& g, int d, void* base) {
 // Backward over a caller's key-tile lists: the inverse CSR built on the device, then the
 // same D and dQ accumulator scratch as dsa_bwd.
 struct ListBwdWorkspace {
-  int32_t* counts;   // [n_tiles] scratch of the inversion
-  int32_t* row_ptr;  // [n_tiles + 1] inverse CSR
+  int32_t* counts;   // [n_lists, n_tiles] scratch of the inversion
+  int32_t* row_ptr;  // [n_lists, n_tiles + 1] inverse CSR
   int32_t* q_tiles;  // [nnz]
   float* delta;      // [BH, N]
   float* dq_acc;     // [BH, N, d]
   size_t bytes;
 };
 
-ListBwdWorkspace list_bwd_workspace(const Geom& g, int d, int nnz, void* base) {
+ListBwdWorkspace list_bwd_workspace(const Geom& g, int d, int nnz, int n_lists, void* base) {
   ListBwdWorkspace w;
   uint8_t* b = static_cast<uint8_t*>(base);
   size_t off = 0;
   w.counts = reinterpret_cast<int32_t*>(b + off);
-  off += round_up(sizeof(int32_t) * g.n_tiles, kAlign);
+  off += round_up(sizeof(int32_t) * static_cast<size_t>(n_lists) * g.n_tiles, kAlign);
   w.row_ptr = reinterpret_cast<int32_t*>(b + off);
-  off += round_up(sizeof(int32_t) * (g.n_tiles + 1), kAlign);
+  off += round_up(sizeof(int32_t) * static_cast<size_t>(n_lists) * (g.n_tiles + 1), kAlign);
   w.q_tiles = reinterpret_cast<int32_t*>(b + off);
   off += round_up(sizeof(int32_t) * static_cast<size_t>(nnz > 0 ? nnz : 1), kAlign);
   w.delta = reinterpret_cast<float*>(b + off);
@@ -231,12 +231,14 @@ bool make_row_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, con
 }
 
 // Validation of a caller's CSR on the device (records DSA_DEV_BOUNDS; never faults).
-dsa_status_t launch_list_check(const Geom& g, const int32_t* row_ptr, const int32_t* list, int nnz, cudaStream_t s) {
-  const int64_t work = g.n_tiles > nnz ? g.n_tiles : nnz;
+dsa_status_t launch_list_check(const Geom& g, const int32_t* row_ptr, const int32_t* list, int n_lists, int nnz,
+                               cudaStream_t s) {
+  const int64_t n_ptr = static_cast<int64_t>(n_lists) * (g.n_tiles + 1);
+  const int64_t work = n_ptr > nnz ? n_ptr : nnz;
   int64_t blocks = (work + 255) / 256;
   if (blocks < 1) blocks = 1;
   if (blocks > 1024) blocks = 1024;
-  dsa::list_check_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(row_ptr, list, g.n_tiles, nnz);
+  dsa::list_check_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(row_ptr, list, g.n_tiles, n_lists, nnz);
   return launch_status();
 }
 
@@ -250,7 +252,7 @@ dsa_status_t launch_plan(const Geom& g, const int32_t* offsets, int32_t* starts,
 // with its CSR offsets row_ptr [n_tiles + 1] and nnz entries (bf16 only).
 dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
                         const int32_t* kv_tiles, void* out, float* lse, cudaStream_t s,
-                        const int32_t* row_ptr = nullptr, int nnz = 0) {
+                        const int32_t* row_ptr = nullptr, int nnz = 0, int rp_head_stride = 0) {
   if (p->dtype == DSA_F32) {
     dsa::FwdF32Params fp;
     fp.q = static_cast<const float*>(q);
@@ -285,6 +287,7 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   dsa::FwdBf16Params bp;
   bp.kv_tiles = kv_tiles;
   bp.row_ptr = row_ptr;
+  bp.rp_head_stride = rp_head_stride;
   bp.nnz = nnz;
   bp.out = static_cast<__nv_bfloat16*>(out);
   bp.lse = lse;
@@ -322,7 +325,7 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
 dsa_status_t launch_bwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
                         const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
                         const int32_t* q_tiles, float* delta, float* dq_acc, void* dq, void* dk, void* dv,
-                        cudaStream_t s) {
+                        cudaStream_t s, int rp_head_stride = 0) {
   dsa_status_t st;
   const int64_t rows = g.BH * g.N;
   dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
@@ -336,6 +339,7 @@ dsa_status_t launch_bwd(const dsa_problem_t* p, const Geom& g, const void* q, co
     return DSA_ERR_CUDA;
   dsa::BwdBf16Params bp;
   bp.row_ptr = row_ptr;
+  bp.rp_head_stride = rp_head_stride;
   bp.q_tiles = q_tiles;
   bp.dq_acc = dq_acc;
   bp.dk = static_cast<__nv_bfloat16*>(dk);
@@ -504,58 +508,88 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
   return launch_bwd(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, ws.delta, ws.dq_acc, dq, dk, dv, s);
 }
 
-size_t dsa_list_workspace_size(const dsa_problem_t* p, int32_t nnz, int32_t kind) {
+size_t dsa_list_workspace_size(const dsa_problem_t* p, int32_t nnz, int32_t per_head, int32_t kind) {
   Geom g;
   if (check_shape(p, &g) != DSA_OK || nnz < 0) return 0;
   if (kind == DSA_WS_FWD) return 0;
-  if (kind == DSA_WS_BWD) return list_bwd_workspace(g, p->d, nnz, nullptr).bytes;
+  if (kind == DSA_WS_BWD) return list_bwd_workspace(g, p->d, nnz, per_head ? static_cast<int>(g.BH) : 1, nullptr).bytes;
   return 0;
 }
 
-dsa_status_t dsa_fwd_list(const dsa_problem_t* p, const void* q, const void* k, const void* v,
-                          const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, void* out, float* lse,
-                          void* stream) {
+dsa_status_t dsa_plan_heads(const dsa_problem_t* p, const int32_t* tile_offsets, int32_t* kv_row_ptr, int32_t* kv_list,
+                            void* stream) {
   Geom g;
   dsa_status_t st = check_shape(p, &g);
   if (st != DSA_OK) return st;
-  if (!q || !k || !v || !kv_row_ptr || !out || !lse || nnz < 0 || (nnz > 0 && !kv_list)) return DSA_ERR_INVALID_ARG;
+  if (!tile_offsets || !kv_row_ptr || !kv_list) return DSA_ERR_INVALID_ARG;
+  if (g.BH > 65535 || g.BH * g.n_tiles * static_cast<int64_t>(g.Wt) > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (!aligned(tile_offsets, 4) || !aligned(kv_row_ptr, 4) || !aligned(kv_list, 4)) return DSA_ERR_INVALID_ARG;
+  dsa::plan_heads_kernel<<<static_cast<unsigned>(g.BH), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      plan_geom(g), tile_offsets, kv_row_ptr, kv_list);
+  return launch_status();
+}
+
+namespace {
+// Argument checks shared by the list entry points; n_lists = 1 or B*heads.
+dsa_status_t check_lists(const Geom& g, const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz,
+                         int32_t per_head, int* n_lists) {
+  if (!kv_row_ptr || nnz < 0 || (nnz > 0 && !kv_list) || (per_head != 0 && per_head != 1)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(kv_row_ptr, 4) || (kv_list && !aligned(kv_list, 4))) return DSA_ERR_INVALID_ARG;
+  *n_lists = per_head ? static_cast<int>(g.BH) : 1;
+  if (static_cast<int64_t>(*n_lists) * (g.n_tiles + 1) > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+}  // namespace
+
+dsa_status_t dsa_fwd_list(const dsa_problem_t* p, const void* q, const void* k, const void* v,
+                          const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, int32_t per_head, void* out,
+                          float* lse, void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !out || !lse) return DSA_ERR_INVALID_ARG;
+  int n_lists = 1;
+  st = check_lists(g, kv_row_ptr, kv_list, nnz, per_head, &n_lists);
+  if (st != DSA_OK) return st;
   if (p->dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
   st = check_kernel_limits(p, g, false);
   if (st != DSA_OK) return st;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
-      !aligned(kv_row_ptr, 4) || (kv_list && !aligned(kv_list, 4)))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
     return DSA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_list_check(g, kv_row_ptr, kv_list, nnz, s);
+  st = launch_list_check(g, kv_row_ptr, kv_list, n_lists, nnz, s);
   if (st != DSA_OK) return st;
-  return launch_fwd(p, g, q, k, v, kv_list, out, lse, s, kv_row_ptr, nnz);
+  return launch_fwd(p, g, q, k, v, kv_list, out, lse, s, kv_row_ptr, nnz, per_head ? g.n_tiles + 1 : 0);
 }
 
 dsa_status_t dsa_bwd_list(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,
                           const float* lse, const void* dout, const int32_t* kv_row_ptr, const int32_t* kv_list,
-                          int32_t nnz, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream) {
+                          int32_t nnz, int32_t per_head, void* dq, void* dk, void* dv, void* workspace,
+                          size_t ws_bytes, void* stream) {
   Geom g;
   dsa_status_t st = check_shape(p, &g);
   if (st != DSA_OK) return st;
-  if (!q || !k || !v || !out || !lse || !dout || !kv_row_ptr || !dq || !dk || !dv || nnz < 0 ||
-      (nnz > 0 && !kv_list))
-    return DSA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return DSA_ERR_INVALID_ARG;
+  int n_lists = 1;
+  st = check_lists(g, kv_row_ptr, kv_list, nnz, per_head, &n_lists);
+  if (st != DSA_OK) return st;
   st = check_kernel_limits(p, g, true);
   if (st != DSA_OK) return st;
   const void* ptrs[] = {q, k, v, out, dout, dq, dk, dv};
   for (const void* ptr : ptrs)
     if (!aligned(ptr, 16)) return DSA_ERR_INVALID_ARG;
-  if (!aligned(lse, 4) || !aligned(kv_row_ptr, 4) || (kv_list && !aligned(kv_list, 4))) return DSA_ERR_INVALID_ARG;
-  ListBwdWorkspace ws = list_bwd_workspace(g, p->d, nnz, workspace);
+  if (!aligned(lse, 4)) return DSA_ERR_INVALID_ARG;
+  ListBwdWorkspace ws = list_bwd_workspace(g, p->d, nnz, n_lists, workspace);
   if (workspace == nullptr || ws_bytes < ws.bytes || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_list_check(g, kv_row_ptr, kv_list, nnz, s);
+  st = launch_list_check(g, kv_row_ptr, kv_list, n_lists, nnz, s);
   if (st != DSA_OK) return st;
-  dsa::invert_lists_kernel<<<1, 1024, 0, s>>>(kv_row_ptr, kv_list, g.n_tiles, nnz, ws.counts, ws.row_ptr,
-                                              ws.q_tiles);
+  dsa::invert_lists_kernel<<<static_cast<unsigned>(n_lists), 1024, 0, s>>>(kv_row_ptr, kv_list, g.n_tiles, nnz,
+                                                                           ws.counts, ws.row_ptr, ws.q_tiles);
   st = launch_status();
   if (st != DSA_OK) return st;
-  return launch_bwd(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, ws.delta, ws.dq_acc, dq, dk, dv, s);
+  return launch_bwd(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, ws.delta, ws.dq_acc, dq, dk, dv, s,
+                    per_head ? g.n_tiles + 1 : 0);
 }
 
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {

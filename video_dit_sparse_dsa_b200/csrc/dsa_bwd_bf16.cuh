@@ -21,7 +21,8 @@
 namespace dsa {
 
 struct BwdBf16Params {
-  const int32_t* row_ptr;  // [n_tiles + 1] inverse plan
+  const int32_t* row_ptr;  // inverse plan: [n_tiles + 1], or per (batch, head) [B*heads, n_tiles + 1]
+  int rp_head_stride;      // 0 (one inverse map for every head) or n_tiles + 1
   const int32_t* q_tiles;  // [n_tiles * Wt]
   float* dq_acc;           // [BH, N, 128] fp32, zeroed by bwd_preprocess
   __nv_bfloat16* dk;       // [BH, N, 128]
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         int bh, kt, ku;
         unit_of(u, bh, kt, ku);
-        const int row0 = p.row_ptr[kt], n = (p.row_ptr[kt + 1] - row0) * p.QS;
+        const int row0 = p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt], n = (p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt + 1] - row0) * p.QS;
         if (n == 0) continue;
         ok = mbar_wait(kv_free, (uc & 1) ^ 1, abort, 50);
         if (!ok) break;
@@ -255,7 +256,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         int bh, kt, ku;
         unit_of(u, bh, kt, ku);
-        const int n = (p.row_ptr[kt + 1] - p.row_ptr[kt]) * p.QS;
+        const int n = (p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt + 1] - p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt]) * p.QS;
         if (n == 0) continue;
         ok = __all_sync(0xffffffffu, mbar_wait(kv_full, uc & 1, abort, 60));
         if (!ok) break;
@@ -327,7 +328,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       int bh, kt, ku;
       unit_of(u, bh, kt, ku);
-      const int n = (p.row_ptr[kt + 1] - p.row_ptr[kt]) * p.QS;
+      const int n = (p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt + 1] - p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt]) * p.QS;
       for (int c = 0; c < n; ++c, ++cc, ++ld) {
         const int b = cc & 1;
         ok = mbar_wait(s_full + b, (cc >> 1) & 1, abort, 70);
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       int bh, kt, ku;
       unit_of(u, bh, kt, ku);
-      const int row0 = p.row_ptr[kt], n = (p.row_ptr[kt + 1] - row0) * p.QS;
+      const int row0 = p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt], n = (p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt + 1] - row0) * p.QS;
       const int64_t slice = static_cast<int64_t>(bh) * p.N;
       for (int c = 0; c < n; ++c, ++cc) {
         const int b = cc & 1;

@@ -53,7 +53,8 @@ namespace dsa {
 
 struct FwdBf16Params {
   const int32_t* kv_tiles;  // window form: [n_tiles, Wt]; list form: the caller's list [nnz]
-  const int32_t* row_ptr;   // list form: [n_tiles + 1] CSR offsets into kv_tiles; null: window form
+  const int32_t* row_ptr;   // list form: CSR offsets into kv_tiles; null: window form
+  int rp_head_stride;       // list form: 0 (one list for every head) or n_tiles + 1 (one per head)
   int nnz;                  // list form: entries of the list
   __nv_bfloat16* out;       // [B*heads, N, 128]
   float* lse;               // [B*heads, N]
@@ -114,12 +115,13 @@ struct Unit {
 // Key tiles of query tile `tile` and their count: the window's Wt tiles, or the tile's
 // row of the caller's list with every index clamped into the list (an invalid list gives
 // wrong numbers and a device error from the list check, never an access outside it).
-__device__ __forceinline__ const int32_t* unit_keys(const FwdBf16Params& p, int tile, int& n_list) {
+__device__ __forceinline__ const int32_t* unit_keys(const FwdBf16Params& p, int bh, int tile, int& n_list) {
   if (p.row_ptr == nullptr) {
     n_list = p.Wt;
     return p.kv_tiles + static_cast<int64_t>(tile) * p.Wt;
   }
-  const int a = min(max(p.row_ptr[tile], 0), p.nnz), b = min(max(p.row_ptr[tile + 1], a), p.nnz);
+  const int32_t* rp = p.row_ptr + static_cast<int64_t>(bh) * p.rp_head_stride;
+  const int a = min(max(rp[tile], 0), p.nnz), b = min(max(rp[tile + 1], a), p.nnz);
   n_list = b - a;
   return p.kv_tiles + a;
 }
@@ -378,7 +380,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
           const Unit x = decode(p, u);
           int n_list;
-          const int32_t* kv = unit_keys(p, x.tile, n_list);
+          const int32_t* kv = unit_keys(p, x.bh, x.tile, n_list);
           const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
           if (n_chunks == 0) continue;  // nothing to load: the softmax warps write O = 0
           if (is_k) {
@@ -431,7 +433,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         int n_list;
-        unit_keys(p, decode(p, u).tile, n_list);
+        const Unit xm = decode(p, u);
+        unit_keys(p, xm.bh, xm.tile, n_list);
         const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
         if (n_chunks == 0) continue;
         ok = warp_wait(q_full, uc & 1, abort, 30);
@@ -500,7 +503,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
       const Unit x = decode(p, u);
       int n_list;
-      unit_keys(p, x.tile, n_list);
+      unit_keys(p, x.bh, x.tile, n_list);
       const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
       if (n_chunks == 0) {
         // no keys: O = 0 and LSE = ln 0 = -inf (the softmax of an empty set has no value;

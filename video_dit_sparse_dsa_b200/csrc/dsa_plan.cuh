@@ -109,4 +109,29 @@ __global__ void __launch_bounds__(1024) plan_kernel(PlanGeom g, const int32_t* _
   }
 }
 
+// Per-(batch, head) windows as key-tile lists: head h (blockIdx.x) plans its own offsets
+// offsets[h][nTiles][3] into kv_list[h * nTiles * Wt ...] (ascending key tiles per window,
+// as above) with CSR offsets row_ptr[h][i] = (h * nTiles + i) * Wt, so the heads' lists
+// follow one another and the flattened row_ptr is non-decreasing.
+__global__ void __launch_bounds__(256) plan_heads_kernel(PlanGeom g, const int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ row_ptr, int32_t* __restrict__ kv_list) {
+  const int n = g.n_tiles, h = blockIdx.x;
+  const int64_t base = static_cast<int64_t>(h) * n;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int32_t* off = offsets + (base + i) * 3;
+    const int it = i / (g.G[1] * g.G[2]), ih = (i / g.G[2]) % g.G[1], iw = i % g.G[2];
+    const int st = plan_axis_start(it, off[0], g.w[0], g.G[0]);
+    const int sh = plan_axis_start(ih, off[1], g.w[1], g.G[1]);
+    const int sw = plan_axis_start(iw, off[2], g.w[2], g.G[2]);
+    const int64_t first = (base + i) * g.n_window_tiles;
+    row_ptr[static_cast<int64_t>(h) * (n + 1) + i] = static_cast<int32_t>(first);
+    int32_t* dst = kv_list + first;
+    int e = 0;
+    for (int a = st; a < st + g.w[0]; ++a)
+      for (int b = sh; b < sh + g.w[1]; ++b)
+        for (int c = sw; c < sw + g.w[2]; ++c) dst[e++] = (a * g.G[1] + b) * g.G[2] + c;
+  }
+  if (threadIdx.x == 0) row_ptr[static_cast<int64_t>(h) * (n + 1) + n] = static_cast<int32_t>((base + n) * g.n_window_tiles);
+}
+
 }  // namespace dsa
