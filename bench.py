@@ -54,7 +54,7 @@ def peaks():
 # single-pass ncu capture summarised in profiles/fwd_bf16_kernel__bf16_720p_dram.md.  The
 # figure holds only for the kernel sources it was taken on, identified by a hash of them;
 # with any other sources the line reports null.
-FWD_TRAFFIC = {"bf16_720p": (4.99e9, "619b1a789b3ad6c1")}
+FWD_TRAFFIC = {"bf16_720p": (5.30e9, "4a20b269f448ba37")}
 FWD_SOURCES = ("dsa_fwd_bf16.cuh", "sm100.cuh")
 
 
@@ -235,6 +235,35 @@ def run_workload(dsa, w: Workload, device, steps: int, warmup: int, seed_offset:
     return res
 
 
+def run_list_workload(dsa, w: Workload, device, steps: int, warmup: int, n_keep: int):
+    """Block-sparse form on the grid of w: every (batch, head, query tile) keeps n_keep key
+    tiles chosen at random (seeded) from the whole tile grid, as per-head key-tile lists
+    (head-adaptive block masks); the forward's FLOPs count n_keep tiles per query."""
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    q, k, v, _, _ = device_inputs(w, device)
+    BH = w.B * w.heads
+    g = torch.Generator(device=device).manual_seed(7000 + w.seed)
+    pick = torch.rand((BH, w.n_tiles, w.n_tiles), generator=g, device=device).argsort(dim=-1)[..., :n_keep]
+    kv_list = pick.sort(dim=-1).values.to(torch.int32).reshape(-1).contiguous()
+    row_ptr = (torch.arange(BH * (w.n_tiles + 1), device=device, dtype=torch.int64).reshape(BH, w.n_tiles + 1)
+               - torch.arange(BH, device=device, dtype=torch.int64)[:, None])
+    row_ptr = (row_ptr * n_keep).to(torch.int32).contiguous()
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:5], dtype=torch.float32, device=device)
+
+    def fwd():
+        dsa.forward_list(q, k, v, row_ptr, kv_list, w.tile, w.scale, out=out, lse=lse, stream=stream)
+
+    fwd()
+    ms = time_steps(fwd, steps, warmup, stream, record=False)
+    flops = 4.0 * w.B * w.heads * w.n_tokens * (n_keep * w.tile_tokens) * w.d
+    st = dsa.device_status(stream)
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st} after the key-tile-list forward")
+    return {"fwd_ms": ms, "fwd_tflops": flops / (ms * 1e-3) / 1e12, "keys_per_query": n_keep * w.tile_tokens}
+
+
 def run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream):
     """Same forward through the host-buffer entry point: H2D of q, k, v, offsets from pinned
     memory, planner + forward, D2H of out and lse, all inside the timed region."""
@@ -384,6 +413,13 @@ def main():
                 extra[name] = {k2: round(v2, 4) for k2, v2 in r.items()
                                if k2.endswith("_ms") or k2.endswith("_tflops")}
             except Exception as e:  # report, do not hide: the line carries the error
+                extra[name] = {"error": str(e)}
+        if w.dtype == "bf16":
+            name = f"{w.name}_lists{w.window_tiles}"
+            try:
+                r = run_list_workload(dsa, w, device, max(3, args.steps // 2), 3, w.window_tiles)
+                extra[name] = {k2: (round(v2, 4) if isinstance(v2, float) else v2) for k2, v2 in r.items()}
+            except Exception as e:
                 extra[name] = {"error": str(e)}
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
