@@ -264,6 +264,38 @@ def run_list_workload(dsa, w: Workload, device, steps: int, warmup: int, n_keep:
     return {"fwd_ms": ms, "fwd_tflops": flops / (ms * 1e-3) / 1e12, "keys_per_query": n_keep * w.tile_tokens}
 
 
+def run_dense_map_workload(dsa, w: Workload, device, steps: int, warmup: int):
+    """Dense attention on the grid of w (every tile listed for every query tile) and its
+    block attention mass: times the dense forward and the map pass separately.  The map
+    pass recomputes the scores only: 2 * B * heads * N^2 * d FLOP."""
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    q, k, v, _, _ = device_inputs(w, device)
+    n = w.n_tiles
+    row_ptr = torch.arange(n + 1, dtype=torch.int32, device=device) * n
+    kv_list = torch.arange(n, dtype=torch.int32, device=device).repeat(n).contiguous()
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:5], dtype=torch.float32, device=device)
+    bmap = torch.empty((w.B * w.heads, n, n), dtype=torch.float32, device=device)
+
+    def fwd():
+        dsa.forward_list(q, k, v, row_ptr, kv_list, w.tile, w.scale, out=out, lse=lse, stream=stream)
+
+    def bm():
+        dsa.block_map(q, k, lse, row_ptr, kv_list, w.tile, w.scale, out=bmap, stream=stream)
+
+    fwd()
+    bm()
+    f_ms = time_steps(fwd, steps, warmup, stream, record=False)
+    m_ms = time_steps(bm, steps, warmup, stream, record=False)
+    st = dsa.device_status(stream)
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st} after the dense map")
+    pairs = float(w.B * w.heads) * w.n_tokens * w.n_tokens
+    return {"fwd_ms": f_ms, "fwd_tflops": 4.0 * pairs * w.d / (f_ms * 1e-3) / 1e12,
+            "map_ms": m_ms, "map_tflops": 2.0 * pairs * w.d / (m_ms * 1e-3) / 1e12}
+
+
 def run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream):
     """Same forward through the host-buffer entry point: H2D of q, k, v, offsets from pinned
     memory, planner + forward, D2H of out and lse, all inside the timed region."""
@@ -414,6 +446,13 @@ def main():
                                if k2.endswith("_ms") or k2.endswith("_tflops")}
             except Exception as e:  # report, do not hide: the line carries the error
                 extra[name] = {"error": str(e)}
+        dense = WORKLOADS.get("bf16_16x32x32")
+        if dense is not None:
+            try:
+                r = run_dense_map_workload(dsa, dense, device, max(3, args.steps // 2), 3)
+                extra["bf16_16x32x32_dense_map"] = {k2: round(v2, 4) for k2, v2 in r.items()}
+            except Exception as e:
+                extra["bf16_16x32x32_dense_map"] = {"error": str(e)}
         if w.dtype == "bf16":
             name = f"{w.name}_lists{w.window_tiles}"
             try:

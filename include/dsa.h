@@ -168,6 +168,22 @@ dsa_status_t dsa_bwd_list(const dsa_problem_t* p, const void* q, const void* k, 
                           int32_t nnz, int32_t per_head, void* dq, void* dk, void* dv, void* workspace,
                           size_t ws_bytes, void* stream);
 
+/* Block attention mass (the sparsity map that block masks are chosen from; MOD-DiT page,
+ * Method section and project structure: attention fused with a sparsity map): for every
+ * (batch, head) h, query tile i and key tile j,
+ *   map[h][i][j] = (1 / tile tokens) * sum over the query tokens n of tile i and the
+ *                  tokens m of key tile j in i's list of exp(scale * q_n . k_m - lse_n),
+ * the mean attention probability tile i's queries put on tile j (each listed occurrence of
+ * j counts; j not listed: 0).  lse: the LSE dsa_fwd_list wrote for the same inputs and lists
+ * (then every non-empty row of the map sums to one); dense attention is the list of every
+ * tile.  Lists as dsa_fwd_list.  map: device fp32 [B * heads, nTiles, nTiles], overwritten.
+ * The scores are recomputed on the tensor cores; sums over a tile pair are accumulated in
+ * fp32 in an order that depends on timing (results may differ in the last bits between
+ * runs).  bf16, d = 128. */
+dsa_status_t dsa_block_map(const dsa_problem_t* p, const void* q, const void* k, const float* lse,
+                           const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, int32_t per_head, float* map,
+                           void* stream);
+
 /* Per-(batch, head) window offsets as per-head key-tile lists: head h = b * heads + j
  * plans its own offsets tile_offsets[h][i][3] (device int32 [B * heads, nTiles, 3], the
  * window rule of dsa_plan) into kv_list[(h * nTiles + i) * Wt ...] (device int32

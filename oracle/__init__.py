@@ -70,8 +70,10 @@ def _load():
                                            i32p, dp]
         lib.oracle_bwd_dkdv_list.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, fp, i32p, i32p, ctypes.c_int32,
                                              i32p, i32p, dp, dp]
+        lib.oracle_block_map_list.argtypes = [ctypes.POINTER(_Problem), fp, fp, i32p, i32p, ctypes.c_int32, i32p,
+                                              i32p, dp]
         for f in (lib.oracle_plan, lib.oracle_fwd, lib.oracle_bwd_dq, lib.oracle_bwd_dkdv, lib.oracle_fwd_list,
-                  lib.oracle_bwd_dq_list, lib.oracle_bwd_dkdv_list):
+                  lib.oracle_bwd_dq_list, lib.oracle_bwd_dkdv_list, lib.oracle_block_map_list):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -371,3 +373,31 @@ def backward_list(geo: Geometry, q, k, v, dout, row_ptr, kv_list):
     (dq,), _ = _run_by_head_lists(geo, (q, k, v, dout), row_ptr, kv_list, None, 1, call_dq)
     (dk, dv), _ = _run_by_head_lists(geo, (q, k, v, dout), row_ptr, kv_list, None, 2, call_dkdv)
     return _scatter(geo, dq), _scatter(geo, dk), _scatter(geo, dv)
+
+
+def block_map_list(geo: Geometry, q, k, row_ptr, kv_list, sel=None):
+    """Block attention mass over key-tile lists: map[bh, i, j] = mean over the query tokens
+    of tile i of the attention probability on the tokens of key tile j (dsa_oracle.c).
+    With sel=None: [B * heads, nTiles, nTiles]; with sel=(bh, tiles): [n_sel, nTiles]."""
+    lib = _load()
+    D = ctypes.c_double
+    I = ctypes.c_int32
+    bh, tiles = _selection(geo, sel)
+    res = np.zeros((len(bh), geo.n_tiles), np.float64)
+    one = Geometry(1, 1, geo.d, geo.grid, geo.tile, (1, 1, 1), geo.scale)
+    p = one.c_problem()
+    for h in np.unique(bh):
+        rows = np.nonzero(bh == h)[0]
+        rp, kl = _head_lists(geo, row_ptr, kv_list, int(h))
+        sq, sk = _head_slice(q, geo, int(h)), _head_slice(k, geo, int(h))
+        sel_t = np.ascontiguousarray(tiles[rows])
+        sel_b = np.zeros(len(rows), np.int32)
+        part = np.zeros((len(rows), geo.n_tiles), np.float64)
+        rc = lib.oracle_block_map_list(ctypes.byref(p), _ptr(sq, D), _ptr(sk, D), _ptr(rp, I), _ptr(kl, I),
+                                       len(rows), _ptr(sel_b, I), _ptr(sel_t, I), _ptr(part, D))
+        if rc:
+            raise RuntimeError(f"oracle block map failed ({rc})")
+        res[rows] = part
+    if sel is not None:
+        return res
+    return res.reshape(geo.B * geo.heads, geo.n_tiles, geo.n_tiles)

@@ -594,3 +594,52 @@ int oracle_bwd_dkdv_list(const oracle_problem* p, const double* q, const double*
     free(q_list);
     return status;
 }
+
+/* ---------------------------------------------------------------------------------- */
+/* Block attention mass (the sparsity map of a key-tile-list attention): for query tile i
+ * and key tile j, the mean over the query tokens n of tile i of the attention probability
+ * that n puts on the tokens of tile j,
+ *     map[i][j] = (1 / tile_tokens) * sum_{n in i} sum over the positions of j's tokens in
+ *                 K(i) of exp(s_nm - lse_n),
+ * with K(i), lse_n as in oracle_fwd_list (a tile listed twice counts twice; tiles not
+ * listed get 0; an empty list gives a zero row).  The rows of a non-empty list sum to one.
+ * Selected (bh, query tile) pairs; map: [n_sel][nTiles]. */
+int oracle_block_map_list(const oracle_problem* p, const double* q, const double* k, const int32_t* row_ptr,
+                          const int32_t* list, int32_t n_sel, const int32_t* sel_bh, const int32_t* sel_tile,
+                          double* map) {
+    geometry g;
+    if (make_geometry(p, &g) || check_lists(&g, row_ptr, list)) return 1;
+    const int64_t nk_max = longest_list(&g, row_ptr) * g.tile_tokens + 1;
+    const int64_t slice = (int64_t)g.n_tokens * p->d;
+    int status = 0;
+    memset(map, 0, sizeof(double) * n_sel * g.n_tiles);
+#pragma omp parallel
+    {
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * nk_max);
+        double* P = (double*)malloc(sizeof(double) * nk_max);
+        double* row = (double*)malloc(sizeof(double) * g.n_tiles);
+        if (!keys || !P || !row) {
+#pragma omp atomic write
+            status = 2;
+        }
+#pragma omp for schedule(dynamic)
+        for (int32_t s = 0; s < n_sel; ++s) {
+            if (!keys || !P || !row) continue;
+            const int32_t i = sel_tile[s];
+            const double* qb = q + sel_bh[s] * slice;
+            const double* kb = k + sel_bh[s] * slice;
+            int64_t nk = list_key_set(p, &g, row_ptr, list, i, keys);
+            for (int32_t j = 0; j < g.n_tiles; ++j) row[j] = 0.0;
+            for (int32_t r = 0; r < g.tile_tokens && nk > 0; ++r) {
+                int64_t n = tile_token(p, &g, i, r);
+                softmax_row(p, qb + n * p->d, kb, keys, nk, P);
+                for (int64_t m = 0; m < nk; ++m) row[list[row_ptr[i] + m / g.tile_tokens]] += P[m];
+            }
+            for (int32_t j = 0; j < g.n_tiles; ++j) map[(int64_t)s * g.n_tiles + j] = row[j] / g.tile_tokens;
+        }
+        free(keys);
+        free(P);
+        free(row);
+    }
+    return status;
+}

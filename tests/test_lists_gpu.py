@@ -214,3 +214,59 @@ def test_per_head_offsets_against_the_windowed_oracle():
         rq, rk, rv = oracle.backward(one, *sl, offs[h])
         for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
             assert_close(got[b, j].float().cpu().numpy(), ref[0, 0], "bf16", f"{name} head {h}")
+
+
+# ------------------------------------------------------------------------------------
+# block attention mass (sparsity map).  Tolerance: the map is a mean of probabilities
+# exp(s - lse) with s from bf16 products and lse from the bf16 forward (LSE gate 1e-3),
+# so entries carry a relative error near 1e-3: max-abs 3e-3 and row sums within 3e-3 of 1.
+MAP_MAX_ABS = 3e-3
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("per_head", [False, True], ids=["shared", "per_head"])
+def test_block_map_against_oracle(w, per_head):
+    inp = make_inputs(w)
+    geo = oracle.Geometry.of(w)
+    if per_head:
+        row_ptr, kv_list = per_head_lists(geo, w.B, w.heads, w.seed + 300, 6)
+    else:
+        row_ptr, kv_list = random_lists(geo.n_tiles, w.seed + 300, 6)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    rp, kl = torch.from_numpy(row_ptr).cuda(), torch.from_numpy(kv_list).cuda()
+    _, lse = dsa.forward_list(q, k, v, rp, kl, w.tile, w.scale)
+    bm = dsa.block_map(q, k, lse, rp, kl, w.tile, w.scale)
+    st, site, _ = dsa.device_status()
+    assert st == 0, f"device status {st} at site {site}"
+    ref = oracle.block_map_list(geo, inp.q, inp.k, row_ptr, kv_list)
+    got = bm.cpu().numpy()
+    err = np.abs(got - ref).max()
+    assert err <= MAP_MAX_ABS, f"block map max-abs {err:.2e}"
+    sums = got.sum(axis=-1)
+    ref_sums = ref.sum(axis=-1)
+    assert np.all(np.abs(sums[ref_sums > 0] - 1.0) <= MAP_MAX_ABS)
+    assert np.all(sums[ref_sums == 0] == 0.0)
+
+
+def test_dense_block_map_sampled():
+    """Dense attention (every tile listed for every query tile) on the 16x32x32 grid: the
+    block map of sampled query tiles against the oracle; every row sums to one."""
+    w = Workload("dense_map", 1, 4, 128, (16, 32, 32), (4, 8, 8), (1, 1, 1), (0, 0), "bf16", 46)
+    inp = make_inputs(w)
+    geo = oracle.Geometry.of(w)
+    n = geo.n_tiles
+    row_ptr = torch.arange(n + 1, dtype=torch.int32, device="cuda") * n
+    kv_list = torch.arange(n, dtype=torch.int32, device="cuda").repeat(n).contiguous()
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    _, lse = dsa.forward_list(q, k, v, row_ptr, kv_list, w.tile, w.scale)
+    bm = dsa.block_map(q, k, lse, row_ptr, kv_list, w.tile, w.scale)
+    assert dsa.device_status()[0] == 0
+    got = bm.cpu().numpy()
+    np.testing.assert_allclose(got.sum(axis=-1), 1.0, rtol=0, atol=MAP_MAX_ABS)
+    rng = np.random.default_rng(8)
+    bh = rng.integers(0, w.B * w.heads, 6).astype(np.int32)
+    tiles = rng.integers(0, n, 6).astype(np.int32)
+    ref = oracle.block_map_list(geo, inp.q, inp.k, row_ptr.cpu().numpy(), kv_list.cpu().numpy(), sel=(bh, tiles))
+    for s in range(len(bh)):
+        err = np.abs(got[bh[s], tiles[s]] - ref[s]).max()
+        assert err <= MAP_MAX_ABS, f"sample {s}: max-abs {err:.2e}"

@@ -511,3 +511,27 @@ def test_lists_per_head_equal_multiset_attention_per_head():
         (o * sl[3]).sum().backward()
         for got, ref in ((dq, qr.grad), (dk, kr.grad), (dv, vr.grad)):
             np.testing.assert_allclose(got[b, j], ref.numpy()[0, 0], rtol=0, atol=1e-11)
+
+
+def test_block_map_equals_blocked_dense_probabilities():
+    """The block attention mass is the dense softmax matrix summed over key tiles and
+    averaged over query tiles (weighted by list multiplicity); rows sum to one."""
+    geo = oracle.Geometry(1, 2, 16, (2, 4, 6), (1, 2, 2), (1, 1, 1))
+    q, k, _, _ = small_inputs(geo, 3)
+    row_ptr, kv_list = random_lists(geo, 3, 5)
+    bm = oracle.block_map_list(geo, q, k, row_ptr, kv_list)
+    tot = tile_of_token(geo)
+    cnt = torch.tensor(list_counts(geo, row_ptr, kv_list)[tot][:, tot], dtype=torch.float64)
+    BH = geo.B * geo.heads
+    s = torch.einsum("hnd,hmd->hnm", q.reshape(BH, -1, geo.d), k.reshape(BH, -1, geo.d)) * geo.scale
+    has = (cnt > 0).any(dim=-1)  # rows with at least one key
+    z = torch.where(cnt > 0, s + torch.log(cnt.clamp(min=1)), torch.full_like(s, -torch.inf))
+    z = torch.where(has[:, None], z, torch.zeros_like(z))  # a finite stand-in for empty rows
+    P = (torch.softmax(z, dim=-1) * has[:, None]).numpy()  # [BH, N, N], multiplicity-weighted
+    onehot_t = np.eye(geo.n_tiles)[tot]  # [N, nTiles]
+    ref = np.einsum("hnm,mj,ni->hij", P, onehot_t, onehot_t) / geo.tile_tokens
+    np.testing.assert_allclose(bm, ref, rtol=0, atol=1e-13)
+    sums = bm.sum(axis=-1)
+    empty = np.diff(row_ptr) == 0
+    np.testing.assert_allclose(sums[:, ~empty], 1.0, rtol=0, atol=1e-13)
+    assert np.all(sums[:, empty] == 0.0)

@@ -35,7 +35,7 @@ _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_size", "dsa_plan", "dsa_fwd",
            "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status", "dsa_fwd_noalloc",
-           "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads")
+           "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map")
 
 
 class DsaError(RuntimeError):
@@ -84,8 +84,9 @@ def load_library(path: Optional[str] = None):
     lib.dsa_fwd_list.argtypes = [pp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp]
     lib.dsa_bwd_list.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]
     lib.dsa_plan_heads.argtypes = [pp, vp, vp, vp, vp]
+    lib.dsa_block_map.argtypes = [pp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
     for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status",
-                 "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads"):
+                 "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -312,6 +313,27 @@ def backward_list(q, k, v, out, lse, dout, row_ptr, kv_list, tile, scale=None, d
                             _ptr(row_ptr), lst, nnz, per_head, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
                             ctypes.c_void_p(_stream(stream))), "dsa_bwd_list")
     return dq, dk, dv
+
+
+def block_map(q: torch.Tensor, k: torch.Tensor, lse: torch.Tensor, row_ptr: torch.Tensor, kv_list: torch.Tensor,
+              tile: Sequence[int], scale: Optional[float] = None, out: Optional[torch.Tensor] = None, stream=None):
+    """Block attention mass [B * heads, nTiles, nTiles] (fp32): mean attention probability
+    of each query tile's tokens on each key tile, against the LSE forward_list wrote for
+    the same lists."""
+    lib = load_library()
+    p = _problem_of(q, tile, (1, 1, 1), scale)
+    _need(q, "q", q)
+    _need(k, "k", q, q.dtype)
+    _need(lse, "lse", q, torch.float32)
+    n_tiles, _ = plan_shape(p)
+    lst, nnz, per_head = _list_args(q, row_ptr, kv_list, n_tiles)
+    BH = q.shape[0] * q.shape[1]
+    if out is None:
+        out = torch.empty((BH, n_tiles, n_tiles), dtype=torch.float32, device=q.device)
+    _need(out, "out", q, torch.float32)
+    _check(lib.dsa_block_map(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(lse), _ptr(row_ptr), lst, nnz, per_head,
+                             _ptr(out), ctypes.c_void_p(_stream(stream))), "dsa_block_map")
+    return out
 
 
 def plan_heads(problem: Problem, offsets: torch.Tensor, stream=None):

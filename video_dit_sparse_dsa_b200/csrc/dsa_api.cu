@@ -252,7 +252,8 @@ dsa_status_t launch_plan(const Geom& g, const int32_t* offsets, int32_t* starts,
 // with its CSR offsets row_ptr [n_tiles + 1] and nnz entries (bf16 only).
 dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
                         const int32_t* kv_tiles, void* out, float* lse, cudaStream_t s,
-                        const int32_t* row_ptr = nullptr, int nnz = 0, int rp_head_stride = 0) {
+                        const int32_t* row_ptr = nullptr, int nnz = 0, int rp_head_stride = 0,
+                        const float* lse_in = nullptr, float* bmap = nullptr) {
   if (p->dtype == DSA_F32) {
     dsa::FwdF32Params fp;
     fp.q = static_cast<const float*>(q);
@@ -289,6 +290,8 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.row_ptr = row_ptr;
   bp.rp_head_stride = rp_head_stride;
   bp.nnz = nnz;
+  bp.lse_in = lse_in;
+  bp.bmap = bmap;
   bp.out = static_cast<__nv_bfloat16*>(out);
   bp.lse = lse;
   bp.n_tiles = g.n_tiles;
@@ -306,17 +309,18 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.N = static_cast<int>(g.N);
   bp.scale_log2 = p->scale * 1.4426950408889634f;
   bp.n_units = static_cast<int>(g.BH * bp.S * g.n_tiles);
-  if (cudaFuncSetAttribute(dsa::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dsa::fwd::kSmemBytes) != cudaSuccess)
+  const bool map_mode = bmap != nullptr;
+  auto kernel = map_mode ? dsa::fwd_bf16_kernel<true> : dsa::fwd_bf16_kernel<false>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::fwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
   // the kernel's setmaxnreg split needs exactly the registers it was compiled for at launch
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, dsa::fwd_bf16_kernel) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
   if (fa.numRegs < dsa::fwd::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
   int sms = 0;
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
-  dsa::fwd_bf16_kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, bp);
+  kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, bp);
   return launch_status();
 }
 
@@ -590,6 +594,30 @@ dsa_status_t dsa_bwd_list(const dsa_problem_t* p, const void* q, const void* k, 
   if (st != DSA_OK) return st;
   return launch_bwd(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, ws.delta, ws.dq_acc, dq, dk, dv, s,
                     per_head ? g.n_tiles + 1 : 0);
+}
+
+dsa_status_t dsa_block_map(const dsa_problem_t* p, const void* q, const void* k, const float* lse,
+                           const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, int32_t per_head, float* map,
+                           void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !lse || !map) return DSA_ERR_INVALID_ARG;
+  int n_lists = 1;
+  st = check_lists(g, kv_row_ptr, kv_list, nnz, per_head, &n_lists);
+  if (st != DSA_OK) return st;
+  if (p->dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  st = check_kernel_limits(p, g, false);
+  if (st != DSA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(lse, 4) || !aligned(map, 4)) return DSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t map_bytes = sizeof(float) * static_cast<size_t>(g.BH) * g.n_tiles * g.n_tiles;
+  if (cudaMemsetAsync(map, 0, map_bytes, s) != cudaSuccess) return DSA_ERR_CUDA;
+  st = launch_list_check(g, kv_row_ptr, kv_list, n_lists, nnz, s);
+  if (st != DSA_OK) return st;
+  // map mode reads no V (its tensor map is given K's) and writes no O or LSE
+  return launch_fwd(p, g, q, k, k, kv_list, nullptr, nullptr, s, kv_row_ptr, nnz, per_head ? g.n_tiles + 1 : 0, lse,
+                    map);
 }
 
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {

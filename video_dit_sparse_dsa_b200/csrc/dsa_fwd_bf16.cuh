@@ -65,6 +65,10 @@ struct FwdBf16Params {
   int tt, th, tw, tcs;      // tile shape; t-extent of one 128-token chunk
   int T, H, W, N;
   float scale_log2;         // scale * log2(e)
+  // block-map mode only: the forward's LSE for the same lists and the map it adds into,
+  // [B*heads, n_tiles, n_tiles] (zeroed by the caller)
+  const float* lse_in;
+  float* bmap;
 };
 
 namespace fwd {
@@ -303,6 +307,11 @@ __device__ __forceinline__ void store_o(uint32_t tO, int groups, float inv, uint
 }
 }  // namespace fwd
 
+// kMap = false: the forward (O, LSE).  kMap = true: the block attention mass of the same
+// units against a given LSE, bmap[bh][query tile][key tile] += (1 / tile tokens) *
+// sum over the unit's rows and the key tile's keys of exp(scale q.k - lse) -- the scores are
+// recomputed with the same products and ring, without V, P.V, the row max or the epilogue.
+template <bool kMap>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, FwdBf16Params p) {
@@ -371,7 +380,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 
   if (warp >= kProducerWarp) {
     setmaxnreg_dec<kRegsAux>();
-    if (warp == kProducerWarp || warp == kVProducerWarp) {
+    if (warp == kProducerWarp || (warp == kVProducerWarp && !kMap)) {
       // ------------------------------------------------------------------ TMA producers
       if (lane == 0) {
         const bool is_k = warp == kProducerWarp;
@@ -462,6 +471,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             ++ks;
             if (t + 2 == n_steps) mma_commit_warp(q_empty);  // every score of this unit issued
           }
+          if constexpr (kMap) continue;  // scores only
           ok = warp_wait(p_full + e, ph, abort, 33);
           if (ok && t == 0) ok = warp_wait(o_free, (uc & 1) ^ 1, abort, 34);
           const int nb = 2 * t + 1 < n_chunks ? 2 : 1;
@@ -476,13 +486,70 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           mma_commit_warp(o_done);
         }
         if (!ok) break;
-        mma_commit_warp(o_final);
+        if constexpr (!kMap) mma_commit_warp(o_final);
         g += n_steps;
         ++uc;
       }
     }
   } else {
     setmaxnreg_inc<kRegsSoftmax>();
+    if constexpr (kMap) {
+      // ---------------------------------------------------------------- block attention mass
+      const int i = warp >> 2;
+      const int r = tid & 127;
+      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const float inv_rows = 1.f / static_cast<float>(p.S * 128);
+      int sc0 = 0, sc1 = 0, g = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit x = decode(p, u);
+        int n_list;
+        const int32_t* kv = unit_keys(p, x.bh, x.tile, n_list);
+        const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
+        if (n_chunks == 0) continue;
+        const int64_t tok = chunk_token(p, x.tile, x.sub, r);
+        const float neg_lse = -p.lse_in[static_cast<int64_t>(x.bh) * p.N + tok] * 1.4426950408889634f;
+        float* mrow = p.bmap + (static_cast<int64_t>(x.bh) * p.n_tiles + x.tile) * p.n_tiles;
+        for (int t = 0; t < n_steps && ok; ++t) {
+          const int e = (g + t) & 1;
+          ok = warp_wait(s_full + e, (e == 0 ? sc0++ : sc1++) & 1, abort, 49);
+          if (!ok) break;
+          tc_fence_after();
+          const bool full = 2 * t + 1 < n_chunks;
+          uint32_t sv[128];
+          float sum = 0.f;
+          if (full) {
+            tmem_ld128_wait(tmem + col_s(e) + 128 * i + lane_off, sv);
+          } else {
+            uint32_t (&half)[64] = *reinterpret_cast<uint32_t(*)[64]>(sv);
+            tmem_ld64_wait(tmem + col_s(e) + 64 * i + lane_off, half);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_read + e);  // the scores' columns may be overwritten
+          const int nc = full ? 128 : 64;
+          float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            if (c < nc) {
+              float x0, x1;
+              ffma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), p.scale_log2, p.scale_log2, neg_lse,
+                    neg_lse);
+              fadd2(sa[(c >> 1) & 3], sb[(c >> 1) & 3], sa[(c >> 1) & 3], sb[(c >> 1) & 3], ex2_approx(x0),
+                    ex2_approx(x1));
+            }
+          }
+          sum = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          // this thread's keys: chunk 2t + i of a full step, or half i of the single chunk 2t
+          const int c = full ? 2 * t + i : 2 * t;
+          const int kt = min(max(kv[c / p.S], 0), p.n_tiles - 1);
+          if (lane == 0) atomicAdd(mrow + kt, sum * inv_rows);
+        }
+        g += n_steps;
+      }
+    } else {
     // ------------------------------------------------------------------ softmax
     // Every barrier is waited on at most one phase behind its count of completions: the
     // score and P barriers alternate with the step parity and each of their phases needs
@@ -559,6 +626,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       }
       g += n_steps;
       ++uc;
+    }
     }
   }
 
