@@ -296,6 +296,31 @@ def run_dense_map_workload(dsa, w: Workload, device, steps: int, warmup: int):
             "map_ms": m_ms, "map_tflops": 2.0 * pairs * w.d / (m_ms * 1e-3) / 1e12}
 
 
+def run_lstsq_workload(dsa, device, steps: int, warmup: int, m: int = 300 * 300, p: int = 3, batch: int = 24):
+    """Pattern intensities of the 720p block maps: m = 300 x 300 map entries, p = 3 bases,
+    one map per head (batch 24); the factor is computed once, the solve is timed.  Bound:
+    HBM, reading S once (batch * m * 4 bytes) plus M (m * p * 4 bytes)."""
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    g = torch.Generator(device=device).manual_seed(123)
+    M = torch.rand((m, p), generator=g, device=device)
+    S = torch.rand((batch, m), generator=g, device=device)
+    L = dsa.lstsq_factor(M, 1e-3, stream=stream)
+    X = torch.empty((batch, p), dtype=torch.float32, device=device)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device=device)
+
+    def solve():
+        dsa.lstsq_solve(M, L, S, X=X, ws=ws, stream=stream)
+
+    solve()
+    ms = time_steps(solve, steps, warmup, stream, record=False)
+    st = dsa.device_status(stream)
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st} after the least-squares solve")
+    gb = (batch * m + m * p) * 4 / 1e9
+    return {"solve_ms": ms, "solve_gbs": gb / (ms * 1e-3)}
+
+
 def run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream):
     """Same forward through the host-buffer entry point: H2D of q, k, v, offsets from pinned
     memory, planner + forward, D2H of out and lse, all inside the timed region."""
@@ -446,6 +471,11 @@ def main():
                                if k2.endswith("_ms") or k2.endswith("_tflops")}
             except Exception as e:  # report, do not hide: the line carries the error
                 extra[name] = {"error": str(e)}
+        try:
+            r = run_lstsq_workload(dsa, device, max(10, args.steps), 5)
+            extra["lstsq_24x90000x3"] = {k2: round(v2, 4) for k2, v2 in r.items()}
+        except Exception as e:
+            extra["lstsq_24x90000x3"] = {"error": str(e)}
         dense = WORKLOADS.get("bf16_16x32x32")
         if dense is not None:
             try:

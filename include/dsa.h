@@ -193,6 +193,24 @@ dsa_status_t dsa_block_map(const dsa_problem_t* p, const void* q, const void* k,
 dsa_status_t dsa_plan_heads(const dsa_problem_t* p, const int32_t* tile_offsets, int32_t* kv_row_ptr, int32_t* kv_list,
                             void* stream);
 
+/* Regularised least squares with a cached factorisation (the MOD-DiT page, Method
+ * section, Stage 1 "Sparsity Map Reconstruction": pattern intensities X from
+ * (M^T M + lambda I) X = M^T S_t, where the design matrix M depends only on the sequence
+ * geometry, so its factorisation is computed once and reused across heads and steps).
+ * The page does not define the structural bases that make up M, so M is the caller's:
+ *   M: device fp32 [m, p] row-major (m observations, e.g. the entries of a block map;
+ *      p patterns, 1 <= p <= 32); lambda >= 0.
+ * dsa_lstsq_factor writes the Cholesky factor L of M^T M + lambda I (lower triangle, device
+ * fp64 [p, p], upper triangle zero); a matrix that is not positive definite is recorded as
+ * DSA_ERR_DEVICE (site 95).  dsa_lstsq_solve solves for a batch of right-hand sides
+ * S (device fp32 [batch, m], one map per row, batch <= 65535) into X (device fp32
+ * [batch, p]) with L from dsa_lstsq_factor; workspace: dsa_lstsq_workspace_size(m, p, batch)
+ * bytes, 256-byte aligned.  Sums and solves run in fp64 in a fixed order. */
+size_t dsa_lstsq_workspace_size(int32_t m, int32_t p, int32_t batch);
+dsa_status_t dsa_lstsq_factor(int32_t m, int32_t p, const float* M, float lambda, double* L, void* stream);
+dsa_status_t dsa_lstsq_solve(int32_t m, int32_t p, int32_t batch, const float* M, const double* L, const float* S,
+                             float* X, void* workspace, size_t ws_bytes, void* stream);
+
 /* Waits for `stream`, then reads and clears the device status word of the current device.
  * Returns DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE (or DSA_ERR_CUDA if the read failed);
  * site / block (either may be NULL) receive where the first failure was raised. */

@@ -401,3 +401,17 @@ def block_map_list(geo: Geometry, q, k, row_ptr, kv_list, sel=None):
     if sel is not None:
         return res
     return res.reshape(geo.B * geo.heads, geo.n_tiles, geo.n_tiles)
+
+
+# ------------------------------------------------------------------------------------------
+# Regularised least squares of the structural decomposition (the MOD-DiT page, Method
+# section, Stage 1 "Sparsity Map Reconstruction"): X with (M^T M + lam I) X = M^T S_t.
+
+
+def lstsq(M, lam: float, S) -> np.ndarray:
+    """X [batch, p] for every row s_b of S [batch, m]: the normal equations of the page,
+    solved in float64 (a library solve as the only step)."""
+    M = _f64(M)
+    S = _f64(S)
+    G = M.T @ M + float(lam) * np.eye(M.shape[1])
+    return np.linalg.solve(G, M.T @ S.T).T

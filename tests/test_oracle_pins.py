@@ -535,3 +535,27 @@ def test_block_map_equals_blocked_dense_probabilities():
     empty = np.diff(row_ptr) == 0
     np.testing.assert_allclose(sums[:, ~empty], 1.0, rtol=0, atol=1e-13)
     assert np.all(sums[:, empty] == 0.0)
+
+
+# ------------------------------------------------------------------------------------
+# regularised least squares: pinned to a different algorithm and to exact recovery
+
+def test_lstsq_equals_augmented_least_squares():
+    """(M^T M + lam I) x = M^T s is the minimiser of |M x - s|^2 + lam |x|^2, which numpy's
+    SVD-based lstsq finds from the augmented system [M; sqrt(lam) I] x = [s; 0]."""
+    rng = np.random.default_rng(0)
+    for m, p, lam in ((200, 3, 0.1), (500, 17, 1e-3), (50, 32, 2.0)):
+        M = rng.standard_normal((m, p))
+        S = rng.standard_normal((6, m))
+        X = oracle.lstsq(M, lam, S)
+        A = np.vstack([M, np.sqrt(lam) * np.eye(p)])
+        for b in range(S.shape[0]):
+            ref = np.linalg.lstsq(A, np.concatenate([S[b], np.zeros(p)]), rcond=None)[0]
+            np.testing.assert_allclose(X[b], ref, rtol=0, atol=1e-10)
+
+
+def test_lstsq_recovers_exact_intensities():
+    rng = np.random.default_rng(1)
+    M = rng.standard_normal((300, 3))
+    X0 = rng.standard_normal((4, 3))
+    np.testing.assert_allclose(oracle.lstsq(M, 0.0, X0 @ M.T), X0, rtol=0, atol=1e-12)

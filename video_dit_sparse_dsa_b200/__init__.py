@@ -35,7 +35,8 @@ _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_size", "dsa_plan", "dsa_fwd",
            "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status", "dsa_fwd_noalloc",
-           "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map")
+           "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map",
+           "dsa_lstsq_workspace_size", "dsa_lstsq_factor", "dsa_lstsq_solve")
 
 
 class DsaError(RuntimeError):
@@ -85,8 +86,13 @@ def load_library(path: Optional[str] = None):
     lib.dsa_bwd_list.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]
     lib.dsa_plan_heads.argtypes = [pp, vp, vp, vp, vp]
     lib.dsa_block_map.argtypes = [pp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+    lib.dsa_lstsq_workspace_size.restype = sz
+    lib.dsa_lstsq_workspace_size.argtypes = [i32, i32, i32]
+    lib.dsa_lstsq_factor.argtypes = [i32, i32, vp, ctypes.c_float, vp, vp]
+    lib.dsa_lstsq_solve.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]
     for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status",
-                 "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map"):
+                 "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map",
+                 "dsa_lstsq_factor", "dsa_lstsq_solve"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -334,6 +340,37 @@ def block_map(q: torch.Tensor, k: torch.Tensor, lse: torch.Tensor, row_ptr: torc
     _check(lib.dsa_block_map(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(lse), _ptr(row_ptr), lst, nnz, per_head,
                              _ptr(out), ctypes.c_void_p(_stream(stream))), "dsa_block_map")
     return out
+
+
+def lstsq_factor(M: torch.Tensor, lam: float, stream=None) -> torch.Tensor:
+    """Cholesky factor (fp64 [p, p], lower) of M^T M + lam I for a design matrix M (fp32
+    CUDA [m, p], p <= 32), to be reused by lstsq_solve across heads and steps."""
+    lib = load_library()
+    if not M.is_cuda or M.dtype != torch.float32 or not M.is_contiguous() or M.dim() != 2:
+        raise ValueError("M must be a contiguous fp32 CUDA tensor [m, p]")
+    m, p = M.shape
+    L = torch.empty((p, p), dtype=torch.float64, device=M.device)
+    _check(lib.dsa_lstsq_factor(m, p, _ptr(M), float(lam), _ptr(L), ctypes.c_void_p(_stream(stream))),
+           "dsa_lstsq_factor")
+    return L
+
+
+def lstsq_solve(M: torch.Tensor, L: torch.Tensor, S: torch.Tensor, X: Optional[torch.Tensor] = None, ws=None,
+                stream=None) -> torch.Tensor:
+    """X [batch, p] (fp32) with (M^T M + lam I) x_b = M^T s_b for every row s_b of S
+    [batch, m] (fp32 CUDA), L from lstsq_factor."""
+    lib = load_library()
+    m, p = M.shape
+    if not S.is_cuda or S.dtype != torch.float32 or not S.is_contiguous() or S.dim() != 2 or S.shape[1] != m:
+        raise ValueError("S must be a contiguous fp32 CUDA tensor [batch, m]")
+    batch = S.shape[0]
+    if X is None:
+        X = torch.empty((batch, p), dtype=torch.float32, device=S.device)
+    if ws is None:
+        ws = torch.empty(max(int(lib.dsa_lstsq_workspace_size(m, p, batch)), 256), dtype=torch.uint8, device=S.device)
+    _check(lib.dsa_lstsq_solve(m, p, batch, _ptr(M), _ptr(L), _ptr(S), _ptr(X), _ptr(ws), ws.numel(),
+                               ctypes.c_void_p(_stream(stream))), "dsa_lstsq_solve")
+    return X
 
 
 def plan_heads(problem: Problem, offsets: torch.Tensor, stream=None):

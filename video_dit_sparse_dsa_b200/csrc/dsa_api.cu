@@ -14,6 +14,7 @@
 #include "dsa_fwd_bf16.cuh"
 #include "dsa_fwd_f32.cuh"
 #include "dsa_lists.cuh"
+#include "dsa_lstsq.cuh"
 #include "dsa_plan.cuh"
 
 namespace {
@@ -618,6 +619,38 @@ dsa_status_t dsa_block_map(const dsa_problem_t* p, const void* q, const void* k,
   // map mode reads no V (its tensor map is given K's) and writes no O or LSE
   return launch_fwd(p, g, q, k, k, kv_list, nullptr, nullptr, s, kv_row_ptr, nnz, per_head ? g.n_tiles + 1 : 0, lse,
                     map);
+}
+
+size_t dsa_lstsq_workspace_size(int32_t m, int32_t p, int32_t batch) {
+  if (m <= 0 || p <= 0 || p > dsa::kLstsqMaxP || batch <= 0) return 0;
+  const int64_t slices = (m + dsa::kLstsqSliceRows - 1) / dsa::kLstsqSliceRows;
+  return round_up(sizeof(double) * static_cast<size_t>(batch) * slices * p, kAlign);
+}
+
+dsa_status_t dsa_lstsq_factor(int32_t m, int32_t p, const float* M, float lambda, double* L, void* stream) {
+  if (m <= 0 || p <= 0 || !M || !L || !(lambda >= 0.f) || !std::isfinite(lambda)) return DSA_ERR_INVALID_ARG;
+  if (p > dsa::kLstsqMaxP) return DSA_ERR_UNSUPPORTED;
+  if (!aligned(M, 4) || !aligned(L, 8)) return DSA_ERR_INVALID_ARG;
+  dsa::lstsq_factor_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(M, m, p, lambda, L);
+  return launch_status();
+}
+
+dsa_status_t dsa_lstsq_solve(int32_t m, int32_t p, int32_t batch, const float* M, const double* L, const float* S,
+                             float* X, void* workspace, size_t ws_bytes, void* stream) {
+  if (m <= 0 || p <= 0 || batch <= 0 || !M || !L || !S || !X) return DSA_ERR_INVALID_ARG;
+  if (p > dsa::kLstsqMaxP || batch > 65535) return DSA_ERR_UNSUPPORTED;
+  if (!aligned(M, 4) || !aligned(L, 8) || !aligned(S, 4) || !aligned(X, 4)) return DSA_ERR_INVALID_ARG;
+  const size_t need = dsa_lstsq_workspace_size(m, p, batch);
+  if (workspace == nullptr || ws_bytes < need || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int slices = (m + dsa::kLstsqSliceRows - 1) / dsa::kLstsqSliceRows;
+  double* part = static_cast<double*>(workspace);
+  dsa::lstsq_rhs_kernel<<<dim3(static_cast<unsigned>(slices), static_cast<unsigned>(batch)), 256, 0, s>>>(M, S, m, p,
+                                                                                                         part);
+  dsa_status_t st = launch_status();
+  if (st != DSA_OK) return st;
+  dsa::lstsq_solve_kernel<<<static_cast<unsigned>(batch), 32, 0, s>>>(L, part, slices, p, X);
+  return launch_status();
 }
 
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {
