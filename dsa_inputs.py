@@ -127,3 +127,27 @@ def make_inputs(w: Workload, with_dout: Optional[bool] = None, seed: Optional[in
         if dout is not None:
             dout = dout.to(torch.bfloat16)
     return Inputs(q, k, v, dout, offsets)
+
+
+@dataclasses.dataclass
+class TextInputs:
+    q: torch.Tensor  # [B, heads, L_text, d], CPU, same dtype as the video tokens
+    k: torch.Tensor
+    v: torch.Tensor
+
+
+def text_length(w: Workload) -> int:
+    """Text tokens beside a video grid: about 1% of the sequence (the MOD-DiT page,
+    "Token-Type-Aware Masking", puts text at roughly 1% of a unified text + video sequence)."""
+    return max(1, -(-w.n_tokens // 100))
+
+
+def make_text_inputs(w: Workload, L_text: int, seed: int) -> TextInputs:
+    """Seeded text-token q, k, v (N(0,1) fp32 draws in that order, rounded to bf16 for bf16
+    workloads), from their own generator so the video draws are unchanged."""
+    g = torch.Generator().manual_seed(seed)
+    shape = (w.B, w.heads, L_text, w.d)
+    q, k, v = (torch.randn(shape, generator=g, dtype=torch.float32) for _ in range(3))
+    if w.dtype == "bf16":
+        q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    return TextInputs(q, k, v)

@@ -72,8 +72,11 @@ def _load():
                                              i32p, i32p, dp, dp]
         lib.oracle_block_map_list.argtypes = [ctypes.POINTER(_Problem), fp, fp, i32p, i32p, ctypes.c_int32, i32p,
                                               i32p, dp]
+        lib.oracle_fwd_prefix.argtypes = [ctypes.POINTER(_Problem), fp, fp, fp, i32p, ctypes.c_int32, fp, fp,
+                                          ctypes.c_int32, i32p, i32p, dp, dp]
         for f in (lib.oracle_plan, lib.oracle_fwd, lib.oracle_bwd_dq, lib.oracle_bwd_dkdv, lib.oracle_fwd_list,
-                  lib.oracle_bwd_dq_list, lib.oracle_bwd_dkdv_list, lib.oracle_block_map_list):
+                  lib.oracle_bwd_dq_list, lib.oracle_bwd_dkdv_list, lib.oracle_block_map_list,
+                  lib.oracle_fwd_prefix):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -176,9 +179,10 @@ def _head_slice(t, geo: Geometry, bh: int) -> np.ndarray:
     return _f64(np.asarray(t).reshape(geo.B * geo.heads, geo.n_tokens, geo.d)[bh])
 
 
-def _run_by_head(geo: Geometry, tensors, offsets, sel, n_out, call):
+def _run_by_head(geo: Geometry, tensors, offsets, sel, n_out, call, extra=None):
     """Run ``call`` once per (b, head) present in the selection, on that head's slice
-    (heads are independent problems), so host memory holds one head in float64 at a time."""
+    (heads are independent problems), so host memory holds one head in float64 at a time.
+    ``extra(h)``, if given, returns more per-head arrays appended to the slices."""
     bh, tiles = _selection(geo, sel)
     off = _i32(offsets).reshape(geo.n_tiles, 3)
     outs = [np.zeros((len(bh), geo.tile_tokens, geo.d), np.float64) for _ in range(n_out)]
@@ -188,6 +192,8 @@ def _run_by_head(geo: Geometry, tensors, offsets, sel, n_out, call):
     for h in np.unique(bh):
         rows = np.nonzero(bh == h)[0]
         sl = [_head_slice(t, geo, int(h)) for t in tensors]
+        if extra is not None:
+            sl += list(extra(int(h)))
         sel_t = np.ascontiguousarray(tiles[rows])
         sel_b = np.zeros(len(rows), np.int32)
         part = [np.zeros((len(rows), geo.tile_tokens, geo.d), np.float64) for _ in range(n_out)]
@@ -219,6 +225,11 @@ def forward_tiles(geo: Geometry, q, k, v, offsets, sel=None):
 def forward(geo: Geometry, q, k, v, offsets):
     """Full forward: out[B, heads, T, H, W, d] and lse[B, heads, T, H, W] in float64."""
     out_t, lse_t = forward_tiles(geo, q, k, v, offsets)
+    return _scatter_forward(geo, out_t, lse_t)
+
+
+def _scatter_forward(geo: Geometry, out_t, lse_t):
+    """Per-tile rows ([BH * nTiles, tile_tokens, ...]) -> full tensors in token order."""
     tok = geo.tile_token_index()
     BH = geo.B * geo.heads
     out = np.zeros((BH, geo.n_tokens, geo.d), np.float64)
@@ -229,6 +240,64 @@ def forward(geo: Geometry, q, k, v, offsets):
     lse[:, tok.reshape(-1)] = lse_t.reshape(BH, -1)
     return (out.reshape((geo.B, geo.heads) + geo.grid + (geo.d,)),
             lse.reshape((geo.B, geo.heads) + geo.grid))
+
+
+def _text_slice(t, geo: Geometry, bh: int) -> np.ndarray:
+    """float64 copy of one (b, head) slice [L_text, d] of a [B, heads, L_text, d] tensor."""
+    a = t if isinstance(t, torch.Tensor) else torch.from_numpy(np.asarray(t))
+    return _f64(a.reshape(geo.B * geo.heads, -1, geo.d)[bh])
+
+
+def forward_prefix_tiles(geo: Geometry, q, k, v, offsets, k_text, v_text, sel=None):
+    """Text-prefix forward of video query tokens on (bh, query tile) pairs: each attends to
+    its window and to every text token (one softmax over the union).  Returns
+    out[n_sel, tile_tokens, d] and lse[n_sel, tile_tokens] (float64)."""
+    lib = _load()
+    D = ctypes.c_double
+    L_text = int(k_text.shape[2])
+
+    def call(p, sl, off, n, sb, st, part, part_lse):
+        return lib.oracle_fwd_prefix(ctypes.byref(p), _ptr(sl[0], D), _ptr(sl[1], D), _ptr(sl[2], D),
+                                     _ptr(off, ctypes.c_int32), L_text, _ptr(sl[3], D), _ptr(sl[4], D), n,
+                                     _ptr(sb, ctypes.c_int32), _ptr(st, ctypes.c_int32), _ptr(part[0], D),
+                                     _ptr(part_lse, D))
+
+    def text_of(h):
+        return _text_slice(k_text, geo, h), _text_slice(v_text, geo, h)
+
+    (out,), lse = _run_by_head(geo, (q, k, v), offsets, sel, 1, call, extra=text_of)
+    return out, lse
+
+
+def forward_prefix_text(geo: Geometry, q_text, k_text, v_text, k, v, rows=None):
+    """Text-prefix forward of text query tokens: each attends to every text token and every
+    video token (plain dense softmax attention over the concatenated key set, per (b, head)).
+    rows: optional text token indices to compute.  Returns out[B, heads, n_rows, d] and
+    lse[B, heads, n_rows] (float64)."""
+    BH = geo.B * geo.heads
+    L_text = int(q_text.shape[2])
+    idx = np.arange(L_text) if rows is None else np.asarray(rows)
+    out = np.zeros((BH, len(idx), geo.d), np.float64)
+    lse = np.zeros((BH, len(idx)), np.float64)
+    for h in range(BH):
+        qh = _text_slice(q_text, geo, h)[idx]
+        keys = np.concatenate([_text_slice(k_text, geo, h), _head_slice(k, geo, h)], axis=0)
+        vals = np.concatenate([_text_slice(v_text, geo, h), _head_slice(v, geo, h)], axis=0)
+        s = geo.scale * (qh @ keys.T)
+        mx = s.max(axis=1, keepdims=True)
+        l = mx[:, 0] + np.log(np.exp(s - mx).sum(axis=1))
+        out[h] = np.exp(s - l[:, None]) @ vals
+        lse[h] = l
+    return (out.reshape(geo.B, geo.heads, len(idx), geo.d), lse.reshape(geo.B, geo.heads, len(idx)))
+
+
+def forward_prefix(geo: Geometry, q, k, v, offsets, q_text, k_text, v_text):
+    """Full text-prefix forward: (out, lse) of the video tokens as in ``forward`` and
+    (out_text, lse_text) of the text tokens, float64."""
+    out_t, lse_t = forward_prefix_tiles(geo, q, k, v, offsets, k_text, v_text)
+    out, lse = _scatter_forward(geo, out_t, lse_t)
+    out_x, lse_x = forward_prefix_text(geo, q_text, k_text, v_text, k, v)
+    return out, lse, out_x, lse_x
 
 
 def backward_dq_tiles(geo: Geometry, q, k, v, dout, offsets, sel=None):

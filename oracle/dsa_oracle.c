@@ -643,3 +643,65 @@ int oracle_block_map_list(const oracle_problem* p, const double* q, const double
     }
     return status;
 }
+
+/* ---------------------------------------------------------------------------------- */
+
+/* Text prefix, video queries (the MOD-DiT page, "Token-Type-Aware Masking": text tokens
+ * take part in full attention, only video-video attention is sparse).  Video query token
+ * n of tile i attends to K(i) (its window, as oracle_fwd) and to every one of the L_text
+ * text tokens, one softmax over the union:
+ *     s_nm = scale <q_n, k_m> (m in K(i)),  s_nj = scale <q_n, k_text_j>,
+ *     lse_n = ln (sum_m exp s_nm + sum_j exp s_nj),
+ *     o_n = sum_m exp(s_nm - lse_n) v_m + sum_j exp(s_nj - lse_n) v_text_j.
+ * k_text, v_text: [B*heads][L_text][d].  Selection and outputs as oracle_fwd. */
+int oracle_fwd_prefix(const oracle_problem* p, const double* q, const double* k, const double* v,
+                      const int32_t* offsets, int32_t L_text, const double* k_text, const double* v_text,
+                      int32_t n_sel, const int32_t* sel_bh, const int32_t* sel_tile, double* out, double* lse) {
+    geometry g;
+    if (make_geometry(p, &g) || L_text < 0) return 1;
+    const int64_t nw = (int64_t)g.n_window_tiles * g.tile_tokens;
+    const int64_t slice = (int64_t)g.n_tokens * p->d, tslice = (int64_t)L_text * p->d;
+    int status = 0;
+#pragma omp parallel
+    {
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * nw);
+        double* P = (double*)malloc(sizeof(double) * (nw + L_text));
+        if (!keys || !P) {
+#pragma omp atomic write
+            status = 2;
+        }
+#pragma omp for schedule(dynamic)
+        for (int64_t job = 0; job < (int64_t)n_sel * g.tile_tokens; ++job) {
+            if (!keys || !P) continue;
+            int32_t s = (int32_t)(job / g.tile_tokens), r = (int32_t)(job % g.tile_tokens);
+            const double* qb = q + sel_bh[s] * slice;
+            const double* kb = k + sel_bh[s] * slice;
+            const double* vb = v + sel_bh[s] * slice;
+            const double* ktb = k_text + sel_bh[s] * tslice;
+            const double* vtb = v_text + sel_bh[s] * tslice;
+            key_set(p, &g, offsets, sel_tile[s], keys);
+            const double* qn = qb + tile_token(p, &g, sel_tile[s], r) * p->d;
+            /* scores over the union: window keys first, then the text keys */
+            double mx = -INFINITY;
+            for (int64_t m = 0; m < nw + L_text; ++m) {
+                const double* km = m < nw ? kb + keys[m] * p->d : ktb + (m - nw) * p->d;
+                P[m] = p->scale * dot(qn, km, p->d);
+                if (P[m] > mx) mx = P[m];
+            }
+            double sum = 0.0;
+            for (int64_t m = 0; m < nw + L_text; ++m) sum += exp(P[m] - mx);
+            const double l = mx + log(sum);
+            double* o = out + ((int64_t)s * g.tile_tokens + r) * p->d;
+            for (int32_t c = 0; c < p->d; ++c) o[c] = 0.0;
+            for (int64_t m = 0; m < nw + L_text; ++m) {
+                const double w = exp(P[m] - l);
+                const double* vm = m < nw ? vb + keys[m] * p->d : vtb + (m - nw) * p->d;
+                for (int32_t c = 0; c < p->d; ++c) o[c] += w * vm[c];
+            }
+            lse[(int64_t)s * g.tile_tokens + r] = l;
+        }
+        free(keys);
+        free(P);
+    }
+    return status;
+}

@@ -559,3 +559,70 @@ def test_lstsq_recovers_exact_intensities():
     M = rng.standard_normal((300, 3))
     X0 = rng.standard_normal((4, 3))
     np.testing.assert_allclose(oracle.lstsq(M, 0.0, X0 @ M.T), X0, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------
+# text prefix (the MOD-DiT page, "Token-Type-Aware Masking": in a unified text + video
+# sequence, text tokens keep full attention and only video-video attention is sparse)
+
+def rand_text(geo, L, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return [torch.randn((geo.B, geo.heads, L, geo.d), generator=g, dtype=torch.float64) * scale for _ in range(3)]
+
+
+@pytest.mark.parametrize("window,L,lo,hi", [((2, 1, 3), 5, -2, 2), ((1, 2, 2), 1, -1, 1), ((3, 3, 3), 9, 0, 0)])
+def test_prefix_equals_masked_dense_over_unified_sequence(window, L, lo, hi):
+    """Unified sequence [video; text] under the mask: video -> window (brute force) and
+    every text token; text -> everything.  Dense attention over it = the prefix oracle."""
+    geo = oracle.Geometry(1, 2, 8, (3, 4, 6), (1, 2, 2), window)
+    q, k, v, _ = rand_inputs(geo, 31)
+    qt, kt, vt = rand_text(geo, L, 32)
+    off = rand_offsets(geo, lo, hi, 33)
+    out, lse, out_x, lse_x = oracle.forward_prefix(geo, q, k, v, off, qt, kt, vt)
+    N = geo.n_tokens
+    mask = np.ones((N + L, N + L), bool)
+    mask[:N, :N] = brute_mask(geo.grid, geo.tile, geo.window, off.numpy())
+    BH = geo.B * geo.heads
+    cat = [np.concatenate([flat(a, geo), np.asarray(b).reshape(BH, L, geo.d)], axis=1) for a, b in
+           ((q, qt), (k, kt), (v, vt))]
+    ref, ref_lse = dense_attention_np(*cat, geo.scale, mask)
+    np.testing.assert_allclose(flat(out, geo), ref[:, :N], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(BH, N), ref_lse[:, :N], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out_x.reshape(BH, L, geo.d), ref[:, N:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse_x.reshape(BH, L), ref_lse[:, N:], rtol=0, atol=1e-12)
+    sdpa = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(c) for c in cat),
+                                                            attn_mask=torch.from_numpy(mask), scale=geo.scale)
+    np.testing.assert_allclose(flat(out, geo), sdpa.numpy()[:, :N], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out_x.reshape(BH, L, geo.d), sdpa.numpy()[:, N:], rtol=0, atol=1e-12)
+
+
+def test_prefix_without_text_is_the_window_forward():
+    geo = oracle.Geometry(1, 2, 8, (3, 4, 6), (1, 2, 2), (2, 2, 2))
+    q, k, v, _ = rand_inputs(geo, 34)
+    qt, kt, vt = rand_text(geo, 0, 35)
+    off = rand_offsets(geo, -2, 2, 36)
+    out, lse, out_x, lse_x = oracle.forward_prefix(geo, q, k, v, off, qt, kt, vt)
+    ref, ref_lse = oracle.forward(geo, q, k, v, off)
+    np.testing.assert_array_equal(out, ref)
+    np.testing.assert_array_equal(lse, ref_lse)
+    assert out_x.size == 0 and lse_x.size == 0
+
+
+def test_prefix_text_copy_of_video_closed_form():
+    """Text = a copy of every video token and a window covering the grid: every key appears
+    twice, so every output equals dense video attention and every LSE gains ln 2."""
+    geo = oracle.Geometry(1, 2, 8, (2, 4, 4), (1, 2, 2), (2, 2, 2))
+    q, k, v, _ = rand_inputs(geo, 37, scale=2.0)
+    off = torch.zeros((geo.n_tiles, 3), dtype=torch.int32)
+    BH, N = geo.B * geo.heads, geo.n_tokens
+    as_text = [torch.from_numpy(flat(a, geo)).reshape(geo.B, geo.heads, N, geo.d) for a in (q, k, v)]
+    out, lse, out_x, lse_x = oracle.forward_prefix(geo, q, k, v, off, *as_text)
+    dense = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(flat(q, geo)), torch.from_numpy(flat(k, geo)), torch.from_numpy(flat(v, geo)),
+        scale=geo.scale).numpy()
+    s = np.einsum("bnc,bmc->bnm", flat(q, geo), flat(k, geo)) * geo.scale
+    dense_lse = np.log(np.exp(s).sum(-1))
+    np.testing.assert_allclose(flat(out, geo), dense, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out_x.reshape(BH, N, geo.d), dense, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(BH, N), dense_lse + np.log(2.0), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse_x.reshape(BH, N), dense_lse + np.log(2.0), rtol=0, atol=1e-12)
