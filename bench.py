@@ -32,7 +32,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from dsa_inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+from dsa_inputs import WORKLOADS, Workload, make_inputs, make_text_inputs, text_length  # noqa: E402
 
 METRIC = "3D-DSA fwd/bwd effective TFLOP/s and % of B200 dense BF16 peak"
 NOMINAL_BF16_TFLOPS = 2250.0
@@ -264,6 +264,32 @@ def run_list_workload(dsa, w: Workload, device, steps: int, warmup: int, n_keep:
     return {"fwd_ms": ms, "fwd_tflops": flops / (ms * 1e-3) / 1e12, "keys_per_query": n_keep * w.tile_tokens}
 
 
+def run_prefix_workload(dsa, w: Workload, device, steps: int, warmup: int):
+    """Text prefix on the grid of w: about 1% of the sequence as text tokens, which attend to
+    and are attended by every token; the video-video part keeps its windows.  FLOPs:
+    4 * B * heads * d * (N * keys_per_query + 2 * N * L_text + L_text^2)."""
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    q, k, v, _, offsets = device_inputs(w, device)
+    L = text_length(w)
+    txt = make_text_inputs(w, L, seed=1000 + w.seed)
+    qt, kt, vt = (t.to(device) for t in (txt.q, txt.k, txt.v))
+    p = dsa._problem_of(q, w.tile, w.window, w.scale)
+    ws = torch.empty(dsa.prefix_workspace_size(p, L), dtype=torch.uint8, device=device)
+
+    def fwd():
+        dsa.forward_prefix(q, k, v, offsets, qt, kt, vt, w.tile, w.window, w.scale, ws=ws, stream=stream)
+
+    fwd()
+    ms = time_steps(fwd, steps, warmup, stream, record=False)
+    st = dsa.device_status(stream)
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st} after the text-prefix forward")
+    N = w.n_tokens
+    flops = 4.0 * w.B * w.heads * w.d * (N * w.keys_per_query + 2.0 * N * L + float(L) * L)
+    return {"fwd_ms": ms, "fwd_tflops": flops / (ms * 1e-3) / 1e12, "L_text": L}
+
+
 def run_dense_map_workload(dsa, w: Workload, device, steps: int, warmup: int):
     """Dense attention on the grid of w (every tile listed for every query tile) and its
     block attention mass: times the dense forward and the map pass separately.  The map
@@ -487,6 +513,12 @@ def main():
             name = f"{w.name}_lists{w.window_tiles}"
             try:
                 r = run_list_workload(dsa, w, device, max(3, args.steps // 2), 3, w.window_tiles)
+                extra[name] = {k2: (round(v2, 4) if isinstance(v2, float) else v2) for k2, v2 in r.items()}
+            except Exception as e:
+                extra[name] = {"error": str(e)}
+            name = f"{w.name}_text_prefix"
+            try:
+                r = run_prefix_workload(dsa, w, device, max(3, args.steps // 2), 3)
                 extra[name] = {k2: (round(v2, 4) if isinstance(v2, float) else v2) for k2, v2 in r.items()}
             except Exception as e:
                 extra[name] = {"error": str(e)}

@@ -168,6 +168,23 @@ dsa_status_t dsa_bwd_list(const dsa_problem_t* p, const void* q, const void* k, 
                           int32_t nnz, int32_t per_head, void* dq, void* dk, void* dv, void* workspace,
                           size_t ws_bytes, void* stream);
 
+/* Text prefix (token-type-aware attention; the MOD-DiT page, "Token-Type-Aware Masking":
+ * in unified text + video attention, text tokens get full attention and only video-video
+ * attention is sparse).  With L_text text tokens q_text, k_text, v_text (device bf16
+ * [B, heads, L_text, 128]) beside the video tokens q, k, v of p:
+ *   every video query attends to the keys of its window (tile_offsets, as dsa_fwd) and to
+ *   every text key;  every text query attends to every text key and every video key.
+ * Writes out, lse (video, as dsa_fwd) and out_text [B, heads, L_text, 128] bf16, lse_text
+ * [B, heads, L_text] fp32.  The parts are computed on the tensor cores separately (the
+ * window kernel, and dense attention between flat token sequences) and merged exactly by
+ * their LSEs.  L_text = 0 is dsa_fwd (the text pointers may then be NULL).  workspace: at
+ * least dsa_prefix_workspace_size(p, L_text) bytes, 256-byte aligned.  bf16, d = 128. */
+size_t dsa_prefix_workspace_size(const dsa_problem_t* p, int32_t L_text);
+dsa_status_t dsa_fwd_prefix(const dsa_problem_t* p, const void* q, const void* k, const void* v,
+                            const int32_t* tile_offsets, int32_t L_text, const void* q_text, const void* k_text,
+                            const void* v_text, void* out, float* lse, void* out_text, float* lse_text,
+                            void* workspace, size_t ws_bytes, void* stream);
+
 /* Block attention mass (the sparsity map that block masks are chosen from; MOD-DiT page,
  * Method section and project structure: attention fused with a sparsity map): for every
  * (batch, head) h, query tile i and key tile j,

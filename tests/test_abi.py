@@ -119,6 +119,21 @@ def test_list_entry_points_reject_bad_arguments(lib):
     assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, None, f, 4, 0, f, f, f, f, 1 << 30, None) == 1
     assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, f, f, 4, 0, f, f, f, f, 16, None) == 5
     assert lib.dsa_bwd_list(ctypes.byref(p), f, f, f, f, f, f, f, f, 4, 1, f, f, f, None, 1 << 30, None) == 5
+    # text prefix: (p, q, k, v, offsets, L_text, q_text, k_text, v_text, out, lse, out_text, lse_text, ws,
+    # ws_bytes, stream)
+    big = 1 << 40
+    assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, None, 4, f, f, f, f, f, f, f, f, big, None) == 1
+    assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, f, -1, f, f, f, f, f, f, f, f, big, None) == 1
+    assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, f, 4, None, f, f, f, f, f, f, f, big, None) == 1
+    assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, f, 4, f, f, f, f, f, None, f, f, big, None) == 1
+    assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, f, 4, f, ctypes.c_void_p((1 << 20) + 8), f, f, f, f, f,
+                              f, big, None) == 1
+    assert lib.dsa_fwd_prefix(ctypes.byref(p32), f, f, f, f, 4, f, f, f, f, f, f, f, f, big, None) == 2
+    assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, f, 4, f, f, f, f, f, f, f, f, 16, None) == 5
+    assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, f, 4, f, f, f, f, f, f, f, None, big, None) == 5
+    w0 = lib.dsa_prefix_workspace_size(ctypes.byref(p), 0)
+    assert 0 < w0 < lib.dsa_prefix_workspace_size(ctypes.byref(p), 1000)
+    assert lib.dsa_prefix_workspace_size(ctypes.byref(p), -1) == 0
     # per-head planner: (p, offsets, row_ptr, list, stream)
     assert lib.dsa_plan_heads(ctypes.byref(p), None, f, f, None) == 1
     assert lib.dsa_plan_heads(ctypes.byref(_prob(window=(0, 1, 1))), f, f, f, None) == 1

@@ -36,7 +36,8 @@ _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "
 EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_size", "dsa_plan", "dsa_fwd",
            "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status", "dsa_fwd_noalloc",
            "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map",
-           "dsa_lstsq_workspace_size", "dsa_lstsq_factor", "dsa_lstsq_solve")
+           "dsa_lstsq_workspace_size", "dsa_lstsq_factor", "dsa_lstsq_solve", "dsa_prefix_workspace_size",
+           "dsa_fwd_prefix")
 
 
 class DsaError(RuntimeError):
@@ -90,9 +91,12 @@ def load_library(path: Optional[str] = None):
     lib.dsa_lstsq_workspace_size.argtypes = [i32, i32, i32]
     lib.dsa_lstsq_factor.argtypes = [i32, i32, vp, ctypes.c_float, vp, vp]
     lib.dsa_lstsq_solve.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_prefix_workspace_size.restype = sz
+    lib.dsa_prefix_workspace_size.argtypes = [pp, i32]
+    lib.dsa_fwd_prefix.argtypes = [pp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status",
                  "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map",
-                 "dsa_lstsq_factor", "dsa_lstsq_solve"):
+                 "dsa_lstsq_factor", "dsa_lstsq_solve", "dsa_fwd_prefix"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -204,6 +208,43 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, offsets: torch.Te
     _check(lib.dsa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(offsets), _ptr(out), _ptr(lse), _ptr(ws),
                        ws.numel(), ctypes.c_void_p(_stream(stream))), "dsa_fwd")
     return out, lse
+
+
+def prefix_workspace_size(problem: Problem, L_text: int) -> int:
+    return int(load_library().dsa_prefix_workspace_size(ctypes.byref(problem), int(L_text)))
+
+
+def forward_prefix(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, q_text: torch.Tensor,
+                   k_text: torch.Tensor, v_text: torch.Tensor, tile: Sequence[int], window: Sequence[int],
+                   scale: Optional[float] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """3D-DSA with a text prefix: video queries over their windows and every text key, text
+    queries over every key.  q, k, v: [B, heads, T, H, W, 128]; q_text, k_text, v_text:
+    [B, heads, L_text, 128].  Returns (out, lse, out_text, lse_text)."""
+    lib = load_library()
+    p = _problem_of(q, tile, window, scale)
+    for t, name in ((k, "k"), (v, "v")):
+        _need(t, name, q, q.dtype)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
+    _need(q, "q", q)
+    _need(offsets, "offsets", q, torch.int32)
+    if q_text.dim() != 4 or tuple(q_text.shape[:2]) != tuple(q.shape[:2]) or q_text.shape[3] != q.shape[5]:
+        raise ValueError(f"q_text shape {tuple(q_text.shape)} does not match q {tuple(q.shape)}")
+    for t, name in ((q_text, "q_text"), (k_text, "k_text"), (v_text, "v_text")):
+        _need(t, name, q, q.dtype)
+        if t.shape != q_text.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != q_text shape {tuple(q_text.shape)}")
+    L_text = int(q_text.shape[2])
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:5], dtype=torch.float32, device=q.device)
+    out_text = torch.empty_like(q_text)
+    lse_text = torch.empty(q_text.shape[:3], dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = torch.empty(max(prefix_workspace_size(p, L_text), 256), dtype=torch.uint8, device=q.device)
+    _check(lib.dsa_fwd_prefix(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(offsets), L_text, _ptr(q_text),
+                              _ptr(k_text), _ptr(v_text), _ptr(out), _ptr(lse), _ptr(out_text), _ptr(lse_text),
+                              _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream))), "dsa_fwd_prefix")
+    return out, lse, out_text, lse_text
 
 
 def forward_host_bytes(problem: Problem) -> int:

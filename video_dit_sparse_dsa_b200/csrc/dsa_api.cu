@@ -231,6 +231,21 @@ bool make_row_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, con
   return r == CUDA_SUCCESS;
 }
 
+// A flat [BH, L, 128] bf16 token sequence seen as 3-D (128, L, BH); one box is 64 channels
+// of 128 consecutive tokens (rows past L load as zeros).
+bool make_flat_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t L) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(L) * 128 * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Validation of a caller's CSR on the device (records DSA_DEV_BOUNDS; never faults).
 dsa_status_t launch_list_check(const Geom& g, const int32_t* row_ptr, const int32_t* list, int n_lists, int nnz,
                                cudaStream_t s) {
@@ -311,7 +326,7 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.scale_log2 = p->scale * 1.4426950408889634f;
   bp.n_units = static_cast<int>(g.BH * bp.S * g.n_tiles);
   const bool map_mode = bmap != nullptr;
-  auto kernel = map_mode ? dsa::fwd_bf16_kernel<true> : dsa::fwd_bf16_kernel<false>;
+  auto kernel = map_mode ? dsa::fwd_bf16_kernel<dsa::fwd::kModeMap> : dsa::fwd_bf16_kernel<dsa::fwd::kModeFwd>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::fwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
   // the kernel's setmaxnreg split needs exactly the registers it was compiled for at launch
@@ -322,6 +337,43 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
   kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, bp);
+  return launch_status();
+}
+
+// Dense attention of Lq flat query rows over Lk flat key rows ([BH, L, 128] bf16), writing
+// out [BH, Lq, 128] bf16 and lse [BH, Lq] fp32.
+dsa_status_t launch_flat(const void* q, const void* k, const void* v, int64_t BH, int Lq, int Lk, float scale,
+                         void* out, float* lse, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  if (!make_flat_map(&tq, q, BH, Lq) || !make_flat_map(&tk, k, BH, Lk) || !make_flat_map(&tv, v, BH, Lk))
+    return DSA_ERR_CUDA;
+  dsa::FwdBf16Params bp;
+  std::memset(&bp, 0, sizeof(bp));
+  bp.out = static_cast<__nv_bfloat16*>(out);
+  bp.lse = lse;
+  bp.Lq = Lq;
+  bp.Lk = Lk;
+  bp.n_tiles = 1;
+  bp.S = 1;
+  bp.N = Lq;
+  bp.n_units = static_cast<int>(BH * ((Lq + 127) / 128));
+  bp.scale_log2 = scale * 1.4426950408889634f;
+  auto kernel = dsa::fwd_bf16_kernel<dsa::fwd::kModeFlat>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::fwd::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
+  if (fa.numRegs < dsa::fwd::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
+  kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, bp);
+  return launch_status();
+}
+
+dsa_status_t launch_merge(void* o, float* lse, const void* o2, const float* lse2, int64_t rows, cudaStream_t s) {
+  dsa::merge_kernel<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
+      static_cast<__nv_bfloat16*>(o), lse, static_cast<const __nv_bfloat16*>(o2), lse2, rows);
   return launch_status();
 }
 
@@ -651,6 +703,68 @@ dsa_status_t dsa_lstsq_solve(int32_t m, int32_t p, int32_t batch, const float* M
   if (st != DSA_OK) return st;
   dsa::lstsq_solve_kernel<<<static_cast<unsigned>(batch), 32, 0, s>>>(L, part, slices, p, X);
   return launch_status();
+}
+
+size_t dsa_prefix_workspace_size(const dsa_problem_t* p, int32_t L_text) {
+  Geom g;
+  if (check_shape(p, &g) != DSA_OK || L_text < 0) return 0;
+  size_t bytes = fwd_workspace(g, nullptr).bytes;
+  bytes += round_up(sizeof(__nv_bfloat16) * static_cast<size_t>(g.BH) * g.N * 128, kAlign);  // video x text O
+  bytes += round_up(sizeof(float) * static_cast<size_t>(g.BH) * g.N, kAlign);                 // and its LSE
+  bytes += round_up(sizeof(__nv_bfloat16) * static_cast<size_t>(g.BH) * (L_text > 0 ? L_text : 1) * 128, kAlign);
+  bytes += round_up(sizeof(float) * static_cast<size_t>(g.BH) * (L_text > 0 ? L_text : 1), kAlign);
+  return bytes;
+}
+
+dsa_status_t dsa_fwd_prefix(const dsa_problem_t* p, const void* q, const void* k, const void* v,
+                            const int32_t* tile_offsets, int32_t L_text, const void* q_text, const void* k_text,
+                            const void* v_text, void* out, float* lse, void* out_text, float* lse_text,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !tile_offsets || !out || !lse || L_text < 0) return DSA_ERR_INVALID_ARG;
+  if (L_text > 0 && (!q_text || !k_text || !v_text || !out_text || !lse_text)) return DSA_ERR_INVALID_ARG;
+  if (p->dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  st = check_kernel_limits(p, g, false);
+  if (st != DSA_OK) return st;
+  if (g.BH * ((g.N + 127) / 128) > INT32_MAX || g.BH * ((static_cast<int64_t>(L_text) + 127) / 128) > INT32_MAX)
+    return DSA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, out, q_text, k_text, v_text, out_text};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned(ptr, 16)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4) || (lse_text && !aligned(lse_text, 4)) || !aligned(tile_offsets, 4)) return DSA_ERR_INVALID_ARG;
+  const size_t need = dsa_prefix_workspace_size(p, L_text);
+  if (workspace == nullptr || ws_bytes < need || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
+  uint8_t* wb = static_cast<uint8_t*>(workspace);
+  FwdWorkspace fws = fwd_workspace(g, wb);
+  size_t off = fws.bytes;
+  void* o_vt = wb + off;
+  off += round_up(sizeof(__nv_bfloat16) * static_cast<size_t>(g.BH) * g.N * 128, kAlign);
+  float* l_vt = reinterpret_cast<float*>(wb + off);
+  off += round_up(sizeof(float) * static_cast<size_t>(g.BH) * g.N, kAlign);
+  void* o_tv = wb + off;
+  off += round_up(sizeof(__nv_bfloat16) * static_cast<size_t>(g.BH) * (L_text > 0 ? L_text : 1) * 128, kAlign);
+  float* l_tv = reinterpret_cast<float*>(wb + off);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // video queries over their windows
+  st = launch_plan(g, tile_offsets, fws.starts, fws.kv_tiles, nullptr, nullptr, s);
+  if (st != DSA_OK) return st;
+  st = launch_fwd(p, g, q, k, v, fws.kv_tiles, out, lse, s);
+  if (st != DSA_OK || L_text == 0) return st;
+  const int N = static_cast<int>(g.N);
+  // video queries over the text keys, merged into the window result by LSE
+  st = launch_flat(q, k_text, v_text, g.BH, N, L_text, p->scale, o_vt, l_vt, s);
+  if (st != DSA_OK) return st;
+  st = launch_merge(out, lse, o_vt, l_vt, g.BH * g.N, s);
+  if (st != DSA_OK) return st;
+  // text queries over the text keys and over every video key (the video tensor in raster
+  // order is a flat [BH, N, 128] sequence)
+  st = launch_flat(q_text, k_text, v_text, g.BH, L_text, L_text, p->scale, out_text, lse_text, s);
+  if (st != DSA_OK) return st;
+  st = launch_flat(q_text, k, v, g.BH, L_text, N, p->scale, o_tv, l_tv, s);
+  if (st != DSA_OK) return st;
+  return launch_merge(out_text, lse_text, o_tv, l_tv, g.BH * L_text, s);
 }
 
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {

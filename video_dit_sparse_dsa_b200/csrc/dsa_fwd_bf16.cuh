@@ -69,6 +69,9 @@ struct FwdBf16Params {
   // [B*heads, n_tiles, n_tiles] (zeroed by the caller)
   const float* lse_in;
   float* bmap;
+  // flat mode only: dense attention of Lq query rows over Lk key rows of flat
+  // [B*heads, L, 128] tensors (out, lse as [B*heads, Lq, 128] and [B*heads, Lq])
+  int Lq, Lk;
 };
 
 namespace fwd {
@@ -112,8 +115,12 @@ constexpr uint32_t kPolyMask = 0x88u;
 __device__ __forceinline__ uint32_t col_s(int e) { return e ? 128u : 0u; }
 __device__ __forceinline__ uint32_t col_p(int e) { return e ? 256u : 0u; }
 
+// Kernel modes: the window / key-tile-list forward, its block-map pass, and dense attention
+// between flat token sequences (text tokens).
+constexpr int kModeFwd = 0, kModeMap = 1, kModeFlat = 2;
+
 struct Unit {
-  int bh, tile, sub;
+  int bh, tile, sub;  // flat mode: tile = query chunk, sub = 0
 };
 
 // Key tiles of query tile `tile` and their count: the window's Wt tiles, or the tile's
@@ -128,6 +135,17 @@ __device__ __forceinline__ const int32_t* unit_keys(const FwdBf16Params& p, int 
   const int a = min(max(rp[tile], 0), p.nnz), b = min(max(rp[tile + 1], a), p.nnz);
   n_list = b - a;
   return p.kv_tiles + a;
+}
+
+// Flat mode: unit u is query chunk u % nq of (batch, head) u / nq, over all ceil(Lk / 128)
+// key chunks.
+__device__ __forceinline__ Unit decode_flat(const FwdBf16Params& p, int u) {
+  const int nq = (p.Lq + 127) / 128;
+  Unit x;
+  x.bh = u / nq;
+  x.tile = u % nq;
+  x.sub = 0;
+  return x;
 }
 
 __device__ __forceinline__ Unit decode(const FwdBf16Params& p, int u) {
@@ -194,7 +212,8 @@ __device__ __forceinline__ float pair_exchange(float* xbuf, int& xe, int i, int 
 // The softmax of one step for this thread's NC score columns at tS (NC = 128: a full step,
 // NC = 64: a half step): agrees on the row max with the partner thread, writes packed bf16
 // P (NC/2 columns) at tP, updates m_used and l, and returns whether the reference max
-// moved; it arrives on `loaded` as soon as its scores are in registers (alpha: the factor the old O and l take).  With !ok (an earlier wait failed; TMEM
+// moved; it arrives on `loaded` as soon as its scores are in registers.  Columns from
+// nvalid on hold no key (the tail of a flat key sequence) and get probability 0 (alpha: the factor the old O and l take).  With !ok (an earlier wait failed; TMEM
 // stays allocated, so the load is harmless) the thread still takes part in the exchange,
 // so its partner never waits for it, and does nothing else.  The load is unconditional: a
 // load under `ok` with the exchange between it and the use makes the compiler keep far
@@ -202,12 +221,17 @@ __device__ __forceinline__ float pair_exchange(float* xbuf, int& xe, int i, int 
 template <int NC>
 __device__ __forceinline__ bool softmax_step(bool ok, uint32_t tS, uint32_t tP, uint64_t* loaded, float scale_log2,
                                              float& m_used, float& l, float& alpha, float* xbuf, int& xe, int i,
-                                             int r, int bar_id) {
+                                             int r, int bar_id, int nvalid = NC) {
   uint32_t s[NC];
   if constexpr (NC == 128)
     tmem_ld128_wait(tS, s);
   else
     tmem_ld64_wait(tS, s);
+  if (nvalid < NC) {  // columns past the end of a flat key sequence: no key, score -inf
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+      if (c >= nvalid) s[c] = 0xff800000u;
+  }
   if (ok) {  // the scores are in registers: their TMEM columns may be overwritten
     tc_fence_before();
     __syncwarp();
@@ -288,8 +312,9 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, int groups, float alpha) 
   }
 }
 
-// Writes O row columns [0, 32 * groups) from tO, times inv, as bf16 to dst.
-__device__ __forceinline__ void store_o(uint32_t tO, int groups, float inv, uint4* dst) {
+// Writes O row columns [0, 32 * groups) from tO, times inv, as bf16 to dst (only where
+// `write`: the TMEM loads are warp-collective and run on every lane regardless).
+__device__ __forceinline__ void store_o(uint32_t tO, int groups, float inv, uint4* dst, bool write = true) {
 #pragma unroll 1
   for (int g = 0; g < groups; ++g) {
     uint32_t o[32];
@@ -301,21 +326,24 @@ __device__ __forceinline__ void store_o(uint32_t tO, int groups, float inv, uint
       v.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
       v.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
       v.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-      dst[4 * g + c] = v;
+      if (write) dst[4 * g + c] = v;
     }
   }
 }
 }  // namespace fwd
 
-// kMap = false: the forward (O, LSE).  kMap = true: the block attention mass of the same
+// kMode = kModeFwd: the forward (O, LSE).  kModeMap: the block attention mass of the same
 // units against a given LSE, bmap[bh][query tile][key tile] += (1 / tile tokens) *
 // sum over the unit's rows and the key tile's keys of exp(scale q.k - lse) -- the scores are
 // recomputed with the same products and ring, without V, P.V, the row max or the epilogue.
-template <bool kMap>
+// kModeFlat: dense attention between flat sequences (rank-3 tensor maps [128, L, B*heads]):
+// every query chunk over every key chunk, the tail of the last key chunk masked.
+template <int kMode>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, FwdBf16Params p) {
   using namespace fwd;
+  constexpr bool kMap = kMode == kModeMap, kFlat = kMode == kModeFlat;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
@@ -387,19 +415,24 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         int ld = 0, uc = 0;  // ring entries loaded, units with keys
         bool ok = true;
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-          const Unit x = decode(p, u);
-          int n_list;
-          const int32_t* kv = unit_keys(p, x.bh, x.tile, n_list);
-          const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
+          const Unit x = kFlat ? decode_flat(p, u) : decode(p, u);
+          int n_list = 0;
+          const int32_t* kv = kFlat ? nullptr : unit_keys(p, x.bh, x.tile, n_list);
+          const int n_chunks = kFlat ? (p.Lk + 127) / 128 : n_list * p.S, n_steps = (n_chunks + 1) / 2;
           if (n_chunks == 0) continue;  // nothing to load: the softmax warps write O = 0
           if (is_k) {
-            const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
             ok = mbar_wait(q_empty, (uc & 1) ^ 1, abort, 20);
             if (!ok) break;
             mbar_arrive_expect_tx(q_full, kTileBytes);
-            const int tq0 = qt * p.tt + x.sub * p.tcs;
-            tma_load_5d(smem + kOffQ, &tmQ, q_full, 0, qw * p.tw, qh * p.th, tq0, x.bh);
-            tma_load_5d(smem + kOffQ + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, tq0, x.bh);
+            if constexpr (kFlat) {
+              tma_load_3d(smem + kOffQ, &tmQ, q_full, 0, 128 * x.tile, x.bh);
+              tma_load_3d(smem + kOffQ + kHalfBytes, &tmQ, q_full, 64, 128 * x.tile, x.bh);
+            } else {
+              const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
+              const int tq0 = qt * p.tt + x.sub * p.tcs;
+              tma_load_5d(smem + kOffQ, &tmQ, q_full, 0, qw * p.tw, qh * p.th, tq0, x.bh);
+              tma_load_5d(smem + kOffQ + kHalfBytes, &tmQ, q_full, 64, qw * p.tw, qh * p.th, tq0, x.bh);
+            }
           }
           ++uc;
           // K: one stage per step, chunk b's channel half h at h * 32 KB + b * 16 KB;
@@ -415,6 +448,18 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             mbar_arrive_expect_tx(full, nb * kTileBytes);
             for (int b = 0; b < nb; ++b) {
               const int c = is_k ? 2 * j + b : j;
+              if constexpr (kFlat) {  // rows past Lk load as zeros (and are masked)
+                if (is_k) {
+                  uint8_t* dst = smem + kOffK + st * kStageBytes + b * kHalfBytes;
+                  tma_load_3d(dst, &tmK, full, 0, 128 * c, x.bh);
+                  tma_load_3d(dst + kTileBytes, &tmK, full, 64, 128 * c, x.bh);
+                } else {
+                  uint8_t* dst = smem + kOffV + st * kTileBytes;
+                  tma_load_3d(dst, &tmV, full, 0, 128 * c, x.bh);
+                  tma_load_3d(dst + kHalfBytes, &tmV, full, 64, 128 * c, x.bh);
+                }
+                continue;
+              }
               const int kt = min(max(kv[c / p.S], 0), p.n_tiles - 1), ks = c % p.S;
               const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
               const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
@@ -441,10 +486,12 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       int pc0 = 0, pc1 = 0;           // phases of p_full[0 / 1] and s_read[0 / 1] consumed
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        int n_list;
-        const Unit xm = decode(p, u);
-        unit_keys(p, xm.bh, xm.tile, n_list);
-        const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
+        int n_list = 0;
+        if constexpr (!kFlat) {
+          const Unit xm = decode(p, u);
+          unit_keys(p, xm.bh, xm.tile, n_list);
+        }
+        const int n_chunks = kFlat ? (p.Lk + 127) / 128 : n_list * p.S, n_steps = (n_chunks + 1) / 2;
         if (n_chunks == 0) continue;
         ok = warp_wait(q_full, uc & 1, abort, 30);
         if (ok) ok = warp_wait(k_full + ks % kKStages, (ks / kKStages) & 1, abort, 31);
@@ -568,18 +615,21 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     int xe = 0;            // pair exchanges so far
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-      const Unit x = decode(p, u);
-      int n_list;
-      unit_keys(p, x.bh, x.tile, n_list);
-      const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
+      const Unit x = kFlat ? decode_flat(p, u) : decode(p, u);
+      int n_list = 0;
+      if constexpr (!kFlat) unit_keys(p, x.bh, x.tile, n_list);
+      const int n_chunks = kFlat ? (p.Lk + 127) / 128 : n_list * p.S, n_steps = (n_chunks + 1) / 2;
       if (n_chunks == 0) {
         // no keys: O = 0 and LSE = ln 0 = -inf (the softmax of an empty set has no value;
         // this is the limit the oracle and the list form define)
-        const int64_t tok = chunk_token(p, x.tile, x.sub, r);
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * p.N + tok) * 128) + 8 * i;
+        const int64_t rows = kFlat ? p.Lq : p.N;
+        const int64_t tok = kFlat ? 128 * static_cast<int64_t>(x.tile) + r : chunk_token(p, x.tile, x.sub, r);
+        if (tok < rows) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * rows + tok) * 128) + 8 * i;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-        if (i == 0) p.lse[static_cast<int64_t>(x.bh) * p.N + tok] = -INFINITY;
+          for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+          if (i == 0) p.lse[static_cast<int64_t>(x.bh) * rows + tok] = -INFINITY;
+        }
         continue;
       }
       float m_used = -INFINITY, l = 0.f;
@@ -589,12 +639,19 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (ok) tc_fence_after();
         float alpha;
         bool need;
-        if (2 * t + 1 < n_chunks)
+        // flat mode: keys of this thread's columns that exist (the last chunk may be partial)
+        const bool full = 2 * t + 1 < n_chunks;
+        int nvalid = full ? 128 : 64;
+        if constexpr (kFlat) {
+          const int first = full ? 128 * (2 * t + i) : 256 * t + 64 * i;
+          nvalid = min(max(p.Lk - first, 0), nvalid);
+        }
+        if (full)
           need = softmax_step<128>(ok, tmem + col_s(e) + 128 * i + lane_off, tmem + col_p(e) + 64 * i + lane_off,
-                                   s_read + e, p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id);
+                                   s_read + e, p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id, nvalid);
         else
           need = softmax_step<64>(ok, tmem + col_s(e) + 64 * i + lane_off, tmem + col_p(e) + 32 * i + lane_off,
-                                  s_read + e, p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id);
+                                  s_read + e, p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id, nvalid);
         if (ok && t > 0 && __any_sync(0xffffffffu, need)) {
           // O holds sum P V up to step t-1 with the old reference max: rescale this
           // warpgroup's channels of it
@@ -616,10 +673,18 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const float l_all = l + pair_exchange(xbuf, xe, i, r, bar_id, l);
       if (ok) {
         tc_fence_after();
-        const int64_t tok = chunk_token(p, x.tile, x.sub, r);
+        // row of the output: the token of the tile (window / list form) or of the flat
+        // query sequence (rows past Lq of the last query chunk have no output)
+        const int64_t rows = kFlat ? p.Lq : p.N;
+        const int64_t tok = kFlat ? 128 * static_cast<int64_t>(x.tile) + r : chunk_token(p, x.tile, x.sub, r);
+        // (the TMEM loads of store_o are warp-collective: every lane takes part, and only
+        // rows that exist are written)
+        const bool row_ok = tok < rows;
         store_o(tO, 2, 1.f / l_all,
-                reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * p.N + tok) * 128) + 8 * i);
-        if (i == 0) p.lse[static_cast<int64_t>(x.bh) * p.N + tok] = (m_used + __log2f(l_all)) * 0.69314718055994531f;
+                reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * rows + (row_ok ? tok : 0)) * 128) +
+                    8 * i,
+                row_ok);
+        if (i == 0 && row_ok) p.lse[static_cast<int64_t>(x.bh) * rows + tok] = (m_used + __log2f(l_all)) * 0.69314718055994531f;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_free);
@@ -636,6 +701,38 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Merge of two attentions of the same queries over disjoint key sets: with
+// L = ln(e^lse + e^lse2),  o <- e^(lse - L) o + e^(lse2 - L) o2,  lse <- L  (exact: the
+// softmax over the union, written through the two partial normalisations).  A part with
+// lse = -inf (no keys) has weight 0.  16 threads per 128-channel row, 8 channels each.
+__global__ void __launch_bounds__(256) merge_kernel(__nv_bfloat16* o, float* lse, const __nv_bfloat16* o2,
+                                                    const float* lse2, int64_t rows) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 16;
+  const int part = threadIdx.x % 16;
+  if (row >= rows) return;
+  const float a = lse[row], b = lse2[row];
+  const float m = fmaxf(a, b);
+  float wa = 0.f, wb = 0.f, L = -INFINITY;
+  if (m != -INFINITY) {
+    const float ea = __expf(a - m), eb = __expf(b - m);
+    L = m + __logf(ea + eb);
+    wa = __expf(a - L);
+    wb = __expf(b - L);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(o + row * 128) + part;
+  const uint4 x = *dst, y = reinterpret_cast<const uint4*>(o2 + row * 128)[part];
+  const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+  uint32_t r[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float x0 = __uint_as_float(xs[e] << 16), x1 = __uint_as_float(xs[e] & 0xffff0000u);
+    const float y0 = __uint_as_float(ys[e] << 16), y1 = __uint_as_float(ys[e] & 0xffff0000u);
+    r[e] = pack_bf16x2(wa * x0 + wb * y0, wa * x1 + wb * y1);
+  }
+  *dst = make_uint4(r[0], r[1], r[2], r[3]);
+  if (part == 0) lse[row] = L;
 }
 
 }  // namespace dsa
