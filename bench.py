@@ -141,15 +141,84 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
-        rows = self.parse(self.lines)
-        inside = [r for r in rows if any(a <= r[0] <= b for a, b in windows)]
-        use = inside if inside else rows
-        power = [r[3] for r in use if r[3] is not None]
-        return {"sm_mhz": statistics.median(r[1] for r in use) if use else None,
-                "sm_max_mhz": max(r[2] for r in use) if use else None,
-                "power_w": statistics.median(power) if power else None,
-                "samples": len(use), "in_timed_region": bool(inside),
-                "reasons": sorted(set().union(*[r[4] for r in use])) if use else []}
+        return summarise_clocks(self.parse(self.lines), windows)
+
+
+def summarise_clocks(rows, windows):
+    """Median SM clock and power, max clock and the union of active reasons over the samples
+    (epoch seconds, sm MHz, max sm MHz, power W, reasons) inside the timed windows."""
+    inside = [r for r in rows if any(a <= r[0] <= b for a, b in windows)]
+    use = inside if inside else rows
+    power = [r[3] for r in use if r[3] is not None]
+    return {"sm_mhz": statistics.median(r[1] for r in use) if use else None,
+            "sm_max_mhz": max(r[2] for r in use) if use else None,
+            "power_w": statistics.median(power) if power else None,
+            "samples": len(use), "in_timed_region": bool(inside),
+            "reasons": sorted(set().union(*[r[4] for r in use])) if use else []}
+
+
+class NvmlSampler:
+    """Samples the SM clock, power and throttle reasons through NVML (read-only queries)
+    every 2 ms from a thread, so that even a timed region of a tenth of a second holds
+    dozens of samples; same stop() result as ClockSampler."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, nvml, handle, period_s: float = 0.002):
+        self.nvml, self.handle, self.period = nvml, handle, period_s
+        self.rows = []
+        self.stop_flag = threading.Event()
+        self.thread = None
+
+    @classmethod
+    def for_device(cls, device_index: int):
+        """The sampler of the CUDA device (matched by UUID, then PCI bus id), or None."""
+        try:
+            import pynvml as nvml
+
+            nvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            handle = None
+            try:
+                uuid = str(props.uuid)
+                handle = nvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                handle = nvml.nvmlDeviceGetHandleByPciBusId(bus)
+            return cls(nvml, handle)
+        except Exception:
+            return None
+
+    def _sample(self):
+        n = self.nvml
+        smax = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
+        while not self.stop_flag.is_set():
+            try:
+                t = time.time()
+                sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                pw = n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                reasons = {name for name, attr in self.REASONS if mask & getattr(n, attr, 0)}
+                self.rows.append((t, float(sm), float(smax), pw, reasons))
+            except Exception:
+                pass
+            self.stop_flag.wait(self.period)
+
+    def start(self):
+        self.thread = threading.Thread(target=self._sample, daemon=True)
+        self.thread.start()
+
+    def stop(self, windows):
+        self.stop_flag.set()
+        if self.thread:
+            self.thread.join(timeout=2)
+        out = summarise_clocks(list(self.rows), windows)
+        out["source"] = "nvml"
+        return out
 
 
 # host wall-clock intervals of the CUDA-event-timed loops of the headline workload
@@ -471,7 +540,9 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    sampler = ClockSampler(local) if rank == 0 else None
+    sampler = None
+    if rank == 0:
+        sampler = NvmlSampler.for_device(device.index if device.index is not None else 0) or ClockSampler(local)
     barrier()
     if sampler:
         sampler.start()

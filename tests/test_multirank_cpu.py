@@ -91,3 +91,37 @@ def test_traffic_is_reported_only_for_the_profiled_kernel_sources(monkeypatch):
     assert bench.fwd_traffic("w") == 123.0
     assert bench.fwd_traffic("stale") is None
     assert bench.fwd_traffic("unknown") is None
+
+
+def test_nvml_sampler_reads_reasons_from_a_fake_nvml():
+    """The NVML sampler decodes the clock-event bitmask and keeps only timed-region samples."""
+    import time as _time
+
+    class FakeNvml:
+        NVML_CLOCK_SM = 1
+        nvmlClocksEventReasonSwPowerCap = 0x4
+        nvmlClocksEventReasonHwSlowdown = 0x8
+        nvmlClocksEventReasonSwThermalSlowdown = 0x20
+        nvmlClocksEventReasonHwThermalSlowdown = 0x40
+        nvmlClocksEventReasonHwPowerBrakeSlowdown = 0x80
+
+        def nvmlDeviceGetMaxClockInfo(self, h, which):
+            return 1965
+
+        def nvmlDeviceGetClockInfo(self, h, which):
+            return 1500
+
+        def nvmlDeviceGetPowerUsage(self, h):
+            return 990_000
+
+        def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+            return 0x4 | 0x1  # power cap and idle (idle is not a slowdown reason)
+
+    s = bench.NvmlSampler(FakeNvml(), handle=None, period_s=0.001)
+    t0 = _time.time()
+    s.start()
+    _time.sleep(0.05)
+    got = s.stop([(t0, _time.time())])
+    assert got["samples"] > 5 and got["in_timed_region"]
+    assert got["sm_mhz"] == 1500 and got["sm_max_mhz"] == 1965 and got["power_w"] == 990.0
+    assert got["reasons"] == ["sw_power_cap"] and got["source"] == "nvml"
