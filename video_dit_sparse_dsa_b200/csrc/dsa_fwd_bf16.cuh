@@ -148,13 +148,16 @@ __device__ __forceinline__ Unit decode_flat(const FwdBf16Params& p, int u) {
   return x;
 }
 
+// Units run head-major, then tile, then the tile's 128-row chunks: the chunks of a tile
+// (same key set) are neighbouring units, so the persistent CTAs take them at the same time
+// and each key tile is read from DRAM about once per head.
 __device__ __forceinline__ Unit decode(const FwdBf16Params& p, int u) {
   Unit x;
   const int per_bh = p.S * p.n_tiles;
   x.bh = u / per_bh;
   const int rem = u % per_bh;
-  x.sub = rem / p.n_tiles;
-  x.tile = rem % p.n_tiles;
+  x.tile = rem / p.S;
+  x.sub = rem % p.S;
   return x;
 }
 
