@@ -106,9 +106,14 @@ dsa_status_t dsa_fwd(const dsa_problem_t* p, const void* q, const void* k, const
 
 /* Forward from and to HOST memory (pinned, for asynchronous copies): copies q, k, v and
  * tile_offsets into the caller's device buffer `dev`, runs dsa_fwd there, and copies out and
- * lse back, all on `stream`.  dev: at least dsa_fwd_host_bytes(p) bytes of device memory,
- * 256-byte aligned.  The host buffers must stay valid until the stream reaches the end of
- * the call. */
+ * lse back.  The work is pipelined over up to 8 groups of (batch, head) slices: copies in
+ * run on one internal stream, the forward of each group on `stream`, copies back on a
+ * second internal stream, ordered by events, so both copy directions overlap the kernels.
+ * Everything the call enqueues happens after the work already on `stream`, and `stream`
+ * reaches the end of the call only after the last copy back.  dev: at least
+ * dsa_fwd_host_bytes(p) bytes of device memory, 256-byte aligned.  The host buffers must
+ * stay valid until the stream reaches the end of the call (after an error return, until
+ * the device is idle). */
 size_t dsa_fwd_host_bytes(const dsa_problem_t* p);
 dsa_status_t dsa_fwd_host(const dsa_problem_t* p, const void* q_host, const void* k_host, const void* v_host,
                           const int32_t* tile_offsets_host, void* out_host, float* lse_host, void* dev,

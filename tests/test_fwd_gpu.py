@@ -164,8 +164,15 @@ def test_bf16_workload_sampled(name):
     compare_sampled(w, inp, out, lse)
 
 
-def test_forward_host_matches_device():
-    w = SMALL_BF16[0]
+HOST_CASES = [SMALL_BF16[0],
+              # ten (batch, head) slices: the host path pipelines them in five groups of two
+              Workload("bf16_host_10", 2, 5, 128, (8, 16, 16), (4, 8, 8), (3, 3, 3), (-2, 2), "bf16", 24)]
+
+
+@pytest.mark.parametrize("w", HOST_CASES, ids=lambda w: w.name)
+def test_forward_host_matches_device(w):
+    """The host-buffer entry point (copies pipelined over head groups on internal streams)
+    gives bit-for-bit the device entry point's results."""
     inp = make_inputs(w)
     out, lse = run_gpu(w, inp)
     p = dsa.make_problem(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale, dsa.DSA_BF16)

@@ -500,6 +500,43 @@ dsa_status_t dsa_fwd(const dsa_problem_t* p, const void* q, const void* k, const
   return launch_fwd(p, g, q, k, v, ws.kv_tiles, out, lse, s);
 }
 
+namespace {
+// Groups of (batch, head) slices the host-buffer forward pipelines over.
+constexpr int64_t kHostGroups = 8;
+
+// Internal streams and events of one host-buffer forward call, released when the call
+// returns (the runtime keeps destroyed streams and events alive until their work is done).
+struct HostPipeline {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t ev_in[kHostGroups] = {}, ev_fwd[kHostGroups] = {};
+  int n = 0;
+  bool init(int groups) {
+    n = groups;
+    if (cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&start, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&end, cudaEventDisableTiming) != cudaSuccess)
+      return false;
+    for (int i = 0; i < n; ++i)
+      if (cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&ev_fwd[i], cudaEventDisableTiming) != cudaSuccess)
+        return false;
+    return true;
+  }
+  ~HostPipeline() {
+    for (int i = 0; i < n; ++i) {
+      if (ev_in[i]) cudaEventDestroy(ev_in[i]);
+      if (ev_fwd[i]) cudaEventDestroy(ev_fwd[i]);
+    }
+    if (start) cudaEventDestroy(start);
+    if (end) cudaEventDestroy(end);
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+  }
+};
+}  // namespace
+
 size_t dsa_fwd_host_bytes(const dsa_problem_t* p) {
   Geom g;
   if (check_shape(p, &g) != DSA_OK) return 0;
@@ -531,15 +568,50 @@ dsa_status_t dsa_fwd_host(const dsa_problem_t* p, const void* q_host, const void
   int32_t* doff = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(dlse) + round_up(lse_bytes, kAlign));
   uint8_t* ws = reinterpret_cast<uint8_t*>(doff) + round_up(off_bytes, kAlign);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(dq, q_host, tok, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k_host, tok, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v_host, tok, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(doff, tile_offsets_host, off_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+  // Pipelined over groups of (batch, head) slices, which are independent problems: the
+  // host-to-device copies of group i + 1 run on one internal stream while the forward of
+  // group i runs on the caller's stream and the copy back of group i - 1 on another, so
+  // the two copy directions and the kernels overlap.  Events order each group's three
+  // stages; the caller's stream waits for the last copy back before the call's end.
+  const int64_t n_groups = g.BH < kHostGroups ? g.BH : kHostGroups;
+  const int64_t per = (g.BH + n_groups - 1) / n_groups;
+  const size_t head_tok = static_cast<size_t>(g.N) * p->d * elem, head_lse = sizeof(float) * g.N;
+  HostPipeline pl;
+  if (!pl.init(static_cast<int>(n_groups))) return DSA_ERR_CUDA;
+  if (cudaEventRecord(pl.start, s) != cudaSuccess || cudaStreamWaitEvent(pl.in, pl.start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(pl.out, pl.start, 0) != cudaSuccess)
     return DSA_ERR_CUDA;
-  st = dsa_fwd(p, dq, dk, dv, doff, dout, dlse, ws, fwd_workspace(g, nullptr).bytes, stream);
-  if (st != DSA_OK) return st;
-  if (cudaMemcpyAsync(out_host, dout, tok, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaMemcpyAsync(lse_host, dlse, lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+  if (cudaMemcpyAsync(doff, tile_offsets_host, off_bytes, cudaMemcpyHostToDevice, pl.in) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  for (int64_t gi = 0; gi < n_groups; ++gi) {
+    const int64_t h0 = gi * per, cnt = (h0 + per <= g.BH ? per : g.BH - h0);
+    if (cnt <= 0) break;
+    const size_t o_tok = static_cast<size_t>(h0) * head_tok, o_lse = static_cast<size_t>(h0) * head_lse;
+    const size_t n_tok = static_cast<size_t>(cnt) * head_tok, n_lse = static_cast<size_t>(cnt) * head_lse;
+    const uint8_t* qh = static_cast<const uint8_t*>(q_host) + o_tok;
+    const uint8_t* kh = static_cast<const uint8_t*>(k_host) + o_tok;
+    const uint8_t* vh = static_cast<const uint8_t*>(v_host) + o_tok;
+    uint8_t *qd = static_cast<uint8_t*>(dq) + o_tok, *kd = static_cast<uint8_t*>(dk) + o_tok,
+            *vd = static_cast<uint8_t*>(dv) + o_tok, *od = static_cast<uint8_t*>(dout) + o_tok;
+    float* ld = dlse + static_cast<size_t>(h0) * g.N;
+    if (cudaMemcpyAsync(qd, qh, n_tok, cudaMemcpyHostToDevice, pl.in) != cudaSuccess ||
+        cudaMemcpyAsync(kd, kh, n_tok, cudaMemcpyHostToDevice, pl.in) != cudaSuccess ||
+        cudaMemcpyAsync(vd, vh, n_tok, cudaMemcpyHostToDevice, pl.in) != cudaSuccess ||
+        cudaEventRecord(pl.ev_in[gi], pl.in) != cudaSuccess || cudaStreamWaitEvent(s, pl.ev_in[gi], 0) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    dsa_problem_t sub = *p;
+    sub.B = 1;
+    sub.heads = static_cast<int32_t>(cnt);
+    st = dsa_fwd(&sub, qd, kd, vd, doff, od, ld, ws, fwd_workspace(g, nullptr).bytes, stream);
+    if (st != DSA_OK) return st;
+    if (cudaEventRecord(pl.ev_fwd[gi], s) != cudaSuccess || cudaStreamWaitEvent(pl.out, pl.ev_fwd[gi], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(out_host) + o_tok, od, n_tok, cudaMemcpyDeviceToHost, pl.out) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(reinterpret_cast<uint8_t*>(lse_host) + o_lse, ld, n_lse, cudaMemcpyDeviceToHost, pl.out) !=
+            cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  if (cudaEventRecord(pl.end, pl.out) != cudaSuccess || cudaStreamWaitEvent(s, pl.end, 0) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;
 }
