@@ -269,7 +269,8 @@ dsa_status_t launch_plan(const Geom& g, const int32_t* offsets, int32_t* starts,
 dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
                         const int32_t* kv_tiles, void* out, float* lse, cudaStream_t s,
                         const int32_t* row_ptr = nullptr, int nnz = 0, int rp_head_stride = 0,
-                        const float* lse_in = nullptr, float* bmap = nullptr) {
+                        const float* lse_in = nullptr, float* bmap = nullptr, const void* kx = nullptr,
+                        const void* vx = nullptr, int Lx = 0) {
   if (p->dtype == DSA_F32) {
     dsa::FwdF32Params fp;
     fp.q = static_cast<const float*>(q);
@@ -298,10 +299,20 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
       dsa::fwd_f32_kernel<128><<<grid, dsa::kF32Threads, 0, s>>>(fp);
     return launch_status();
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tkx, tvx;
   if (!make_token_map(&tq, q, p, g, 128) || !make_token_map(&tk, k, p, g, 128) || !make_token_map(&tv, v, p, g, 128))
     return DSA_ERR_CUDA;
+  if (Lx > 0) {  // extra (text) keys after every query tile's own
+    if (bmap != nullptr || !make_flat_map(&tkx, kx, g.BH, Lx) || !make_flat_map(&tvx, vx, g.BH, Lx))
+      return DSA_ERR_CUDA;
+  } else {
+    tkx = tk;
+    tvx = tv;
+  }
   dsa::FwdBf16Params bp;
+  std::memset(&bp, 0, sizeof(bp));
+  bp.Lx = Lx > 0 ? Lx : 0;
+  bp.n_split = 1;
   bp.kv_tiles = kv_tiles;
   bp.row_ptr = row_ptr;
   bp.rp_head_stride = rp_head_stride;
@@ -336,27 +347,39 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   int sms = 0;
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
-  kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, bp);
+  kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, tkx, tvx, bp);
   return launch_status();
 }
 
-// Dense attention of Lq flat query rows over Lk flat key rows ([BH, L, 128] bf16), writing
-// out [BH, Lq, 128] bf16 and lse [BH, Lq] fp32.
-dsa_status_t launch_flat(const void* q, const void* k, const void* v, int64_t BH, int Lq, int Lk, float scale,
-                         void* out, float* lse, cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
+// Dense attention of Lq flat query rows over Lk flat key rows and Lx flat extra key rows
+// ([BH, L, 128] bf16 each), the main keys cut into n_split parts: part j writes
+// out + j * part_out ([BH, Lq, 128] bf16) and lse + j * part_lse ([BH, Lq] fp32).
+dsa_status_t launch_flat(const void* q, const void* k, const void* v, const void* kx, const void* vx, int64_t BH,
+                         int Lq, int Lk, int Lx, int n_split, float scale, void* out, float* lse, int64_t part_out,
+                         int64_t part_lse, cudaStream_t s) {
+  CUtensorMap tq, tk, tv, tkx, tvx;
   if (!make_flat_map(&tq, q, BH, Lq) || !make_flat_map(&tk, k, BH, Lk) || !make_flat_map(&tv, v, BH, Lk))
     return DSA_ERR_CUDA;
+  if (Lx > 0) {
+    if (!make_flat_map(&tkx, kx, BH, Lx) || !make_flat_map(&tvx, vx, BH, Lx)) return DSA_ERR_CUDA;
+  } else {
+    tkx = tk;
+    tvx = tv;
+  }
   dsa::FwdBf16Params bp;
   std::memset(&bp, 0, sizeof(bp));
   bp.out = static_cast<__nv_bfloat16*>(out);
   bp.lse = lse;
   bp.Lq = Lq;
   bp.Lk = Lk;
+  bp.Lx = Lx > 0 ? Lx : 0;
+  bp.n_split = n_split;
+  bp.part_out = part_out;
+  bp.part_lse = part_lse;
   bp.n_tiles = 1;
   bp.S = 1;
   bp.N = Lq;
-  bp.n_units = static_cast<int>(BH * ((Lq + 127) / 128));
+  bp.n_units = static_cast<int>(BH * ((Lq + 127) / 128) * n_split);
   bp.scale_log2 = scale * 1.4426950408889634f;
   auto kernel = dsa::fwd_bf16_kernel<dsa::fwd::kModeFlat>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::fwd::kSmemBytes) != cudaSuccess)
@@ -367,13 +390,15 @@ dsa_status_t launch_flat(const void* q, const void* k, const void* v, int64_t BH
   int sms = 0;
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
-  kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, bp);
+  kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, tkx, tvx, bp);
   return launch_status();
 }
 
-dsa_status_t launch_merge(void* o, float* lse, const void* o2, const float* lse2, int64_t rows, cudaStream_t s) {
-  dsa::merge_kernel<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
-      static_cast<__nv_bfloat16*>(o), lse, static_cast<const __nv_bfloat16*>(o2), lse2, rows);
+dsa_status_t launch_merge_parts(const void* o, const float* lse, int n_parts, int64_t part_out, int64_t part_lse,
+                                int64_t rows, void* out, float* lse_out, cudaStream_t s) {
+  dsa::merge_parts_kernel<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(o), lse, n_parts, part_out, part_lse, rows, static_cast<__nv_bfloat16*>(out),
+      lse_out);
   return launch_status();
 }
 
@@ -777,15 +802,49 @@ dsa_status_t dsa_lstsq_solve(int32_t m, int32_t p, int32_t batch, const float* M
   return launch_status();
 }
 
+namespace {
+// Parts the text queries' key sequence (every video token) is cut into: enough units for
+// about four waves of persistent CTAs, at most one part per 128-key chunk.
+int prefix_split(const Geom& g, int32_t L_text) {
+  const int64_t units = g.BH * ((static_cast<int64_t>(L_text) + 127) / 128);
+  const int64_t n_main = (g.N + 127) / 128;
+  int64_t n = (4 * 148 + units - 1) / (units > 0 ? units : 1);
+  if (n > n_main) n = n_main;
+  if (n > 16) n = 16;
+  return static_cast<int>(n < 1 ? 1 : n);
+}
+
+struct PrefixWorkspace {
+  int32_t* starts;
+  int32_t* kv_tiles;
+  void* o_parts;   // [n_split][BH, L_text, 128] bf16 (n_split > 1 only)
+  float* l_parts;  // [n_split][BH, L_text] fp32
+  int n_split;
+  size_t bytes;
+};
+
+PrefixWorkspace prefix_workspace(const Geom& g, int32_t L_text, void* base) {
+  PrefixWorkspace w;
+  FwdWorkspace f = fwd_workspace(g, base);
+  w.starts = f.starts;
+  w.kv_tiles = f.kv_tiles;
+  w.n_split = prefix_split(g, L_text);
+  size_t off = f.bytes;
+  const size_t rows = static_cast<size_t>(g.BH) * (L_text > 0 ? L_text : 0);
+  uint8_t* b = static_cast<uint8_t*>(base);
+  w.o_parts = b ? b + off : nullptr;
+  if (w.n_split > 1) off += round_up(sizeof(__nv_bfloat16) * rows * 128 * w.n_split, kAlign);
+  w.l_parts = b ? reinterpret_cast<float*>(b + off) : nullptr;
+  if (w.n_split > 1) off += round_up(sizeof(float) * rows * w.n_split, kAlign);
+  w.bytes = off;
+  return w;
+}
+}  // namespace
+
 size_t dsa_prefix_workspace_size(const dsa_problem_t* p, int32_t L_text) {
   Geom g;
   if (check_shape(p, &g) != DSA_OK || L_text < 0) return 0;
-  size_t bytes = fwd_workspace(g, nullptr).bytes;
-  bytes += round_up(sizeof(__nv_bfloat16) * static_cast<size_t>(g.BH) * g.N * 128, kAlign);  // video x text O
-  bytes += round_up(sizeof(float) * static_cast<size_t>(g.BH) * g.N, kAlign);                 // and its LSE
-  bytes += round_up(sizeof(__nv_bfloat16) * static_cast<size_t>(g.BH) * (L_text > 0 ? L_text : 1) * 128, kAlign);
-  bytes += round_up(sizeof(float) * static_cast<size_t>(g.BH) * (L_text > 0 ? L_text : 1), kAlign);
-  return bytes;
+  return prefix_workspace(g, L_text, nullptr).bytes;
 }
 
 dsa_status_t dsa_fwd_prefix(const dsa_problem_t* p, const void* q, const void* k, const void* v,
@@ -800,43 +859,31 @@ dsa_status_t dsa_fwd_prefix(const dsa_problem_t* p, const void* q, const void* k
   if (p->dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
   st = check_kernel_limits(p, g, false);
   if (st != DSA_OK) return st;
-  if (g.BH * ((g.N + 127) / 128) > INT32_MAX || g.BH * ((static_cast<int64_t>(L_text) + 127) / 128) > INT32_MAX)
-    return DSA_ERR_UNSUPPORTED;
+  if (g.BH * ((static_cast<int64_t>(L_text) + 127) / 128) * 16 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k, v, out, q_text, k_text, v_text, out_text};
   for (const void* ptr : ptrs)
     if (ptr && !aligned(ptr, 16)) return DSA_ERR_INVALID_ARG;
   if (!aligned(lse, 4) || (lse_text && !aligned(lse_text, 4)) || !aligned(tile_offsets, 4)) return DSA_ERR_INVALID_ARG;
-  const size_t need = dsa_prefix_workspace_size(p, L_text);
-  if (workspace == nullptr || ws_bytes < need || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
-  uint8_t* wb = static_cast<uint8_t*>(workspace);
-  FwdWorkspace fws = fwd_workspace(g, wb);
-  size_t off = fws.bytes;
-  void* o_vt = wb + off;
-  off += round_up(sizeof(__nv_bfloat16) * static_cast<size_t>(g.BH) * g.N * 128, kAlign);
-  float* l_vt = reinterpret_cast<float*>(wb + off);
-  off += round_up(sizeof(float) * static_cast<size_t>(g.BH) * g.N, kAlign);
-  void* o_tv = wb + off;
-  off += round_up(sizeof(__nv_bfloat16) * static_cast<size_t>(g.BH) * (L_text > 0 ? L_text : 1) * 128, kAlign);
-  float* l_tv = reinterpret_cast<float*>(wb + off);
+  if (workspace == nullptr || ws_bytes < prefix_workspace(g, L_text, nullptr).bytes || !aligned(workspace, kAlign))
+    return DSA_ERR_WORKSPACE;
+  const PrefixWorkspace ws = prefix_workspace(g, L_text, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // video queries over their windows
-  st = launch_plan(g, tile_offsets, fws.starts, fws.kv_tiles, nullptr, nullptr, s);
+  // video queries: their windows, then every text key, in one softmax
+  st = launch_plan(g, tile_offsets, ws.starts, ws.kv_tiles, nullptr, nullptr, s);
   if (st != DSA_OK) return st;
-  st = launch_fwd(p, g, q, k, v, fws.kv_tiles, out, lse, s);
+  st = launch_fwd(p, g, q, k, v, ws.kv_tiles, out, lse, s, nullptr, 0, 0, nullptr, nullptr, k_text, v_text, L_text);
   if (st != DSA_OK || L_text == 0) return st;
+  // text queries: every video key (the video tensor in raster order is a flat sequence of N
+  // rows), cut into parts for load balance, then every text key (with part 0)
   const int N = static_cast<int>(g.N);
-  // video queries over the text keys, merged into the window result by LSE
-  st = launch_flat(q, k_text, v_text, g.BH, N, L_text, p->scale, o_vt, l_vt, s);
+  const int64_t rows = g.BH * L_text;
+  if (ws.n_split == 1)
+    return launch_flat(q_text, k, v, k_text, v_text, g.BH, L_text, N, L_text, 1, p->scale, out_text, lse_text, 0, 0,
+                       s);
+  st = launch_flat(q_text, k, v, k_text, v_text, g.BH, L_text, N, L_text, ws.n_split, p->scale, ws.o_parts,
+                   ws.l_parts, rows * 128, rows, s);
   if (st != DSA_OK) return st;
-  st = launch_merge(out, lse, o_vt, l_vt, g.BH * g.N, s);
-  if (st != DSA_OK) return st;
-  // text queries over the text keys and over every video key (the video tensor in raster
-  // order is a flat [BH, N, 128] sequence)
-  st = launch_flat(q_text, k_text, v_text, g.BH, L_text, L_text, p->scale, out_text, lse_text, s);
-  if (st != DSA_OK) return st;
-  st = launch_flat(q_text, k, v, g.BH, L_text, N, p->scale, o_tv, l_tv, s);
-  if (st != DSA_OK) return st;
-  return launch_merge(out_text, lse_text, o_tv, l_tv, g.BH * L_text, s);
+  return launch_merge_parts(ws.o_parts, ws.l_parts, ws.n_split, rows * 128, rows, rows, out_text, lse_text, s);
 }
 
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {

@@ -72,6 +72,13 @@ struct FwdBf16Params {
   // flat mode only: dense attention of Lq query rows over Lk key rows of flat
   // [B*heads, L, 128] tensors (out, lse as [B*heads, Lq, 128] and [B*heads, Lq])
   int Lq, Lk;
+  // extra (text) keys appended to every unit's keys in the forward and flat modes: Lx rows
+  // of a flat [B*heads, Lx, 128] pair of tensors (0: none)
+  int Lx;
+  // flat mode only: the main key chunks are cut into n_split parts, one unit each; part j
+  // writes out + j * part_out and lse + j * part_lse (the extra keys go with part 0)
+  int n_split;
+  int64_t part_out, part_lse;
 };
 
 namespace fwd {
@@ -137,15 +144,47 @@ __device__ __forceinline__ const int32_t* unit_keys(const FwdBf16Params& p, int 
   return p.kv_tiles + a;
 }
 
-// Flat mode: unit u is query chunk u % nq of (batch, head) u / nq, over all ceil(Lk / 128)
-// key chunks.
+// Flat mode: units run (batch, head), then part of the key chunks, then query chunk, so
+// the query chunks that read the same keys are neighbours.
 __device__ __forceinline__ Unit decode_flat(const FwdBf16Params& p, int u) {
-  const int nq = (p.Lq + 127) / 128;
+  const int nq = (p.Lq + 127) / 128, per_bh = nq * p.n_split;
   Unit x;
-  x.bh = u / nq;
-  x.tile = u % nq;
-  x.sub = 0;
+  x.bh = u / per_bh;
+  const int rem = u % per_bh;
+  x.sub = rem / nq;  // part
+  x.tile = rem % nq;
   return x;
+}
+
+// Key chunks of a unit: nm main chunks from main chunk c0 (the tiles' 128-row chunks, or
+// rows of the flat key sequence), then nx chunks of the extra keys.
+struct Chunks {
+  int c0, nm, nx;
+};
+
+template <bool kFlat>
+__device__ __forceinline__ Chunks unit_chunks(const FwdBf16Params& p, const Unit& x, int n_list) {
+  Chunks k;
+  const int nx = (p.Lx + 127) / 128;
+  if constexpr (kFlat) {
+    const int n_main = (p.Lk + 127) / 128, per = (n_main + p.n_split - 1) / p.n_split;
+    k.c0 = x.sub * per;
+    k.nm = max(min(per, n_main - k.c0), 0);
+    k.nx = x.sub == 0 ? nx : 0;
+  } else {
+    k.c0 = 0;
+    k.nm = n_list * p.S;
+    k.nx = nx;
+  }
+  return k;
+}
+
+// Keys present in local chunk j of a unit: the last chunk of a flat sequence and of the
+// extra keys can be partial.
+template <bool kFlat>
+__device__ __forceinline__ int chunk_valid(const FwdBf16Params& p, const Chunks& k, int j) {
+  if (j < k.nm) return kFlat ? min(p.Lk - 128 * (k.c0 + j), 128) : 128;
+  return min(p.Lx - 128 * (j - k.nm), 128);
 }
 
 // Units run head-major, then tile, then the tile's 128-row chunks: the chunks of a tile
@@ -344,7 +383,8 @@ __device__ __forceinline__ void store_o(uint32_t tO, int groups, float inv, uint
 template <int kMode>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, FwdBf16Params p) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKx,
+                    const __grid_constant__ CUtensorMap tmVx, FwdBf16Params p) {
   using namespace fwd;
   constexpr bool kMap = kMode == kModeMap, kFlat = kMode == kModeFlat;
   extern __shared__ uint8_t smem_raw[];
@@ -379,6 +419,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     tma_prefetch_map(&tmQ);
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
+    if (p.Lx > 0) {
+      tma_prefetch_map(&tmKx);
+      tma_prefetch_map(&tmVx);
+    }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < kKStages; ++s) {
@@ -421,7 +465,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           const Unit x = kFlat ? decode_flat(p, u) : decode(p, u);
           int n_list = 0;
           const int32_t* kv = kFlat ? nullptr : unit_keys(p, x.bh, x.tile, n_list);
-          const int n_chunks = kFlat ? (p.Lk + 127) / 128 : n_list * p.S, n_steps = (n_chunks + 1) / 2;
+          const Chunks ck = unit_chunks<kFlat>(p, x, n_list);
+          const int n_chunks = ck.nm + ck.nx, n_steps = (n_chunks + 1) / 2;
           if (n_chunks == 0) continue;  // nothing to load: the softmax warps write O = 0
           if (is_k) {
             ok = mbar_wait(q_empty, (uc & 1) ^ 1, abort, 20);
@@ -450,7 +495,21 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             uint64_t* full = (is_k ? k_full : v_full) + st;
             mbar_arrive_expect_tx(full, nb * kTileBytes);
             for (int b = 0; b < nb; ++b) {
-              const int c = is_k ? 2 * j + b : j;
+              const int jc = is_k ? 2 * j + b : j;  // the unit's chunk
+              if (jc >= ck.nm) {  // extra keys (rows past Lx load as zeros and are masked)
+                const int row = 128 * (jc - ck.nm);
+                if (is_k) {
+                  uint8_t* dst = smem + kOffK + st * kStageBytes + b * kHalfBytes;
+                  tma_load_3d(dst, &tmKx, full, 0, row, x.bh);
+                  tma_load_3d(dst + kTileBytes, &tmKx, full, 64, row, x.bh);
+                } else {
+                  uint8_t* dst = smem + kOffV + st * kTileBytes;
+                  tma_load_3d(dst, &tmVx, full, 0, row, x.bh);
+                  tma_load_3d(dst + kHalfBytes, &tmVx, full, 64, row, x.bh);
+                }
+                continue;
+              }
+              const int c = ck.c0 + jc;
               if constexpr (kFlat) {  // rows past Lk load as zeros (and are masked)
                 if (is_k) {
                   uint8_t* dst = smem + kOffK + st * kStageBytes + b * kHalfBytes;
@@ -490,11 +549,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         int n_list = 0;
-        if constexpr (!kFlat) {
-          const Unit xm = decode(p, u);
-          unit_keys(p, xm.bh, xm.tile, n_list);
-        }
-        const int n_chunks = kFlat ? (p.Lk + 127) / 128 : n_list * p.S, n_steps = (n_chunks + 1) / 2;
+        const Unit xm = kFlat ? decode_flat(p, u) : decode(p, u);
+        if constexpr (!kFlat) unit_keys(p, xm.bh, xm.tile, n_list);
+        const Chunks ck = unit_chunks<kFlat>(p, xm, n_list);
+        const int n_chunks = ck.nm + ck.nx, n_steps = (n_chunks + 1) / 2;
         if (n_chunks == 0) continue;
         ok = warp_wait(q_full, uc & 1, abort, 30);
         if (ok) ok = warp_wait(k_full + ks % kKStages, (ks / kKStages) & 1, abort, 31);
@@ -621,17 +679,21 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const Unit x = kFlat ? decode_flat(p, u) : decode(p, u);
       int n_list = 0;
       if constexpr (!kFlat) unit_keys(p, x.bh, x.tile, n_list);
-      const int n_chunks = kFlat ? (p.Lk + 127) / 128 : n_list * p.S, n_steps = (n_chunks + 1) / 2;
+      const Chunks ck = unit_chunks<kFlat>(p, x, n_list);
+      const int n_chunks = ck.nm + ck.nx, n_steps = (n_chunks + 1) / 2;
+      // flat mode: part x.sub of the key chunks writes its own partial output
+      const int64_t po = kFlat ? static_cast<int64_t>(x.sub) * p.part_out : 0;
+      const int64_t pl = kFlat ? static_cast<int64_t>(x.sub) * p.part_lse : 0;
       if (n_chunks == 0) {
         // no keys: O = 0 and LSE = ln 0 = -inf (the softmax of an empty set has no value;
         // this is the limit the oracle and the list form define)
         const int64_t rows = kFlat ? p.Lq : p.N;
         const int64_t tok = kFlat ? 128 * static_cast<int64_t>(x.tile) + r : chunk_token(p, x.tile, x.sub, r);
         if (tok < rows) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * rows + tok) * 128) + 8 * i;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + po + (static_cast<int64_t>(x.bh) * rows + tok) * 128) + 8 * i;
 #pragma unroll
           for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-          if (i == 0) p.lse[static_cast<int64_t>(x.bh) * rows + tok] = -INFINITY;
+          if (i == 0) p.lse[pl + static_cast<int64_t>(x.bh) * rows + tok] = -INFINITY;
         }
         continue;
       }
@@ -642,13 +704,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (ok) tc_fence_after();
         float alpha;
         bool need;
-        // flat mode: keys of this thread's columns that exist (the last chunk may be partial)
+        // keys present in this thread's columns (a flat sequence's or the extra keys' last
+        // chunk may be partial): chunk 2t + i of a full step, half i of chunk 2t otherwise
         const bool full = 2 * t + 1 < n_chunks;
-        int nvalid = full ? 128 : 64;
-        if constexpr (kFlat) {
-          const int first = full ? 128 * (2 * t + i) : 256 * t + 64 * i;
-          nvalid = min(max(p.Lk - first, 0), nvalid);
-        }
+        const int nvalid = full ? chunk_valid<kFlat>(p, ck, 2 * t + i)
+                                : min(max(chunk_valid<kFlat>(p, ck, 2 * t) - 64 * i, 0), 64);
         if (full)
           need = softmax_step<128>(ok, tmem + col_s(e) + 128 * i + lane_off, tmem + col_p(e) + 64 * i + lane_off,
                                    s_read + e, p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id, nvalid);
@@ -684,10 +744,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         // rows that exist are written)
         const bool row_ok = tok < rows;
         store_o(tO, 2, 1.f / l_all,
-                reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(x.bh) * rows + (row_ok ? tok : 0)) * 128) +
+                reinterpret_cast<uint4*>(p.out + po + (static_cast<int64_t>(x.bh) * rows + (row_ok ? tok : 0)) * 128) +
                     8 * i,
                 row_ok);
-        if (i == 0 && row_ok) p.lse[static_cast<int64_t>(x.bh) * rows + tok] = (m_used + __log2f(l_all)) * 0.69314718055994531f;
+        if (i == 0 && row_ok)
+          p.lse[pl + static_cast<int64_t>(x.bh) * rows + tok] = (m_used + __log2f(l_all)) * 0.69314718055994531f;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_free);
@@ -706,36 +767,40 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   }
 }
 
-// Merge of two attentions of the same queries over disjoint key sets: with
-// L = ln(e^lse + e^lse2),  o <- e^(lse - L) o + e^(lse2 - L) o2,  lse <- L  (exact: the
-// softmax over the union, written through the two partial normalisations).  A part with
-// lse = -inf (no keys) has weight 0.  16 threads per 128-channel row, 8 channels each.
-__global__ void __launch_bounds__(256) merge_kernel(__nv_bfloat16* o, float* lse, const __nv_bfloat16* o2,
-                                                    const float* lse2, int64_t rows) {
+// Merge of n attentions of the same rows over disjoint key sets (parts j = 0..n-1 at
+// o + j * part_out, lse + j * part_lse):  L = ln sum_j e^lse_j,  O = sum_j e^(lse_j - L) O_j
+// (exact: the softmax over the union, written through the parts' own normalisations).  A
+// part with lse = -inf (no keys) has weight 0.  16 threads per 128-channel row, 8 channels
+// each; fp32 sums, bf16 result.
+__global__ void __launch_bounds__(256) merge_parts_kernel(const __nv_bfloat16* o, const float* lse, int n_parts,
+                                                          int64_t part_out, int64_t part_lse, int64_t rows,
+                                                          __nv_bfloat16* out, float* lse_out) {
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 16;
   const int part = threadIdx.x % 16;
   if (row >= rows) return;
-  const float a = lse[row], b = lse2[row];
-  const float m = fmaxf(a, b);
-  float wa = 0.f, wb = 0.f, L = -INFINITY;
+  float m = -INFINITY;
+  for (int j = 0; j < n_parts; ++j) m = fmaxf(m, lse[j * part_lse + row]);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float L = -INFINITY;
   if (m != -INFINITY) {
-    const float ea = __expf(a - m), eb = __expf(b - m);
-    L = m + __logf(ea + eb);
-    wa = __expf(a - L);
-    wb = __expf(b - L);
-  }
-  uint4* dst = reinterpret_cast<uint4*>(o + row * 128) + part;
-  const uint4 x = *dst, y = reinterpret_cast<const uint4*>(o2 + row * 128)[part];
-  const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
-  uint32_t r[4];
+    float sum = 0.f;
+    for (int j = 0; j < n_parts; ++j) sum += __expf(lse[j * part_lse + row] - m);
+    L = m + __logf(sum);
+    for (int j = 0; j < n_parts; ++j) {
+      const float w = __expf(lse[j * part_lse + row] - L);
+      const uint4 x = reinterpret_cast<const uint4*>(o + j * part_out + row * 128)[part];
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float x0 = __uint_as_float(xs[e] << 16), x1 = __uint_as_float(xs[e] & 0xffff0000u);
-    const float y0 = __uint_as_float(ys[e] << 16), y1 = __uint_as_float(ys[e] & 0xffff0000u);
-    r[e] = pack_bf16x2(wa * x0 + wb * y0, wa * x1 + wb * y1);
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += w * __uint_as_float(xs[e] << 16);
+        acc[2 * e + 1] += w * __uint_as_float(xs[e] & 0xffff0000u);
+      }
+    }
   }
-  *dst = make_uint4(r[0], r[1], r[2], r[3]);
-  if (part == 0) lse[row] = L;
+  reinterpret_cast<uint4*>(out + row * 128)[part] =
+      make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                 pack_bf16x2(acc[6], acc[7]));
+  if (part == 0) lse_out[row] = L;
 }
 
 }  // namespace dsa
