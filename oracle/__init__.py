@@ -300,6 +300,58 @@ def forward_prefix(geo: Geometry, q, k, v, offsets, q_text, k_text, v_text):
     return out, lse, out_x, lse_x
 
 
+def _prefix_key_mask(geo: Geometry, offsets, L_text: int, rows) -> np.ndarray:
+    """Boolean [len(rows), N + L_text]: which keys of the unified [video; text] sequence
+    query row r (r < N: video token r, else text token r - N) attends to: a video token its
+    window's key tiles (the oracle's plan) and every text token; a text token everything."""
+    N = geo.n_tokens
+    _, kv, _, _ = plan(geo.G, geo.window, offsets)
+    tile_of = np.zeros(N, np.int64)
+    tile_of[geo.tile_token_index().reshape(-1)] = np.repeat(np.arange(geo.n_tiles), geo.tile_tokens)
+    allowed = np.zeros((geo.n_tiles, geo.n_tiles), bool)
+    allowed[np.repeat(np.arange(geo.n_tiles), kv.shape[1]), kv.reshape(-1)] = True
+    rows = np.asarray(rows)
+    mask = np.ones((len(rows), N + L_text), bool)
+    vid = rows < N
+    mask[np.nonzero(vid)[0], :N] = allowed[tile_of[rows[vid]]][:, tile_of]
+    return mask
+
+
+def backward_prefix(geo: Geometry, q, k, v, dout, offsets, q_text, k_text, v_text, dout_text, block: int = 512):
+    """Text-prefix backward of L = sum(O * dO) over the unified sequence: the plain softmax
+    attention gradients (P = exp(s - lse), D = rowsum(dO * O), dS = P (dP - D),
+    dq = scale dS K, dk = scale dS^T Q, dv = P^T dO), each query row over its key set (video:
+    window and every text token; text: everything), in float64, query rows in blocks of
+    `block` with library matmuls.  Returns (dq, dk, dv) as [B, heads, T, H, W, d] and
+    (dq_text, dk_text, dv_text) as [B, heads, L_text, d]."""
+    BH, N, d = geo.B * geo.heads, geo.n_tokens, geo.d
+    L = int(q_text.shape[2])
+    outs = [np.zeros((BH, N + L, d), np.float64) for _ in range(3)]
+    for h in range(BH):
+        def cat(a, b):
+            return np.concatenate([_head_slice(a, geo, h), _text_slice(b, geo, h)], axis=0)
+
+        Q, K, V, dO = cat(q, q_text), cat(k, k_text), cat(v, v_text), cat(dout, dout_text)
+        dq, dk, dv = (o[h] for o in outs)
+        for r0 in range(0, N + L, block):
+            rows = np.arange(r0, min(r0 + block, N + L))
+            m = _prefix_key_mask(geo, offsets, L, rows)
+            s = np.where(m, geo.scale * (Q[rows] @ K.T), -np.inf)
+            mx = s.max(axis=1, keepdims=True)
+            lse = mx + np.log(np.exp(s - mx).sum(axis=1, keepdims=True))
+            P = np.exp(s - lse)
+            O = P @ V
+            dP = dO[rows] @ V.T
+            D = (dO[rows] * O).sum(axis=1, keepdims=True)
+            dS = P * (dP - D)
+            dq[rows] = geo.scale * (dS @ K)
+            dk += geo.scale * (dS.T @ Q[rows])
+            dv += P.T @ dO[rows]
+    shape_v = (geo.B, geo.heads) + geo.grid + (d,)
+    shape_t = (geo.B, geo.heads, L, d)
+    return (tuple(o[:, :N].reshape(shape_v) for o in outs), tuple(o[:, N:].reshape(shape_t) for o in outs))
+
+
 def backward_dq_tiles(geo: Geometry, q, k, v, dout, offsets, sel=None):
     """dq on (bh, query tile) pairs: [n_sel, tile_tokens, d] float64."""
     lib = _load()

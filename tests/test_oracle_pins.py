@@ -626,3 +626,47 @@ def test_prefix_text_copy_of_video_closed_form():
     np.testing.assert_allclose(out_x.reshape(BH, N, geo.d), dense, rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse.reshape(BH, N), dense_lse + np.log(2.0), rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse_x.reshape(BH, N), dense_lse + np.log(2.0), rtol=0, atol=1e-12)
+
+
+def _unified_autograd(geo, tensors, text, mask):
+    """Masked dense attention over the unified [video; text] sequence in float64 and the
+    autograd gradients of sum(O * dO) (written independently of the oracle)."""
+    BH = geo.B * geo.heads
+    L = text[0].shape[2]
+    cat = [torch.cat([torch.as_tensor(flat(a, geo)), torch.as_tensor(np.asarray(b)).reshape(BH, L, geo.d)], 1)
+           for a, b in zip(tensors, text)]
+    q, k, v = (c.clone().requires_grad_(True) for c in cat[:3])
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(mask), scale=geo.scale)
+    (o * cat[3]).sum().backward()
+    return q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+@pytest.mark.parametrize("window,L,lo,hi", [((2, 1, 3), 5, -2, 2), ((1, 2, 2), 1, -1, 1), ((3, 3, 3), 9, 0, 0)])
+def test_prefix_backward_equals_autograd_of_unified_attention(window, L, lo, hi):
+    geo = oracle.Geometry(1, 2, 8, (3, 4, 6), (1, 2, 2), window)
+    q, k, v, do = rand_inputs(geo, 41)
+    qt, kt, vt = rand_text(geo, L, 42)
+    dot = rand_text(geo, L, 43)[0]
+    off = rand_offsets(geo, lo, hi, 44)
+    (dq, dk, dv), (dqt, dkt, dvt) = oracle.backward_prefix(geo, q, k, v, do, off, qt, kt, vt, dot, block=7)
+    N = geo.n_tokens
+    mask = np.ones((N + L, N + L), bool)
+    mask[:N, :N] = brute_mask(geo.grid, geo.tile, geo.window, off.numpy())
+    gq, gk, gv = _unified_autograd(geo, (q, k, v, do), (qt, kt, vt, dot), mask)
+    BH = geo.B * geo.heads
+    for got_v, got_t, ref, name in ((dq, dqt, gq, "dq"), (dk, dkt, gk, "dk"), (dv, dvt, gv, "dv")):
+        np.testing.assert_allclose(flat(got_v, geo), ref[:, :N], rtol=0, atol=1e-11, err_msg=name)
+        np.testing.assert_allclose(np.asarray(got_t).reshape(BH, L, geo.d), ref[:, N:], rtol=0, atol=1e-11,
+                                   err_msg=name + "_text")
+
+
+def test_prefix_backward_without_text_is_the_window_backward():
+    geo = oracle.Geometry(1, 2, 8, (3, 4, 6), (1, 2, 2), (2, 2, 2))
+    q, k, v, do = rand_inputs(geo, 45)
+    qt, kt, vt = rand_text(geo, 0, 46)
+    off = rand_offsets(geo, -2, 2, 47)
+    (dq, dk, dv), (dqt, _, _) = oracle.backward_prefix(geo, q, k, v, do, off, qt, kt, vt, qt)
+    rq, rk, rv = oracle.backward(geo, q, k, v, do, off)
+    for a, b in ((dq, rq), (dk, rk), (dv, rv)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    assert dqt.size == 0
