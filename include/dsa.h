@@ -190,6 +190,24 @@ dsa_status_t dsa_fwd_prefix(const dsa_problem_t* p, const void* q, const void* k
                             const void* v_text, void* out, float* lse, void* out_text, float* lse_text,
                             void* workspace, size_t ws_bytes, void* stream);
 
+/* Backward of dsa_fwd_prefix: gradients of L = sum(O * dO) over both token types, each
+ * query's softmax over its key set as in dsa_fwd_prefix, given that call's out, lse,
+ * out_text, lse_text and the output gradients dout [B, heads, T, H, W, 128] and dout_text
+ * [B, heads, L_text, 128] (bf16).  Writes dq, dk, dv (video, the layout of q) and dq_text,
+ * dk_text, dv_text (the layout of q_text), bf16.  Video keys are reduced over their windows'
+ * queries and every text query by the window backward kernel; text keys over every video
+ * and text query by the same kernel in a flat-key mode (query chunks cut into parts for
+ * load balance, fp32 partial dK / dV summed at the end).  L_text = 0 is dsa_bwd (text
+ * pointers may be NULL).  workspace: at least dsa_bwd_prefix_workspace_size(p, L_text)
+ * bytes, 256-byte aligned.  bf16, d = 128. */
+size_t dsa_bwd_prefix_workspace_size(const dsa_problem_t* p, int32_t L_text);
+dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,
+                            const float* lse, const void* dout, const int32_t* tile_offsets, int32_t L_text,
+                            const void* q_text, const void* k_text, const void* v_text, const void* out_text,
+                            const float* lse_text, const void* dout_text, void* dq, void* dk, void* dv,
+                            void* dq_text, void* dk_text, void* dv_text, void* workspace, size_t ws_bytes,
+                            void* stream);
+
 /* Block attention mass (the sparsity map that block masks are chosen from; MOD-DiT page,
  * Method section and project structure: attention fused with a sparsity map): for every
  * (batch, head) h, query tile i and key tile j,

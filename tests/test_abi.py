@@ -131,6 +131,20 @@ def test_list_entry_points_reject_bad_arguments(lib):
     assert lib.dsa_fwd_prefix(ctypes.byref(p32), f, f, f, f, 4, f, f, f, f, f, f, f, f, big, None) == 2
     assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, f, 4, f, f, f, f, f, f, f, f, 16, None) == 5
     assert lib.dsa_fwd_prefix(ctypes.byref(p), f, f, f, f, 4, f, f, f, f, f, f, f, None, big, None) == 5
+    # prefix backward: (p, q, k, v, out, lse, dout, offsets, L_text, q_text, k_text, v_text, out_text,
+    # lse_text, dout_text, dq, dk, dv, dq_text, dk_text, dv_text, ws, ws_bytes, stream)
+    fb = [f] * 7
+    tb = [f] * 6
+    gb = [f] * 6
+    assert lib.dsa_bwd_prefix(ctypes.byref(p), *fb[:6], None, 4, *tb, *gb, f, big, None) == 1   # no offsets
+    assert lib.dsa_bwd_prefix(ctypes.byref(p), *fb, -3, *tb, *gb, f, big, None) == 1             # negative length
+    assert lib.dsa_bwd_prefix(ctypes.byref(p), *fb, 4, None, *tb[1:], *gb, f, big, None) == 1    # text q missing
+    assert lib.dsa_bwd_prefix(ctypes.byref(p), *fb, 4, *tb, *gb[:5], None, f, big, None) == 1    # dv_text missing
+    assert lib.dsa_bwd_prefix(ctypes.byref(p32), *fb, 4, *tb, *gb, f, big, None) == 2
+    assert lib.dsa_bwd_prefix(ctypes.byref(p), *fb, 4, *tb, *gb, f, 16, None) == 5
+    b0 = lib.dsa_bwd_prefix_workspace_size(ctypes.byref(p), 0)
+    assert 0 < b0 < lib.dsa_bwd_prefix_workspace_size(ctypes.byref(p), 1000)
+    assert lib.dsa_bwd_prefix_workspace_size(ctypes.byref(p), -1) == 0
     w0 = lib.dsa_prefix_workspace_size(ctypes.byref(p), 0)
     assert 0 < w0 < lib.dsa_prefix_workspace_size(ctypes.byref(p), 1000)
     assert lib.dsa_prefix_workspace_size(ctypes.byref(p), -1) == 0

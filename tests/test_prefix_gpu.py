@@ -92,3 +92,69 @@ def test_prefix_720p_sampled():
     ref_x, ref_lse_x = oracle.forward_prefix_text(geo, txt.q, txt.k, txt.v, inp.k, inp.v, rows)
     assert_close(out_x[:, :, rows].float().cpu().numpy(), ref_x, w.dtype, "text out")
     assert_lse_close(lse_x[:, :, rows].cpu().numpy(), ref_lse_x, w.dtype, "text lse")
+
+
+# ------------------------------------------------------------------------------------
+# backward of the text prefix
+
+
+def _dout(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def run_backward(w, inp, txt, seed):
+    dev = torch.device("cuda")
+    q, k, v, off = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), inp.offsets.to(dev)
+    qt, kt, vt = txt.q.to(dev), txt.k.to(dev), txt.v.to(dev)
+    out, lse, out_t, lse_t = dsa.forward_prefix(q, k, v, off, qt, kt, vt, w.tile, w.window, w.scale)
+    do, do_t = _dout(tuple(q.shape), seed), _dout(tuple(qt.shape), seed + 1)
+    grads = dsa.backward_prefix(q, k, v, out, lse, do.to(dev), off, qt, kt, vt, out_t, lse_t, do_t.to(dev), w.tile,
+                                w.window, w.scale)
+    torch.cuda.synchronize()
+    st, site, _ = dsa.device_status()
+    assert st == 0, f"device status {st} at site {site}"
+    return grads, do, do_t
+
+
+def check_backward(w, inp, txt, grads, do, do_t):
+    geo = oracle.Geometry.of(w)
+    (rq, rk, rv), (rqt, rkt, rvt) = oracle.backward_prefix(geo, inp.q, inp.k, inp.v, do, inp.offsets, txt.q, txt.k,
+                                                           txt.v, do_t)
+    for got, ref, name in zip(grads, (rq, rk, rv, rqt, rkt, rvt), ("dq", "dk", "dv", "dq_text", "dk_text", "dv_text")):
+        assert_close(got.float().cpu().numpy(), ref, w.dtype, name)
+
+
+@pytest.mark.parametrize("L", [1, 77, 200])
+def test_prefix_backward_small_full(L):
+    w = SMALL
+    inp = make_inputs(w)
+    txt = make_text_inputs(w, L, seed=200 + L)
+    grads, do, do_t = run_backward(w, inp, txt, 300 + L)
+    check_backward(w, inp, txt, grads, do, do_t)
+
+
+def test_prefix_backward_without_text_is_the_window_backward():
+    w = SMALL
+    inp = make_inputs(w)
+    txt = make_text_inputs(w, 0, seed=9)
+    grads, do, _ = run_backward(w, inp, txt, 11)
+    dev = torch.device("cuda")
+    q, k, v, off = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), inp.offsets.to(dev)
+    out, lse = dsa.forward(q, k, v, off, w.tile, w.window, w.scale)
+    ref = dsa.backward(q, k, v, out, lse, do.to(dev), off, w.tile, w.window, w.scale)
+    # dK, dV accumulate in a fixed order: bit-exact; dQ is summed with fp32 atomics in
+    # timing-dependent order, so it may differ in the last bf16 place
+    assert torch.equal(grads[1], ref[1]) and torch.equal(grads[2], ref[2])
+    assert float((grads[0].float() - ref[0].float()).abs().max()) <= 1e-3
+    assert all(g.numel() == 0 for g in grads[3:])
+
+
+def test_prefix_backward_16x32x32_grid_full():
+    """A 16384-token grid (64 tiles, 3x3x3 windows) with 163 text tokens: every text key
+    sees 256 video query chunks cut into parts."""
+    w = Workload("prefix_16x32x32", 1, 1, 128, (16, 32, 32), (4, 8, 8), (3, 3, 3), (-1, 1), "bf16", 61)
+    inp = make_inputs(w)
+    txt = make_text_inputs(w, 163, seed=62)
+    grads, do, do_t = run_backward(w, inp, txt, 63)
+    check_backward(w, inp, txt, grads, do, do_t)

@@ -37,7 +37,7 @@ EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_
            "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status", "dsa_fwd_noalloc",
            "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map",
            "dsa_lstsq_workspace_size", "dsa_lstsq_factor", "dsa_lstsq_solve", "dsa_prefix_workspace_size",
-           "dsa_fwd_prefix")
+           "dsa_fwd_prefix", "dsa_bwd_prefix_workspace_size", "dsa_bwd_prefix")
 
 
 class DsaError(RuntimeError):
@@ -94,9 +94,13 @@ def load_library(path: Optional[str] = None):
     lib.dsa_prefix_workspace_size.restype = sz
     lib.dsa_prefix_workspace_size.argtypes = [pp, i32]
     lib.dsa_fwd_prefix.argtypes = [pp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_bwd_prefix_workspace_size.restype = sz
+    lib.dsa_bwd_prefix_workspace_size.argtypes = [pp, i32]
+    lib.dsa_bwd_prefix.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                   vp, vp, sz, vp]
     for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status",
                  "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map",
-                 "dsa_lstsq_factor", "dsa_lstsq_solve", "dsa_fwd_prefix"):
+                 "dsa_lstsq_factor", "dsa_lstsq_solve", "dsa_fwd_prefix", "dsa_bwd_prefix"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -245,6 +249,44 @@ def forward_prefix(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, offsets: t
                               _ptr(k_text), _ptr(v_text), _ptr(out), _ptr(lse), _ptr(out_text), _ptr(lse_text),
                               _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream))), "dsa_fwd_prefix")
     return out, lse, out_text, lse_text
+
+
+def prefix_bwd_workspace_size(problem: Problem, L_text: int) -> int:
+    return int(load_library().dsa_bwd_prefix_workspace_size(ctypes.byref(problem), int(L_text)))
+
+
+def backward_prefix(q, k, v, out, lse, dout, offsets, q_text, k_text, v_text, out_text, lse_text, dout_text,
+                    tile: Sequence[int], window: Sequence[int], scale: Optional[float] = None,
+                    ws: Optional[torch.Tensor] = None, stream=None):
+    """Backward of forward_prefix (gradients of sum(out * dout) + sum(out_text * dout_text)).
+    Returns (dq, dk, dv, dq_text, dk_text, dv_text)."""
+    lib = load_library()
+    p = _problem_of(q, tile, window, scale)
+    for t, name in ((k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, name, q, q.dtype)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
+    _need(q, "q", q)
+    _need(lse, "lse", q, torch.float32)
+    _need(offsets, "offsets", q, torch.int32)
+    if q_text.dim() != 4 or tuple(q_text.shape[:2]) != tuple(q.shape[:2]) or q_text.shape[3] != q.shape[5]:
+        raise ValueError(f"q_text shape {tuple(q_text.shape)} does not match q {tuple(q.shape)}")
+    for t, name in ((q_text, "q_text"), (k_text, "k_text"), (v_text, "v_text"), (out_text, "out_text"),
+                    (dout_text, "dout_text")):
+        _need(t, name, q, q.dtype)
+        if t.shape != q_text.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != q_text shape {tuple(q_text.shape)}")
+    _need(lse_text, "lse_text", q, torch.float32)
+    L_text = int(q_text.shape[2])
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dqt, dkt, dvt = torch.empty_like(q_text), torch.empty_like(q_text), torch.empty_like(q_text)
+    if ws is None:
+        ws = torch.empty(max(prefix_bwd_workspace_size(p, L_text), 256), dtype=torch.uint8, device=q.device)
+    _check(lib.dsa_bwd_prefix(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                              _ptr(offsets), L_text, _ptr(q_text), _ptr(k_text), _ptr(v_text), _ptr(out_text),
+                              _ptr(lse_text), _ptr(dout_text), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dqt), _ptr(dkt),
+                              _ptr(dvt), _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream))), "dsa_bwd_prefix")
+    return dq, dk, dv, dqt, dkt, dvt
 
 
 def forward_host_bytes(problem: Problem) -> int:

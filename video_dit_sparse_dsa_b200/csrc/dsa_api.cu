@@ -232,16 +232,31 @@ bool make_row_map(CUtensorMap* map, const void* ptr, const dsa_problem_t* p, con
 }
 
 // A flat [BH, L, 128] bf16 token sequence seen as 3-D (128, L, BH); one box is 64 channels
-// of 128 consecutive tokens (rows past L load as zeros).
-bool make_flat_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t L) {
+// of box_rows consecutive tokens (rows past L load as zeros).
+bool make_flat_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t L, int box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(L) * 128 * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// fp32 rows [BH, L] (L * 4 bytes a multiple of 16) seen as 2-D (L, BH); one box is 64
+// consecutive rows of one (batch, head) (rows past L load as zeros).
+bool make_vec_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t L) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(L) * 4};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -404,10 +419,43 @@ dsa_status_t launch_merge_parts(const void* o, const float* lse, int n_parts, in
 
 // The backward after planning: D preprocess (and zeroing of the dQ accumulator), the
 // key-major kernel over the inverse CSR (row_ptr, q_tiles), and the dQ conversion.
+// Extra (text) query rows of a backward: flat q, dO [BH, L, 128] bf16, LSE and D copies
+// padded to [BH, Lp] fp32, and their fp32 dQ accumulator.
+struct ExtraQueries {
+  const void* q;
+  const void* dout;
+  const float* lse_pad;
+  const float* delta_pad;
+  float* dq_acc;
+  int L, Lp;
+};
+
+template <bool kFlatK>
+dsa_status_t launch_bwd_kernel(const dsa::BwdBf16Params& bp, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tlse,
+                               const CUtensorMap& tdel, const ExtraQueries* x, int64_t BH, cudaStream_t s) {
+  CUtensorMap tqx = tq, tdox = tdo, tlsex = tlse, tdx = tdel;
+  if (x != nullptr && x->L > 0) {
+    if (!make_flat_map(&tqx, x->q, BH, x->L, 64) || !make_flat_map(&tdox, x->dout, BH, x->L, 64) ||
+        !make_vec_map(&tlsex, x->lse_pad, BH, x->Lp) || !make_vec_map(&tdx, x->delta_pad, BH, x->Lp))
+      return DSA_ERR_CUDA;
+  }
+  auto kernel = dsa::bwd_bf16_kernel<kFlatK>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::bwd::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
+  kernel<<<grid, dsa::bwd::kThreads, dsa::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tlse, tdel, tqx, tdox, tlsex, tdx,
+                                                                 bp);
+  return launch_status();
+}
+
 dsa_status_t launch_bwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
                         const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
                         const int32_t* q_tiles, float* delta, float* dq_acc, void* dq, void* dk, void* dv,
-                        cudaStream_t s, int rp_head_stride = 0) {
+                        cudaStream_t s, int rp_head_stride = 0, const ExtraQueries* x = nullptr,
+                        bool convert_dq = true) {
   dsa_status_t st;
   const int64_t rows = g.BH * g.N;
   dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
@@ -443,15 +491,18 @@ dsa_status_t launch_bwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.N = static_cast<int>(g.N);
   bp.scale = p->scale;
   bp.scale_log2 = p->scale * 1.4426950408889634f;
-  if (cudaFuncSetAttribute(dsa::bwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dsa::bwd::kSmemBytes) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  int sms = 0;
-  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
-  dsa::bwd_bf16_kernel<<<grid, dsa::bwd::kThreads, dsa::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tlse, tdel, bp);
-  st = launch_status();
-  if (st != DSA_OK) return st;
+  bp.Lxq = 0;
+  bp.dq_acc_x = nullptr;
+  bp.Lk = bp.Nq = 0;
+  bp.n_split = 1;
+  bp.dk_part = bp.dv_part = nullptr;
+  bp.part_stride = 0;
+  if (x != nullptr) {  // extra (text) queries after every key unit's own
+    bp.Lxq = x->L;
+    bp.dq_acc_x = x->dq_acc;
+  }
+  st = launch_bwd_kernel<false>(bp, tq, tk, tv, tdo, tlse, tdel, x, g.BH, s);
+  if (st != DSA_OK || !convert_dq) return st;
   const int64_t n8 = rows * p->d / 8;
   dsa::bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
       dq_acc, static_cast<__nv_bfloat16*>(dq), p->scale, n8);
@@ -884,6 +935,145 @@ dsa_status_t dsa_fwd_prefix(const dsa_problem_t* p, const void* q, const void* k
                    ws.l_parts, rows * 128, rows, s);
   if (st != DSA_OK) return st;
   return launch_merge_parts(ws.o_parts, ws.l_parts, ws.n_split, rows * 128, rows, rows, out_text, lse_text, s);
+}
+
+namespace {
+// Parts the query chunks of the text keys' backward are cut into: enough units for about
+// four waves of persistent CTAs, at most one part per 64-query chunk of the video.
+int prefix_bwd_split(const Geom& g, int32_t L_text) {
+  const int64_t units = g.BH * ((static_cast<int64_t>(L_text) + 127) / 128);
+  const int64_t nqm = (g.N + 63) / 64;
+  int64_t n = (4 * 148 + units - 1) / (units > 0 ? units : 1);
+  if (n > nqm) n = nqm;
+  if (n > 16) n = 16;
+  return static_cast<int>(n < 1 ? 1 : n);
+}
+
+struct PrefixBwdWorkspace {
+  BwdWorkspace video;
+  float* lse_pad;    // [BH, Lp] text LSE, zeros past L
+  float* delta_pad;  // [BH, Lp] text D
+  float* dq_acc_x;   // [BH, L, 128] fp32
+  float* dk_part;    // [n_split][BH, L, 128] fp32
+  float* dv_part;
+  int Lp, n_split;
+  size_t bytes;
+};
+
+PrefixBwdWorkspace prefix_bwd_workspace(const Geom& g, int32_t L, void* base) {
+  PrefixBwdWorkspace w;
+  w.video = bwd_workspace(g, 128, base);
+  uint8_t* b = static_cast<uint8_t*>(base);
+  size_t off = w.video.bytes;
+  w.Lp = (L + 63) / 64 * 64;
+  w.n_split = prefix_bwd_split(g, L);
+  const size_t rows = static_cast<size_t>(g.BH) * L, rows_p = static_cast<size_t>(g.BH) * w.Lp;
+  auto take = [&](size_t bytes) {
+    float* ptr = b ? reinterpret_cast<float*>(b + off) : nullptr;
+    off += round_up(bytes, kAlign);
+    return ptr;
+  };
+  w.lse_pad = take(sizeof(float) * rows_p);
+  w.delta_pad = take(sizeof(float) * rows_p);
+  w.dq_acc_x = take(sizeof(float) * rows * 128);
+  w.dk_part = take(sizeof(float) * rows * 128 * w.n_split);
+  w.dv_part = take(sizeof(float) * rows * 128 * w.n_split);
+  w.bytes = off;
+  return w;
+}
+}  // namespace
+
+size_t dsa_bwd_prefix_workspace_size(const dsa_problem_t* p, int32_t L_text) {
+  Geom g;
+  if (check_shape(p, &g) != DSA_OK || L_text < 0) return 0;
+  return prefix_bwd_workspace(g, L_text, nullptr).bytes;
+}
+
+dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,
+                            const float* lse, const void* dout, const int32_t* tile_offsets, int32_t L_text,
+                            const void* q_text, const void* k_text, const void* v_text, const void* out_text,
+                            const float* lse_text, const void* dout_text, void* dq, void* dk, void* dv,
+                            void* dq_text, void* dk_text, void* dv_text, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  Geom g;
+  dsa_status_t st = check_shape(p, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !k || !v || !out || !lse || !dout || !tile_offsets || !dq || !dk || !dv || L_text < 0)
+    return DSA_ERR_INVALID_ARG;
+  if (L_text > 0 && (!q_text || !k_text || !v_text || !out_text || !lse_text || !dout_text || !dq_text || !dk_text ||
+                     !dv_text))
+    return DSA_ERR_INVALID_ARG;
+  if (p->dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  st = check_kernel_limits(p, g, true);
+  if (st != DSA_OK) return st;
+  if (g.BH * ((static_cast<int64_t>(L_text) + 127) / 128) * 16 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, out, dout, dq, dk, dv, q_text, k_text, v_text, out_text, dout_text, dq_text, dk_text,
+                        dv_text};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned(ptr, 16)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4) || (lse_text && !aligned(lse_text, 4)) || !aligned(tile_offsets, 4)) return DSA_ERR_INVALID_ARG;
+  if (workspace == nullptr || ws_bytes < prefix_bwd_workspace(g, L_text, nullptr).bytes || !aligned(workspace, kAlign))
+    return DSA_ERR_WORKSPACE;
+  const PrefixBwdWorkspace ws = prefix_bwd_workspace(g, L_text, workspace);
+  const BwdWorkspace& wv = ws.video;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_plan(g, tile_offsets, wv.starts, wv.kv_tiles, wv.row_ptr, wv.q_tiles, s);
+  if (st != DSA_OK) return st;
+  if (L_text == 0)
+    return launch_bwd(p, g, q, k, v, out, lse, dout, wv.row_ptr, wv.q_tiles, wv.delta, wv.dq_acc, dq, dk, dv, s);
+  // text rows: D, padded LSE / D copies, zeroed dQ accumulator
+  const int64_t prow = g.BH * ws.Lp;
+  dsa::bwd_preprocess_flat<<<static_cast<unsigned>((prow * 16 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(out_text), static_cast<const __nv_bfloat16*>(dout_text), lse_text,
+      ws.delta_pad, ws.lse_pad, ws.dq_acc_x, L_text, ws.Lp, g.BH);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  const ExtraQueries xq{q_text, dout_text, ws.lse_pad, ws.delta_pad, ws.dq_acc_x, L_text, ws.Lp};
+  // video keys: their windows' query chunks, then every text query chunk (dK, dV final)
+  st = launch_bwd(p, g, q, k, v, out, lse, dout, wv.row_ptr, wv.q_tiles, wv.delta, wv.dq_acc, dq, dk, dv, s, 0, &xq,
+                  false);
+  if (st != DSA_OK) return st;
+  // text keys: every video query chunk (the video as flat rows), in parts, then every text
+  // query chunk; fp32 partial dK, dV per part
+  CUtensorMap tq, tk, tv, tdo, tlse, tdel;
+  if (!make_flat_map(&tq, q, g.BH, g.N, 64) || !make_flat_map(&tk, k_text, g.BH, L_text, 128) ||
+      !make_flat_map(&tv, v_text, g.BH, L_text, 128) || !make_flat_map(&tdo, dout, g.BH, g.N, 64) ||
+      !make_vec_map(&tlse, lse, g.BH, g.N) || !make_vec_map(&tdel, wv.delta, g.BH, g.N))
+    return DSA_ERR_CUDA;
+  dsa::BwdBf16Params bp;
+  std::memset(&bp, 0, sizeof(bp));
+  bp.dq_acc = wv.dq_acc;
+  bp.N = static_cast<int>(g.N);
+  bp.scale = p->scale;
+  bp.scale_log2 = p->scale * 1.4426950408889634f;
+  bp.Lxq = L_text;
+  bp.dq_acc_x = ws.dq_acc_x;
+  bp.Lk = L_text;
+  bp.Nq = static_cast<int>(g.N);
+  bp.n_split = ws.n_split;
+  bp.dk_part = ws.dk_part;
+  bp.dv_part = ws.dv_part;
+  bp.part_stride = g.BH * static_cast<int64_t>(L_text) * 128;
+  bp.n_units = static_cast<int>(g.BH * ((L_text + 127) / 128) * ws.n_split);
+  bp.tt = bp.th = bp.tw = 1;  // no tile geometry in the flat-key mode
+  bp.T = bp.H = bp.W = 1;
+  st = launch_bwd_kernel<true>(bp, tq, tk, tv, tdo, tlse, tdel, &xq, g.BH, s);
+  if (st != DSA_OK) return st;
+  // dQ of both token types, dK and dV of the text
+  const int64_t n8v = g.BH * g.N * 128 / 8, n8t = g.BH * static_cast<int64_t>(L_text) * 128 / 8;
+  dsa::bwd_dq_convert<<<static_cast<unsigned>((n8v + 255) / 256), 256, 0, s>>>(
+      wv.dq_acc, static_cast<__nv_bfloat16*>(dq), p->scale, n8v);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  dsa::bwd_dq_convert<<<static_cast<unsigned>((n8t + 255) / 256), 256, 0, s>>>(
+      ws.dq_acc_x, static_cast<__nv_bfloat16*>(dq_text), p->scale, n8t);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  const int64_t n4 = 2 * n8t;
+  dsa::bwd_kv_combine<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
+      ws.dk_part, ws.dv_part, ws.n_split, bp.part_stride, p->scale, n4, static_cast<__nv_bfloat16*>(dk_text),
+      static_cast<__nv_bfloat16*>(dv_text));
+  return launch_status();
 }
 
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block) {

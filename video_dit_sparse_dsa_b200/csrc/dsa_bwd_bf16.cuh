@@ -37,6 +37,17 @@ struct BwdBf16Params {
   int qcs;                 // t-extent of a 64-token query chunk
   int T, H, W, N;
   float scale, scale_log2;
+  // extra (text) query rows after every unit's own query chunks: flat [B*heads, Lxq, 128] Q
+  // and dO, [B*heads, Lxq] LSE and D; their dQ goes to dq_acc_x [B*heads, Lxq, 128] fp32
+  int Lxq;
+  float* dq_acc_x;
+  // flat-key mode: the keys are Lk rows of a flat sequence and the main query rows Nq rows
+  // of another, in 64-row chunks cut into n_split parts; part j writes fp32 dK, dV at
+  // dk_part / dv_part + j * part_stride (the extra queries go with part 0)
+  int Lk, Nq, n_split;
+  float* dk_part;
+  float* dv_part;
+  int64_t part_stride;
 };
 
 namespace bwd {
@@ -63,6 +74,64 @@ constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, 64, 1, 1);    // K^T dS^T
 // A byte offset added to a shared-memory descriptor's address field (16-byte units).
 __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
 }  // namespace bwd
+
+// A work unit: (batch, head), key tile and its 128-key chunk (flat-key mode: the 128-row key
+// chunk kt and the part of the query chunks).
+struct BwdUnit {
+  int bh, kt, ku, part;
+};
+
+template <bool kFlatK>
+__device__ __forceinline__ BwdUnit bwd_unit(const BwdBf16Params& p, int u) {
+  BwdUnit x;
+  if constexpr (kFlatK) {
+    const int nk = (p.Lk + 127) / 128, per_bh = nk * p.n_split;
+    x.bh = u / per_bh;
+    const int rem = u % per_bh;
+    x.part = rem / nk;
+    x.kt = rem % nk;
+    x.ku = 0;
+  } else {
+    x.ku = u % p.KU;
+    x.kt = (u / p.KU) % p.n_tiles;
+    x.bh = u / (p.KU * p.n_tiles);
+    x.part = 0;
+  }
+  return x;
+}
+
+// The unit's 64-query chunks: nm main chunks (the query tiles of CSR row kt of the inverse
+// plan from entry row0, or flat chunks from c0), then nx chunks of the extra queries.
+struct BwdChunks {
+  int row0, c0, nm, nx;
+};
+
+template <bool kFlatK>
+__device__ __forceinline__ BwdChunks bwd_chunks(const BwdBf16Params& p, const BwdUnit& x) {
+  BwdChunks q;
+  const int nx = (p.Lxq + 63) / 64;
+  if constexpr (kFlatK) {
+    const int nqm = (p.Nq + 63) / 64, per = (nqm + p.n_split - 1) / p.n_split;
+    q.row0 = 0;
+    q.c0 = x.part * per;
+    q.nm = max(min(per, nqm - q.c0), 0);
+    q.nx = x.part == 0 ? nx : 0;
+  } else {
+    const int32_t* rp = p.row_ptr + static_cast<int64_t>(x.bh) * p.rp_head_stride + x.kt;
+    q.row0 = rp[0];
+    q.c0 = 0;
+    q.nm = (rp[1] - rp[0]) * p.QS;
+    q.nx = nx;
+  }
+  return q;
+}
+
+// Query rows present in the unit's chunk c (a flat sequence's last chunk can be partial).
+template <bool kFlatK>
+__device__ __forceinline__ int bwd_qvalid(const BwdBf16Params& p, const BwdChunks& q, int c) {
+  if (c < q.nm) return kFlatK ? min(p.Nq - 64 * (q.c0 + c), 64) : 64;
+  return min(p.Lxq - 64 * (c - q.nm), 64);
+}
 
 __device__ __forceinline__ int64_t chunk_row_token(int r, int t0, int h0, int w0, int th, int tw, int H, int W) {
   const int lw = r % tw, lh = (r / tw) % th, lt = r / (tw * th);
@@ -98,6 +167,47 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __res
   if (row < rows && part == 0) delta[row] = s;
 }
 
+// bwd_preprocess for flat rows ([B*heads, L, 128]) whose LSE and D are read by 64-row TMA
+// boxes: D and a copy of the LSE go to [B*heads, Lp] arrays (Lp a multiple of 64, so every
+// box starts 16-byte aligned) with zeros past L; the fp32 dQ accumulator [B*heads, L, 128]
+// is zeroed.
+__global__ void __launch_bounds__(256) bwd_preprocess_flat(const __nv_bfloat16* __restrict__ o,
+                                                           const __nv_bfloat16* __restrict__ dout,
+                                                           const float* __restrict__ lse, float* __restrict__ delta_pad,
+                                                           float* __restrict__ lse_pad, float* __restrict__ dq_acc,
+                                                           int L, int Lp, int64_t BH) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 16;
+  const int part = threadIdx.x % 16;
+  const bool in = r < BH * Lp;
+  const int64_t bh = in ? r / Lp : 0;
+  const int i = in ? static_cast<int>(r % Lp) : L;
+  const bool live = in && i < L;
+  const int64_t row = bh * L + i;
+  float s = 0.f;
+  if (live) {
+    const uint4 a = reinterpret_cast<const uint4*>(o + row * 128)[part];
+    const uint4 b = reinterpret_cast<const uint4*>(dout + row * 128)[part];
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 x = __bfloat1622float2(pa[k]);
+      const float2 y = __bfloat1622float2(pb[k]);
+      s = fmaf(x.x, y.x, s);
+      s = fmaf(x.y, y.y, s);
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * 128) + part * 2;
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int o2 = 8; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
+  if (in && part == 0) {
+    delta_pad[r] = s;
+    lse_pad[r] = live ? lse[row] : 0.f;
+  }
+}
+
 __global__ void __launch_bounds__(256) bwd_dq_convert(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
                                                       float scale, int64_t n8) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -110,6 +220,24 @@ __global__ void __launch_bounds__(256) bwd_dq_convert(const float* __restrict__ 
   v.z = pack_bf16x2(b.x * scale, b.y * scale);
   v.w = pack_bf16x2(b.z * scale, b.w * scale);
   reinterpret_cast<uint4*>(dq)[i] = v;
+}
+
+// dK = scale * sum of the parts' dK, dV = sum of their dV (fp32 parts of flat keys), bf16.
+__global__ void __launch_bounds__(256) bwd_kv_combine(const float* __restrict__ dk_part,
+                                                      const float* __restrict__ dv_part, int n_parts,
+                                                      int64_t part_stride, float scale, int64_t n4,
+                                                      __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+  for (int j = 0; j < n_parts; ++j) {
+    const float4 x = reinterpret_cast<const float4*>(dk_part + j * part_stride)[i];
+    const float4 y = reinterpret_cast<const float4*>(dv_part + j * part_stride)[i];
+    a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+    b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+  }
+  reinterpret_cast<uint2*>(dk)[i] = make_uint2(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale));
+  reinterpret_cast<uint2*>(dv)[i] = make_uint2(pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
 
 // Persistent, warp-specialised backward; one CTA per SM, one 128-key chunk of a key tile
@@ -129,10 +257,17 @@ __global__ void __launch_bounds__(256) bwd_dq_convert(const float* __restrict__ 
 //               the end of a unit, one thread per key row writes dV and scale * dK as bf16.
 // Barriers advance at most one phase ahead of their waiters (each refill of a buffer waits
 // for the previous consumer), so waiting by phase parity is unambiguous.
+//
+// kFlatK: the keys and the main queries are flat sequences (rank-3 / rank-2 maps); rows past
+// the end of either load as zeros and get P = dS = 0, and their gradients are not written.
+// Extra queries (Lxq > 0, flat maps tmQx, tmDOx, tmLsex, tmDx) follow every unit's own.
+template <bool kFlatK>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmLse, const __grid_constant__ CUtensorMap tmD,
+                    const __grid_constant__ CUtensorMap tmQx, const __grid_constant__ CUtensorMap tmDOx,
+                    const __grid_constant__ CUtensorMap tmLsex, const __grid_constant__ CUtensorMap tmDx,
                     BwdBf16Params p) {
   using namespace bwd;
   extern __shared__ uint8_t smem_raw[];
@@ -164,6 +299,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     tma_prefetch_map(&tmDO);
     tma_prefetch_map(&tmLse);
     tma_prefetch_map(&tmD);
+    if (p.Lxq > 0) {
+      tma_prefetch_map(&tmQx);
+      tma_prefetch_map(&tmDOx);
+      tma_prefetch_map(&tmLsex);
+      tma_prefetch_map(&tmDx);
+    }
     mbar_init(kv_full, 1);
     mbar_init(kv_free, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -181,7 +322,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     *abort = 0;
     fence_mbar_init();
   }
-  if (tid < 64) {
+  if (!kFlatK && tid < 64) {
     // token offset of row n of a 64-query chunk box, relative to the box origin
     const int lw = tid % p.tw, lh = (tid / p.tw) % p.th, lt = tid / (p.tw * p.th);
     rel[tid] = (lt * p.H + lh) * p.W + lw;
@@ -196,48 +337,61 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tDV = tmem, tDK = tmem + 128, tS = tmem + 256, tDP = tmem + 384;
 
-  // unit u -> (bh, key tile, 128-key chunk); its query chunks come from CSR row kt
-  auto unit_of = [&](int u, int& bh, int& kt, int& ku) {
-    ku = u % p.KU;
-    kt = (u / p.KU) % p.n_tiles;
-    bh = u / (p.KU * p.n_tiles);
-  };
-
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int ld = 0, uc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        int bh, kt, ku;
-        unit_of(u, bh, kt, ku);
-        const int row0 = p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt], n = (p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt + 1] - row0) * p.QS;
+        const BwdUnit x = bwd_unit<kFlatK>(p, u);
+        const BwdChunks qc = bwd_chunks<kFlatK>(p, x);
+        const int bh = x.bh, n = qc.nm + qc.nx;
         if (n == 0) continue;
         ok = mbar_wait(kv_free, (uc & 1) ^ 1, abort, 50);
         if (!ok) break;
         ++uc;
-        const int k_t0 = (kt / (p.G1 * p.G2)) * p.tt + ku * p.kcs;
-        const int k_h0 = ((kt / p.G2) % p.G1) * p.th, k_w0 = (kt % p.G2) * p.tw;
         mbar_arrive_expect_tx(kv_full, 2 * kKBytes);
-        tma_load_5d(smem + kOffK, &tmK, kv_full, 0, k_w0, k_h0, k_t0, bh);
-        tma_load_5d(smem + kOffK + kKHalf, &tmK, kv_full, 64, k_w0, k_h0, k_t0, bh);
-        tma_load_5d(smem + kOffV, &tmV, kv_full, 0, k_w0, k_h0, k_t0, bh);
-        tma_load_5d(smem + kOffV + kKHalf, &tmV, kv_full, 64, k_w0, k_h0, k_t0, bh);
+        if constexpr (kFlatK) {  // rows past Lk load as zeros
+          tma_load_3d(smem + kOffK, &tmK, kv_full, 0, 128 * x.kt, bh);
+          tma_load_3d(smem + kOffK + kKHalf, &tmK, kv_full, 64, 128 * x.kt, bh);
+          tma_load_3d(smem + kOffV, &tmV, kv_full, 0, 128 * x.kt, bh);
+          tma_load_3d(smem + kOffV + kKHalf, &tmV, kv_full, 64, 128 * x.kt, bh);
+        } else {
+          const int k_t0 = (x.kt / (p.G1 * p.G2)) * p.tt + x.ku * p.kcs;
+          const int k_h0 = ((x.kt / p.G2) % p.G1) * p.th, k_w0 = (x.kt % p.G2) * p.tw;
+          tma_load_5d(smem + kOffK, &tmK, kv_full, 0, k_w0, k_h0, k_t0, bh);
+          tma_load_5d(smem + kOffK + kKHalf, &tmK, kv_full, 64, k_w0, k_h0, k_t0, bh);
+          tma_load_5d(smem + kOffV, &tmV, kv_full, 0, k_w0, k_h0, k_t0, bh);
+          tma_load_5d(smem + kOffV + kKHalf, &tmV, kv_full, 64, k_w0, k_h0, k_t0, bh);
+        }
         for (int c = 0; c < n && ok; ++c, ++ld) {
-          const int qi = p.q_tiles[row0 + c / p.QS], qs = c % p.QS;
-          const int q_t0 = (qi / (p.G1 * p.G2)) * p.tt + qs * p.qcs;
-          const int q_h0 = ((qi / p.G2) % p.G1) * p.th, q_w0 = (qi % p.G2) * p.tw;
           const int st = ld % kStages;
           ok = mbar_wait(ld_empty + st, ((ld / kStages) & 1) ^ 1, abort, 51);
           if (!ok) break;
           uint8_t* dst = smem + kOffStage + st * kStageBytes;
           mbar_arrive_expect_tx(ld_full + st, 2 * kQBytes + 512);
-          tma_load_5d(dst, &tmQ, ld_full + st, 0, q_w0, q_h0, q_t0, bh);
-          tma_load_5d(dst + kQHalf, &tmQ, ld_full + st, 64, q_w0, q_h0, q_t0, bh);
-          tma_load_5d(dst + kQBytes, &tmDO, ld_full + st, 0, q_w0, q_h0, q_t0, bh);
-          tma_load_5d(dst + kQBytes + kQHalf, &tmDO, ld_full + st, 64, q_w0, q_h0, q_t0, bh);
-          tma_load_4d(dst + 2 * kQBytes, &tmLse, ld_full + st, q_w0, q_h0, q_t0, bh);
-          tma_load_4d(dst + 2 * kQBytes + 512, &tmD, ld_full + st, q_w0, q_h0, q_t0, bh);
+          if (c >= qc.nm || kFlatK) {  // flat rows (past the end: zeros)
+            const bool extra = c >= qc.nm;
+            const int row = extra ? 64 * (c - qc.nm) : 64 * (qc.c0 + c);
+            const CUtensorMap* mq = extra ? &tmQx : &tmQ;
+            const CUtensorMap* mdo = extra ? &tmDOx : &tmDO;
+            tma_load_3d(dst, mq, ld_full + st, 0, row, bh);
+            tma_load_3d(dst + kQHalf, mq, ld_full + st, 64, row, bh);
+            tma_load_3d(dst + kQBytes, mdo, ld_full + st, 0, row, bh);
+            tma_load_3d(dst + kQBytes + kQHalf, mdo, ld_full + st, 64, row, bh);
+            tma_load_2d(dst + 2 * kQBytes, extra ? &tmLsex : &tmLse, ld_full + st, row, bh);
+            tma_load_2d(dst + 2 * kQBytes + 512, extra ? &tmDx : &tmD, ld_full + st, row, bh);
+          } else {
+            const int qi = p.q_tiles[qc.row0 + c / p.QS], qs = c % p.QS;
+            const int q_t0 = (qi / (p.G1 * p.G2)) * p.tt + qs * p.qcs;
+            const int q_h0 = ((qi / p.G2) % p.G1) * p.th, q_w0 = (qi % p.G2) * p.tw;
+            tma_load_5d(dst, &tmQ, ld_full + st, 0, q_w0, q_h0, q_t0, bh);
+            tma_load_5d(dst + kQHalf, &tmQ, ld_full + st, 64, q_w0, q_h0, q_t0, bh);
+            tma_load_5d(dst + kQBytes, &tmDO, ld_full + st, 0, q_w0, q_h0, q_t0, bh);
+            tma_load_5d(dst + kQBytes + kQHalf, &tmDO, ld_full + st, 64, q_w0, q_h0, q_t0, bh);
+            tma_load_4d(dst + 2 * kQBytes, &tmLse, ld_full + st, q_w0, q_h0, q_t0, bh);
+            tma_load_4d(dst + 2 * kQBytes + 512, &tmD, ld_full + st, q_w0, q_h0, q_t0, bh);
+          }
         }
       }
     }
@@ -254,9 +408,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       int ld = 0, uc = 0, sc = 0, pc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        int bh, kt, ku;
-        unit_of(u, bh, kt, ku);
-        const int n = (p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt + 1] - p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt]) * p.QS;
+        const BwdChunks qc = bwd_chunks<kFlatK>(p, bwd_unit<kFlatK>(p, u));
+        const int n = qc.nm + qc.nx;
         if (n == 0) continue;
         ok = __all_sync(0xffffffffu, mbar_wait(kv_full, uc & 1, abort, 60));
         if (!ok) break;
@@ -326,10 +479,14 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     int cc = 0, ld = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      int bh, kt, ku;
-      unit_of(u, bh, kt, ku);
-      const int n = (p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt + 1] - p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt]) * p.QS;
+      const BwdUnit x = bwd_unit<kFlatK>(p, u);
+      const BwdChunks qc = bwd_chunks<kFlatK>(p, x);
+      const int n = qc.nm + qc.nx;
+      // flat keys: this thread's key row may lie past the end (zeros, no gradient)
+      const bool k_ok = !kFlatK || 128 * x.kt + m < p.Lk;
       for (int c = 0; c < n; ++c, ++cc, ++ld) {
+        const int nvq = bwd_qvalid<kFlatK>(p, qc, c);
+        const bool masked = !k_ok || nvq < 64;  // P = dS = 0 for missing keys and queries
         const int b = cc & 1;
         ok = mbar_wait(s_full + b, (cc >> 1) & 1, abort, 70);
         if (ok) ok = mbar_wait(ld_full + ld % kStages, (ld / kStages) & 1, abort, 71);
@@ -348,9 +505,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int n0 = 8 * g + 2 * e;
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[n0]), p.scale_log2, -lse[n0] * 1.4426950408889634f));
-            const float p1 =
-                ex2_approx(fmaf(__uint_as_float(sr[n0 + 1]), p.scale_log2, -lse[n0 + 1] * 1.4426950408889634f));
+            float p0 = ex2_approx(fmaf(__uint_as_float(sr[n0]), p.scale_log2, -lse[n0] * 1.4426950408889634f));
+            float p1 = ex2_approx(fmaf(__uint_as_float(sr[n0 + 1]), p.scale_log2, -lse[n0 + 1] * 1.4426950408889634f));
+            if (masked) {
+              if (!k_ok || n0 >= nvq) p0 = 0.f;
+              if (!k_ok || n0 + 1 >= nvq) p1 = 0.f;
+            }
             pk[e] = pack_bf16x2(p0, p1);
             dk2[e] = pack_bf16x2(p0 * (__uint_as_float(dr[n0]) - dd[n0]), p1 * (__uint_as_float(dr[n0 + 1]) - dd[n0 + 1]));
           }
@@ -379,9 +539,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     int cc = 0, uc = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      int bh, kt, ku;
-      unit_of(u, bh, kt, ku);
-      const int row0 = p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt], n = (p.row_ptr[static_cast<int64_t>(bh) * p.rp_head_stride + kt + 1] - row0) * p.QS;
+      const BwdUnit x = bwd_unit<kFlatK>(p, u);
+      const BwdChunks qc = bwd_chunks<kFlatK>(p, x);
+      const int bh = x.bh, kt = x.kt, ku = x.ku, n = qc.nm + qc.nx;
       const int64_t slice = static_cast<int64_t>(bh) * p.N;
       for (int c = 0; c < n; ++c, ++cc) {
         const int b = cc & 1;
@@ -394,20 +554,46 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_free + b);
-        const int qi = p.q_tiles[row0 + c / p.QS], qs = c % p.QS;
-        const int q_t0 = (qi / (p.G1 * p.G2)) * p.tt + qs * p.qcs;
-        const int q_h0 = ((qi / p.G2) % p.G1) * p.th, q_w0 = (qi % p.G2) * p.tw;
-        float* base = p.dq_acc + (slice + (static_cast<int64_t>(q_t0) * p.H + q_h0) * p.W + q_w0) * 128 + t;
+        if (c >= qc.nm || kFlatK) {  // flat query rows: consecutive, the last chunk maybe partial
+          const bool extra = c >= qc.nm;
+          const int nvq = bwd_qvalid<kFlatK>(p, qc, c);
+          float* base = extra ? p.dq_acc_x + (static_cast<int64_t>(bh) * p.Lxq + 64 * (c - qc.nm)) * 128 + t
+                              : p.dq_acc + (static_cast<int64_t>(bh) * p.Nq + 64 * (qc.c0 + c)) * 128 + t;
 #pragma unroll
-        for (int nn = 0; nn < 64; ++nn) atomicAdd(base + static_cast<int64_t>(rel[nn]) * 128, __uint_as_float(r[nn]));
+          for (int nn = 0; nn < 64; ++nn)
+            if (nn < nvq) atomicAdd(base + static_cast<int64_t>(nn) * 128, __uint_as_float(r[nn]));
+        } else {
+          const int qi = p.q_tiles[qc.row0 + c / p.QS], qs = c % p.QS;
+          const int q_t0 = (qi / (p.G1 * p.G2)) * p.tt + qs * p.qcs;
+          const int q_h0 = ((qi / p.G2) % p.G1) * p.th, q_w0 = (qi % p.G2) * p.tw;
+          float* base = p.dq_acc + (slice + (static_cast<int64_t>(q_t0) * p.H + q_h0) * p.W + q_w0) * 128 + t;
+#pragma unroll
+          for (int nn = 0; nn < 64; ++nn) atomicAdd(base + static_cast<int64_t>(rel[nn]) * 128, __uint_as_float(r[nn]));
+        }
       }
       if (!ok) break;
-      // dV and scale * dK of the unit's 128 keys; zeros for a key tile no window holds
-      const int k_t0 = (kt / (p.G1 * p.G2)) * p.tt + ku * p.kcs;
-      const int k_h0 = ((kt / p.G2) % p.G1) * p.th, k_w0 = (kt % p.G2) * p.tw;
-      const int64_t ktok = chunk_row_token(t, k_t0, k_h0, k_w0, p.th, p.tw, p.H, p.W);
+      // dV and scale * dK of the unit's 128 keys; zeros for a key tile no window holds.
+      // Flat keys: fp32 partial sums of this part (unscaled dK), rows past Lk not written.
+      int64_t ktok;
+      bool k_row_ok = true;
+      if constexpr (kFlatK) {
+        ktok = 128 * static_cast<int64_t>(kt) + t;
+        k_row_ok = ktok < p.Lk;
+        if (!k_row_ok) ktok = 0;
+      } else {
+        const int k_t0 = (kt / (p.G1 * p.G2)) * p.tt + ku * p.kcs;
+        const int k_h0 = ((kt / p.G2) % p.G1) * p.th, k_w0 = (kt % p.G2) * p.tw;
+        ktok = chunk_row_token(t, k_t0, k_h0, k_w0, p.th, p.tw, p.H, p.W);
+      }
       uint4* dv_dst = reinterpret_cast<uint4*>(p.dv + (slice + ktok) * 128);
       uint4* dk_dst = reinterpret_cast<uint4*>(p.dk + (slice + ktok) * 128);
+      float4* dvp = nullptr;
+      float4* dkp = nullptr;
+      if constexpr (kFlatK) {
+        const int64_t o = static_cast<int64_t>(x.part) * p.part_stride + (static_cast<int64_t>(bh) * p.Lk + ktok) * 128;
+        dvp = reinterpret_cast<float4*>(p.dv_part + o);
+        dkp = reinterpret_cast<float4*>(p.dk_part + o);
+      }
       if (n > 0) {
         ok = mbar_wait(dkv_full, uc & 1, abort, 81);
         ok = __all_sync(0xffffffffu, ok);
@@ -424,19 +610,31 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) a[j] = bb[j] = 0u;
         }
+        if constexpr (kFlatK) {
+          if (k_row_ok) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 x, y;
-          x.x = pack_bf16x2(__uint_as_float(a[8 * j + 0]), __uint_as_float(a[8 * j + 1]));
-          x.y = pack_bf16x2(__uint_as_float(a[8 * j + 2]), __uint_as_float(a[8 * j + 3]));
-          x.z = pack_bf16x2(__uint_as_float(a[8 * j + 4]), __uint_as_float(a[8 * j + 5]));
-          x.w = pack_bf16x2(__uint_as_float(a[8 * j + 6]), __uint_as_float(a[8 * j + 7]));
-          y.x = pack_bf16x2(__uint_as_float(bb[8 * j + 0]) * p.scale, __uint_as_float(bb[8 * j + 1]) * p.scale);
-          y.y = pack_bf16x2(__uint_as_float(bb[8 * j + 2]) * p.scale, __uint_as_float(bb[8 * j + 3]) * p.scale);
-          y.z = pack_bf16x2(__uint_as_float(bb[8 * j + 4]) * p.scale, __uint_as_float(bb[8 * j + 5]) * p.scale);
-          y.w = pack_bf16x2(__uint_as_float(bb[8 * j + 6]) * p.scale, __uint_as_float(bb[8 * j + 7]) * p.scale);
-          dv_dst[g * 4 + j] = x;
-          dk_dst[g * 4 + j] = y;
+            for (int j = 0; j < 8; ++j) {
+              dvp[g * 8 + j] = make_float4(__uint_as_float(a[4 * j]), __uint_as_float(a[4 * j + 1]),
+                                           __uint_as_float(a[4 * j + 2]), __uint_as_float(a[4 * j + 3]));
+              dkp[g * 8 + j] = make_float4(__uint_as_float(bb[4 * j]), __uint_as_float(bb[4 * j + 1]),
+                                           __uint_as_float(bb[4 * j + 2]), __uint_as_float(bb[4 * j + 3]));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 x, y;
+            x.x = pack_bf16x2(__uint_as_float(a[8 * j + 0]), __uint_as_float(a[8 * j + 1]));
+            x.y = pack_bf16x2(__uint_as_float(a[8 * j + 2]), __uint_as_float(a[8 * j + 3]));
+            x.z = pack_bf16x2(__uint_as_float(a[8 * j + 4]), __uint_as_float(a[8 * j + 5]));
+            x.w = pack_bf16x2(__uint_as_float(a[8 * j + 6]), __uint_as_float(a[8 * j + 7]));
+            y.x = pack_bf16x2(__uint_as_float(bb[8 * j + 0]) * p.scale, __uint_as_float(bb[8 * j + 1]) * p.scale);
+            y.y = pack_bf16x2(__uint_as_float(bb[8 * j + 2]) * p.scale, __uint_as_float(bb[8 * j + 3]) * p.scale);
+            y.z = pack_bf16x2(__uint_as_float(bb[8 * j + 4]) * p.scale, __uint_as_float(bb[8 * j + 5]) * p.scale);
+            y.w = pack_bf16x2(__uint_as_float(bb[8 * j + 6]) * p.scale, __uint_as_float(bb[8 * j + 7]) * p.scale);
+            dv_dst[g * 4 + j] = x;
+            dk_dst[g * 4 + j] = y;
+          }
         }
       }
       if (n > 0) {
