@@ -356,7 +356,26 @@ def run_prefix_workload(dsa, w: Workload, device, steps: int, warmup: int):
         raise RuntimeError(f"device status {st} after the text-prefix forward")
     N = w.n_tokens
     flops = 4.0 * w.B * w.heads * w.d * (N * w.keys_per_query + 2.0 * N * L + float(L) * L)
-    return {"fwd_ms": ms, "fwd_tflops": flops / (ms * 1e-3) / 1e12, "L_text": L}
+    res = {"fwd_ms": ms, "fwd_tflops": flops / (ms * 1e-3) / 1e12, "L_text": L}
+    # backward of the same call (2.5x the forward's FLOPs), dO drawn like the inputs
+    out, lse, out_t, lse_t = dsa.forward_prefix(q, k, v, offsets, qt, kt, vt, w.tile, w.window, w.scale, ws=ws,
+                                                stream=stream)
+    g = torch.Generator(device=device).manual_seed(9000 + w.seed)
+    do = torch.randn(q.shape, generator=g, device=device, dtype=torch.float32).to(q.dtype)
+    do_t = torch.randn(qt.shape, generator=g, device=device, dtype=torch.float32).to(q.dtype)
+    ws_b = torch.empty(dsa.prefix_bwd_workspace_size(p, L), dtype=torch.uint8, device=device)
+
+    def bwd():
+        dsa.backward_prefix(q, k, v, out, lse, do, offsets, qt, kt, vt, out_t, lse_t, do_t, w.tile, w.window, w.scale,
+                            ws=ws_b, stream=stream)
+
+    bwd()
+    b_ms = time_steps(bwd, steps, warmup, stream, record=False)
+    st = dsa.device_status(stream)
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st} after the text-prefix backward")
+    res.update({"bwd_ms": b_ms, "bwd_tflops": 2.5 * flops / (b_ms * 1e-3) / 1e12})
+    return res
 
 
 def run_dense_map_workload(dsa, w: Workload, device, steps: int, warmup: int):

@@ -352,7 +352,8 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.scale_log2 = p->scale * 1.4426950408889634f;
   bp.n_units = static_cast<int>(g.BH * bp.S * g.n_tiles);
   const bool map_mode = bmap != nullptr;
-  auto kernel = map_mode ? dsa::fwd_bf16_kernel<dsa::fwd::kModeMap> : dsa::fwd_bf16_kernel<dsa::fwd::kModeFwd>;
+  auto kernel = map_mode ? dsa::fwd_bf16_kernel<dsa::fwd::kModeMap>
+                         : (bp.Lx > 0 ? dsa::fwd_bf16_kernel<dsa::fwd::kModeFwdX> : dsa::fwd_bf16_kernel<dsa::fwd::kModeFwd>);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::fwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
   // the kernel's setmaxnreg split needs exactly the registers it was compiled for at launch
@@ -430,7 +431,7 @@ struct ExtraQueries {
   int L, Lp;
 };
 
-template <bool kFlatK>
+template <bool kFlatK, bool kExtra>
 dsa_status_t launch_bwd_kernel(const dsa::BwdBf16Params& bp, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tlse,
                                const CUtensorMap& tdel, const ExtraQueries* x, int64_t BH, cudaStream_t s) {
@@ -440,7 +441,7 @@ dsa_status_t launch_bwd_kernel(const dsa::BwdBf16Params& bp, const CUtensorMap& 
         !make_vec_map(&tlsex, x->lse_pad, BH, x->Lp) || !make_vec_map(&tdx, x->delta_pad, BH, x->Lp))
       return DSA_ERR_CUDA;
   }
-  auto kernel = dsa::bwd_bf16_kernel<kFlatK>;
+  auto kernel = dsa::bwd_bf16_kernel<kFlatK, kExtra>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::bwd::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
   int sms = 0;
@@ -501,7 +502,8 @@ dsa_status_t launch_bwd(const dsa_problem_t* p, const Geom& g, const void* q, co
     bp.Lxq = x->L;
     bp.dq_acc_x = x->dq_acc;
   }
-  st = launch_bwd_kernel<false>(bp, tq, tk, tv, tdo, tlse, tdel, x, g.BH, s);
+  st = bp.Lxq > 0 ? launch_bwd_kernel<false, true>(bp, tq, tk, tv, tdo, tlse, tdel, x, g.BH, s)
+                  : launch_bwd_kernel<false, false>(bp, tq, tk, tv, tdo, tlse, tdel, x, g.BH, s);
   if (st != DSA_OK || !convert_dq) return st;
   const int64_t n8 = rows * p->d / 8;
   dsa::bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
@@ -1057,7 +1059,7 @@ dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k
   bp.n_units = static_cast<int>(g.BH * ((L_text + 127) / 128) * ws.n_split);
   bp.tt = bp.th = bp.tw = 1;  // no tile geometry in the flat-key mode
   bp.T = bp.H = bp.W = 1;
-  st = launch_bwd_kernel<true>(bp, tq, tk, tv, tdo, tlse, tdel, &xq, g.BH, s);
+  st = launch_bwd_kernel<true, true>(bp, tq, tk, tv, tdo, tlse, tdel, &xq, g.BH, s);
   if (st != DSA_OK) return st;
   // dQ of both token types, dK and dV of the text
   const int64_t n8v = g.BH * g.N * 128 / 8, n8t = g.BH * static_cast<int64_t>(L_text) * 128 / 8;

@@ -106,10 +106,10 @@ struct BwdChunks {
   int row0, c0, nm, nx;
 };
 
-template <bool kFlatK>
+template <bool kFlatK, bool kExtra>
 __device__ __forceinline__ BwdChunks bwd_chunks(const BwdBf16Params& p, const BwdUnit& x) {
   BwdChunks q;
-  const int nx = (p.Lxq + 63) / 64;
+  const int nx = kExtra ? (p.Lxq + 63) / 64 : 0;
   if constexpr (kFlatK) {
     const int nqm = (p.Nq + 63) / 64, per = (nqm + p.n_split - 1) / p.n_split;
     q.row0 = 0;
@@ -127,8 +127,9 @@ __device__ __forceinline__ BwdChunks bwd_chunks(const BwdBf16Params& p, const Bw
 }
 
 // Query rows present in the unit's chunk c (a flat sequence's last chunk can be partial).
-template <bool kFlatK>
+template <bool kFlatK, bool kExtra>
 __device__ __forceinline__ int bwd_qvalid(const BwdBf16Params& p, const BwdChunks& q, int c) {
+  if (!kFlatK && !kExtra) return 64;
   if (c < q.nm) return kFlatK ? min(p.Nq - 64 * (q.c0 + c), 64) : 64;
   return min(p.Lxq - 64 * (c - q.nm), 64);
 }
@@ -260,8 +261,9 @@ __global__ void __launch_bounds__(256) bwd_kv_combine(const float* __restrict__ 
 //
 // kFlatK: the keys and the main queries are flat sequences (rank-3 / rank-2 maps); rows past
 // the end of either load as zeros and get P = dS = 0, and their gradients are not written.
-// Extra queries (Lxq > 0, flat maps tmQx, tmDOx, tmLsex, tmDx) follow every unit's own.
-template <bool kFlatK>
+// kExtra: extra queries (p.Lxq of them, flat maps tmQx, tmDOx, tmLsex, tmDx) follow every
+// unit's own.
+template <bool kFlatK, bool kExtra>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -299,7 +301,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     tma_prefetch_map(&tmDO);
     tma_prefetch_map(&tmLse);
     tma_prefetch_map(&tmD);
-    if (p.Lxq > 0) {
+    if (kExtra && p.Lxq > 0) {
       tma_prefetch_map(&tmQx);
       tma_prefetch_map(&tmDOx);
       tma_prefetch_map(&tmLsex);
@@ -344,7 +346,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const BwdUnit x = bwd_unit<kFlatK>(p, u);
-        const BwdChunks qc = bwd_chunks<kFlatK>(p, x);
+        const BwdChunks qc = bwd_chunks<kFlatK, kExtra>(p, x);
         const int bh = x.bh, n = qc.nm + qc.nx;
         if (n == 0) continue;
         ok = mbar_wait(kv_free, (uc & 1) ^ 1, abort, 50);
@@ -370,7 +372,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           if (!ok) break;
           uint8_t* dst = smem + kOffStage + st * kStageBytes;
           mbar_arrive_expect_tx(ld_full + st, 2 * kQBytes + 512);
-          if (c >= qc.nm || kFlatK) {  // flat rows (past the end: zeros)
+          if ((kExtra && c >= qc.nm) || kFlatK) {  // flat rows (past the end: zeros)
             const bool extra = c >= qc.nm;
             const int row = extra ? 64 * (c - qc.nm) : 64 * (qc.c0 + c);
             const CUtensorMap* mq = extra ? &tmQx : &tmQ;
@@ -408,7 +410,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       int ld = 0, uc = 0, sc = 0, pc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const BwdChunks qc = bwd_chunks<kFlatK>(p, bwd_unit<kFlatK>(p, u));
+        const BwdChunks qc = bwd_chunks<kFlatK, kExtra>(p, bwd_unit<kFlatK>(p, u));
         const int n = qc.nm + qc.nx;
         if (n == 0) continue;
         ok = __all_sync(0xffffffffu, mbar_wait(kv_full, uc & 1, abort, 60));
@@ -480,12 +482,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const BwdUnit x = bwd_unit<kFlatK>(p, u);
-      const BwdChunks qc = bwd_chunks<kFlatK>(p, x);
+      const BwdChunks qc = bwd_chunks<kFlatK, kExtra>(p, x);
       const int n = qc.nm + qc.nx;
       // flat keys: this thread's key row may lie past the end (zeros, no gradient)
       const bool k_ok = !kFlatK || 128 * x.kt + m < p.Lk;
       for (int c = 0; c < n; ++c, ++cc, ++ld) {
-        const int nvq = bwd_qvalid<kFlatK>(p, qc, c);
+        const int nvq = bwd_qvalid<kFlatK, kExtra>(p, qc, c);
         const bool masked = !k_ok || nvq < 64;  // P = dS = 0 for missing keys and queries
         const int b = cc & 1;
         ok = mbar_wait(s_full + b, (cc >> 1) & 1, abort, 70);
@@ -540,7 +542,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const BwdUnit x = bwd_unit<kFlatK>(p, u);
-      const BwdChunks qc = bwd_chunks<kFlatK>(p, x);
+      const BwdChunks qc = bwd_chunks<kFlatK, kExtra>(p, x);
       const int bh = x.bh, kt = x.kt, ku = x.ku, n = qc.nm + qc.nx;
       const int64_t slice = static_cast<int64_t>(bh) * p.N;
       for (int c = 0; c < n; ++c, ++cc) {
@@ -554,9 +556,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_free + b);
-        if (c >= qc.nm || kFlatK) {  // flat query rows: consecutive, the last chunk maybe partial
+        if ((kExtra && c >= qc.nm) || kFlatK) {  // flat query rows: consecutive, the last chunk maybe partial
           const bool extra = c >= qc.nm;
-          const int nvq = bwd_qvalid<kFlatK>(p, qc, c);
+          const int nvq = bwd_qvalid<kFlatK, kExtra>(p, qc, c);
           float* base = extra ? p.dq_acc_x + (static_cast<int64_t>(bh) * p.Lxq + 64 * (c - qc.nm)) * 128 + t
                               : p.dq_acc + (static_cast<int64_t>(bh) * p.Nq + 64 * (qc.c0 + c)) * 128 + t;
 #pragma unroll

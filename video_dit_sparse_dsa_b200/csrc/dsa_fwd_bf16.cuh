@@ -122,9 +122,10 @@ constexpr uint32_t kPolyMask = 0x88u;
 __device__ __forceinline__ uint32_t col_s(int e) { return e ? 128u : 0u; }
 __device__ __forceinline__ uint32_t col_p(int e) { return e ? 256u : 0u; }
 
-// Kernel modes: the window / key-tile-list forward, its block-map pass, and dense attention
-// between flat token sequences (text tokens).
-constexpr int kModeFwd = 0, kModeMap = 1, kModeFlat = 2;
+// Kernel modes: the window / key-tile-list forward, its block-map pass, dense attention
+// between flat token sequences (text tokens), and the window forward with extra (text)
+// keys after every unit's own.
+constexpr int kModeFwd = 0, kModeMap = 1, kModeFlat = 2, kModeFwdX = 3;
 
 struct Unit {
   int bh, tile, sub;  // flat mode: tile = query chunk, sub = 0
@@ -162,10 +163,10 @@ struct Chunks {
   int c0, nm, nx;
 };
 
-template <bool kFlat>
+template <bool kFlat, bool kExtra>
 __device__ __forceinline__ Chunks unit_chunks(const FwdBf16Params& p, const Unit& x, int n_list) {
   Chunks k;
-  const int nx = (p.Lx + 127) / 128;
+  const int nx = kExtra ? (p.Lx + 127) / 128 : 0;
   if constexpr (kFlat) {
     const int n_main = (p.Lk + 127) / 128, per = (n_main + p.n_split - 1) / p.n_split;
     k.c0 = x.sub * per;
@@ -181,8 +182,9 @@ __device__ __forceinline__ Chunks unit_chunks(const FwdBf16Params& p, const Unit
 
 // Keys present in local chunk j of a unit: the last chunk of a flat sequence and of the
 // extra keys can be partial.
-template <bool kFlat>
+template <bool kFlat, bool kExtra>
 __device__ __forceinline__ int chunk_valid(const FwdBf16Params& p, const Chunks& k, int j) {
+  if (!kFlat && !kExtra) return 128;
   if (j < k.nm) return kFlat ? min(p.Lk - 128 * (k.c0 + j), 128) : 128;
   return min(p.Lx - 128 * (j - k.nm), 128);
 }
@@ -380,6 +382,7 @@ __device__ __forceinline__ void store_o(uint32_t tO, int groups, float inv, uint
 // recomputed with the same products and ring, without V, P.V, the row max or the epilogue.
 // kModeFlat: dense attention between flat sequences (rank-3 tensor maps [128, L, B*heads]):
 // every query chunk over every key chunk, the tail of the last key chunk masked.
+// kModeFwdX: kModeFwd with p.Lx extra (text) keys after every unit's own (maps tmKx, tmVx).
 template <int kMode>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -387,6 +390,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
                     const __grid_constant__ CUtensorMap tmVx, FwdBf16Params p) {
   using namespace fwd;
   constexpr bool kMap = kMode == kModeMap, kFlat = kMode == kModeFlat;
+  constexpr bool kExtra = kFlat || kMode == kModeFwdX;  // extra keys possible (p.Lx > 0)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
@@ -419,7 +423,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     tma_prefetch_map(&tmQ);
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
-    if (p.Lx > 0) {
+    if (kExtra && p.Lx > 0) {
       tma_prefetch_map(&tmKx);
       tma_prefetch_map(&tmVx);
     }
@@ -465,7 +469,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           const Unit x = kFlat ? decode_flat(p, u) : decode(p, u);
           int n_list = 0;
           const int32_t* kv = kFlat ? nullptr : unit_keys(p, x.bh, x.tile, n_list);
-          const Chunks ck = unit_chunks<kFlat>(p, x, n_list);
+          const Chunks ck = unit_chunks<kFlat, kExtra>(p, x, n_list);
           const int n_chunks = ck.nm + ck.nx, n_steps = (n_chunks + 1) / 2;
           if (n_chunks == 0) continue;  // nothing to load: the softmax warps write O = 0
           if (is_k) {
@@ -496,7 +500,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             mbar_arrive_expect_tx(full, nb * kTileBytes);
             for (int b = 0; b < nb; ++b) {
               const int jc = is_k ? 2 * j + b : j;  // the unit's chunk
-              if (jc >= ck.nm) {  // extra keys (rows past Lx load as zeros and are masked)
+              if (kExtra && jc >= ck.nm) {  // extra keys (rows past Lx load as zeros and are masked)
                 const int row = 128 * (jc - ck.nm);
                 if (is_k) {
                   uint8_t* dst = smem + kOffK + st * kStageBytes + b * kHalfBytes;
@@ -551,7 +555,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         int n_list = 0;
         const Unit xm = kFlat ? decode_flat(p, u) : decode(p, u);
         if constexpr (!kFlat) unit_keys(p, xm.bh, xm.tile, n_list);
-        const Chunks ck = unit_chunks<kFlat>(p, xm, n_list);
+        const Chunks ck = unit_chunks<kFlat, kExtra>(p, xm, n_list);
         const int n_chunks = ck.nm + ck.nx, n_steps = (n_chunks + 1) / 2;
         if (n_chunks == 0) continue;
         ok = warp_wait(q_full, uc & 1, abort, 30);
@@ -679,7 +683,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const Unit x = kFlat ? decode_flat(p, u) : decode(p, u);
       int n_list = 0;
       if constexpr (!kFlat) unit_keys(p, x.bh, x.tile, n_list);
-      const Chunks ck = unit_chunks<kFlat>(p, x, n_list);
+      const Chunks ck = unit_chunks<kFlat, kExtra>(p, x, n_list);
       const int n_chunks = ck.nm + ck.nx, n_steps = (n_chunks + 1) / 2;
       // flat mode: part x.sub of the key chunks writes its own partial output
       const int64_t po = kFlat ? static_cast<int64_t>(x.sub) * p.part_out : 0;
@@ -707,8 +711,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         // keys present in this thread's columns (a flat sequence's or the extra keys' last
         // chunk may be partial): chunk 2t + i of a full step, half i of chunk 2t otherwise
         const bool full = 2 * t + 1 < n_chunks;
-        const int nvalid = full ? chunk_valid<kFlat>(p, ck, 2 * t + i)
-                                : min(max(chunk_valid<kFlat>(p, ck, 2 * t) - 64 * i, 0), 64);
+        const int nvalid = full ? chunk_valid<kFlat, kExtra>(p, ck, 2 * t + i)
+                                : min(max(chunk_valid<kFlat, kExtra>(p, ck, 2 * t) - 64 * i, 0), 64);
         if (full)
           need = softmax_step<128>(ok, tmem + col_s(e) + 128 * i + lane_off, tmem + col_p(e) + 64 * i + lane_off,
                                    s_read + e, p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id, nvalid);
