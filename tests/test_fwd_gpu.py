@@ -77,6 +77,10 @@ SMALL_BF16 = [
     Workload("bf16_small_dense", 1, 2, 128, (8, 8, 16), (4, 8, 8), (9, 9, 9), (0, 0), "bf16", 25),
     # 1x1x1 window: block-diagonal
     Workload("bf16_small_diag", 1, 2, 128, (8, 16, 16), (4, 8, 8), (1, 1, 1), (0, 0), "bf16", 26),
+    # a grid of one tile (every window is that tile, whatever the offsets)
+    Workload("bf16_one_tile", 1, 3, 128, (4, 8, 8), (4, 8, 8), (3, 3, 3), (-2, 2), "bf16", 27),
+    # many (batch, head) slices on a small grid: 160 of them
+    Workload("bf16_many_heads", 8, 20, 128, (4, 16, 8), (4, 8, 8), (1, 3, 1), (-1, 1), "bf16", 28),
 ]
 
 
