@@ -636,7 +636,8 @@ def main():
                         f"{src}_{burst:g}": 100 * fwd_tflops / burst},
         "roofline": {"bound": "tensor", "kernel": "fwd_bf16_kernel (timed with the planner, one dsa_fwd call)",
                      "achieved": fwd_tflops, "peak": burst, "peak_kind": f"{src} burst bf16", "unit": "TFLOP/s",
-                     "frac": fwd_tflops / burst, "traffic": fwd_traffic(w.name), "traffic_unit": "bytes per launch"},
+                     "frac": fwd_tflops / burst, "traffic": fwd_traffic(w.name), "traffic_unit": "bytes per launch",
+                     "peak_sustained": sustained, "frac_sustained": fwd_tflops / sustained},
         "e2e": e2e, "gpu_launches": res["launches_per_step"] * args.steps, "clocks": clocks,
         "cpu_baseline": cpu, "workloads": extra,
     }
