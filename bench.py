@@ -484,6 +484,14 @@ def oracle_sample_rate(w: Workload, target_s: float, max_tiles: int = 4096):
         threads, dt_s
 
 
+def workload_config(w: Workload, world: int) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": list(w.grid), "tile": list(w.tile),
+            "window": list(w.window), "offsets": list(w.offset_range), "keys_per_query": w.keys_per_query,
+            "pass": "fwd+bwd" if w.backward else "fwd", "l2": "inputs larger than L2 (no flush)",
+            "parallelism": f"independent problem per rank x{world}"}
+
+
 def reference_arm(args, w: Workload):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -500,8 +508,7 @@ def reference_arm(args, w: Workload):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops / (value * 1e12) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": list(w.grid),
-                       "tile": list(w.tile), "window": list(w.window), "pass": "fwd"},
+            "config": workload_config(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -628,10 +635,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": list(w.grid),
-                   "tile": list(w.tile), "window": list(w.window), "offsets": list(w.offset_range),
-                   "keys_per_query": w.keys_per_query, "pass": "fwd+bwd" if w.backward else "fwd",
-                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"independent problem per rank x{world}"},
+        "config": workload_config(w, world),
         "pct_of_peak": {"nominal_2250": 100 * fwd_tflops / NOMINAL_BF16_TFLOPS,
                         f"{src}_{burst:g}": 100 * fwd_tflops / burst},
         "roofline": {"bound": "tensor", "kernel": "fwd_bf16_kernel (timed with the planner, one dsa_fwd call)",
