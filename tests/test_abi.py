@@ -77,6 +77,8 @@ def _fwd(lib, p, **kw):
     (dict(tile=(4, 3, 8), grid=(16, 30, 32)), 2),  # a 128-token chunk is not whole (h, w) planes
     (dict(tile=(1, 8, 8), grid=(16, 32, 32)), 2),  # 64-token tile: no whole 128-token chunk
     (dict(d=96, dtype=dsa.DSA_F32), 2),      # fp32 path: d in {64, 128}
+    (dict(B=4096, heads=4096), 2),           # 2^31 or more 128-row units: past the kernel's int32 unit index
+    (dict(B=256, heads=512, d=64, dtype=dsa.DSA_F32, grid=(4, 8, 8), tile=(1, 4, 4)), 2),  # fp32 grid y > 65535
 ])
 def test_fwd_rejects_bad_problems(lib, kw, status):
     assert _fwd(lib, _prob(**kw)) == status
