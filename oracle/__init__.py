@@ -352,6 +352,83 @@ def backward_prefix(geo: Geometry, q, k, v, dout, offsets, q_text, k_text, v_tex
     return (tuple(o[:, :N].reshape(shape_v) for o in outs), tuple(o[:, N:].reshape(shape_t) for o in outs))
 
 
+def backward_prefix_sampled(geo: Geometry, q, k, v, dout, offsets, q_text, k_text, v_text, dout_text, h: int,
+                            q_rows, qt_rows, k_rows, kt_rows):
+    """Text-prefix backward of (b, head) h on selected rows only, from the definition: the
+    forward of every query row of the head (video rows through the C oracle over their window
+    and the text keys, text rows over every key) gives lse and O, D = rowsum(dO * O); then
+    dq of the selected video query rows q_rows and text query rows qt_rows over their key sets,
+    and dk, dv of the selected video key rows k_rows (over the video queries whose window
+    holds the key's tile, and every text query) and text key rows kt_rows (over every query).
+    Returns (dq[len(q_rows)], dq_text[len(qt_rows)], dk, dv [len(k_rows)], dk_text, dv_text
+    [len(kt_rows)]), each row [d], float64."""
+    N, d, sc = geo.n_tokens, geo.d, geo.scale
+    one = Geometry(1, 1, d, geo.grid, geo.tile, geo.window, geo.scale)
+    Q, K, V, dO = (_head_slice(t, geo, h) for t in (q, k, v, dout))
+    Qt, Kt, Vt, dOt = (_text_slice(t, geo, h) for t in (q_text, k_text, v_text, dout_text))
+    Lt = Qt.shape[0]
+    # forward of every video row of the head (window + text keys), in token order
+    sel = (np.zeros(geo.n_tiles, np.int32), np.arange(geo.n_tiles, dtype=np.int32))
+    as_head = [torch.from_numpy(a).reshape((1, 1) + geo.grid + (d,)) for a in (Q, K, V)]
+    out_t, lse_t = forward_prefix_tiles(one, *as_head, offsets, torch.from_numpy(Kt).reshape(1, 1, Lt, d),
+                                        torch.from_numpy(Vt).reshape(1, 1, Lt, d), sel)
+    tok = geo.tile_token_index().reshape(-1)
+    O = np.zeros((N, d))
+    lse = np.zeros(N)
+    O[tok] = out_t.reshape(-1, d)
+    lse[tok] = lse_t.reshape(-1)
+    D = (dO * O).sum(axis=1)
+    # text rows over every key (text first, then video)
+    keys, vals = np.concatenate([Kt, K]), np.concatenate([Vt, V])
+    st = sc * (Qt @ keys.T)
+    mx = st.max(axis=1, keepdims=True)
+    lse_x = mx[:, 0] + np.log(np.exp(st - mx).sum(axis=1))
+    Ot = np.exp(st - lse_x[:, None]) @ vals
+    Dt = (dOt * Ot).sum(axis=1)
+    # key sets of the video query tiles (the oracle's plan)
+    _, kv, _, _ = plan(geo.G, geo.window, offsets)
+    tile_of = np.zeros(N, np.int64)
+    tile_of[tok] = np.repeat(np.arange(geo.n_tiles), geo.tile_tokens)
+    tiles_tok = geo.tile_token_index()
+
+    def grad_rows(qv, dov, lsev, Dv, kk, vv):
+        """dq of query rows (one row per call) over keys kk, vv: P, dS and sum dS k."""
+        s = sc * (kk @ qv)
+        P = np.exp(s - lsev)
+        dS = P * (vv @ dov - Dv)
+        return sc * (dS @ kk)
+
+    dq = np.array([grad_rows(Q[n], dO[n], lse[n], D[n],
+                             np.concatenate([K[tiles_tok[kv[tile_of[n]]].reshape(-1)], Kt]),
+                             np.concatenate([V[tiles_tok[kv[tile_of[n]]].reshape(-1)], Vt])) for n in q_rows])
+    dq_t = np.array([grad_rows(Qt[j], dOt[j], lse_x[j], Dt[j], keys, vals) for j in qt_rows])
+
+    def key_grads(km, vm, qs, dos, lses, Ds):
+        """dk, dv of one key over the query rows qs (with their dO, lse, D)."""
+        s = sc * (qs @ km)
+        P = np.exp(s - lses)
+        dS = P * (dos @ vm - Ds)
+        return sc * (dS @ qs), P @ dos
+
+    dk, dv = [], []
+    for m in k_rows:
+        holders = np.nonzero((kv == tile_of[m]).any(axis=1))[0]  # query tiles whose window holds m
+        rows = tiles_tok[holders].reshape(-1)
+        qs = np.concatenate([Q[rows], Qt])
+        g = key_grads(K[m], V[m], qs, np.concatenate([dO[rows], dOt]), np.concatenate([lse[rows], lse_x]),
+                      np.concatenate([D[rows], Dt]))
+        dk.append(g[0])
+        dv.append(g[1])
+    dkt, dvt = [], []
+    Qall, dOall = np.concatenate([Q, Qt]), np.concatenate([dO, dOt])
+    lall, Dall = np.concatenate([lse, lse_x]), np.concatenate([D, Dt])
+    for j in kt_rows:
+        g = key_grads(Kt[j], Vt[j], Qall, dOall, lall, Dall)
+        dkt.append(g[0])
+        dvt.append(g[1])
+    return dq, dq_t, np.array(dk), np.array(dv), np.array(dkt), np.array(dvt)
+
+
 def backward_dq_tiles(geo: Geometry, q, k, v, dout, offsets, sel=None):
     """dq on (bh, query tile) pairs: [n_sel, tile_tokens, d] float64."""
     lib = _load()

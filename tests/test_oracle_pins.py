@@ -670,3 +670,21 @@ def test_prefix_backward_without_text_is_the_window_backward():
     for a, b in ((dq, rq), (dk, rk), (dv, rv)):
         np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
     assert dqt.size == 0
+
+
+def test_prefix_backward_sampled_rows_equal_the_full_oracle():
+    """The row-sampled prefix backward (used at full sizes) agrees with the full one."""
+    geo = oracle.Geometry(1, 2, 8, (4, 4, 6), (2, 2, 2), (2, 1, 2))
+    q, k, v, do = rand_inputs(geo, 51)
+    L = 6
+    qt, kt, vt = rand_text(geo, L, 52)
+    dot = rand_text(geo, L, 53)[0]
+    off = rand_offsets(geo, -2, 2, 54)
+    (dq, dk, dv), (dqt, dkt, dvt) = oracle.backward_prefix(geo, q, k, v, do, off, qt, kt, vt, dot)
+    N, h = geo.n_tokens, 1
+    qr, kr, tr = np.array([0, 7, N - 1]), np.array([3, 40, N - 2]), np.array([0, L - 1])
+    got = oracle.backward_prefix_sampled(geo, q, k, v, do, off, qt, kt, vt, dot, h, qr, tr, kr, tr)
+    f = lambda a: np.asarray(a).reshape(geo.B * geo.heads, -1, geo.d)[h]
+    refs = (f(dq)[qr], f(dqt)[tr], f(dk)[kr], f(dv)[kr], f(dkt)[tr], f(dvt)[tr])
+    for a, b in zip(got, refs):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
