@@ -106,7 +106,7 @@ dsa_status_t dsa_fwd(const dsa_problem_t* p, const void* q, const void* k, const
 
 /* Forward from and to HOST memory (pinned, for asynchronous copies): copies q, k, v and
  * tile_offsets into the caller's device buffer `dev`, runs dsa_fwd there, and copies out and
- * lse back.  The work is pipelined over up to 8 groups of (batch, head) slices: copies in
+ * lse back.  The work is pipelined over up to 24 groups of (batch, head) slices: copies in
  * run on one internal stream, the forward of each group on `stream`, copies back on a
  * second internal stream, ordered by events, so both copy directions overlap the kernels.
  * Everything the call enqueues happens after the work already on `stream`, and `stream`

@@ -169,7 +169,7 @@ def test_bf16_workload_sampled(name):
 
 
 HOST_CASES = [SMALL_BF16[0],
-              # ten (batch, head) slices: the host path pipelines them in five groups of two
+              # ten (batch, head) slices: the host path pipelines them in ten groups of one
               Workload("bf16_host_10", 2, 5, 128, (8, 16, 16), (4, 8, 8), (3, 3, 3), (-2, 2), "bf16", 24)]
 
 

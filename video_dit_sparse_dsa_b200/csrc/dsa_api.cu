@@ -580,7 +580,7 @@ dsa_status_t dsa_fwd(const dsa_problem_t* p, const void* q, const void* k, const
 
 namespace {
 // Groups of (batch, head) slices the host-buffer forward pipelines over.
-constexpr int64_t kHostGroups = 8;
+constexpr int64_t kHostGroups = 24;
 
 // Internal streams and events of one host-buffer forward call, released when the call
 // returns (the runtime keeps destroyed streams and events alive until their work is done).
