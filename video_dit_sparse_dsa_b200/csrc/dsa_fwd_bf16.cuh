@@ -128,7 +128,7 @@ __device__ __forceinline__ uint32_t col_p(int e) { return e ? 256u : 0u; }
 constexpr int kModeFwd = 0, kModeMap = 1, kModeFlat = 2, kModeFwdX = 3;
 
 struct Unit {
-  int bh, tile, sub;  // flat mode: tile = query chunk, sub = 0
+  int bh, tile, sub;  // flat mode: tile = query chunk, sub = part of the key chunks
 };
 
 // Key tiles of query tile `tile` and their count: the window's Wt tiles, or the tile's
