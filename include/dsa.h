@@ -256,6 +256,14 @@ dsa_status_t dsa_lstsq_solve(int32_t m, int32_t p, int32_t batch, const float* M
  * site / block (either may be NULL) receive where the first failure was raised. */
 dsa_status_t dsa_device_status(void* stream, int32_t* site, int32_t* block);
 
+/* Failure-path self-test: enqueues one small kernel that waits on a barrier nothing ever
+ * completes, through the same bounded wait every kernel of the library uses.  After the
+ * wait's limit (2 s of the device clock) it records DSA_DEV_TIMEOUT at site 99 and returns,
+ * so dsa_device_status() then reports DSA_ERR_TIMEOUT with *site = 99 and the context stays
+ * usable.  Nothing faults, traps or hangs. */
+#define DSA_SELFTEST_SITE 99
+dsa_status_t dsa_selftest_wait(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

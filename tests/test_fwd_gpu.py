@@ -187,3 +187,18 @@ def test_forward_host_matches_device(w):
     dsa.forward_host(p, qh, kh, vh, inp.offsets.contiguous(), oh, lh, dev)
     torch.cuda.synchronize()
     assert torch.equal(oh, out.cpu()) and torch.equal(lh, lse.cpu())
+
+
+def test_bounded_wait_runs_out_and_the_context_survives():
+    """The failure path every kernel relies on: a wait nothing completes runs out after its
+    limit, the device status reports DSA_ERR_TIMEOUT at the self-test's site, and the next
+    forward on the same context runs and is correct."""
+    dsa.device_status()  # start from a clear status word
+    dsa.selftest_wait()
+    st, site, _ = dsa.device_status()
+    assert st == 4 and site == 99, (st, site)  # DSA_ERR_TIMEOUT
+    w = SMALL_BF16[0]
+    inp = make_inputs(w)
+    out, lse = run_gpu(w, inp)
+    assert dsa.device_status()[0] == 0
+    compare_full(w, inp, out, lse)

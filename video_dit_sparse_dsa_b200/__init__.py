@@ -37,7 +37,7 @@ EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_
            "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status", "dsa_fwd_noalloc",
            "dsa_list_workspace_size", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map",
            "dsa_lstsq_workspace_size", "dsa_lstsq_factor", "dsa_lstsq_solve", "dsa_prefix_workspace_size",
-           "dsa_fwd_prefix", "dsa_bwd_prefix_workspace_size", "dsa_bwd_prefix")
+           "dsa_fwd_prefix", "dsa_bwd_prefix_workspace_size", "dsa_bwd_prefix", "dsa_selftest_wait")
 
 
 class DsaError(RuntimeError):
@@ -94,13 +94,15 @@ def load_library(path: Optional[str] = None):
     lib.dsa_prefix_workspace_size.restype = sz
     lib.dsa_prefix_workspace_size.argtypes = [pp, i32]
     lib.dsa_fwd_prefix.argtypes = [pp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_selftest_wait.argtypes = [vp]
     lib.dsa_bwd_prefix_workspace_size.restype = sz
     lib.dsa_bwd_prefix_workspace_size.argtypes = [pp, i32]
     lib.dsa_bwd_prefix.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                    vp, vp, sz, vp]
     for name in ("dsa_plan_shape", "dsa_plan", "dsa_fwd", "dsa_fwd_host", "dsa_bwd", "dsa_device_status",
                  "dsa_fwd_noalloc", "dsa_fwd_list", "dsa_bwd_list", "dsa_plan_heads", "dsa_block_map",
-                 "dsa_lstsq_factor", "dsa_lstsq_solve", "dsa_fwd_prefix", "dsa_bwd_prefix"):
+                 "dsa_lstsq_factor", "dsa_lstsq_solve", "dsa_fwd_prefix", "dsa_bwd_prefix",
+                 "dsa_selftest_wait"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -249,6 +251,12 @@ def forward_prefix(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, offsets: t
                               _ptr(k_text), _ptr(v_text), _ptr(out), _ptr(lse), _ptr(out_text), _ptr(lse_text),
                               _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream))), "dsa_fwd_prefix")
     return out, lse, out_text, lse_text
+
+
+def selftest_wait(stream=None):
+    """Enqueue the failure-path self-test (a bounded wait that runs out after 2 s and records
+    DSA_ERR_TIMEOUT at site 99); read the result with device_status()."""
+    _check(load_library().dsa_selftest_wait(ctypes.c_void_p(_stream(stream))), "dsa_selftest_wait")
 
 
 def prefix_bwd_workspace_size(problem: Problem, L_text: int) -> int:

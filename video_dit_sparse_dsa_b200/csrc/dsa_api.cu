@@ -247,6 +247,20 @@ bool make_flat_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t L, int
   return r == CUDA_SUCCESS;
 }
 
+// A wait on a barrier that nothing completes: the library's bounded wait runs out, records
+// DSA_DEV_TIMEOUT at `site` and the kernel returns (the failure path, exercised on purpose).
+__global__ void selftest_wait_kernel(int site) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    dsa::mbar_init(&bar, 1);
+    abort_flag = 0;
+    dsa::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) dsa::mbar_wait(&bar, 0, &abort_flag, site);
+}
+
 // fp32 rows [BH, L] (L * 4 bytes a multiple of 16) seen as 2-D (L, BH); one box is 64
 // consecutive rows of one (batch, head) (rows past L load as zeros).
 bool make_vec_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t L) {
@@ -1076,6 +1090,11 @@ dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k
   dsa::bwd_kv_combine<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
       ws.dk_part, ws.dv_part, ws.n_split, bp.part_stride, p->scale, n4, static_cast<__nv_bfloat16*>(dk_text),
       static_cast<__nv_bfloat16*>(dv_text));
+  return launch_status();
+}
+
+dsa_status_t dsa_selftest_wait(void* stream) {
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(DSA_SELFTEST_SITE);
   return launch_status();
 }
 
