@@ -584,7 +584,9 @@ def main():
     if rank == 0:
         e2e = dict(res["e2e"])
         e2e["value"] = res["e2e"]["value"] * world  # every rank runs the same host-buffer path
-    if rank == 0 and not args.no_extra:
+    # the per-workload table and the CPU baseline run at N = 1 only (the scaling runs time
+    # the headline workload alone, and the other ranks do not wait at a barrier meanwhile)
+    if rank == 0 and world == 1 and not args.no_extra:
         for name, ow in WORKLOADS.items():
             if ow.dtype != "bf16" or name == w.name:
                 continue
@@ -620,7 +622,7 @@ def main():
             except Exception as e:
                 extra[name] = {"error": str(e)}
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, desc, threads, secs = oracle_sample_rate(w, 12.0)
         cpu = {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc + f", {secs:.1f} s"}
