@@ -572,18 +572,21 @@ def main():
     barrier()
     if sampler:
         sampler.start()
-    res = run_workload(dsa, w, device, args.steps, args.warmup, seed_offset=rank, with_e2e=(rank == 0))
+    res = run_workload(dsa, w, device, args.steps, args.warmup, seed_offset=rank, with_e2e=True)
     barrier()
     timed = list(TIMED_WINDOWS)
     clocks = sampler.stop(timed) if sampler else None
     step_ms = max_over_ranks(res["step_ms"], dist, device)
     value, _ = aggregate([step_ms] * world, res["step_flops"])
 
+    # every rank runs the host-buffer path on its own problem: whole-job rate over the slowest
+    e2e_ms = max_over_ranks(res["e2e"]["ms_per_step"], dist, device)
     e2e = None
     extra = {}
     if rank == 0:
         e2e = dict(res["e2e"])
-        e2e["value"] = res["e2e"]["value"] * world  # every rank runs the same host-buffer path
+        e2e["ms_per_step"] = e2e_ms
+        e2e["value"] = aggregate([e2e_ms] * world, w.fwd_flops())[0]
     # the per-workload table and the CPU baseline run at N = 1 only (the scaling runs time
     # the headline workload alone, and the other ranks do not wait at a barrier meanwhile)
     if rank == 0 and world == 1 and not args.no_extra:
