@@ -540,6 +540,8 @@ def main():
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the per-workload table")
+    ap.add_argument("--extra-only", choices=["text_prefix", "lists", "dense_map", "lstsq"],
+                    help="run one entry of the per-workload table on the workload alone and print it (profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
@@ -560,6 +562,15 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     dsa.load_library()
+    if args.extra_only:
+        if world > 1:
+            raise SystemExit("--extra-only runs on one GPU")
+        runs = {"text_prefix": lambda: run_prefix_workload(dsa, w, device, args.steps, args.warmup),
+                "lists": lambda: run_list_workload(dsa, w, device, args.steps, args.warmup, w.window_tiles),
+                "dense_map": lambda: run_dense_map_workload(dsa, w, device, args.steps, args.warmup),
+                "lstsq": lambda: run_lstsq_workload(dsa, device, args.steps, args.warmup)}
+        print(json.dumps({"extra": args.extra_only, "workload": w.name, **runs[args.extra_only]()}), flush=True)
+        return
 
     def barrier():
         if dist is not None:
