@@ -248,11 +248,12 @@ __global__ void __launch_bounds__(256) bwd_kv_combine(const float* __restrict__ 
 //               through a 3-stage ring;
 //   warp 9      MMA issuer, per chunk c (buffer b = c % 2):
 //                 S^T_b = K Q_c^T, dP^T_b = V dO_c^T                 (TMEM, 64 columns each)
-//                 dV += P^T dO_c (P^T read from TMEM), dK += dS^T Q_c (dS^T from smem)
+//                 dV += P^T dO_c, dK += dS^T Q_c (P^T and dS^T read from TMEM)
 //                 dQ^T_c = K^T dS^T into the dP^T_b columns
 //               so the scores of chunk c+1 are ready while chunk c's softmax runs;
 //   warps 0-3   one thread per key row: P^T = exp2(S^T * scale * log2 e - LSE_n * log2 e),
-//               dS^T = P^T (dP^T - D_n); P^T goes back into TMEM as bf16, dS^T into smem;
+//               dS^T = P^T (dP^T - D_n); P^T and dS^T go back into TMEM as bf16 (the dV and dK
+//               products read them there), dS^T also into smem (the B operand of dQ^T);
 //   warps 4-7   one thread per channel d: reads dQ^T_c and adds it to the fp32 dQ
 //               accumulator (a warp covers 32 consecutive channels of one query row); at
 //               the end of a unit, one thread per key row writes dV and scale * dK as bf16.
@@ -435,8 +436,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
               mma_ts_warp(tDV, tS + b * 64 + kk * 8, desc_add(do_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-              mma_ss_warp(tDK, desc_add(ds_k, kk * 32), desc_add(q_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
+            for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q (dS^T from TMEM, beside P^T)
+              mma_ts_warp(tDK, tS + b * 64 + 32 + kk * 8, desc_add(q_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
               mma_ss_warp(tDP + b * 64, desc_add(dKt, kk * 2048), desc_add(ds_m, kk * 2048), kIdescDQ, kk > 0);
@@ -518,6 +519,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) sr[4 * g + e] = pk[e];  // packed P^T of columns 8g..8g+7
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dr[4 * g + e] = dk2[e];  // packed dS^T (dP^T of these columns is used)
           st_shared_v4(dsrow + ((g ^ (m & 7)) << 4), dk2[0], dk2[1], dk2[2], dk2[3]);
         }
         {
@@ -525,6 +528,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) w[e] = sr[e];
           tmem_st32(tS + lane_off + b * 64, w);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w[e] = dr[e];
+          tmem_st32(tS + lane_off + b * 64 + 32, w);
         }
         fence_proxy_async_smem();
         tmem_wait_st();
