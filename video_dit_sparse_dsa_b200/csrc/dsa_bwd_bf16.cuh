@@ -406,7 +406,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const uint64_t dKt = smem_desc_sw128(sbase + kOffK, kKHalf, 1024);       // K^T, MN-major
       const uint64_t dQk = smem_desc_sw128(sbase + kOffStage, 16, 1024);       // stage 0 Q, K-major
       const uint64_t dQm = smem_desc_sw128(sbase + kOffStage, kQHalf, 1024);   // stage 0 Q, MN-major
-      const uint64_t dSk = smem_desc_sw128(sbase + kOffDS, 16, 1024);          // dS^T buffer 0, K-major
       const uint64_t dSm = smem_desc_sw128(sbase + kOffDS, kKHalf, 1024);      // dS^T buffer 0, MN-major
       int ld = 0, uc = 0, sc = 0, pc = 0;
       bool ok = true;
@@ -431,7 +430,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             tc_fence_after();
             const uint32_t so = ((ld0 + cc) % kStages) * kStageBytes;
             const uint64_t q_m = desc_add(dQm, so), do_m = desc_add(dQm, so + kQBytes);
-            const uint64_t ds_k = desc_add(dSk, b * kDSBytes), ds_m = desc_add(dSm, b * kDSBytes);
+            const uint64_t ds_m = desc_add(dSm, b * kDSBytes);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
               mma_ts_warp(tDV, tS + b * 64 + kk * 8, desc_add(do_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
