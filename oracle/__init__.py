@@ -16,7 +16,10 @@ gradients are written out in the header of ``dsa_oracle.c``.
 The key-tile-list functions (``forward_list``, ``backward_list``) take a CSR of key tiles
 per query tile instead of window offsets: the block-sparse generalisation of the window
 (the MOD-DiT page, Method section, Stage 2 "Online Block Masking", attends over selected
-blocks of keys).
+blocks of keys).  The block attention mass (``block_map_list``), the text prefix
+(``forward_prefix*``, ``backward_prefix*``: the MOD-DiT page, "Token-Type-Aware Masking") and
+the regularised least squares (``lstsq``: the MOD-DiT page, Method, Stage 1) follow their
+definitions in the same plain way.
 
 Every function here is pinned by the CPU tests in ``tests/test_oracle_pins.py``.
 """

@@ -37,11 +37,18 @@
  *   K(i) is every token of the tiles listed for i in a CSR (row_ptr, list); a tile listed
  *   twice counts twice; an empty list gives o = 0 and lse = -inf.  Functions *_list.
  *
+ *   Block attention mass (oracle_block_map_list): the mean over a query tile's tokens of
+ *   the probability mass each listed key tile receives.
+ *
+ *   Text prefix (oracle_fwd_prefix; the MOD-DiT page, "Token-Type-Aware Masking"): a video
+ *   query attends to its window and to every text token in one softmax.
+ *
  * Parity pins (tests, CPU only): a window covering the grid equals dense attention; a
  * 1x1x1 window equals block-diagonal attention; softmax rows sum to one; brute-force
  * membership by nearest window centre; backward against central finite differences;
  * lists: multiset-weighted dense attention and its autograd backward, doubled lists
- * (same o, lse + ln 2), lists of the window plan equal the window form.
+ * (same o, lse + ln 2), lists of the window plan equal the window form; block map: blocked
+ * dense probabilities; text prefix: masked dense attention over the unified sequence.
  */
 #include <math.h>
 #include <stdint.h>
