@@ -647,8 +647,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
               float x0, x1;
               ffma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), p.scale_log2, p.scale_log2, neg_lse,
                     neg_lse);
-              fadd2(sa[(c >> 1) & 3], sb[(c >> 1) & 3], sa[(c >> 1) & 3], sb[(c >> 1) & 3], ex2_approx(x0),
-                    ex2_approx(x1));
+              float p0, p1;
+              if ((kPolyMask >> (c >> 4)) & 1u) {  // the forward's share of 2^x on the FMA pipe
+                exp2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              fadd2(sa[(c >> 1) & 3], sb[(c >> 1) & 3], sa[(c >> 1) & 3], sb[(c >> 1) & 3], p0, p1);
             }
           }
           sum = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
