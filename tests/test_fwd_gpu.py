@@ -170,7 +170,9 @@ def test_bf16_workload_sampled(name):
 
 HOST_CASES = [SMALL_BF16[0],
               # ten (batch, head) slices: the host path pipelines them in ten groups of one
-              Workload("bf16_host_10", 2, 5, 128, (8, 16, 16), (4, 8, 8), (3, 3, 3), (-2, 2), "bf16", 24)]
+              Workload("bf16_host_10", 2, 5, 128, (8, 16, 16), (4, 8, 8), (3, 3, 3), (-2, 2), "bf16", 24),
+              # the exact-fp32 path through the same pipeline
+              WORKLOADS["tiny_f32"]]
 
 
 @pytest.mark.parametrize("w", HOST_CASES, ids=lambda w: w.name)
@@ -179,7 +181,8 @@ def test_forward_host_matches_device(w):
     gives bit-for-bit the device entry point's results."""
     inp = make_inputs(w)
     out, lse = run_gpu(w, inp)
-    p = dsa.make_problem(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale, dsa.DSA_BF16)
+    p = dsa.make_problem(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale,
+                         dsa.DSA_BF16 if w.dtype == "bf16" else dsa.DSA_F32)
     dev = torch.empty(dsa.forward_host_bytes(p), dtype=torch.uint8, device="cuda")
     qh, kh, vh = inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory()
     oh = torch.empty_like(qh).pin_memory()
