@@ -39,7 +39,7 @@
  *
  * Supported: bf16 with d = 128 on the tensor-core path, where 64-token key chunks and
  * 128-token query chunks of a tile must be whole (h, w) planes (th*tw divides 64 and
- * 128/(th*tw) divides tt);
+ * 128/(th*tw) divides tt), and for the backward tw a multiple of 4;
  * fp32 with d in {64, 128} on the exact-fp32 path (any tile shape).  Pointers of the bf16
  * path must be 16-byte aligned.
  */

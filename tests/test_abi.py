@@ -99,6 +99,9 @@ def test_fwd_rejects_bad_pointers_and_workspace(lib):
 def test_bwd_rejects_bad_arguments(lib):
     p = _prob()
     f = FAKE
+    # 8 x 2 tile planes: the backward refuses them before any launch (LSE / D boxes of 8 bytes)
+    narrow = _prob(tile=(16, 8, 2), grid=(32, 16, 8))
+    assert lib.dsa_bwd(ctypes.byref(narrow), f, f, f, f, f, f, f, f, f, f, f, 1 << 30, None) == 2
     assert lib.dsa_bwd(ctypes.byref(p), f, f, f, f, f, f, f, f, f, None, f, 1 << 30, None) == 1
     p32 = _prob(d=64, dtype=dsa.DSA_F32, grid=(4, 8, 8), tile=(1, 4, 4))
     assert lib.dsa_bwd(ctypes.byref(p32), f, f, f, f, f, f, f, f, f, f, f, 1 << 30, None) == 2

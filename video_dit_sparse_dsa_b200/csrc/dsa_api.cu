@@ -68,6 +68,9 @@ dsa_status_t check_kernel_limits(const dsa_problem_t* p, const Geom& g, bool bac
   const int plane = p->tile[1] * p->tile[2];
   if (plane > 64 || 64 % plane != 0) return DSA_ERR_UNSUPPORTED;
   if (p->tile[0] % (128 / plane) != 0) return DSA_ERR_UNSUPPORTED;
+  // the backward reads a query chunk's LSE and D rows as TMA boxes of tw fp32 values, which
+  // must be a multiple of 16 bytes
+  if (backward && p->tile[2] % 4 != 0) return DSA_ERR_UNSUPPORTED;
   if (g.BH * g.n_tiles * (g.tile_tokens / 128) > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
 }
