@@ -30,7 +30,7 @@ def random_workload(seed: int) -> Workload:
                     backward=True)
 
 
-@pytest.mark.parametrize("seed", range(8))
+@pytest.mark.parametrize("seed", range(16))
 def test_random_shape_forward_and_backward(seed):
     w = random_workload(seed)
     inp = make_inputs(w)
