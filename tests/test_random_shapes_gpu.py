@@ -53,3 +53,37 @@ def test_random_shape_forward_and_backward(seed):
     rq, rk, rv = oracle.backward(geo, inp.q, inp.k, inp.v, inp.dout, inp.offsets)
     for got, r, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
         assert_close(got.float().cpu().numpy(), r, w.dtype, f"{w.name} {name} {w.tile} {w.grid} {w.window}")
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_shape_text_prefix(seed):
+    """Random shapes with a random number of text tokens: prefix forward and backward in full."""
+    w = random_workload(100 + seed)
+    if w.tile[2] % 4 != 0:  # keep the backward's tile-width rule
+        w = w.replace(tile=(w.tile[0], w.tile[2], w.tile[1]), grid=(w.grid[0], w.grid[2], w.grid[1]))
+    rng = np.random.default_rng(900 + seed)
+    L = int(rng.integers(1, 400))
+    from dsa_inputs import make_text_inputs
+
+    inp = make_inputs(w)
+    txt = make_text_inputs(w, L, seed=950 + seed)
+    dev = torch.device("cuda")
+    q, k, v, off = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), inp.offsets.to(dev)
+    qt, kt, vt = txt.q.to(dev), txt.k.to(dev), txt.v.to(dev)
+    out, lse, out_t, lse_t = dsa.forward_prefix(q, k, v, off, qt, kt, vt, w.tile, w.window, w.scale)
+    do_t = torch.randn(tuple(qt.shape), generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16)
+    grads = dsa.backward_prefix(q, k, v, out, lse, inp.dout.to(dev), off, qt, kt, vt, out_t, lse_t, do_t.to(dev),
+                                w.tile, w.window, w.scale)
+    st, site, _ = dsa.device_status()
+    assert st == 0, f"{w}, L={L}: device status {st} at site {site}"
+    geo = oracle.Geometry.of(w)
+    ro, rl, rot, rlt = oracle.forward_prefix(geo, inp.q, inp.k, inp.v, inp.offsets, txt.q, txt.k, txt.v)
+    tag = f"{w.name} {w.tile} {w.grid} {w.window} L={L}"
+    assert_close(out.float().cpu().numpy(), ro, w.dtype, f"out {tag}")
+    assert_close(out_t.float().cpu().numpy(), rot, w.dtype, f"out_text {tag}")
+    assert_lse_close(lse.cpu().numpy(), rl, w.dtype, f"lse {tag}")
+    assert_lse_close(lse_t.cpu().numpy(), rlt, w.dtype, f"lse_text {tag}")
+    (rq, rk, rv), (rqt, rkt, rvt) = oracle.backward_prefix(geo, inp.q, inp.k, inp.v, inp.dout, inp.offsets, txt.q,
+                                                           txt.k, txt.v, do_t)
+    for got, r, name in zip(grads, (rq, rk, rv, rqt, rkt, rvt), ("dq", "dk", "dv", "dq_text", "dk_text", "dv_text")):
+        assert_close(got.float().cpu().numpy(), r, w.dtype, f"{name} {tag}")
