@@ -1,4 +1,5 @@
-"""Seeded random problem shapes through the bf16 tensor-core path, forward and backward,
+"""Seeded random problem shapes through the bf16 tensor-core path (window, text-prefix and
+key-tile-list forms), forward and backward,
 each compared in full with the fp64 oracle: tile planes of 8x8, 4x8, 8x4, 4x4, 2x8 and 8x2
 tokens (a 128-token chunk spans 128 / (th tw) t-planes), tile grids of 1-3 tiles per axis,
 windows of 1-4 tiles (often wider than the grid), offsets in [-2, 2], 1-2 batch entries
@@ -87,3 +88,49 @@ def test_random_shape_text_prefix(seed):
                                                            txt.k, txt.v, do_t)
     for got, r, name in zip(grads, (rq, rk, rv, rqt, rkt, rvt), ("dq", "dk", "dv", "dq_text", "dk_text", "dv_text")):
         assert_close(got.float().cpu().numpy(), r, w.dtype, f"{name} {tag}")
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_shape_key_tile_lists(seed):
+    """Random shapes with random per-(batch, head) key-tile lists (empty rows, repeats):
+    forward, backward and block map in full against the oracle's list form."""
+    w = random_workload(200 + seed)
+    if w.tile[2] % 4 != 0:
+        w = w.replace(tile=(w.tile[0], w.tile[2], w.tile[1]), grid=(w.grid[0], w.grid[2], w.grid[1]))
+    geo = oracle.Geometry.of(w)
+    rng = np.random.default_rng(700 + seed)
+    BH, n = w.B * w.heads, geo.n_tiles
+    rows, row_ptr = [], np.zeros((BH, n + 1), np.int64)
+    total = 0
+    for h in range(BH):
+        row_ptr[h, 0] = total  # absolute positions: head h's rows continue where head h - 1's end
+        for i in range(n):
+            cnt = int(rng.integers(0, 6))
+            rows.append(rng.integers(0, n, cnt))
+            total += cnt
+            row_ptr[h, i + 1] = total
+    kv_list = np.concatenate(rows).astype(np.int32) if total else np.zeros(0, np.int32)
+    rp = row_ptr.astype(np.int32)
+    inp = make_inputs(w)
+    dev = torch.device("cuda")
+    q, k, v, dout = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), inp.dout.to(dev)
+    rpd, kvd = torch.from_numpy(rp).to(dev), torch.from_numpy(kv_list).to(dev)
+    out, lse = dsa.forward_list(q, k, v, rpd, kvd, w.tile, w.scale)
+    dq, dk, dv = dsa.backward_list(q, k, v, out, lse, dout, rpd, kvd, w.tile, w.scale)
+    bmap = dsa.block_map(q, k, lse, rpd, kvd, w.tile, w.scale)
+    st, site, _ = dsa.device_status()
+    assert st == 0, f"{w}: device status {st} at site {site}"
+    tag = f"{w.name} {w.tile} {w.grid}"
+    ref, ref_lse = oracle.forward_list(geo, inp.q, inp.k, inp.v, rp, kv_list)
+    got_o, got_l = out.float().cpu().numpy(), lse.cpu().numpy()
+    finite = np.isfinite(ref_lse)  # empty lists: O = 0, LSE = -inf on both sides
+    assert np.array_equal(np.isfinite(got_l), finite)
+    assert_close(got_o, ref, w.dtype, f"out {tag}")
+    assert_lse_close(got_l[finite], ref_lse[finite], w.dtype, f"lse {tag}")
+    rq, rk, rv = oracle.backward_list(geo, inp.q, inp.k, inp.v, inp.dout, rp, kv_list)
+    for got, r, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        assert_close(got.float().cpu().numpy(), r, w.dtype, f"{name} {tag}")
+    # block map: the list tests' gate (entries carry the bf16 forward's LSE error, ~1e-3 relative)
+    rmap = np.asarray(oracle.block_map_list(geo, inp.q, inp.k, rp, kv_list)).reshape(bmap.shape)
+    err = float(np.abs(bmap.cpu().numpy() - rmap).max())
+    assert err <= 3e-3, f"map {tag}: max-abs {err:.2e}"
