@@ -30,6 +30,8 @@ SMALL = [
     Workload("bwd_small_c", 1, 2, 128, (16, 8, 8), (8, 4, 4), (1, 3, 3), (-1, 1), "bf16", 33, backward=True),
     # offsets of 3 leave some key tiles in no window at all: their dK, dV must be zero
     Workload("bwd_small_shift", 1, 1, 128, (8, 32, 32), (4, 8, 8), (1, 1, 1), (3, 3), "bf16", 34, backward=True),
+    # 64 (batch, head) slices on a small grid
+    Workload("bwd_many_heads", 4, 16, 128, (4, 16, 8), (4, 8, 8), (1, 3, 1), (-1, 1), "bf16", 35, backward=True),
 ]
 
 
