@@ -30,7 +30,10 @@
  * dsa_fwd_host) is DEVICE memory owned by the caller.  The library allocates no memory:
  * scratch lives in the caller's workspace (dsa_workspace_size).  All work is enqueued on
  * `stream` (a cudaStream_t; NULL = the legacy default stream) and returns without waiting.
- * The library holds no per-call state and may be called from several threads.
+ * The library holds no per-call state and may be called from several threads.  The device-
+ * buffer entry points allocate and synchronise nothing, so they can be captured in a CUDA
+ * graph (after one call outside the capture); dsa_fwd_host creates streams and events and
+ * cannot.
  *
  * Errors.  Argument errors are returned synchronously and nothing is launched.  A launch
  * error returns DSA_ERR_CUDA.  Kernels never trap: a device-side failure (a bounded wait

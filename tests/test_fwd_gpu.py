@@ -205,3 +205,40 @@ def test_bounded_wait_runs_out_and_the_context_survives():
     out, lse = run_gpu(w, inp)
     assert dsa.device_status()[0] == 0
     compare_full(w, inp, out, lse)
+
+
+def test_forward_and_backward_replay_from_a_cuda_graph():
+    """The planner, forward and backward launches can be captured in a CUDA graph and
+    replayed (every launch goes to the caller's stream; no allocation, no synchronisation
+    inside the calls); replays give the eager results."""
+    w = Workload("graph_bf16", 1, 2, 128, (8, 16, 16), (4, 8, 8), (3, 3, 3), (-1, 1), "bf16", 29, backward=True)
+    inp = make_inputs(w)
+    q, k, v, dout, off = inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.dout.cuda(), inp.offsets.cuda()
+    p = dsa.make_problem(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale)
+    ws_f, ws_b = dsa.workspace(p, q.device), dsa.workspace(p, q.device, backward=True)
+    out, lse = torch.empty_like(q), torch.empty(q.shape[:5], dtype=torch.float32, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ref_o, ref_l = dsa.forward(q, k, v, off, w.tile, w.window, w.scale)
+    ref_g = dsa.backward(q, k, v, ref_o, ref_l, dout, off, w.tile, w.window, w.scale)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up outside the capture (attribute setup, encoder lookup)
+        dsa.forward(q, k, v, off, w.tile, w.window, w.scale, out=out, lse=lse, ws=ws_f, stream=s)
+        dsa.backward(q, k, v, out, lse, dout, off, w.tile, w.window, w.scale, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dsa.forward(q, k, v, off, w.tile, w.window, w.scale, out=out, lse=lse, ws=ws_f, stream=s)
+        dsa.backward(q, k, v, out, lse, dout, off, w.tile, w.window, w.scale, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=s)
+    for tensor in (out, lse, dq, dk, dv):
+        tensor.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert dsa.device_status()[0] == 0
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+    assert torch.equal(dk, ref_g[1]) and torch.equal(dv, ref_g[2])  # dQ sums with atomics: compare loosely
+    assert float((dq.float() - ref_g[0].float()).abs().max()) <= 1e-3
+    del g
