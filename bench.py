@@ -50,10 +50,10 @@ def peaks():
 
 
 # ----------------------------------------------------------------------------- DRAM traffic
-# DRAM bytes (read + write) of one fwd_bf16_kernel launch per workload, from the
-# single-pass ncu capture summarised in profiles/fwd_bf16_kernel__bf16_720p_dram.md.  The
-# figure holds only for the kernel sources it was taken on, identified by a hash of them;
-# with any other sources the line reports null.
+# DRAM bytes (read + write) of one fwd_bf16_kernel launch per workload, from a
+# single-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the full-size
+# launch.  The figure holds only for the kernel sources it was taken on, identified by a
+# hash of them; with any other sources the line reports null.
 FWD_TRAFFIC = {"bf16_720p": (3.54e9, "cafcb10850cbd1e3")}
 FWD_SOURCES = ("dsa_fwd_bf16.cuh", "sm100.cuh")
 
@@ -226,43 +226,51 @@ TIMED_WINDOWS = []
 
 
 # ----------------------------------------------------------------------------- inputs
-def device_inputs(w: Workload, device, seed_offset: int = 0):
-    """Seeded synthetic inputs drawn on the device (same distributions as dsa_inputs, which
-    draws on the CPU for the parity tests)."""
-    g = torch.Generator(device=device).manual_seed(1000 + w.seed + seed_offset)
-    shape = (w.B, w.heads) + tuple(w.grid) + (w.d,)
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    q = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt)
-    k = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt)
-    v = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt)
-    dout = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dt) if w.backward else None
-    gc = torch.Generator().manual_seed(w.seed + seed_offset)
-    lo, hi = w.offset_range
-    off = torch.randint(lo, hi + 1, (w.n_tiles, 3), generator=gc).to(torch.int32).to(device)
-    return q, k, v, dout, off
+def host_inputs(w: Workload, rank: int = 0):
+    """The seeded inputs of the parity tests (dsa_inputs, drawn on the CPU); rank r > 0 of a
+    multi-GPU run draws its own independent problem of the same shape from seed + r."""
+    return make_inputs(w, seed=w.seed + rank) if rank else make_inputs(w)
+
+
+def device_inputs(w: Workload, device, rank: int = 0):
+    inp = host_inputs(w, rank)
+    dout = inp.dout.to(device) if inp.dout is not None else None
+    return inp.q.to(device), inp.k.to(device), inp.v.to(device), dout, inp.offsets.to(device), inp
 
 
 # ----------------------------------------------------------------------------- GPU arm
 def time_steps(step, steps: int, warmup: int, stream, record: bool = True):
+    """W untimed steps, then K steps each between two CUDA events on `stream`, with a
+    synchronize before and after.  Returns {median, mean, min, max} ms per step."""
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     t0 = time.time()
-    start.record(stream)
-    for _ in range(steps):
+    ev[0].record(stream)
+    for i in range(steps):
         step()
-    end.record(stream)
+        ev[i + 1].record(stream)
     torch.cuda.synchronize()
     if record:
         TIMED_WINDOWS.append((t0, time.time()))
-    return start.elapsed_time(end) / steps  # ms per step
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    return {"median": statistics.median(per), "mean": ev[0].elapsed_time(ev[steps]) / steps, "min": min(per),
+            "max": max(per)}
 
 
-def run_workload(dsa, w: Workload, device, steps: int, warmup: int, seed_offset: int = 0, with_e2e: bool = False):
+def pct_of_peaks(tflops: float) -> dict:
+    burst, sustained, src = peaks()
+    return {"pct_nominal_2250": 100 * tflops / NOMINAL_BF16_TFLOPS, f"pct_{src}_burst": 100 * tflops / burst}
+
+
+def run_workload(dsa, w: Workload, device, steps: int, warmup: int, rank: int = 0, with_e2e: bool = False,
+                 record: bool = True):
+    """Times the forward (planner + kernel, one dsa_fwd call) and, for workloads with a
+    backward, the backward (one dsa_bwd call) on the workload's seeded inputs.  Times are
+    medians over `steps` timed steps after `warmup` untimed ones."""
     stream = torch.cuda.current_stream(device)
-    q, k, v, dout, off = device_inputs(w, device, seed_offset)
+    q, k, v, dout, off, host = device_inputs(w, device, rank)
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:5], dtype=torch.float32, device=device)
     p = dsa.make_problem(w.B, w.heads, w.d, w.grid, w.tile, w.window, w.scale,
@@ -274,10 +282,13 @@ def run_workload(dsa, w: Workload, device, steps: int, warmup: int, seed_offset:
         dsa.forward(q, k, v, off, w.tile, w.window, w.scale, out=out, lse=lse, ws=ws_f, stream=stream)
 
     fwd()
-    res["fwd_ms"] = time_steps(fwd, steps, warmup, stream)
+    t = time_steps(fwd, steps, warmup, stream, record)
+    res["fwd_ms"] = t["median"]
+    res["fwd_ms_mean"] = t["mean"]
     res["fwd_tflops"] = w.fwd_flops() / (res["fwd_ms"] * 1e-3) / 1e12
-    launches = 2  # planner + forward
+    launches = dsa.FWD_LAUNCHES
     step_ms = res["fwd_ms"]
+    step_ms_mean = t["mean"]
     step_flops = w.fwd_flops()
     if w.backward:
         ws_b = dsa.workspace(p, device, backward=True)
@@ -288,19 +299,23 @@ def run_workload(dsa, w: Workload, device, steps: int, warmup: int, seed_offset:
                          stream=stream)
 
         bwd()
-        res["bwd_ms"] = time_steps(bwd, steps, warmup, stream)
+        t = time_steps(bwd, steps, warmup, stream, record)
+        res["bwd_ms"] = t["median"]
+        res["bwd_ms_mean"] = t["mean"]
         res["bwd_tflops"] = w.bwd_flops() / (res["bwd_ms"] * 1e-3) / 1e12
         step_ms += res["bwd_ms"]
+        step_ms_mean += t["mean"]
         step_flops += w.bwd_flops()
-        launches += 4  # planner (with inverse map), D preprocess, backward, dQ convert
+        launches += dsa.BWD_LAUNCHES
     res["step_ms"] = step_ms
+    res["step_ms_mean"] = step_ms_mean
     res["step_flops"] = step_flops
     res["launches_per_step"] = launches
     st = dsa.device_status(stream)
     if st[0] != 0:
         raise RuntimeError(f"device status {st} after {w.name}")
     if with_e2e:
-        res["e2e"] = run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream)
+        res["e2e"] = run_e2e(dsa, w, p, host, device, steps, warmup, stream)
     return res
 
 
@@ -310,7 +325,7 @@ def run_list_workload(dsa, w: Workload, device, steps: int, warmup: int, n_keep:
     (head-adaptive block masks); the forward's FLOPs count n_keep tiles per query."""
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
-    q, k, v, _, _ = device_inputs(w, device)
+    q, k, v, _, _, _ = device_inputs(w, device)
     BH = w.B * w.heads
     g = torch.Generator(device=device).manual_seed(7000 + w.seed)
     pick = torch.rand((BH, w.n_tiles, w.n_tiles), generator=g, device=device).argsort(dim=-1)[..., :n_keep]
@@ -325,7 +340,7 @@ def run_list_workload(dsa, w: Workload, device, steps: int, warmup: int, n_keep:
         dsa.forward_list(q, k, v, row_ptr, kv_list, w.tile, w.scale, out=out, lse=lse, stream=stream)
 
     fwd()
-    ms = time_steps(fwd, steps, warmup, stream, record=False)
+    ms = time_steps(fwd, steps, warmup, stream, record=False)["median"]
     flops = 4.0 * w.B * w.heads * w.n_tokens * (n_keep * w.tile_tokens) * w.d
     st = dsa.device_status(stream)
     if st[0] != 0:
@@ -339,7 +354,7 @@ def run_prefix_workload(dsa, w: Workload, device, steps: int, warmup: int):
     4 * B * heads * d * (N * keys_per_query + 2 * N * L_text + L_text^2)."""
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
-    q, k, v, _, offsets = device_inputs(w, device)
+    q, k, v, _, offsets, _ = device_inputs(w, device)
     L = text_length(w)
     txt = make_text_inputs(w, L, seed=1000 + w.seed)
     qt, kt, vt = (t.to(device) for t in (txt.q, txt.k, txt.v))
@@ -350,7 +365,7 @@ def run_prefix_workload(dsa, w: Workload, device, steps: int, warmup: int):
         dsa.forward_prefix(q, k, v, offsets, qt, kt, vt, w.tile, w.window, w.scale, ws=ws, stream=stream)
 
     fwd()
-    ms = time_steps(fwd, steps, warmup, stream, record=False)
+    ms = time_steps(fwd, steps, warmup, stream, record=False)["median"]
     st = dsa.device_status(stream)
     if st[0] != 0:
         raise RuntimeError(f"device status {st} after the text-prefix forward")
@@ -370,7 +385,7 @@ def run_prefix_workload(dsa, w: Workload, device, steps: int, warmup: int):
                             ws=ws_b, stream=stream)
 
     bwd()
-    b_ms = time_steps(bwd, steps, warmup, stream, record=False)
+    b_ms = time_steps(bwd, steps, warmup, stream, record=False)["median"]
     st = dsa.device_status(stream)
     if st[0] != 0:
         raise RuntimeError(f"device status {st} after the text-prefix backward")
@@ -384,7 +399,7 @@ def run_dense_map_workload(dsa, w: Workload, device, steps: int, warmup: int):
     pass recomputes the scores only: 2 * B * heads * N^2 * d FLOP."""
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
-    q, k, v, _, _ = device_inputs(w, device)
+    q, k, v, _, _, _ = device_inputs(w, device)
     n = w.n_tiles
     row_ptr = torch.arange(n + 1, dtype=torch.int32, device=device) * n
     kv_list = torch.arange(n, dtype=torch.int32, device=device).repeat(n).contiguous()
@@ -400,8 +415,8 @@ def run_dense_map_workload(dsa, w: Workload, device, steps: int, warmup: int):
 
     fwd()
     bm()
-    f_ms = time_steps(fwd, steps, warmup, stream, record=False)
-    m_ms = time_steps(bm, steps, warmup, stream, record=False)
+    f_ms = time_steps(fwd, steps, warmup, stream, record=False)["median"]
+    m_ms = time_steps(bm, steps, warmup, stream, record=False)["median"]
     st = dsa.device_status(stream)
     if st[0] != 0:
         raise RuntimeError(f"device status {st} after the dense map")
@@ -427,7 +442,7 @@ def run_lstsq_workload(dsa, device, steps: int, warmup: int, m: int = 300 * 300,
         dsa.lstsq_solve(M, L, S, X=X, ws=ws, stream=stream)
 
     solve()
-    ms = time_steps(solve, steps, warmup, stream, record=False)
+    ms = time_steps(solve, steps, warmup, stream, record=False)["median"]
     st = dsa.device_status(stream)
     if st[0] != 0:
         raise RuntimeError(f"device status {st} after the least-squares solve")
@@ -435,11 +450,11 @@ def run_lstsq_workload(dsa, device, steps: int, warmup: int, m: int = 300 * 300,
     return {"solve_ms": ms, "solve_gbs": gb / (ms * 1e-3)}
 
 
-def run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream):
+def run_e2e(dsa, w, p, host, device, steps, warmup, stream):
     """Same forward through the host-buffer entry point: H2D of q, k, v, offsets from pinned
     memory, planner + forward, D2H of out and lse, all inside the timed region."""
-    qh, kh, vh = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
-    oh_ = off.cpu().pin_memory()
+    qh, kh, vh = host.q.pin_memory(), host.k.pin_memory(), host.v.pin_memory()
+    oh_ = host.offsets.pin_memory()
     outh = torch.empty_like(qh).pin_memory()
     lseh = torch.empty(qh.shape[:5], dtype=torch.float32).pin_memory()
     dev = torch.empty(dsa.forward_host_bytes(p), dtype=torch.uint8, device=device)
@@ -447,7 +462,7 @@ def run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream):
     def step():
         dsa.forward_host(p, qh, kh, vh, oh_, outh, lseh, dev, stream=stream)
 
-    ms = time_steps(step, max(1, steps // 2), max(1, warmup // 2), stream, record=False)
+    ms = time_steps(step, max(1, steps // 2), max(1, warmup // 2), stream, record=False)["median"]
     h2d = 3 * qh.numel() * qh.element_size() + oh_.numel() * 4
     d2h = outh.numel() * outh.element_size() + lseh.numel() * 4
     return {"value": w.fwd_flops() / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
@@ -455,61 +470,120 @@ def run_e2e(dsa, w, p, q, k, v, off, device, steps, warmup, stream):
 
 
 # ----------------------------------------------------------------------------- oracle timing
-def oracle_sample_rate(w: Workload, target_s: float, max_tiles: int = 4096):
-    """Time the fp64 oracle (as it stands) on a growing sample of query tiles of head 0
-    until one run takes about target_s.  Returns (TFLOP/s, sample description, threads)."""
+def _slice0(w: Workload, host):
+    """(workload of one (batch, head), its tensors): the first slice of the inputs the GPU ran."""
+    one = w.replace(B=1, heads=1)
+    sl = [None if t is None else t[:1, :1].contiguous() for t in (host.q, host.k, host.v, host.dout)]
+    return one, sl
+
+
+def _grow(run, n_max: int, target_s: float):
+    """Calls run(n) with growing n (1, then scaled up to reach target_s) until one call takes
+    at least target_s or n reaches n_max.  Returns (n, seconds of that call)."""
+    n = 1
+    while True:
+        t0 = time.perf_counter()
+        run(n)
+        dt_s = time.perf_counter() - t0
+        if dt_s >= target_s or n >= n_max:
+            return n, dt_s
+        n = min(n_max, max(n + 1, int(n * min(8.0, 1.2 * target_s / max(dt_s, 1e-3)))))
+
+
+def oracle_fwd_rate(w: Workload, host, target_s: float):
+    """The fp64 oracle (as it stands) timed on the query tiles of the first (batch, head)
+    slice of the GPU's inputs, in raster order: growing samples until one run takes
+    target_s, or the whole slice.  Returns a cpu_baseline object (TFLOP/s)."""
     import oracle
 
-    inp_w = w.replace(B=1, heads=1)
-    g = torch.Generator().manual_seed(w.seed)
-    shape = (1, 1) + tuple(w.grid) + (w.d,)
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    q, k, v = (torch.randn(shape, generator=g).to(dt) for _ in range(3))
-    lo, hi = w.offset_range
-    off = torch.randint(lo, hi + 1, (w.n_tiles, 3), generator=g).to(torch.int32)
-    geo = oracle.Geometry.of(inp_w)
+    one, (q, k, v, _) = _slice0(w, host)
+    geo = oracle.Geometry.of(one)
     per_tile = 4.0 * w.tile_tokens * w.keys_per_query * w.d
-    n = 1
-    rng = np.random.default_rng(0)
-    while True:
-        tiles = rng.integers(0, geo.n_tiles, n).astype(np.int32)
-        t0 = time.perf_counter()
-        oracle.forward_tiles(geo, q, k, v, off, (np.zeros(n, np.int32), tiles))
-        dt_s = time.perf_counter() - t0
-        if dt_s >= target_s or n >= max_tiles:
-            break
-        n = min(max_tiles, max(n + 1, int(n * min(8.0, 1.2 * target_s / max(dt_s, 1e-3)))))
-    threads = len(os.sched_getaffinity(0))
-    return per_tile * n / dt_s / 1e12, f"{n} query tiles of one head ({n * w.tile_tokens} query rows), forward", \
-        threads, dt_s
+
+    def run(n):
+        oracle.forward_tiles(geo, q, k, v, host.offsets, (np.zeros(n, np.int32), np.arange(n, dtype=np.int32)))
+
+    n, secs = _grow(run, geo.n_tiles, target_s)
+    whole = n == geo.n_tiles
+    return {"value": per_tile * n / secs / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle", "seconds": secs, "extrapolated": not whole,
+            "sample": ("the whole first (batch, head) slice" if whole else
+                       f"query tiles 0..{n - 1} of {geo.n_tiles} of the first (batch, head) slice") +
+                      f" ({n * w.tile_tokens} query rows), forward, {secs:.1f} s"}
+
+
+def oracle_bwd_rate(w: Workload, host, target_s: float):
+    """The fp64 oracle's backward timed on query tiles 0..n-1 (dQ) and key tiles 0..n-1
+    (dK, dV) of the first (batch, head) slice, n grown until one run takes target_s.  Its
+    effective FLOP: 2.5 x 4d x (query-key pairs of the dQ sample + pairs of the dK/dV
+    sample) / 2, since every pair of the full backward is counted once for dQ and once for
+    dK, dV."""
+    import oracle
+
+    one, (q, k, v, do) = _slice0(w, host)
+    geo = oracle.Geometry.of(one)
+    _, _, row_ptr, _ = oracle.plan(geo.G, geo.window, host.offsets)
+    indeg = np.diff(row_ptr)
+    tt = w.tile_tokens
+
+    def run(n):
+        sel = (np.zeros(n, np.int32), np.arange(n, dtype=np.int32))
+        oracle.backward_dq_tiles(geo, q, k, v, do, host.offsets, sel)
+        oracle.backward_dkdv_tiles(geo, q, k, v, do, host.offsets, sel)
+
+    n, secs = _grow(run, geo.n_tiles, target_s)
+    pairs = n * tt * w.keys_per_query + int(indeg[:n].sum()) * tt * tt
+    return {"value": 2.5 * 4.0 * w.d * pairs / 2 / secs / 1e12, "unit": "TFLOP/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle", "seconds": secs, "extrapolated": True,
+            "sample": f"dQ of query tiles 0..{n - 1} and dK, dV of key tiles 0..{n - 1} of {geo.n_tiles}, first "
+                      f"(batch, head) slice, backward, {secs:.1f} s"}
 
 
 def workload_config(w: Workload, world: int) -> dict:
     """The `config` object of both arms' JSON lines."""
     return {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": list(w.grid), "tile": list(w.tile),
             "window": list(w.window), "offsets": list(w.offset_range), "keys_per_query": w.keys_per_query,
-            "pass": "fwd+bwd" if w.backward else "fwd", "l2": "inputs larger than L2 (no flush)",
+            "dtype": w.dtype, "pass": "fwd+bwd" if w.backward else "fwd",
+            "l2": "inputs larger than L2 (no flush)" if 3 * w.B * w.heads * w.n_tokens * w.d * 2 > 126e6 else
+                  "inputs smaller than L2 (no flush; L2-resident)",
+            "inputs": "dsa_inputs seeded CPU draws (the parity tests' inputs)",
             "parallelism": f"independent problem per rank x{world}"}
 
 
 def reference_arm(args, w: Workload):
+    """The oracle as it stands on the host cores: each step is a bounded sample of the
+    workload (forward query tiles, plus the backward sample for workloads with one), and the
+    line's ms_per_step is the measured time of one such sample step."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    host = host_inputs(w.replace(B=1, heads=1))
     per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
-    rates = []
-    desc, threads = "", 0
+    rates, secs = [], []
+    fwd = bwd = None
     for i in range(args.warmup + args.steps):
-        r, desc, threads, _ = oracle_sample_rate(w, per_step)
+        fwd = oracle_fwd_rate(w, host, per_step)
+        t = fwd["seconds"]
+        r = fwd["value"]
+        if w.backward:
+            bwd = oracle_bwd_rate(w, host, per_step)
+            t += bwd["seconds"]
+            # the step's rate: fwd + bwd effective FLOP of the samples over their time
+            r = (fwd["value"] * fwd["seconds"] + bwd["value"] * bwd["seconds"]) / t
         if i >= args.warmup:
             rates.append(r)
+            secs.append(t)
     value = statistics.median(rates)
     flops = w.fwd_flops() + (w.bwd_flops() if w.backward else 0)
+    sample = fwd["sample"] + ("; " + bwd["sample"] if bwd else "")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops / (value * 1e12) * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(secs) * 1e3,
+            "ms_per_step_is": "measured time of one bounded sample step (not the whole workload)",
+            "full_workload_ms_extrapolated": flops / (value * 1e12) * 1e3, "extrapolated": True,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, args.gpus),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": fwd["cores"], "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -536,7 +610,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="bf16_720p", choices=[k for k, w in WORKLOADS.items() if w.dtype == "bf16"])
+    ap.add_argument("--workload", default="bf16_720p", choices=list(WORKLOADS))
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the per-workload table")
@@ -583,63 +657,74 @@ def main():
     barrier()
     if sampler:
         sampler.start()
-    res = run_workload(dsa, w, device, args.steps, args.warmup, seed_offset=rank, with_e2e=True)
+    res = run_workload(dsa, w, device, args.steps, args.warmup, rank=rank, with_e2e=True)
     barrier()
     timed = list(TIMED_WINDOWS)
     clocks = sampler.stop(timed) if sampler else None
     step_ms = max_over_ranks(res["step_ms"], dist, device)
+    step_ms_mean = max_over_ranks(res["step_ms_mean"], dist, device)
     value, _ = aggregate([step_ms] * world, res["step_flops"])
 
     # every rank runs the host-buffer path on its own problem: whole-job rate over the slowest
     e2e_ms = max_over_ranks(res["e2e"]["ms_per_step"], dist, device)
     e2e = None
     extra = {}
+    cpu = None
     if rank == 0:
         e2e = dict(res["e2e"])
         e2e["ms_per_step"] = e2e_ms
         e2e["value"] = aggregate([e2e_ms] * world, w.fwd_flops())[0]
-    # the per-workload table and the CPU baseline run at N = 1 only (the scaling runs time
-    # the headline workload alone, and the other ranks do not wait at a barrier meanwhile)
+    # the per-workload table (every configuration, each with the oracle timed beside it on
+    # this machine's host cores) and the CPU baseline run at N = 1 only (the scaling runs time the
+    # headline workload alone, and the other ranks do not wait at a barrier meanwhile)
     if rank == 0 and world == 1 and not args.no_extra:
         for name, ow in WORKLOADS.items():
-            if ow.dtype != "bf16" or name == w.name:
-                continue
             try:
-                r = run_workload(dsa, ow, device, max(3, args.steps // 2), 3)
-                extra[name] = {k2: round(v2, 4) for k2, v2 in r.items()
-                               if k2.endswith("_ms") or k2.endswith("_tflops")}
+                r = res if name == w.name else run_workload(dsa, ow, device, max(20, args.steps),
+                                                            max(5, args.warmup), record=False)
+                row = {k2: round(v2, 4) for k2, v2 in r.items() if k2.endswith("_ms") or k2.endswith("_tflops")
+                       or k2.endswith("_ms_mean")}
+                row["steps"], row["warmup"] = max(20, args.steps), max(5, args.warmup)
+                row["fwd_pct"] = {k2: round(v2, 2) for k2, v2 in pct_of_peaks(r["fwd_tflops"]).items()}
+                if "bwd_tflops" in r:
+                    row["bwd_pct"] = {k2: round(v2, 2) for k2, v2 in pct_of_peaks(r["bwd_tflops"]).items()}
+                if not args.no_cpu_baseline:
+                    host = host_inputs(ow.replace(B=1, heads=1))
+                    row["oracle_fwd"] = oracle_fwd_rate(ow, host, 12.0 if name == w.name else 6.0)
+                    if name == w.name:
+                        cpu = dict(row["oracle_fwd"])
+                    if ow.backward:
+                        row["oracle_bwd"] = oracle_bwd_rate(ow, host, 8.0)
+                extra[name] = row
             except Exception as e:  # report, do not hide: the line carries the error
                 extra[name] = {"error": str(e)}
         try:
-            r = run_lstsq_workload(dsa, device, max(10, args.steps), 5)
+            r = run_lstsq_workload(dsa, device, max(20, args.steps), 5)
             extra["lstsq_24x90000x3"] = {k2: round(v2, 4) for k2, v2 in r.items()}
         except Exception as e:
             extra["lstsq_24x90000x3"] = {"error": str(e)}
         dense = WORKLOADS.get("bf16_16x32x32")
         if dense is not None:
             try:
-                r = run_dense_map_workload(dsa, dense, device, max(3, args.steps // 2), 3)
+                r = run_dense_map_workload(dsa, dense, device, max(20, args.steps), 5)
                 extra["bf16_16x32x32_dense_map"] = {k2: round(v2, 4) for k2, v2 in r.items()}
             except Exception as e:
                 extra["bf16_16x32x32_dense_map"] = {"error": str(e)}
         if w.dtype == "bf16":
             name = f"{w.name}_lists{w.window_tiles}"
             try:
-                r = run_list_workload(dsa, w, device, max(3, args.steps // 2), 3, w.window_tiles)
+                r = run_list_workload(dsa, w, device, max(20, args.steps), 5, w.window_tiles)
                 extra[name] = {k2: (round(v2, 4) if isinstance(v2, float) else v2) for k2, v2 in r.items()}
             except Exception as e:
                 extra[name] = {"error": str(e)}
             name = f"{w.name}_text_prefix"
             try:
-                r = run_prefix_workload(dsa, w, device, max(3, args.steps // 2), 3)
+                r = run_prefix_workload(dsa, w, device, max(20, args.steps), 5)
                 extra[name] = {k2: (round(v2, 4) if isinstance(v2, float) else v2) for k2, v2 in r.items()}
             except Exception as e:
                 extra[name] = {"error": str(e)}
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, threads, secs = oracle_sample_rate(w, 12.0)
-        cpu = {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": desc + f", {secs:.1f} s"}
+    elif rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_fwd_rate(w, host_inputs(w.replace(B=1, heads=1)), 12.0)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -649,8 +734,10 @@ def main():
     fwd_tflops = res["fwd_tflops"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "warmup": args.warmup, "ms_per_step": step_ms, "ms_per_step_mean": step_ms_mean,
+        "timing": "median of the per-step CUDA-event times of the timed steps (max over ranks)",
+        "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": workload_config(w, world),
         "pct_of_peak": {"nominal_2250": 100 * fwd_tflops / NOMINAL_BF16_TFLOPS,
                         f"{src}_{burst:g}": 100 * fwd_tflops / burst},

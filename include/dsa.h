@@ -139,9 +139,12 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
  * inside the library, held by every GPU that loads it until the process exits, so a
  * problem must satisfy  roundup(3 * nTiles, 64) + nTiles * Wt <= 65536;  larger ones
  * return DSA_ERR_UNSUPPORTED before anything is launched.  The first call on each device
- * looks up the array's device address (make that first call before any stream capture).
- * All calls on a device share the array: calls whose work overlaps on the GPU (other
- * streams, other threads) race and must be serialized by the caller. */
+ * looks up the array's device address (make that first call before any stream capture);
+ * the address is cached with the context it was found in and looked up again, on the next
+ * call, if the device's context has changed (after cudaDeviceReset).  All calls on a
+ * device share the array and each call's planner rewrites every entry its forward reads:
+ * calls whose work overlaps on the GPU (other streams, other threads) race and must be
+ * serialized by the caller. */
 dsa_status_t dsa_fwd_noalloc(const dsa_problem_t* p, const void* q, const void* k, const void* v,
                              const int32_t* tile_offsets, void* out, float* lse, void* stream);
 

@@ -461,6 +461,37 @@ def backward_dkdv_tiles(geo: Geometry, q, k, v, dout, offsets, sel=None):
     return dk, dv
 
 
+def backward_head(geo: Geometry, q, k, v, dout, offsets, h: int):
+    """Full backward of one (b, head) slice h: dq, dk, dv as [N, d] float64 (token order).
+
+    The definition of the header of dsa_oracle.c, grouped by query tile: for each query tile
+    i with key set K(i) (the oracle's plan), S = scale Q_i K^T, lse by max subtraction,
+    P = exp(S - lse), dP = dO_i V^T, dS = P (dP - rowsum(P dP)); then dq_i = scale dS K,
+    and every key row m of K(i) gains scale dS^T Q_i (dk) and P^T dO_i (dv), so dk_m and
+    dv_m sum over every query token whose key set holds m.  numpy fp64 matrix products
+    serve as the sums; one head is a few seconds (the C functions recompute each query
+    row's softmax per key tile, which is far slower for whole heads)."""
+    N, d, sc = geo.n_tokens, geo.d, geo.scale
+    Q, K, V, dO = (_head_slice(t, geo, h) for t in (q, k, v, dout))
+    _, kv, _, _ = plan(geo.G, geo.window, offsets)
+    tiles_tok = geo.tile_token_index()
+    dq, dk, dv = np.zeros((N, d)), np.zeros((N, d)), np.zeros((N, d))
+    for i in range(geo.n_tiles):
+        rows = tiles_tok[i]
+        keys = tiles_tok[kv[i]].reshape(-1)
+        s = sc * (Q[rows] @ K[keys].T)
+        mx = s.max(axis=1, keepdims=True)
+        lse = mx + np.log(np.exp(s - mx).sum(axis=1, keepdims=True))
+        P = np.exp(s - lse)
+        dP = dO[rows] @ V[keys].T
+        dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+        dq[rows] = sc * (dS @ K[keys])
+        # a window lists each of its tiles once, so `keys` has no repeated row
+        dk[keys] += sc * (dS.T @ Q[rows])
+        dv[keys] += P.T @ dO[rows]
+    return dq, dk, dv
+
+
 def backward(geo: Geometry, q, k, v, dout, offsets):
     """Full backward: dq, dk, dv as [B, heads, T, H, W, d] float64."""
     dq_t = backward_dq_tiles(geo, q, k, v, dout, offsets)

@@ -1,7 +1,8 @@
 """GPU backward (dQ, dK, dV of sum(O * dO)) against the fp64 oracle.
 
-Small problems are compared in full; the full-size adaptation workload on sampled query
-tiles (dQ) and key tiles (dK, dV), with the forward outputs the GPU produced."""
+Small problems are compared in full; the full-size adaptation workload on two whole
+(batch, head) slices and on sampled query tiles (dQ) and key tiles (dK, dV) of the others,
+with the forward outputs the GPU produced."""
 import numpy as np
 import pytest
 import torch
@@ -46,6 +47,11 @@ def test_bwd_small_full(w):
 
 
 def test_bwd_adaptation_workload_sampled():
+    """The full-size adaptation workload (B2 h12, 480p grid, 140 tiles, 3x3x5 windows):
+    every dQ, dK, dV element of two whole (batch, head) slices (the first and the last, so
+    every tile, both grid corners and every in-degree of the inverse plan), then 16 query
+    tiles (dQ) and 16 key tiles (dK, dV) spread over the other slices: the key tiles with the
+    largest and the smallest inverse-plan rows, the eight grid corners and random tiles."""
     w = WORKLOADS["adapt_480p_b2"]
     inp = make_inputs(w)
     dq, dk, dv = run_gpu(w, inp)
@@ -54,21 +60,34 @@ def test_bwd_adaptation_workload_sampled():
     tok = geo.tile_token_index()
     rng = np.random.default_rng(1)
 
+    def head(t, bh):
+        return t.reshape(BH, geo.n_tokens, w.d)[bh].float().cpu().numpy()
+
+    for bh in (0, BH - 1):
+        ref = oracle.backward_head(geo, inp.q, inp.k, inp.v, inp.dout, inp.offsets, bh)
+        for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+            assert_close(head(got, bh), r, "bf16", f"{name} of (batch, head) {bh}")
+
     def gather(t, bh, tiles):
         flat = t.reshape(BH, geo.n_tokens, w.d)
         ib = torch.as_tensor(np.repeat(bh, geo.tile_tokens), device=t.device, dtype=torch.long)
         it = torch.as_tensor(tok[tiles].reshape(-1), device=t.device, dtype=torch.long)
         return flat[ib, it].float().cpu().numpy().reshape(len(bh), geo.tile_tokens, w.d)
 
-    bh = np.array([0, BH - 1, int(rng.integers(0, BH))], np.int32)
-    qt = np.array([0, geo.n_tiles - 1, int(rng.integers(0, geo.n_tiles))], np.int32)
-    ref_dq = oracle.backward_dq_tiles(geo, inp.q, inp.k, inp.v, inp.dout, inp.offsets, (bh, qt))
-    assert_close(gather(dq, bh, qt), ref_dq, "bf16", "dq")
-    kb = np.array([BH - 1, int(rng.integers(0, BH))], np.int32)
-    kt = np.array([geo.n_tiles - 1, int(rng.integers(0, geo.n_tiles))], np.int32)
+    _, _, row_ptr, _ = oracle.plan(geo.G, geo.window, inp.offsets)
+    indeg = np.diff(row_ptr)
+    Gt, Gh, Gw = geo.G
+    corners = [(t * Gh + h) * Gw + x for t in (0, Gt - 1) for h in (0, Gh - 1) for x in (0, Gw - 1)]
+    kt = np.array([int(np.argmax(indeg)), int(np.argmin(indeg))] + corners, np.int32)
+    kt = np.concatenate([kt, rng.choice(geo.n_tiles, 16 - len(kt), replace=False)]).astype(np.int32)
+    kb = rng.integers(1, BH - 1, len(kt)).astype(np.int32)
     ref_dk, ref_dv = oracle.backward_dkdv_tiles(geo, inp.q, inp.k, inp.v, inp.dout, inp.offsets, (kb, kt))
     assert_close(gather(dk, kb, kt), ref_dk, "bf16", "dk")
     assert_close(gather(dv, kb, kt), ref_dv, "bf16", "dv")
+    qt = np.concatenate([np.array(corners, np.int32), rng.choice(geo.n_tiles, 8, replace=False)]).astype(np.int32)
+    qb = rng.integers(1, BH - 1, len(qt)).astype(np.int32)
+    ref_dq = oracle.backward_dq_tiles(geo, inp.q, inp.k, inp.v, inp.dout, inp.offsets, (qb, qt))
+    assert_close(gather(dq, qb, qt), ref_dq, "bf16", "dq")
 
 
 def test_bwd_every_gradient_written():

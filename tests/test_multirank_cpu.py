@@ -1,6 +1,7 @@
-"""Multi-rank host logic of the benchmark on CPU with two gloo ranks: every rank solves an
-independent problem (no data-path collective); the step time is the max over ranks and the
-whole-job value counts the work of all ranks."""
+"""Multi-rank host logic on CPU with gloo ranks: in the benchmark every rank solves an
+independent problem (no data-path collective), the step time is the max over ranks and the
+whole-job value counts the work of all ranks; one problem split over ranks by (batch, head)
+slices reassembles exactly."""
 import os
 import socket
 
@@ -125,3 +126,77 @@ def test_nvml_sampler_reads_reasons_from_a_fake_nvml():
     assert got["samples"] > 5 and got["in_timed_region"]
     assert got["sm_mhz"] == 1500 and got["sm_max_mhz"] == 1965 and got["power_w"] == 990.0
     assert got["reasons"] == ["sw_power_cap"] and got["source"] == "nvml"
+
+
+def test_head_range_covers_every_slice_once():
+    import video_dit_sparse_dsa_b200 as dsa
+
+    for n in (1, 2, 5, 24, 48):
+        for world in (1, 2, 3, 4, 8):
+            ranges = [dsa.head_range(n, r, world) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == n
+            assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+            sizes = [hi - lo for lo, hi in ranges]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def _head_split_worker(rank, world, port, q):
+    # one OpenMP thread: the oracle's dK, dV sums then run in one fixed order, so results
+    # can be compared bit for bit (torch shares the process's OpenMP runtime with the
+    # oracle's library and sets its thread count)
+    torch.set_num_threads(1)
+    import numpy as np
+
+    import oracle
+    import video_dit_sparse_dsa_b200 as dsa
+    from dsa_inputs import Workload, make_inputs
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = Workload("split", 2, 3, 16, (4, 4, 6), (2, 2, 2), (2, 1, 3), (-2, 2), "bf16", 71, backward=True)
+        inp = make_inputs(w)
+        BH = w.B * w.heads
+        lo, hi = dsa.head_range(BH, rank, world)
+        flat = lambda t: t.reshape((BH, 1) + tuple(w.grid) + (w.d,))[lo:hi]
+        part = w.replace(B=hi - lo, heads=1)
+        geo = oracle.Geometry.of(part)
+        out, lse = oracle.forward(geo, flat(inp.q), flat(inp.k), flat(inp.v), inp.offsets)
+        grads = oracle.backward(geo, flat(inp.q), flat(inp.k), flat(inp.v), flat(inp.dout), inp.offsets)
+        # ranks hold different numbers of slices: pad to the longest, gather, trim
+        most = -(-BH // world)
+        pieces = []
+        for a in (out, lse) + tuple(grads):
+            a = torch.from_numpy(np.ascontiguousarray(a.reshape(hi - lo, -1)))
+            pad = torch.zeros((most, a.shape[1]), dtype=a.dtype)
+            pad[: hi - lo] = a
+            got = [torch.zeros_like(pad) for _ in range(world)]
+            dist.all_gather(got, pad)
+            pieces.append(torch.cat([g[: dsa.head_range(BH, r, world)[1] - dsa.head_range(BH, r, world)[0]]
+                                     for r, g in enumerate(got)]))
+        if rank == 0:
+            full = oracle.Geometry.of(w)
+            ref_o, ref_l = oracle.forward(full, inp.q, inp.k, inp.v, inp.offsets)
+            ref_g = oracle.backward(full, inp.q, inp.k, inp.v, inp.dout, inp.offsets)
+            refs = [ref_o, ref_l] + list(ref_g)
+            same = [bool(np.array_equal(p.numpy(), np.asarray(r).reshape(BH, -1))) for p, r in zip(pieces, refs)]
+            q.put(same)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_one_problem_split_by_heads_over_two_gloo_ranks_reassembles_exactly():
+    """Two gloo ranks each take their (batch, head) slices of one seeded problem, run the
+    forward and backward oracle on them alone and gather the results: bit for bit the
+    single-rank oracle's (slices are independent, so the split needs no other exchange)."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_head_split_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+        assert p.exitcode == 0
+    assert q.get(timeout=5) == [True] * 5

@@ -14,7 +14,9 @@ tile-granular sliding-window form of "Fast Video Generation with Sliding Tile At
 * softmax rows sum to one (V = 1 gives O = 1; V = identity exposes P), and the LSE
   normalises each row;
 * masked dense attention with the brute-force mask = the windowed oracle;
-* backward = central finite differences of L = sum(O * dO) in float64;
+* backward = central finite differences of L = sum(O * dO) in float64 (the per-tile C
+  functions and the whole-head function grouped by query tile), and with a covering window
+  the whole-head backward = torch autograd of dense attention;
 * dv = P^T dO with P read off the forward (V = identity).
 """
 import os
@@ -320,6 +322,57 @@ def test_backward_selection_matches_full():
         np.testing.assert_allclose(dq_t[s], flat(dq, geo)[bh, tok[t]], rtol=0, atol=1e-13)
         np.testing.assert_allclose(dk_t[s], flat(dk, geo)[bh, tok[t]], rtol=0, atol=1e-13)
         np.testing.assert_allclose(dv_t[s], flat(dv, geo)[bh, tok[t]], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("window", [(2, 1, 2), (3, 2, 2)])
+def test_backward_head_finite_differences(window):
+    """The whole-head backward (grouped by query tile) against central finite differences of
+    L = sum(O * dO), computed from the forward alone."""
+    geo = oracle.Geometry(1, 2, 3, (3, 2, 4), (1, 2, 2), window)
+    q, k, v, dout = rand_inputs(geo, 18)
+    off = rand_offsets(geo, -1, 1, 19)
+    h, hh = 1e-5, 1
+    grads = oracle.backward_head(geo, q, k, v, dout, off, hh)
+    for x, g, name in zip((q, k, v), grads, ("q", "k", "v")):
+        xf = x.reshape(geo.B * geo.heads, -1)[hh]
+        fd = np.zeros(xf.numel())
+        for e in range(xf.numel()):
+            old = float(xf[e])
+            xf[e] = old + h
+            lp = _loss(geo, q, k, v, dout, off)
+            xf[e] = old - h
+            lm = _loss(geo, q, k, v, dout, off)
+            xf[e] = old
+            fd[e] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g.reshape(-1), fd, rtol=0, atol=2e-9, err_msg=name)
+
+
+def test_backward_head_full_window_is_autograd_of_dense_attention():
+    """With a window covering the grid, the whole-head backward is the gradient of dense
+    softmax attention (torch autograd, float64)."""
+    geo = oracle.Geometry(1, 2, 8, (2, 4, 4), (1, 2, 2), (2, 2, 2))
+    q, k, v, dout = rand_inputs(geo, 20)
+    off = rand_offsets(geo, -2, 2, 21)
+    BH, N, d = geo.B * geo.heads, geo.n_tokens, geo.d
+    qa, ka, va = (t.reshape(BH, N, d).clone().requires_grad_(True) for t in (q, k, v))
+    o = torch.softmax(geo.scale * qa @ ka.transpose(1, 2), dim=-1) @ va
+    (o * dout.reshape(BH, N, d)).sum().backward()
+    for hh in range(BH):
+        got = oracle.backward_head(geo, q, k, v, dout, off, hh)
+        for g, ref in zip(got, (qa.grad[hh], ka.grad[hh], va.grad[hh])):
+            np.testing.assert_allclose(g, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_backward_head_equals_tile_functions():
+    """The whole-head backward equals the C oracle's per-tile backward on every head."""
+    geo = oracle.Geometry(2, 2, 16, (4, 4, 6), (2, 2, 2), (2, 1, 3))
+    q, k, v, dout = rand_inputs(geo, 22)
+    off = rand_offsets(geo, -2, 2, 23)
+    dq, dk, dv = oracle.backward(geo, q, k, v, dout, off)
+    for hh in range(geo.B * geo.heads):
+        got = oracle.backward_head(geo, q, k, v, dout, off, hh)
+        for g, ref in zip(got, (dq, dk, dv)):
+            np.testing.assert_allclose(g, flat(ref, geo)[hh], rtol=0, atol=1e-12)
 
 
 # ------------------------------------------------------------------------------------

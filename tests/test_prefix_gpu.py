@@ -161,8 +161,9 @@ def test_prefix_backward_16x32x32_grid_full():
 
 
 def test_prefix_backward_720p_sampled():
-    """The 720p grid with its ~1% of text tokens, as the benchmark times it: gradients of one
-    (batch, head) on sampled rows (video and text queries and keys, first and last rows)."""
+    """The 720p grid with its ~1% of text tokens, as the benchmark times it: gradients of two
+    (batch, head) slices on sampled rows (video and text queries and keys, first and last
+    rows)."""
     w = WORKLOADS["bf16_720p"]
     L = text_length(w)
     inp = make_inputs(w)
@@ -170,19 +171,19 @@ def test_prefix_backward_720p_sampled():
     grads, do, do_t = run_backward(w, inp, txt, 77)
     geo = oracle.Geometry.of(w)
     rng = np.random.default_rng(6)
-    h = 7
     N = geo.n_tokens
-    q_rows = np.concatenate([[0, N - 1], rng.integers(0, N, 4)])
-    k_rows = np.concatenate([[1, N - 2], rng.integers(0, N, 4)])
-    t_rows = np.concatenate([[0, L - 1], rng.integers(0, L, 3)])
-    ref = oracle.backward_prefix_sampled(geo, inp.q, inp.k, inp.v, do, inp.offsets, txt.q, txt.k, txt.v, do_t, h,
-                                         q_rows, t_rows, k_rows, t_rows)
     BH = w.B * w.heads
+    for h in (7, BH - 1):
+        q_rows = np.concatenate([[0, N - 1], rng.integers(0, N, 6)])
+        k_rows = np.concatenate([[1, N - 2], rng.integers(0, N, 6)])
+        t_rows = np.concatenate([[0, L - 1], rng.integers(0, L, 4)])
+        ref = oracle.backward_prefix_sampled(geo, inp.q, inp.k, inp.v, do, inp.offsets, txt.q, txt.k, txt.v, do_t,
+                                             h, q_rows, t_rows, k_rows, t_rows)
 
-    def rows(t, idx):
-        return t.reshape(BH, -1, w.d)[h][torch.as_tensor(idx, device=t.device)].float().cpu().numpy()
+        def rows(t, idx):
+            return t.reshape(BH, -1, w.d)[h][torch.as_tensor(idx, device=t.device)].float().cpu().numpy()
 
-    got = (rows(grads[0], q_rows), rows(grads[3], t_rows), rows(grads[1], k_rows), rows(grads[2], k_rows),
-           rows(grads[4], t_rows), rows(grads[5], t_rows))
-    for g, r, name in zip(got, ref, ("dq", "dq_text", "dk", "dv", "dk_text", "dv_text")):
-        assert_close(g, r, w.dtype, name)
+        got = (rows(grads[0], q_rows), rows(grads[3], t_rows), rows(grads[1], k_rows), rows(grads[2], k_rows),
+               rows(grads[4], t_rows), rows(grads[5], t_rows))
+        for g, r, name in zip(got, ref, ("dq", "dq_text", "dk", "dv", "dk_text", "dv_text")):
+            assert_close(g, r, w.dtype, f"{name} of (batch, head) {h}")

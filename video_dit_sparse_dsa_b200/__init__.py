@@ -32,6 +32,11 @@ DSA_WS_FWD, DSA_WS_BWD = 0, 1
 _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_CUDA",
            4: "DSA_ERR_TIMEOUT", 5: "DSA_ERR_WORKSPACE", 6: "DSA_ERR_DEVICE"}
 
+# kernel launches of one dsa_fwd call (planner, forward) and of one dsa_bwd call (planner,
+# the inverse map's count, scan and fill, D preprocess, backward, dQ conversion)
+FWD_LAUNCHES = 2
+BWD_LAUNCHES = 7
+
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_version", "dsa_status_string", "dsa_plan_shape", "dsa_workspace_size", "dsa_plan", "dsa_fwd",
            "dsa_fwd_host_bytes", "dsa_fwd_host", "dsa_bwd", "dsa_device_status", "dsa_fwd_noalloc",
@@ -107,6 +112,19 @@ def load_library(path: Optional[str] = None):
     if path is None:
         _lib = lib
     return lib
+
+
+def head_range(n_slices: int, rank: int, world: int):
+    """The (batch, head) slices [lo, hi) of a problem with n_slices = B * heads that rank
+    `rank` of `world` takes when one problem is split over GPUs by heads.  Slices are
+    independent problems (each has its own softmax), so ranks run the same calls on their
+    slices with no collective; contiguous ranges of near-equal size, the first
+    n_slices % world ranks one slice longer."""
+    if world <= 0 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of {world}")
+    base, extra = divmod(int(n_slices), world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
 
 
 def make_problem(B, heads, d, grid, tile, window, scale=None, dtype=DSA_BF16) -> Problem:

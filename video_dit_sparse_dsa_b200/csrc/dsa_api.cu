@@ -293,7 +293,22 @@ dsa_status_t launch_list_check(const Geom& g, const int32_t* row_ptr, const int3
 
 dsa_status_t launch_plan(const Geom& g, const int32_t* offsets, int32_t* starts, int32_t* kv_tiles,
                          int32_t* row_ptr, int32_t* q_tiles, cudaStream_t s) {
-  dsa::plan_kernel<<<1, 1024, 0, s>>>(plan_geom(g), offsets, starts, kv_tiles, row_ptr, q_tiles);
+  const dsa::PlanGeom pg = plan_geom(g);
+  dsa::plan_kernel<<<1, 1024, 0, s>>>(pg, offsets, starts, kv_tiles);
+  dsa_status_t st = launch_status();
+  if (st != DSA_OK || row_ptr == nullptr || q_tiles == nullptr) return st;
+  // inverse map: one warp per key tile, at most 8 warps per CTA and 8 CTAs per SM
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  const int64_t want = (static_cast<int64_t>(g.n_tiles) + 7) / 8;
+  const unsigned blocks = static_cast<unsigned>(want < 8 * sms ? want : 8 * sms);
+  dsa::plan_inverse_kernel<false><<<blocks, 256, 0, s>>>(pg, starts, row_ptr, nullptr);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  dsa::plan_scan_kernel<<<1, 1024, 0, s>>>(g.n_tiles, row_ptr);
+  st = launch_status();
+  if (st != DSA_OK) return st;
+  dsa::plan_inverse_kernel<true><<<blocks, 256, 0, s>>>(pg, starts, row_ptr, q_tiles);
   return launch_status();
 }
 
@@ -1132,23 +1147,54 @@ constexpr int kNoAllocPlanInts = 65536;  // 256 KB: 3 starts + Wt key tiles per 
 static __device__ __align__(256) int32_t g_noalloc_plan[kNoAllocPlanInts];
 
 constexpr int kNoAllocMaxDevices = 128;
-int32_t* g_noalloc_addr[kNoAllocMaxDevices];
+struct NoAllocAddr {
+  void* ctx;       // the context the address was looked up in
+  int32_t* addr;   // device address of g_noalloc_plan in that context
+};
+NoAllocAddr g_noalloc_addr[kNoAllocMaxDevices];
 std::mutex g_noalloc_mutex;
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, looked up once through the runtime (no libcuda link).
+CtxGetCurrentFn ctx_get_current_fn() {
+  static const CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(ptr);
+    return nullptr;
+  }();
+  return fn;
+}
+
+void* current_context() {
+  CtxGetCurrentFn fn = ctx_get_current_fn();
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
 // Device address of g_noalloc_plan on the current device.  In host code the array's name
-// is only a host-side stand-in, so the address is looked up once per device, with that
-// device current, and cached.
+// is only a host-side stand-in, so the address is looked up with the device current and
+// cached per device, together with the context it belongs to: if the device's context
+// has changed since (cudaDeviceReset, then a new primary context, into which the module
+// may load elsewhere), the address is looked up again.
 dsa_status_t noalloc_plan_address(int32_t** addr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
   if (dev < 0 || dev >= kNoAllocMaxDevices) return DSA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
+  NoAllocAddr& e = g_noalloc_addr[dev];
+  void* ctx = current_context();
+  if (e.addr == nullptr || ctx == nullptr || ctx != e.ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_plan) != cudaSuccess || ptr == nullptr) return DSA_ERR_CUDA;
-    g_noalloc_addr[dev] = static_cast<int32_t*>(ptr);
+    e.addr = static_cast<int32_t*>(ptr);
+    e.ctx = current_context();  // the lookup makes the device's primary context current
   }
-  *addr = g_noalloc_addr[dev];
+  *addr = e.addr;
   return DSA_OK;
 }
 

@@ -9,8 +9,8 @@
 // Optionally the inverse map is built as CSR: row j lists, ascending, the query tiles whose
 // window holds key tile j (the backward pass walks it key-tile-major).
 //
-// One CTA of 1024 threads: the plans here have at most a few thousand tiles, so the
-// O(nTiles^2) containment scan of the inverse map costs microseconds.
+// The forward plan is one CTA of 1024 threads (a thread per query tile, Wt entries each);
+// the inverse map spreads its containment tests over the whole grid.
 #pragma once
 
 #include <stdint.h>
@@ -38,8 +38,7 @@ __device__ __forceinline__ bool plan_holds(const PlanGeom& g, const int32_t* sta
 }
 
 __global__ void __launch_bounds__(1024) plan_kernel(PlanGeom g, const int32_t* __restrict__ offsets,
-                                                    int32_t* __restrict__ starts, int32_t* __restrict__ kv_tiles,
-                                                    int32_t* __restrict__ row_ptr, int32_t* __restrict__ q_tiles) {
+                                                    int32_t* __restrict__ starts, int32_t* __restrict__ kv_tiles) {
   const int n = g.n_tiles;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const int it = i / (g.G[1] * g.G[2]), ih = (i / g.G[2]) % g.G[1], iw = i % g.G[2];
@@ -55,18 +54,37 @@ __global__ void __launch_bounds__(1024) plan_kernel(PlanGeom g, const int32_t* _
       for (int b = sh; b < sh + g.w[1]; ++b)
         for (int c = sw; c < sw + g.w[2]; ++c) dst[e++] = (a * g.G[1] + b) * g.G[2] + c;
   }
-  if (row_ptr == nullptr || q_tiles == nullptr) return;
-  __syncthreads();
+}
 
-  // in-degree of each key tile, parked in row_ptr[j + 1]
-  for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    int cnt = 0;
-    for (int i = 0; i < n; ++i) cnt += plan_holds(g, starts, i, j) ? 1 : 0;
-    row_ptr[j + 1] = cnt;
+// The inverse map, in three launches after plan_kernel: for every key tile j the query
+// tiles whose window holds j, ascending.  One warp per key tile (grid-stride over the
+// warps of the whole grid) tests the query tiles 32 at a time and takes the hits from a
+// ballot, so each row comes out in ascending order without a sort and the work
+// (nTiles^2 / 32 warp steps) is spread over every SM.
+//   kFill = false: the count of row j goes to row_ptr[j + 1];
+//   kFill = true : row j is written from row_ptr[j] (after plan_scan_kernel).
+template <bool kFill>
+__global__ void __launch_bounds__(256) plan_inverse_kernel(PlanGeom g, const int32_t* __restrict__ starts,
+                                                           int32_t* __restrict__ row_ptr,
+                                                           int32_t* __restrict__ q_tiles) {
+  const int n = g.n_tiles, lane = threadIdx.x & 31;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t j = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; j < n; j += nwarps) {
+    int pos = kFill ? row_ptr[j] : 0;
+    for (int base = 0; base < n; base += 32) {
+      const int i = base + lane;
+      const bool hit = i < n && plan_holds(g, starts, i, static_cast<int>(j));
+      const unsigned m = __ballot_sync(0xffffffffu, hit);
+      if (kFill && hit) q_tiles[pos + __popc(m & ((1u << lane) - 1u))] = i;
+      pos += __popc(m);
+    }
+    if (!kFill && lane == 0) row_ptr[j + 1] = pos;
   }
-  __syncthreads();
+}
 
-  // exclusive scan of the in-degrees, 1024 at a time
+// Exclusive scan of the counts row_ptr[1..n] in place (row_ptr[0] = 0), one CTA of 1024
+// threads, 1024 entries at a time.
+__global__ void __launch_bounds__(1024) plan_scan_kernel(int n, int32_t* __restrict__ row_ptr) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -100,12 +118,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(PlanGeom g, const int32_t* _
     if (j < n) row_ptr[j + 1] = x;
     if (threadIdx.x == blockDim.x - 1) carry = x;
     __syncthreads();
-  }
-
-  for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    int pos = row_ptr[j];
-    for (int i = 0; i < n; ++i)
-      if (plan_holds(g, starts, i, j)) q_tiles[pos++] = i;
   }
 }
 
