@@ -123,8 +123,12 @@ dsa_status_t dsa_fwd_host(const dsa_problem_t* p, const void* q_host, const void
                           size_t dev_bytes, void* stream);
 
 /* Backward of L = sum(out * dout) (gradients of the forward above with respect to q, k, v;
- * the integer offsets have none).  out and lse are the forward's outputs for the same
- * inputs.  Writes dq, dk, dv (dtype of p).  workspace: at least
+ * the integer offsets have none; the full-parameter adaptation of the MegaSlide-DiT
+ * abstract needs them).  out and lse are the forward's outputs for the same inputs.
+ * Writes dq, dk, dv (dtype of p).  Two passes on the tensor cores: a key-major kernel sums
+ * dk and dv of each key row over the query tiles whose window holds it, a query-major
+ * kernel sums dq of each query row over its window; every sum runs in one CTA in a fixed
+ * order, so the gradients are identical from run to run.  workspace: at least
  * dsa_workspace_size(p, DSA_WS_BWD) bytes; its contents on entry do not matter.
  * bf16 only. */
 dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,

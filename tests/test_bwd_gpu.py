@@ -100,3 +100,20 @@ def test_bwd_every_gradient_written():
     torch.cuda.synchronize()
     for t in (dq, dk, dv):
         assert torch.isfinite(t.float()).all()
+
+
+def test_bwd_is_bit_identical_across_runs():
+    """dQ is summed by one CTA per query row in the fixed order of the row's key list, dK and
+    dV by one CTA per key row in the fixed order of the inverse lists: two runs of the
+    backward on the same inputs give the same bits (the adaptation grid, 4 heads)."""
+    w = WORKLOADS["adapt_480p_b2"].replace(name="bwd_repeat", B=1, heads=4, seed=36)
+    inp = make_inputs(w)
+    q, k, v, dout, off = inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.dout.cuda(), inp.offsets.cuda()
+    out, lse = dsa.forward(q, k, v, off, w.tile, w.window, w.scale)
+    first = dsa.backward(q, k, v, out, lse, dout, off, w.tile, w.window, w.scale)
+    for _ in range(2):
+        again = dsa.backward(q, k, v, out, lse, dout, off, w.tile, w.window, w.scale)
+        for a, b, name in zip(first, again, ("dq", "dk", "dv")):
+            assert torch.equal(a, b), f"{name} differs between runs"
+    st = dsa.device_status()
+    assert st[0] == 0, f"device status {st}"

@@ -239,6 +239,6 @@ def test_forward_and_backward_replay_from_a_cuda_graph():
     torch.cuda.synchronize()
     assert dsa.device_status()[0] == 0
     assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
-    assert torch.equal(dk, ref_g[1]) and torch.equal(dv, ref_g[2])  # dQ sums with atomics: compare loosely
-    assert float((dq.float() - ref_g[0].float()).abs().max()) <= 1e-3
+    # every gradient is summed in a fixed order: the replays match the direct call bit for bit
+    assert torch.equal(dq, ref_g[0]) and torch.equal(dk, ref_g[1]) and torch.equal(dv, ref_g[2])
     del g

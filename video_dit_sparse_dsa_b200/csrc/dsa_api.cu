@@ -10,6 +10,7 @@
 
 #include "../../include/dsa.h"
 #include "dsa_bwd_bf16.cuh"
+#include "dsa_bwd_dq.cuh"
 #include "dsa_device_status.cuh"
 #include "dsa_fwd_bf16.cuh"
 #include "dsa_fwd_f32.cuh"
@@ -105,7 +106,7 @@ struct BwdWorkspace {
   size_t bytes;
 };
 
-BwdWorkspace bwd_workspace(const Geom& g, int d, void* base) {
+BwdWorkspace bwd_workspace(const Geom& g, int d, void* base, bool with_dq_acc = false) {
   BwdWorkspace w;
   uint8_t* b = static_cast<uint8_t*>(base);
   size_t off = 0;
@@ -119,20 +120,22 @@ BwdWorkspace bwd_workspace(const Geom& g, int d, void* base) {
   off += round_up(sizeof(int32_t) * static_cast<size_t>(g.n_tiles) * g.Wt, kAlign);
   w.delta = reinterpret_cast<float*>(b + off);
   off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N), kAlign);
-  w.dq_acc = reinterpret_cast<float*>(b + off);
-  off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N) * d, kAlign);
+  w.dq_acc = nullptr;
+  if (with_dq_acc) {
+    w.dq_acc = reinterpret_cast<float*>(b + off);
+    off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N) * d, kAlign);
+  }
   w.bytes = off;
   return w;
 }
 
 // Backward over a caller's key-tile lists: the inverse CSR built on the device, then the
-// same D and dQ accumulator scratch as dsa_bwd.
+// same D scratch as dsa_bwd.
 struct ListBwdWorkspace {
   int32_t* counts;   // [n_lists, n_tiles] scratch of the inversion
   int32_t* row_ptr;  // [n_lists, n_tiles + 1] inverse CSR
   int32_t* q_tiles;  // [nnz]
   float* delta;      // [BH, N]
-  float* dq_acc;     // [BH, N, d]
   size_t bytes;
 };
 
@@ -148,9 +151,8 @@ ListBwdWorkspace list_bwd_workspace(const Geom& g, int d, int nnz, int n_lists, 
   off += round_up(sizeof(int32_t) * static_cast<size_t>(nnz > 0 ? nnz : 1), kAlign);
   w.delta = reinterpret_cast<float*>(b + off);
   off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N), kAlign);
-  w.dq_acc = reinterpret_cast<float*>(b + off);
-  off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N) * d, kAlign);
   w.bytes = off;
+  (void)d;
   return w;
 }
 
@@ -385,6 +387,8 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   bp.scale_log2 = p->scale * 1.4426950408889634f;
   bp.n_units = static_cast<int>(g.BH * bp.S * g.n_tiles);
   const bool map_mode = bmap != nullptr;
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   auto kernel = map_mode ? dsa::fwd_bf16_kernel<dsa::fwd::kModeMap>
                          : (bp.Lx > 0 ? dsa::fwd_bf16_kernel<dsa::fwd::kModeFwdX> : dsa::fwd_bf16_kernel<dsa::fwd::kModeFwd>);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::fwd::kSmemBytes) != cudaSuccess)
@@ -393,8 +397,6 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
   if (fa.numRegs < dsa::fwd::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
-  int sms = 0;
-  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
   kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, tkx, tvx, bp);
   return launch_status();
@@ -475,12 +477,13 @@ dsa_status_t launch_bwd_kernel(const dsa::BwdBf16Params& bp, const CUtensorMap& 
       return DSA_ERR_CUDA;
   }
   auto kernel = dsa::bwd_bf16_kernel<kFlatK, kExtra>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::bwd::kSmemBytes) != cudaSuccess)
+  constexpr uint32_t smem = dsa::bwd::Layout<true>::kSmemBytes;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DSA_ERR_CUDA;
   int sms = 0;
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
-  kernel<<<grid, dsa::bwd::kThreads, dsa::bwd::kSmemBytes, s>>>(tq, tk, tv, tdo, tlse, tdel, tqx, tdox, tlsex, tdx,
+  kernel<<<grid, dsa::bwd::kThreads, smem, s>>>(tq, tk, tv, tdo, tlse, tdel, tqx, tdox, tlsex, tdx,
                                                                  bp);
   return launch_status();
 }
@@ -541,6 +544,110 @@ dsa_status_t launch_bwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   const int64_t n8 = rows * p->d / 8;
   dsa::bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
       dq_acc, static_cast<__nv_bfloat16*>(dq), p->scale, n8);
+  return launch_status();
+}
+
+// Key tiles of each query tile as the forward takes them: the window plan's kv_tiles
+// (row_ptr null) or a caller's CSR (row_ptr, nnz entries, rp_head_stride 0 or nTiles + 1).
+struct FwdKeys {
+  const int32_t* kv;
+  const int32_t* row_ptr;
+  int nnz, rp_head_stride;
+};
+
+// The backward of the window and key-tile-list forms: D = rowsum(dO * O), the key-major
+// kernel for dK and dV over the inverse lists (row_ptr, q_tiles), and the query-major
+// kernel for dQ over the forward's lists; no dQ accumulator, no atomics.
+dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
+                            const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
+                            const int32_t* q_tiles, int inv_head_stride, const FwdKeys& fk, float* delta, void* dq,
+                            void* dk, void* dv, cudaStream_t s) {
+  const int64_t rows = g.BH * g.N;
+  dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta, nullptr, rows);
+  dsa_status_t st = launch_status();
+  if (st != DSA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo, tlse, tdel;
+  if (!make_token_map(&tq, q, p, g, 64) || !make_token_map(&tk, k, p, g, 128) ||
+      !make_token_map(&tv, v, p, g, 128) || !make_token_map(&tdo, dout, p, g, 64) ||
+      !make_row_map(&tlse, lse, p, g, 64) || !make_row_map(&tdel, delta, p, g, 64))
+    return DSA_ERR_CUDA;
+  dsa::BwdBf16Params bp;
+  std::memset(&bp, 0, sizeof(bp));
+  bp.row_ptr = row_ptr;
+  bp.rp_head_stride = inv_head_stride;
+  bp.q_tiles = q_tiles;
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.n_tiles = g.n_tiles;
+  bp.KU = g.tile_tokens / 128;
+  bp.QS = g.tile_tokens / 64;
+  bp.n_units = static_cast<int>(g.BH * g.n_tiles * bp.KU);
+  bp.G1 = g.G[1];
+  bp.G2 = g.G[2];
+  bp.tt = p->tile[0];
+  bp.th = p->tile[1];
+  bp.tw = p->tile[2];
+  bp.kcs = 128 / (p->tile[1] * p->tile[2]);
+  bp.qcs = 64 / (p->tile[1] * p->tile[2]);
+  bp.T = p->T;
+  bp.H = p->H;
+  bp.W = p->W;
+  bp.N = static_cast<int>(g.N);
+  bp.scale = p->scale;
+  bp.scale_log2 = p->scale * 1.4426950408889634f;
+  bp.n_split = 1;
+  {
+    auto kernel = dsa::bwd_bf16_kernel<false, false, false>;
+    constexpr uint32_t smem = dsa::bwd::Layout<false>::kSmemBytes;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    int sms = 0;
+    if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
+    kernel<<<grid, dsa::bwd::kThreads, smem, s>>>(tq, tk, tv, tdo, tlse, tdel, tq, tdo, tlse, tdel, bp);
+    st = launch_status();
+    if (st != DSA_OK) return st;
+  }
+  // dQ: 128-row query chunks over the forward's key lists
+  CUtensorMap tq2, tdo2;
+  if (!make_token_map(&tq2, q, p, g, 128) || !make_token_map(&tdo2, dout, p, g, 128)) return DSA_ERR_CUDA;
+  dsa::BwdDqParams dp;
+  std::memset(&dp, 0, sizeof(dp));
+  dp.kv_tiles = fk.kv;
+  dp.row_ptr = fk.row_ptr;
+  dp.rp_head_stride = fk.rp_head_stride;
+  dp.nnz = fk.nnz;
+  dp.lse = lse;
+  dp.delta = delta;
+  dp.dq = static_cast<__nv_bfloat16*>(dq);
+  dp.n_tiles = g.n_tiles;
+  dp.Wt = g.Wt;
+  dp.S = g.tile_tokens / 128;
+  dp.n_units = static_cast<int>(g.BH * g.n_tiles * dp.S);
+  dp.G1 = g.G[1];
+  dp.G2 = g.G[2];
+  dp.tt = p->tile[0];
+  dp.th = p->tile[1];
+  dp.tw = p->tile[2];
+  dp.tcs = 128 / (p->tile[1] * p->tile[2]);
+  dp.T = p->T;
+  dp.H = p->H;
+  dp.W = p->W;
+  dp.N = static_cast<int>(g.N);
+  dp.scale = p->scale;
+  dp.scale_log2 = p->scale * 1.4426950408889634f;
+  auto kernel = dsa::bwd_dq_kernel;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::bdq::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  // the kernel's setmaxnreg split needs exactly the registers it was compiled for at launch
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
+  if (fa.numRegs < dsa::bdq::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(dp.n_units < sms ? dp.n_units : sms);
+  kernel<<<grid, dsa::bdq::kThreads, dsa::bdq::kSmemBytes, s>>>(tq2, tk, tv, tdo2, dp);
   return launch_status();
 }
 
@@ -745,7 +852,8 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_plan(g, tile_offsets, ws.starts, ws.kv_tiles, ws.row_ptr, ws.q_tiles, s);
   if (st != DSA_OK) return st;
-  return launch_bwd(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, ws.delta, ws.dq_acc, dq, dk, dv, s);
+  return launch_bwd_det(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, 0, FwdKeys{ws.kv_tiles, nullptr, 0, 0},
+                        ws.delta, dq, dk, dv, s);
 }
 
 size_t dsa_list_workspace_size(const dsa_problem_t* p, int32_t nnz, int32_t per_head, int32_t kind) {
@@ -828,8 +936,9 @@ dsa_status_t dsa_bwd_list(const dsa_problem_t* p, const void* q, const void* k, 
                                                                            ws.counts, ws.row_ptr, ws.q_tiles);
   st = launch_status();
   if (st != DSA_OK) return st;
-  return launch_bwd(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, ws.delta, ws.dq_acc, dq, dk, dv, s,
-                    per_head ? g.n_tiles + 1 : 0);
+  const int stride = per_head ? g.n_tiles + 1 : 0;
+  return launch_bwd_det(p, g, q, k, v, out, lse, dout, ws.row_ptr, ws.q_tiles, stride,
+                        FwdKeys{kv_list, kv_row_ptr, nnz, stride}, ws.delta, dq, dk, dv, s);
 }
 
 dsa_status_t dsa_block_map(const dsa_problem_t* p, const void* q, const void* k, const float* lse,
@@ -997,7 +1106,7 @@ struct PrefixBwdWorkspace {
 
 PrefixBwdWorkspace prefix_bwd_workspace(const Geom& g, int32_t L, void* base) {
   PrefixBwdWorkspace w;
-  w.video = bwd_workspace(g, 128, base);
+  w.video = bwd_workspace(g, 128, base, true);
   uint8_t* b = static_cast<uint8_t*>(base);
   size_t off = w.video.bytes;
   w.Lp = (L + 63) / 64 * 64;
@@ -1055,7 +1164,8 @@ dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k
   st = launch_plan(g, tile_offsets, wv.starts, wv.kv_tiles, wv.row_ptr, wv.q_tiles, s);
   if (st != DSA_OK) return st;
   if (L_text == 0)
-    return launch_bwd(p, g, q, k, v, out, lse, dout, wv.row_ptr, wv.q_tiles, wv.delta, wv.dq_acc, dq, dk, dv, s);
+    return launch_bwd_det(p, g, q, k, v, out, lse, dout, wv.row_ptr, wv.q_tiles, 0,
+                          FwdKeys{wv.kv_tiles, nullptr, 0, 0}, wv.delta, dq, dk, dv, s);
   // text rows: D, padded LSE / D copies, zeroed dQ accumulator
   const int64_t prow = g.BH * ws.Lp;
   dsa::bwd_preprocess_flat<<<static_cast<unsigned>((prow * 16 + 255) / 256), 256, 0, s>>>(

@@ -8,10 +8,14 @@
 //   dK_m = scale sum_n dS_nm q_n,   dQ_n = scale sum_m dS_nm k_m,
 // where n runs over the query tokens whose window holds key m.
 //
-// Three kernels:
-//   bwd_preprocess : D = rowsum(dO * O) (fp32) and zeroes the fp32 dQ accumulator;
-//   bwd_bf16_kernel: key-major and persistent (described above the kernel);
+// Kernels:
+//   bwd_preprocess : D = rowsum(dO * O) (fp32), and zeroes the fp32 dQ accumulator of the
+//                    forms that reduce dQ with atomics (the text prefix);
+//   bwd_bf16_kernel: key-major and persistent (described above the kernel): dK and dV, and
+//                    with kDq also dQ, added with fp32 atomics into the accumulator;
 //   bwd_dq_convert : dQ = scale * accumulator, as bf16.
+// The window and key-tile-list backward take dQ from the query-major bwd_dq_kernel
+// (dsa_bwd_dq.cuh) instead: deterministic, with no accumulator.
 #pragma once
 
 #include <stdint.h>
@@ -54,7 +58,6 @@ namespace bwd {
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kStages = 3;
 constexpr uint32_t kKBytes = 128 * 128 * 2;  // K or V of a 128-key unit
 constexpr uint32_t kKHalf = kKBytes / 2;
 constexpr uint32_t kQBytes = 64 * 128 * 2;   // Q or dO of a 64-query chunk
@@ -62,11 +65,20 @@ constexpr uint32_t kQHalf = kQBytes / 2;
 constexpr uint32_t kStageBytes = 2 * kQBytes + 1024;  // Q, dO, LSE (at +0) and D (at +512) vectors
 constexpr uint32_t kOffK = 0, kOffV = kKBytes;
 constexpr uint32_t kOffStage = 2 * kKBytes;
-constexpr uint32_t kOffDS = kOffStage + kStages * kStageBytes;  // 2 buffers of 128 x 64 bf16
 constexpr uint32_t kDSBytes = 128 * 64 * 2;
-constexpr uint32_t kOffRel = kOffDS + 2 * kDSBytes;  // 64 int32 token offsets within a query chunk
-constexpr uint32_t kOffBar = kOffRel + 256;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+// Shared-memory layout: K, V, the query-chunk ring, then (kDq only) two dS^T buffers of
+// 128 x 64 bf16 (the B operand of dQ^T), 64 int32 token offsets within a query chunk, the
+// barriers.  Without dQ the dS^T buffers' room gives the ring a fourth stage.
+template <bool kDq>
+struct Layout {
+  static constexpr int kStages = kDq ? 3 : 4;
+  static constexpr uint32_t kOffDS = kOffStage + kStages * kStageBytes;
+  static constexpr uint32_t kOffRel = kOffDS + (kDq ? 2 * kDSBytes : 0);
+  static constexpr uint32_t kOffBar = kOffRel + 256;
+  static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+};
+static_assert(Layout<true>::kSmemBytes <= 227 * 1024 && Layout<false>::kSmemBytes <= 227 * 1024,
+              "shared memory layout too large");
 constexpr uint32_t kTmemCols = 512;  // dV [0,128), dK [128,256), S^T buffers [256,384), dP^T / dQ^T [384,512)
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // K Q^T and V dO^T
 constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 128, 0, 1);  // P^T dO, dS^T Q
@@ -159,9 +171,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __res
       s = fmaf(x.x, y.x, s);
       s = fmaf(x.y, y.y, s);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + row * 128) + part * 2;
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (dq_acc != nullptr) {
+      float4* z = reinterpret_cast<float4*>(dq_acc + row * 128) + part * 2;
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int o2 = 8; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
@@ -264,7 +278,7 @@ __global__ void __launch_bounds__(256) bwd_kv_combine(const float* __restrict__ 
 // the end of either load as zeros and get P = dS = 0, and their gradients are not written.
 // kExtra: extra queries (p.Lxq of them, flat maps tmQx, tmDOx, tmLsex, tmDx) follow every
 // unit's own.
-template <bool kFlatK, bool kExtra>
+template <bool kFlatK, bool kExtra, bool kDq = true>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -273,13 +287,15 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
                     const __grid_constant__ CUtensorMap tmLsex, const __grid_constant__ CUtensorMap tmDx,
                     BwdBf16Params p) {
   using namespace bwd;
+  using L = Layout<kDq>;
+  constexpr int kStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw + pad;
-  int32_t* rel = reinterpret_cast<int32_t*>(smem + kOffRel);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  int32_t* rel = reinterpret_cast<int32_t*>(smem + L::kOffRel);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_free = bars + 1;
   uint64_t* ld_full = bars + 2;               // [kStages]
@@ -406,7 +422,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const uint64_t dKt = smem_desc_sw128(sbase + kOffK, kKHalf, 1024);       // K^T, MN-major
       const uint64_t dQk = smem_desc_sw128(sbase + kOffStage, 16, 1024);       // stage 0 Q, K-major
       const uint64_t dQm = smem_desc_sw128(sbase + kOffStage, kQHalf, 1024);   // stage 0 Q, MN-major
-      const uint64_t dSm = smem_desc_sw128(sbase + kOffDS, kKHalf, 1024);      // dS^T buffer 0, MN-major
+      const uint64_t dSm = smem_desc_sw128(sbase + L::kOffDS, kKHalf, 1024);      // dS^T buffer 0, MN-major
       int ld = 0, uc = 0, sc = 0, pc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -437,10 +453,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q (dS^T from TMEM, beside P^T)
               mma_ts_warp(tDK, tS + b * 64 + 32 + kk * 8, desc_add(q_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
+            if constexpr (kDq) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
-              mma_ss_warp(tDP + b * 64, desc_add(dKt, kk * 2048), desc_add(ds_m, kk * 2048), kIdescDQ, kk > 0);
-            mma_commit_warp(dq_full + b);
+              for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
+                mma_ss_warp(tDP + b * 64, desc_add(dKt, kk * 2048), desc_add(ds_m, kk * 2048), kIdescDQ, kk > 0);
+              mma_commit_warp(dq_full + b);
+            }
             mma_commit_warp(ld_empty + (ld0 + cc) % kStages);
           }
           if (c < n) {
@@ -456,7 +474,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
               mma_ss_warp(tS + b * 64, desc_add(dK, ko), desc_add(q_k, qo), kIdescS, kk > 0);
             }
             // dP^T overwrites the dQ^T of chunk sc - 2: wait until it has been read out
-            if (sc >= 2) ok = __all_sync(0xffffffffu, mbar_wait(dq_free + b, ((sc >> 1) - 1) & 1, abort, 62));
+            if (kDq && sc >= 2) ok = __all_sync(0xffffffffu, mbar_wait(dq_free + b, ((sc >> 1) - 1) & 1, abort, 62));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -500,7 +518,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         uint32_t sr[64], dr[64];
         tmem_ld64_wait(tS + lane_off + b * 64, sr);
         tmem_ld64_wait(tDP + lane_off + b * 64, dr);
-        const uint32_t dsrow = sbase + kOffDS + b * kDSBytes + (m >> 3) * 1024 + (m & 7) * 128;
+        const uint32_t dsrow = sbase + L::kOffDS + b * kDSBytes + (m >> 3) * 1024 + (m & 7) * 128;
 #pragma unroll
         for (int g = 0; g < 8; ++g) {  // query columns 8g..8g+7 form one 16-byte chunk
           uint32_t pk[4], dk2[4];
@@ -520,7 +538,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           for (int e = 0; e < 4; ++e) sr[4 * g + e] = pk[e];  // packed P^T of columns 8g..8g+7
 #pragma unroll
           for (int e = 0; e < 4; ++e) dr[4 * g + e] = dk2[e];  // packed dS^T (dP^T of these columns is used)
-          st_shared_v4(dsrow + ((g ^ (m & 7)) << 4), dk2[0], dk2[1], dk2[2], dk2[3]);
+          if constexpr (kDq) st_shared_v4(dsrow + ((g ^ (m & 7)) << 4), dk2[0], dk2[1], dk2[2], dk2[3]);
         }
         {
           uint32_t w[32];
@@ -531,7 +549,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           for (int e = 0; e < 32; ++e) w[e] = dr[e];
           tmem_st32(tS + lane_off + b * 64 + 32, w);
         }
-        fence_proxy_async_smem();
+        if constexpr (kDq) fence_proxy_async_smem();
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -550,7 +568,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const BwdChunks qc = bwd_chunks<kFlatK, kExtra>(p, x);
       const int bh = x.bh, kt = x.kt, ku = x.ku, n = qc.nm + qc.nx;
       const int64_t slice = static_cast<int64_t>(bh) * p.N;
-      for (int c = 0; c < n; ++c, ++cc) {
+      for (int c = 0; c < (kDq ? n : 0); ++c, ++cc) {
         const int b = cc & 1;
         ok = mbar_wait(dq_full + b, (cc >> 1) & 1, abort, 80);
         ok = __all_sync(0xffffffffu, ok);
