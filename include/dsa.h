@@ -227,9 +227,10 @@ dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k
  * j counts; j not listed: 0).  lse: the LSE dsa_fwd_list wrote for the same inputs and lists
  * (then every non-empty row of the map sums to one); dense attention is the list of every
  * tile.  Lists as dsa_fwd_list.  map: device fp32 [B * heads, nTiles, nTiles], overwritten.
- * The scores are recomputed on the tensor cores; sums over a tile pair are accumulated in
- * fp32 in an order that depends on timing (results may differ in the last bits between
- * runs).  bf16, d = 128. */
+ * The scores are recomputed on the tensor cores; one CTA sums each row of the map (all
+ * chunks of query tile i) in fp32 in a fixed order, so the map is the same from run to run.
+ * A row of the lists may hold at most 8192 entries here (a longer row is recorded as
+ * DSA_ERR_DEVICE, site 48, and its map row left zero).  bf16, d = 128. */
 dsa_status_t dsa_block_map(const dsa_problem_t* p, const void* q, const void* k, const float* lse,
                            const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, int32_t per_head, float* map,
                            void* stream);
@@ -254,8 +255,10 @@ dsa_status_t dsa_plan_heads(const dsa_problem_t* p, const int32_t* tile_offsets,
  * fp64 [p, p], upper triangle zero); a matrix that is not positive definite is recorded as
  * DSA_ERR_DEVICE (site 95).  dsa_lstsq_solve solves for a batch of right-hand sides
  * S (device fp32 [batch, m], one map per row, batch <= 65535) into X (device fp32
- * [batch, p]) with L from dsa_lstsq_factor; workspace: dsa_lstsq_workspace_size(m, p, batch)
- * bytes, 256-byte aligned.  Sums and solves run in fp64 in a fixed order. */
+ * [batch, p]) with L from dsa_lstsq_factor, in one launch (a cluster of 8 CTAs per map sums
+ * M^T s in fp64 and combines the partial sums through distributed shared memory).  It needs
+ * no workspace: dsa_lstsq_workspace_size returns 0 and workspace may be NULL.  Sums and
+ * solves run in fp64 in a fixed order, so X is the same from run to run. */
 size_t dsa_lstsq_workspace_size(int32_t m, int32_t p, int32_t batch);
 dsa_status_t dsa_lstsq_factor(int32_t m, int32_t p, const float* M, float lambda, double* L, void* stream);
 dsa_status_t dsa_lstsq_solve(int32_t m, int32_t p, int32_t batch, const float* M, const double* L, const float* S,

@@ -217,10 +217,14 @@ def test_per_head_offsets_against_the_windowed_oracle():
 
 
 # ------------------------------------------------------------------------------------
-# block attention mass (sparsity map).  Tolerance: the map is a mean of probabilities
-# exp(s - lse) with s from bf16 products and lse from the bf16 forward (LSE gate 1e-3),
-# so entries carry a relative error near 1e-3: max-abs 3e-3 and row sums within 3e-3 of 1.
-MAP_MAX_ABS = 3e-3
+# block attention mass (sparsity map).  Tolerance: an entry is a mean of probabilities
+# exp(s - lse) <= 1.  The scores are exact products of the bf16 inputs summed in fp32
+# (relative error ~1e-6); lse is the forward's, whose error against the exact value is the
+# relative error of its row sum (fp32 sum of 2^x, each with relative error <= 7.6e-5 on the
+# FMA-pipe share, ~1e-7 on MUFU: well under 1e-4); each probability adds its own 2^x error
+# (<= 7.6e-5).  So an entry's relative error is below 2e-4 and, as entries are <= 1, its
+# absolute error too: max-abs 5e-4 (and row sums within 5e-4 of 1) keeps a margin of 2.5x.
+MAP_MAX_ABS = 5e-4
 
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
@@ -238,6 +242,8 @@ def test_block_map_against_oracle(w, per_head):
     bm = dsa.block_map(q, k, lse, rp, kl, w.tile, w.scale)
     st, site, _ = dsa.device_status()
     assert st == 0, f"device status {st} at site {site}"
+    # one CTA sums each row of the map in a fixed order: a second run gives the same bits
+    assert torch.equal(dsa.block_map(q, k, lse, rp, kl, w.tile, w.scale), bm)
     ref = oracle.block_map_list(geo, inp.q, inp.k, row_ptr, kv_list)
     got = bm.cpu().numpy()
     err = np.abs(got - ref).max()

@@ -51,3 +51,26 @@ def test_singular_system_is_reported():
     dsa.lstsq_factor(M, 0.0)
     st, site, _ = dsa.device_status()
     assert st == 6 and site == 95
+
+
+def test_lstsq_solve_is_one_launch_without_workspace_and_reproducible():
+    """The solve takes no workspace (a null pointer is accepted) and, summing in a fixed order,
+    gives the same bits on every call."""
+    import ctypes
+
+    lib = dsa.load_library()
+    assert lib.dsa_lstsq_workspace_size(90000, 3, 24) == 0
+    g = torch.Generator().manual_seed(5)
+    M = torch.rand((90000, 3), generator=g).cuda()
+    S = torch.rand((24, 90000), generator=g).cuda()
+    L = dsa.lstsq_factor(M, 1e-3)
+    X = torch.empty((24, 3), dtype=torch.float32, device="cuda")
+    st = lib.dsa_lstsq_solve(90000, 3, 24, ctypes.c_void_p(M.data_ptr()), ctypes.c_void_p(L.data_ptr()),
+                             ctypes.c_void_p(S.data_ptr()), ctypes.c_void_p(X.data_ptr()), None, 0,
+                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    again = dsa.lstsq_solve(M, L, S)
+    torch.cuda.synchronize()
+    assert torch.equal(X, again)
+    ref = oracle.lstsq(M.cpu().double(), 1e-3, S.cpu().double())
+    np.testing.assert_allclose(X.cpu().numpy(), ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())

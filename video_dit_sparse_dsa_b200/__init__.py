@@ -475,10 +475,11 @@ def lstsq_solve(M: torch.Tensor, L: torch.Tensor, S: torch.Tensor, X: Optional[t
     batch = S.shape[0]
     if X is None:
         X = torch.empty((batch, p), dtype=torch.float32, device=S.device)
-    if ws is None:
-        ws = torch.empty(max(int(lib.dsa_lstsq_workspace_size(m, p, batch)), 256), dtype=torch.uint8, device=S.device)
-    _check(lib.dsa_lstsq_solve(m, p, batch, _ptr(M), _ptr(L), _ptr(S), _ptr(X), _ptr(ws), ws.numel(),
-                               ctypes.c_void_p(_stream(stream))), "dsa_lstsq_solve")
+    n_ws = int(lib.dsa_lstsq_workspace_size(m, p, batch))
+    if ws is None and n_ws > 0:
+        ws = torch.empty(n_ws, dtype=torch.uint8, device=S.device)
+    _check(lib.dsa_lstsq_solve(m, p, batch, _ptr(M), _ptr(L), _ptr(S), _ptr(X), _ptr(ws),
+                               0 if ws is None else ws.numel(), ctypes.c_void_p(_stream(stream))), "dsa_lstsq_solve")
     return X
 
 

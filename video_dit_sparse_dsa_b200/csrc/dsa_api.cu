@@ -397,7 +397,9 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
   if (fa.numRegs < dsa::fwd::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
-  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
+  // the block-map pass takes whole query tiles (all their chunks) per CTA
+  const int units = map_mode ? bp.n_units / bp.S : bp.n_units;
+  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
   kernel<<<grid, dsa::fwd::kThreads, dsa::fwd::kSmemBytes, s>>>(tq, tk, tv, tkx, tvx, bp);
   return launch_status();
 }
@@ -966,9 +968,10 @@ dsa_status_t dsa_block_map(const dsa_problem_t* p, const void* q, const void* k,
 }
 
 size_t dsa_lstsq_workspace_size(int32_t m, int32_t p, int32_t batch) {
-  if (m <= 0 || p <= 0 || p > dsa::kLstsqMaxP || batch <= 0) return 0;
-  const int64_t slices = (m + dsa::kLstsqSliceRows - 1) / dsa::kLstsqSliceRows;
-  return round_up(sizeof(double) * static_cast<size_t>(batch) * slices * p, kAlign);
+  (void)m;
+  (void)p;
+  (void)batch;
+  return 0;  // the solve keeps its partial sums in shared memory
 }
 
 dsa_status_t dsa_lstsq_factor(int32_t m, int32_t p, const float* M, float lambda, double* L, void* stream) {
@@ -981,19 +984,14 @@ dsa_status_t dsa_lstsq_factor(int32_t m, int32_t p, const float* M, float lambda
 
 dsa_status_t dsa_lstsq_solve(int32_t m, int32_t p, int32_t batch, const float* M, const double* L, const float* S,
                              float* X, void* workspace, size_t ws_bytes, void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
   if (m <= 0 || p <= 0 || batch <= 0 || !M || !L || !S || !X) return DSA_ERR_INVALID_ARG;
   if (p > dsa::kLstsqMaxP || batch > 65535) return DSA_ERR_UNSUPPORTED;
   if (!aligned(M, 4) || !aligned(L, 8) || !aligned(S, 4) || !aligned(X, 4)) return DSA_ERR_INVALID_ARG;
-  const size_t need = dsa_lstsq_workspace_size(m, p, batch);
-  if (workspace == nullptr || ws_bytes < need || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int slices = (m + dsa::kLstsqSliceRows - 1) / dsa::kLstsqSliceRows;
-  double* part = static_cast<double*>(workspace);
-  dsa::lstsq_rhs_kernel<<<dim3(static_cast<unsigned>(slices), static_cast<unsigned>(batch)), 256, 0, s>>>(M, S, m, p,
-                                                                                                         part);
-  dsa_status_t st = launch_status();
-  if (st != DSA_OK) return st;
-  dsa::lstsq_solve_kernel<<<static_cast<unsigned>(batch), 32, 0, s>>>(L, part, slices, p, X);
+  // one cluster of kLstsqCluster CTAs per right-hand side (the cluster shape is compiled in)
+  dim3 grid(dsa::kLstsqCluster, static_cast<unsigned>(batch));
+  dsa::lstsq_solve_kernel<<<grid, dsa::kLstsqThreads, 0, static_cast<cudaStream_t>(stream)>>>(M, S, m, p, L, X);
   return launch_status();
 }
 

@@ -117,6 +117,13 @@ constexpr float kRescaleThreshold = 8.0f;                        // log2 units
 // taken from the FMA-pipe polynomial instead of the MUFU unit, which takes 16 per clock per
 // SM and would otherwise bound the softmax
 constexpr uint32_t kPolyMask = 0x88u;
+// the block-map pass's share of 2^x on the FMA pipe (the forward's: a larger share was
+// slower, the polynomial's issue slots cost more than the MUFU time they free)
+constexpr uint32_t kPolyMaskMap = 0x88u;
+// list positions of a query tile's row the block-map pass keeps totals for (the V ring's
+// shared memory, which the pass does not use)
+constexpr int kMapCap = 8192;
+static_assert(8 * kMapCap <= kVStages * kTileBytes, "map totals must fit in the V ring");
 
 // TMEM columns of the scores and of P for a step of parity e.
 __device__ __forceinline__ uint32_t col_s(int e) { return e ? 128u : 0u; }
@@ -200,6 +207,27 @@ __device__ __forceinline__ Unit decode(const FwdBf16Params& p, int u) {
   x.tile = rem / p.S;
   x.sub = rem % p.S;
   return x;
+}
+
+// The CTA's it-th work unit.  The forward and flat modes stride over the unit sequence; the
+// block-map mode takes every chunk of a query tile in one CTA (tiles strided over the grid,
+// a tile's chunks in order), so that one CTA owns each row of the map and sums it in a fixed
+// order.
+template <int kMode>
+__device__ __forceinline__ bool next_unit(const FwdBf16Params& p, int it, Unit& x) {
+  if constexpr (kMode == kModeMap) {
+    const int64_t tu = blockIdx.x + static_cast<int64_t>(it / p.S) * gridDim.x;
+    if (tu >= p.n_units / p.S) return false;
+    x.bh = static_cast<int>(tu / p.n_tiles);
+    x.tile = static_cast<int>(tu % p.n_tiles);
+    x.sub = it % p.S;
+    return true;
+  } else {
+    const int64_t u = blockIdx.x + static_cast<int64_t>(it) * gridDim.x;
+    if (u >= p.n_units) return false;
+    x = kMode == kModeFlat ? decode_flat(p, static_cast<int>(u)) : decode(p, static_cast<int>(u));
+    return true;
+  }
 }
 
 // Shared-memory descriptors are built once; a byte offset is added in 16-byte units to
@@ -465,8 +493,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         const bool is_k = warp == kProducerWarp;
         int ld = 0, uc = 0;  // ring entries loaded, units with keys
         bool ok = true;
-        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-          const Unit x = kFlat ? decode_flat(p, u) : decode(p, u);
+        Unit x;
+        for (int it = 0; ok && next_unit<kMode>(p, it, x); ++it) {
           int n_list = 0;
           const int32_t* kv = kFlat ? nullptr : unit_keys(p, x.bh, x.tile, n_list);
           const Chunks ck = unit_chunks<kFlat, kExtra>(p, x, n_list);
@@ -551,9 +579,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       int uc = 0, g = 0;              // units and steps so far
       int pc0 = 0, pc1 = 0;           // phases of p_full[0 / 1] and s_read[0 / 1] consumed
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      Unit xm;
+      for (int it = 0; ok && next_unit<kMode>(p, it, xm); ++it) {
         int n_list = 0;
-        const Unit xm = kFlat ? decode_flat(p, u) : decode(p, u);
         if constexpr (!kFlat) unit_keys(p, xm.bh, xm.tile, n_list);
         const Chunks ck = unit_chunks<kFlat, kExtra>(p, xm, n_list);
         const int n_chunks = ck.nm + ck.nx, n_steps = (n_chunks + 1) / 2;
@@ -607,65 +635,112 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     setmaxnreg_inc<kRegsSoftmax>();
     if constexpr (kMap) {
       // ---------------------------------------------------------------- block attention mass
+      // One CTA owns every chunk of a query tile (next_unit), so the tile's row of the map is
+      // summed here in a fixed order and written once: per step each warp sums its 32 rows x
+      // 128 keys, the warps' sums meet in shared memory and one thread adds them, in warp
+      // order, to the list position's total; at the tile's end the totals of each listed key
+      // tile (in list order, so a tile listed twice counts twice) are written to the map.
+      // Every map warp takes every named barrier, even after a failed wait, so none waits
+      // for a warp that has left.
       const int i = warp >> 2;
       const int r = tid & 127;
       const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
       const float inv_rows = 1.f / static_cast<float>(p.S * 128);
+      float* acc = reinterpret_cast<float*>(smem + kOffV);                 // [kMapCap] per list position
+      int32_t* kvs = reinterpret_cast<int32_t*>(smem + kOffV + 4 * kMapCap);  // [kMapCap] the row's key tiles
+      float* stage = xbuf;                                                   // [2][8] warp sums of a step
       int sc0 = 0, sc1 = 0, g = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit x = decode(p, u);
+      Unit x;
+      for (int it = 0; next_unit<kMode>(p, it, x); ++it) {
         int n_list;
         const int32_t* kv = unit_keys(p, x.bh, x.tile, n_list);
         const int n_chunks = n_list * p.S, n_steps = (n_chunks + 1) / 2;
-        if (n_chunks == 0) continue;
+        const bool fits = n_list <= kMapCap;
+        if (x.sub == 0) {  // a new query tile: its totals start at zero
+          named_bar_sync(5, 256);  // the previous tile's row has been written
+          if (fits) {
+            for (int e = tid; e < n_list; e += 256) {
+              acc[e] = 0.f;
+              kvs[e] = min(max(kv[e], 0), p.n_tiles - 1);
+            }
+          } else if (tid == 0) {
+            device_report(DSA_DEV_BOUNDS, 48);  // a list row longer than the map pass takes
+          }
+          named_bar_sync(5, 256);
+        }
         const int64_t tok = chunk_token(p, x.tile, x.sub, r);
         const float neg_lse = -p.lse_in[static_cast<int64_t>(x.bh) * p.N + tok] * 1.4426950408889634f;
-        float* mrow = p.bmap + (static_cast<int64_t>(x.bh) * p.n_tiles + x.tile) * p.n_tiles;
-        for (int t = 0; t < n_steps && ok; ++t) {
+        for (int t = 0; t < n_steps; ++t) {
           const int e = (g + t) & 1;
-          ok = warp_wait(s_full + e, (e == 0 ? sc0++ : sc1++) & 1, abort, 49);
-          if (!ok) break;
-          tc_fence_after();
+          if (ok) ok = warp_wait(s_full + e, (e == 0 ? sc0++ : sc1++) & 1, abort, 49);
           const bool full = 2 * t + 1 < n_chunks;
-          uint32_t sv[128];
           float sum = 0.f;
-          if (full) {
-            tmem_ld128_wait(tmem + col_s(e) + 128 * i + lane_off, sv);
-          } else {
-            uint32_t (&half)[64] = *reinterpret_cast<uint32_t(*)[64]>(sv);
-            tmem_ld64_wait(tmem + col_s(e) + 64 * i + lane_off, half);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s_read + e);  // the scores' columns may be overwritten
-          const int nc = full ? 128 : 64;
-          float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+          if (ok) {
+            tc_fence_after();
+            uint32_t sv[128];
+            if (full) {
+              tmem_ld128_wait(tmem + col_s(e) + 128 * i + lane_off, sv);
+            } else {
+              uint32_t (&half)[64] = *reinterpret_cast<uint32_t(*)[64]>(sv);
+              tmem_ld64_wait(tmem + col_s(e) + 64 * i + lane_off, half);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_read + e);  // the scores' columns may be overwritten
+            const int nc = full ? 128 : 64;
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            if (c < nc) {
-              float x0, x1;
-              ffma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), p.scale_log2, p.scale_log2, neg_lse,
-                    neg_lse);
-              float p0, p1;
-              if ((kPolyMask >> (c >> 4)) & 1u) {  // the forward's share of 2^x on the FMA pipe
-                exp2_poly2(x0, x1, p0, p1);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
+            for (int c = 0; c < 128; c += 2) {
+              if (c < nc) {
+                float x0, x1;
+                ffma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), p.scale_log2, p.scale_log2,
+                      neg_lse, neg_lse);
+                float p0, p1;
+                if ((kPolyMaskMap >> (c >> 4)) & 1u) {  // a share of 2^x on the FMA pipe
+                  exp2_poly2(x0, x1, p0, p1);
+                } else {
+                  p0 = ex2_approx(x0);
+                  p1 = ex2_approx(x1);
+                }
+                fadd2(sa[(c >> 1) & 3], sb[(c >> 1) & 3], sa[(c >> 1) & 3], sb[(c >> 1) & 3], p0, p1);
               }
-              fadd2(sa[(c >> 1) & 3], sb[(c >> 1) & 3], sa[(c >> 1) & 3], sb[(c >> 1) & 3], p0, p1);
+            }
+            sum = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          }
+          if (lane == 0) stage[8 * e + warp] = sum;
+          named_bar_sync(5, 256);
+          if (tid == 0 && fits) {
+            // warpgroup i summed chunk 2t + i of a full step, or half i of the single chunk 2t
+            const float* st = stage + 8 * e;
+            const float s0 = (st[0] + st[1]) + (st[2] + st[3]), s1 = (st[4] + st[5]) + (st[6] + st[7]);
+            if (full) {
+              acc[(2 * t) / p.S] += s0;
+              acc[(2 * t + 1) / p.S] += s1;
+            } else {
+              acc[(2 * t) / p.S] += s0 + s1;
             }
           }
-          sum = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-          // this thread's keys: chunk 2t + i of a full step, or half i of the single chunk 2t
-          const int c = full ? 2 * t + i : 2 * t;
-          const int kt = min(max(kv[c / p.S], 0), p.n_tiles - 1);
-          if (lane == 0) atomicAdd(mrow + kt, sum * inv_rows);
         }
         g += n_steps;
+        if (x.sub == p.S - 1) {
+          named_bar_sync(5, 256);  // the tile's totals are complete
+          float* mrow = p.bmap + (static_cast<int64_t>(x.bh) * p.n_tiles + x.tile) * p.n_tiles;
+          if (fits) {
+            for (int e = tid; e < n_list; e += 256) {
+              const int kt = kvs[e];
+              bool first = true;
+              for (int f = 0; f < e && first; ++f) first = kvs[f] != kt;
+              if (!first) continue;  // counted with the tile's first occurrence
+              float s = 0.f;
+              for (int f = e; f < n_list; ++f)
+                if (kvs[f] == kt) s += acc[f];
+              mrow[kt] = s * inv_rows;
+            }
+          }
+        }
       }
     } else {
     // ------------------------------------------------------------------ softmax
@@ -685,8 +760,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     int uc = 0;            // units with keys before the current one
     int xe = 0;            // pair exchanges so far
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-      const Unit x = kFlat ? decode_flat(p, u) : decode(p, u);
+    Unit x;
+    for (int it = 0; next_unit<kMode>(p, it, x); ++it) {
       int n_list = 0;
       if constexpr (!kFlat) unit_keys(p, x.bh, x.tile, n_list);
       const Chunks ck = unit_chunks<kFlat, kExtra>(p, x, n_list);

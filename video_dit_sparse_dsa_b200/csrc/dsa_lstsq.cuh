@@ -7,19 +7,19 @@
 //
 //   lstsq_factor_kernel : G = M^T M + lambda I, then its Cholesky factor L (lower, fp64,
 //                         [p, p]); one CTA, one warp per entry of G;
-//   lstsq_rhs_kernel    : partial right-hand sides M^T s_b over a slice of the m rows
-//                         (grid: batch x slices), written per slice for a fixed-order sum;
-//   lstsq_solve_kernel  : sums the slices in order and solves L L^T x = r (one warp per b).
+//   lstsq_solve_kernel  : one launch for a batch of right-hand sides: M^T s_b summed by a
+//                         cluster of CTAs per b, then L L^T x = M^T s_b solved.
 #pragma once
 
 #include <stdint.h>
+
+#include <cooperative_groups.h>
 
 #include "dsa_device_status.cuh"
 
 namespace dsa {
 
 constexpr int kLstsqMaxP = 32;
-constexpr int kLstsqSliceRows = 8192;  // rows of M per partial right-hand side
 
 __global__ void __launch_bounds__(256) lstsq_factor_kernel(const float* M, int m, int p, float lambda, double* L) {
   __shared__ double G[kLstsqMaxP][kLstsqMaxP];
@@ -58,50 +58,89 @@ __global__ void __launch_bounds__(256) lstsq_factor_kernel(const float* M, int m
   }
 }
 
-// part: [batch, slices, p] fp64
-__global__ void __launch_bounds__(256) lstsq_rhs_kernel(const float* M, const float* S, int m, int p, double* part) {
-  __shared__ double acc[8][kLstsqMaxP];
-  const int b = blockIdx.y, slice = blockIdx.x, slices = gridDim.x;
+// X[b] = (L L^T)^-1 M^T s_b for every right-hand side b, in one launch: a cluster of
+// kLstsqCluster CTAs per b (grid (kLstsqCluster, batch)).  CTA r of a cluster sums M^T s_b
+// over its contiguous slice of the m rows in fp64 (each thread over rows tid, tid + 512, ...,
+// four rows' loads in flight at a time, then the warps' sums in warp order); the cluster's rank-0 CTA adds the CTAs' partial sums
+// in rank order, read from their shared memory, and one thread solves L y = r, L^T x = y.
+// Every sum runs in a fixed order, so X is the same from run to run.
+constexpr int kLstsqCluster = 8;
+constexpr int kLstsqThreads = 512;
+constexpr int kLstsqUnroll = 4;  // rows per thread whose loads are in flight together
+
+__global__ void __cluster_dims__(kLstsqCluster, 1, 1) __launch_bounds__(kLstsqThreads)
+    lstsq_solve_kernel(const float* __restrict__ M, const float* __restrict__ S, int m, int p,
+                       const double* __restrict__ L, float* __restrict__ X) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ double warp_acc[kLstsqThreads / 32][kLstsqMaxP];
+  __shared__ double part[kLstsqMaxP];
+  const int b = blockIdx.y;
+  const int rank = static_cast<int>(cluster.block_rank());
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = slice * kLstsqSliceRows, r1 = min(r0 + kLstsqSliceRows, m);
+  const int per = (m + kLstsqCluster - 1) / kLstsqCluster;
+  const int r0 = rank * per, r1 = min(r0 + per, m);
   const float* s = S + static_cast<int64_t>(b) * m;
-  for (int a = 0; a < p; ++a) {
-    double x = 0.0;
-    for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x)
-      x += static_cast<double>(s[r]) * static_cast<double>(M[static_cast<int64_t>(r) * p + a]);
+  double acc[kLstsqMaxP];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    if (lane == 0) acc[warp][a] = x;
+  for (int a = 0; a < kLstsqMaxP; ++a) acc[a] = 0.0;
+  for (int r = r0 + threadIdx.x; r < r1; r += kLstsqUnroll * kLstsqThreads) {
+    float sv[kLstsqUnroll];
+#pragma unroll
+    for (int u = 0; u < kLstsqUnroll; ++u) {
+      const int rr = r + u * kLstsqThreads;
+      sv[u] = rr < r1 ? s[rr] : 0.f;
+    }
+#pragma unroll
+    for (int a = 0; a < kLstsqMaxP; ++a) {
+      if (a < p) {
+        float mv[kLstsqUnroll];
+#pragma unroll
+        for (int u = 0; u < kLstsqUnroll; ++u) {
+          const int rr = r + u * kLstsqThreads;
+          mv[u] = rr < r1 ? M[static_cast<int64_t>(rr) * p + a] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kLstsqUnroll; ++u) acc[a] += static_cast<double>(sv[u]) * static_cast<double>(mv[u]);
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < kLstsqMaxP; ++a) {
+    if (a < p) {
+      double x = acc[a];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      if (lane == 0) warp_acc[warp][a] = x;
+    }
   }
   __syncthreads();
   if (threadIdx.x < p) {
     double x = 0.0;
-    for (int w = 0; w < 8; ++w) x += acc[w][threadIdx.x];
-    part[(static_cast<int64_t>(b) * slices + slice) * p + threadIdx.x] = x;
+    for (int w = 0; w < kLstsqThreads / 32; ++w) x += warp_acc[w][threadIdx.x];
+    part[threadIdx.x] = x;
   }
-}
-
-__global__ void __launch_bounds__(32) lstsq_solve_kernel(const double* L, const double* part, int slices, int p,
-                                                         float* X) {
-  const int b = blockIdx.x;
-  if (threadIdx.x != 0) return;
-  double y[kLstsqMaxP];
-  for (int a = 0; a < p; ++a) {
-    double r = 0.0;
-    for (int sl = 0; sl < slices; ++sl) r += part[(static_cast<int64_t>(b) * slices + sl) * p + a];
-    y[a] = r;
+  cluster.sync();  // every CTA's partial sums are in its shared memory
+  if (rank == 0 && threadIdx.x == 0) {
+    double y[kLstsqMaxP];
+    for (int a = 0; a < p; ++a) {
+      double r = 0.0;
+      for (int k = 0; k < kLstsqCluster; ++k) r += cluster.map_shared_rank(part, k)[a];
+      y[a] = r;
+    }
+    for (int i = 0; i < p; ++i) {  // L y = r
+      double t = y[i];
+      for (int j = 0; j < i; ++j) t -= L[i * p + j] * y[j];
+      y[i] = t / L[i * p + i];
+    }
+    for (int i = p - 1; i >= 0; --i) {  // L^T x = y
+      double t = y[i];
+      for (int j = i + 1; j < p; ++j) t -= L[j * p + i] * y[j];
+      y[i] = t / L[i * p + i];
+    }
+    for (int a = 0; a < p; ++a) X[static_cast<int64_t>(b) * p + a] = static_cast<float>(y[a]);
   }
-  for (int i = 0; i < p; ++i) {  // L y = r
-    double s = y[i];
-    for (int t = 0; t < i; ++t) s -= L[i * p + t] * y[t];
-    y[i] = s / L[i * p + i];
-  }
-  for (int i = p - 1; i >= 0; --i) {  // L^T x = y
-    double s = y[i];
-    for (int t = i + 1; t < p; ++t) s -= L[t * p + i] * y[t];
-    y[i] = s / L[i * p + i];
-  }
-  for (int a = 0; a < p; ++a) X[static_cast<int64_t>(b) * p + a] = static_cast<float>(y[a]);
+  cluster.sync();  // the other CTAs' shared memory stays valid until rank 0 has read it
 }
 
 }  // namespace dsa
