@@ -85,6 +85,19 @@ constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 128, 0, 1);  // P^T dO, dS^T 
 constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, 64, 1, 1);    // K^T dS^T
 // A byte offset added to a shared-memory descriptor's address field (16-byte units).
 __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+// Columns (within a chunk's 64-column S^T buffer) of packed bf16 P^T and dS^T for queries
+// [16kk, 16kk + 16).  With kDq one thread per key row handles all 64 queries: P^T in columns
+// [0, 32), dS^T in [32, 64).  Without it two threads share a row, thread h taking queries
+// [32h, 32h + 32) and writing over its own score columns [32h, 32h + 32): P^T in the first
+// 16, dS^T in the next 16.
+template <bool kDq>
+__device__ __forceinline__ uint32_t pt_col(int kk) {
+  return kDq ? 8u * kk : 32u * (kk >> 1) + 8u * (kk & 1);
+}
+template <bool kDq>
+__device__ __forceinline__ uint32_t dst_col(int kk) {
+  return kDq ? 32u + 8u * kk : 32u * (kk >> 1) + 16u + 8u * (kk & 1);
+}
 }  // namespace bwd
 
 // A work unit: (batch, head), key tile and its 128-key chunk (flat-key mode: the 128-row key
@@ -332,12 +345,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(p_full + b, 4);
+      mbar_init(p_full + b, kDq ? 4 : 8);  // the warps that write P^T and dS^T
       mbar_init(dq_full + b, 1);
       mbar_init(dq_free + b, 4);
     }
     mbar_init(dkv_full, 1);
-    mbar_init(dkv_free, 4);
+    mbar_init(dkv_free, kDq ? 4 : 8);  // the warps that read dK and dV out
     *abort = 0;
     fence_mbar_init();
   }
@@ -449,10 +462,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             const uint64_t ds_m = desc_add(dSm, b * kDSBytes);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
-              mma_ts_warp(tDV, tS + b * 64 + kk * 8, desc_add(do_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
+              mma_ts_warp(tDV, tS + b * 64 + pt_col<kDq>(kk), desc_add(do_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q (dS^T from TMEM, beside P^T)
-              mma_ts_warp(tDK, tS + b * 64 + 32 + kk * 8, desc_add(q_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
+              mma_ts_warp(tDK, tS + b * 64 + dst_col<kDq>(kk), desc_add(q_m, kk * 2048), kIdescAcc,
+                          (cc > 0) || (kk > 0));
             if constexpr (kDq) {
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
@@ -489,6 +503,129 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!ok) break;
         mma_commit_warp(dkv_full);
         mma_commit_warp(kv_free);
+        ++uc;
+      }
+    }
+  } else if (!kDq && warp < 8) {
+    // ------------------------------------------------------------------ P^T, dS^T and dK / dV out
+    // Two threads per key row (lane of warps w and w + 4): thread h takes queries [32h, 32h + 32)
+    // of every chunk.  At the end of a unit warps 0-3 write dV and warps 4-7 scale * dK.
+    const int h = warp >> 2;
+    const int m = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float kLog2e = 1.4426950408889634f;
+    int cc = 0, ld = 0, uc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BwdUnit x = bwd_unit<kFlatK>(p, u);
+      const BwdChunks qc = bwd_chunks<kFlatK, kExtra>(p, x);
+      const int n = qc.nm + qc.nx;
+      // flat keys: this thread's key row may lie past the end (zeros, no gradient)
+      const bool k_ok = !kFlatK || 128 * x.kt + m < p.Lk;
+      for (int c = 0; c < n; ++c, ++cc, ++ld) {
+        const int nvq = bwd_qvalid<kFlatK, kExtra>(p, qc, c) - 32 * h;  // valid queries of this half
+        const bool masked = !k_ok || nvq < 32;  // P = dS = 0 for missing keys and queries
+        const int b = cc & 1;
+        ok = mbar_wait(s_full + b, (cc >> 1) & 1, abort, 70);
+        if (ok) ok = mbar_wait(ld_full + ld % kStages, (ld / kStages) & 1, abort, 71);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float4* lse4 =
+            reinterpret_cast<const float4*>(smem + kOffStage + (ld % kStages) * kStageBytes + 2 * kQBytes) + 8 * h;
+        const float4* dd4 = lse4 + 32;  // D at +512 bytes
+        uint32_t sr[32], dr[32];
+        tmem_ld32_wait(tS + lane_off + b * 64 + 32 * h, sr);
+        tmem_ld32_wait(tDP + lane_off + b * 64 + 32 * h, dr);
+        uint32_t pk[16], dk2[16];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {  // queries 32h + 4g .. 32h + 4g + 3
+          const float4 lv = lse4[g], dv = dd4[g];
+          const float nl[4] = {-lv.x * kLog2e, -lv.y * kLog2e, -lv.z * kLog2e, -lv.w * kLog2e};
+          const float dq4[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int n0 = 4 * g + 2 * e;
+            float p0 = ex2_approx(fmaf(__uint_as_float(sr[n0]), p.scale_log2, nl[2 * e]));
+            float p1 = ex2_approx(fmaf(__uint_as_float(sr[n0 + 1]), p.scale_log2, nl[2 * e + 1]));
+            if (masked) {
+              if (!k_ok || n0 >= nvq) p0 = 0.f;
+              if (!k_ok || n0 + 1 >= nvq) p1 = 0.f;
+            }
+            pk[2 * g + e] = pack_bf16x2(p0, p1);
+            dk2[2 * g + e] = pack_bf16x2(p0 * (__uint_as_float(dr[n0]) - dq4[2 * e]),
+                                         p1 * (__uint_as_float(dr[n0 + 1]) - dq4[2 * e + 1]));
+          }
+        }
+        tmem_st16(tS + lane_off + b * 64 + 32 * h, pk);        // P^T over this thread's own score columns
+        tmem_st16(tS + lane_off + b * 64 + 32 * h + 16, dk2);  // dS^T beside it
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + b);
+      }
+      if (!ok) break;
+      // dV (warps 0-3) or scale * dK (warps 4-7) of the unit's 128 keys; zeros for a key tile
+      // no window holds.  Flat keys: fp32 partial sums of this part (unscaled dK), rows past
+      // Lk not written.
+      int64_t ktok;
+      bool k_row_ok = true;
+      if constexpr (kFlatK) {
+        ktok = 128 * static_cast<int64_t>(x.kt) + m;
+        k_row_ok = ktok < p.Lk;
+        if (!k_row_ok) ktok = 0;
+      } else {
+        const int k_t0 = (x.kt / (p.G1 * p.G2)) * p.tt + x.ku * p.kcs;
+        const int k_h0 = ((x.kt / p.G2) % p.G1) * p.th, k_w0 = (x.kt % p.G2) * p.tw;
+        ktok = chunk_row_token(m, k_t0, k_h0, k_w0, p.th, p.tw, p.H, p.W);
+      }
+      const int64_t slice = static_cast<int64_t>(x.bh) * p.N;
+      __nv_bfloat16* outp = h ? p.dk : p.dv;
+      const float sc_out = h ? p.scale : 1.f;
+      uint4* dst = reinterpret_cast<uint4*>(outp + (slice + ktok) * 128);
+      float4* dstp = nullptr;
+      if constexpr (kFlatK) {
+        const int64_t o = static_cast<int64_t>(x.part) * p.part_stride + (static_cast<int64_t>(x.bh) * p.Lk + ktok) * 128;
+        dstp = reinterpret_cast<float4*>((h ? p.dk_part : p.dv_part) + o);
+      }
+      if (n > 0) {
+        ok = mbar_wait(dkv_full, uc & 1, abort, 81);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+      }
+#pragma unroll 1
+      for (int g = 0; g < 4; ++g) {
+        uint32_t a[32];
+        if (n > 0) {
+          tmem_ld32_wait((h ? tDK : tDV) + lane_off + g * 32, a);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) a[j] = 0u;
+        }
+        if constexpr (kFlatK) {
+          if (k_row_ok) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dstp[g * 8 + j] = make_float4(__uint_as_float(a[4 * j]), __uint_as_float(a[4 * j + 1]),
+                                            __uint_as_float(a[4 * j + 2]), __uint_as_float(a[4 * j + 3]));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 y;
+            y.x = pack_bf16x2(__uint_as_float(a[8 * j + 0]) * sc_out, __uint_as_float(a[8 * j + 1]) * sc_out);
+            y.y = pack_bf16x2(__uint_as_float(a[8 * j + 2]) * sc_out, __uint_as_float(a[8 * j + 3]) * sc_out);
+            y.z = pack_bf16x2(__uint_as_float(a[8 * j + 4]) * sc_out, __uint_as_float(a[8 * j + 5]) * sc_out);
+            y.w = pack_bf16x2(__uint_as_float(a[8 * j + 6]) * sc_out, __uint_as_float(a[8 * j + 7]) * sc_out);
+            dst[g * 4 + j] = y;
+          }
+        }
+      }
+      if (n > 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dkv_free);
         ++uc;
       }
     }
