@@ -611,9 +611,11 @@ dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q
     st = launch_status();
     if (st != DSA_OK) return st;
   }
-  // dQ: 128-row query chunks over the forward's key lists
-  CUtensorMap tq2, tdo2;
-  if (!make_token_map(&tq2, q, p, g, 128) || !make_token_map(&tdo2, dout, p, g, 128)) return DSA_ERR_CUDA;
+  // dQ: 128-row query chunks over the forward's key lists, 64 keys per step
+  CUtensorMap tq2, tdo2, tk2, tv2;
+  if (!make_token_map(&tq2, q, p, g, 128) || !make_token_map(&tdo2, dout, p, g, 128) ||
+      !make_token_map(&tk2, k, p, g, 64) || !make_token_map(&tv2, v, p, g, 64))
+    return DSA_ERR_CUDA;
   dsa::BwdDqParams dp;
   std::memset(&dp, 0, sizeof(dp));
   dp.kv_tiles = fk.kv;
@@ -626,6 +628,7 @@ dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q
   dp.n_tiles = g.n_tiles;
   dp.Wt = g.Wt;
   dp.S = g.tile_tokens / 128;
+  dp.KS = g.tile_tokens / 64;
   dp.n_units = static_cast<int>(g.BH * g.n_tiles * dp.S);
   dp.G1 = g.G[1];
   dp.G2 = g.G[2];
@@ -633,6 +636,7 @@ dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q
   dp.th = p->tile[1];
   dp.tw = p->tile[2];
   dp.tcs = 128 / (p->tile[1] * p->tile[2]);
+  dp.kcs = 64 / (p->tile[1] * p->tile[2]);
   dp.T = p->T;
   dp.H = p->H;
   dp.W = p->W;
@@ -649,7 +653,7 @@ dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q
   int sms = 0;
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(dp.n_units < sms ? dp.n_units : sms);
-  kernel<<<grid, dsa::bdq::kThreads, dsa::bdq::kSmemBytes, s>>>(tq2, tk, tv, tdo2, dp);
+  kernel<<<grid, dsa::bdq::kThreads, dsa::bdq::kSmemBytes, s>>>(tq2, tk2, tv2, tdo2, dp);
   return launch_status();
 }
 

@@ -5,7 +5,7 @@
 // For query token n with key set K(i) of its tile i:
 //   P_nm = exp(scale q_n.k_m - LSE_n),  dS_nm = P_nm (dO_n.v_m - D_n),  dQ_n = scale sum_m dS_nm k_m,
 // with LSE the forward's and D_n = dO_n.O_n (bwd_preprocess).  A work unit is one 128-row
-// query chunk of one query tile of one (batch, head); it walks its window's keys 128 at a
+// query chunk of one query tile of one (batch, head); it walks its window's keys 64 at a
 // time ("steps"), recomputes S = Q K^T and dP = dO V^T on the tensor cores, forms dS in
 // registers and accumulates dQ += dS K in TMEM.  Each dQ row is summed by one CTA in the
 // fixed order of the unit's key list and written once as bf16: no atomics, and the result is
@@ -13,23 +13,32 @@
 // passes are the whole backward.)
 //
 // Persistent and warp-specialised, one CTA per SM, 384 threads:
-//   warp 8      TMA producer of Q and dO (once per unit) and of K (a 3-stage ring: a K
-//               chunk is read by the score product of its step and by the dQ product, which
-//               is issued one step later);
-//   warp 10     TMA producer of V (2-stage ring, read by the dP product only);
+//   warp 8      TMA producer of Q and dO (a staging copy per unit, refilled for the next
+//               unit as soon as the elementwise warps have moved it to TMEM) and of K
+//               (64-key chunks, a 6-entry ring: a K chunk is read by the score product of
+//               its step and by the dQ product, issued one step later);
+//   warp 10     TMA producer of V (64-key chunks, 4-entry ring, read by the dP product only);
 //   warp 9      MMA issuer (a converged warp; one elected lane issues), per step t:
-//                 S(t+1) = Q K(t+1)^T and dP(t+1) = dO V(t+1)^T once the elementwise warps
-//                 hold S(t) and dP(t) in registers, then dQ += dS(t) K(t) with dS from TMEM;
+//                 S(t) = Q K(t)^T and dP(t) = dO V(t)^T into TMEM buffer t % 2, with Q and
+//                 dO read from TMEM, then dQ += dS(t-1) K(t-1) once the elementwise warps
+//               have written dS(t-1); the buffers alternate, so the products of step t run
+//               while the elementwise warps work on step t-1;
 //   warp 11     idle (its warpgroup's registers go to the elementwise warpgroups);
-//   warps 0-7   elementwise: warpgroup i (warps 4i..4i+3) takes keys [64i, 64i+64) of every
-//               step, one thread per query row: P = 2^(S scale log2 e - LSE log2 e),
-//               dS = P (dP - D), packed to bf16 into TMEM; at the end of a unit each writes
-//               half of the row's 128 channels of dQ = scale * accumulator.
-// TMEM (512 columns): regions A [0,128), B [128,256), C [256,384) and the dQ accumulator
-// [384,512).  A step of parity e puts S in A (e = 0) or C (e = 1) and dP in B; the dS of
-// keys [64i, 64i+64) goes to columns [64i, 64i+32) of S's region, over the S columns the
-// same threads have already loaded.  So S(t+1) never lands on the dS(t) the dQ product
-// still reads, and dP(t+1) only needs the elementwise warps to have loaded dP(t).
+//   warps 0-7   elementwise: two threads per query row (lane of warps w and w + 4).  At the
+//               start of a unit thread 0 of a row copies the row of Q, thread 1 that of dO,
+//               from the staging copy into TMEM.  Per step thread h takes keys
+//               [32h, 32h + 32): P = 2^(S scale log2 e - LSE log2 e), dS = P (dP - D),
+//               packed to bf16 into TMEM over its own score columns; at the end of a unit
+//               each writes half of the row's 128 channels of dQ = scale * accumulator.
+// Every product takes its A operand (Q, dO or dS) from TMEM, so shared memory only feeds the
+// K and V tiles (B operands) and their fills: 80 KB per 64-key step against 768 cycles of
+// products, inside its bandwidth.
+// TMEM (512 columns): Q [0,64) and dO [64,128) as packed bf16 pairs, S buffers [128,192) and
+// [192,256), dP buffers [256,320) and [320,384), the dQ accumulator [384,512).  The products
+// of step t + 2 reuse step t's buffers only after the dQ product of step t (which reads its
+// dS) is issued, and that waits for the elementwise warps to have written dS(t), so they have
+// loaded S(t) and dP(t) long before.  A unit's Q and dO are overwritten only after the
+// elementwise warps have seen the unit's last scores, i.e. after its last products.
 // Units are ordered head, tile, chunk, as in the forward (the chunks of a tile read the
 // same keys at the same time).
 #pragma once
@@ -49,10 +58,13 @@ struct BwdDqParams {
   const float* delta;       // [B*heads, N] D = rowsum(dO * O)
   __nv_bfloat16* dq;        // [B*heads, N, 128]
   int n_tiles, Wt;
-  int S;                    // 128-row chunks per tile (query chunks and key chunks alike)
+  int S;                    // 128-row chunks per tile (the unit is one of them)
+  int KS;                   // 64-key chunks per tile (a step is one of them)
   int n_units;              // B*heads * n_tiles * S
   int G1, G2;
-  int tt, th, tw, tcs;      // tile shape; t-extent of a 128-token chunk
+  int tt, th, tw;
+  int tcs;                  // t-extent of a 128-token query chunk
+  int kcs;                  // t-extent of a 64-token key chunk
   int T, H, W, N;
   float scale, scale_log2;
 };
@@ -66,42 +78,42 @@ constexpr int kRegsElem = 216;
 constexpr int kRegsAux = 72;
 constexpr int kRegsAtLaunch = (2 * 128 * kRegsElem + 128 * kRegsAux) / kThreads;  // 168
 static_assert(kRegsAtLaunch * kThreads == 2 * 128 * kRegsElem + 128 * kRegsAux, "split must use the launch registers");
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
-constexpr uint32_t kTileBytes = 128 * 128 * 2;  // 128 tokens x 128 channels, bf16
-constexpr uint32_t kHalfBytes = kTileBytes / 2;
+constexpr int kKStages = 6;
+constexpr int kVStages = 4;
+constexpr uint32_t kQTileBytes = 128 * 128 * 2;  // 128 query tokens x 128 channels, bf16
+constexpr uint32_t kQHalfBytes = kQTileBytes / 2;
+constexpr uint32_t kKTileBytes = 64 * 128 * 2;   // 64 keys x 128 channels
+constexpr uint32_t kKHalfBytes = kKTileBytes / 2;
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffDO = kTileBytes;
-constexpr uint32_t kOffK = 2 * kTileBytes;
-constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
+constexpr uint32_t kOffDO = kQTileBytes;
+constexpr uint32_t kOffK = 2 * kQTileBytes;
+constexpr uint32_t kOffV = kOffK + kKStages * kKTileBytes;
+constexpr uint32_t kOffBar = kOffV + kVStages * kKTileBytes;
 constexpr uint32_t kSmemUsed = kOffBar + 256;
 constexpr uint32_t kSmemBytes = 227 * 1024;
 static_assert(kSmemUsed + 1023 <= kSmemBytes, "shared memory layout too large for any base alignment");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColB = 128, kColDQ = 384;
-constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // Q K^T, dO V^T: both K-major
+constexpr uint32_t kColQ = 0, kColDO = 64, kColS = 128, kColDP = 256, kColDQ = 384;
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);    // Q K^T, dO V^T: both K-major, 64 keys
 constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, 128, 0, 1);  // dS (TMEM) K: K as the MN-major B
 __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
-__device__ __forceinline__ uint32_t col_s(int e) { return e ? 256u : 0u; }
 
-// S = A B^T over 128 channels for a K-major 128-row A and B (8 k-steps of 16 in two
-// 64-channel halves).
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc) {
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t o = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    mma_ss_warp(d_tmem, desc_add(a_desc, o), desc_add(b_desc, o), kIdescS, kk > 0);
-  }
-}
-
-// dQ (+)= dS K over one 128-key step: dS of keys [16kk, 16kk+16) at TMEM columns
-// 8kk (kk < 4) and 64 + 8(kk - 4) (kk >= 4) of its region; K an MN-major tile, 16 keys =
-// 2048 bytes per k-step.
-__device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t ds_tmem, uint64_t k_desc, bool accumulate) {
+// D = A B^T over 128 channels for A (128 rows) in TMEM as packed bf16 pairs, 8 columns per
+// 16 channels, and a K-major B of 64 rows in shared memory (two 64-channel halves of 8 KB):
+// 8 k-steps of 16 channels.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc) {
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    mma_ts_warp(d_tmem, ds_tmem + (kk >> 2) * 64 + (kk & 3) * 8, desc_add(k_desc, kk * 2048), kIdescDQ,
+    mma_ts_warp(d_tmem, a_tmem + 8 * kk, desc_add(b_desc, (kk >> 2) * kKHalfBytes + (kk & 3) * 32), kIdescS, kk > 0);
+}
+
+// dQ (+)= dS K over one 64-key step: dS of keys [16kk, 16kk + 16) at TMEM columns
+// 32 (kk >> 1) + 8 (kk & 1) of its buffer (thread h wrote keys [32h, 32h + 32) over its own
+// score columns); K an MN-major tile, 16 keys = 2048 bytes per k-step.
+__device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t ds_tmem, uint64_t k_desc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    mma_ts_warp(d_tmem, ds_tmem + 32 * (kk >> 1) + 8 * (kk & 1), desc_add(k_desc, kk * 2048), kIdescDQ,
                 accumulate || kk > 0);
 }
 
@@ -165,13 +177,13 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
   uint64_t* k_empty = k_full + kKStages;     // [kKStages]
   uint64_t* v_full = k_empty + kKStages;     // [kVStages]
   uint64_t* v_empty = v_full + kVStages;     // [kVStages]
-  uint64_t* s_full = v_empty + kVStages;     // [2] S and dP of a step of parity e ready
-  uint64_t* s_read = s_full + 2;             // [2] ... loaded by the elementwise warps (8)
-  uint64_t* ds_full = s_full + 4;            // [2] dS of a step of parity e written (8)
-  uint64_t* dq_done = s_full + 6;            // every dQ product of a unit done
-  uint64_t* dq_free = s_full + 7;            // dQ read out (8)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
-  volatile int* abort = reinterpret_cast<volatile int*>(s_full + 9);
+  uint64_t* s_full = v_empty + kVStages;     // [2] S and dP of a step in buffer b ready
+  uint64_t* ds_full = s_full + 2;            // [2] dS of a step in buffer b written (8)
+  uint64_t* dq_done = s_full + 4;            // every dQ product of a unit done
+  uint64_t* dq_free = s_full + 5;            // dQ read out (8)
+  uint64_t* qa_full = s_full + 6;            // the unit's Q and dO are in TMEM (8)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 7);
+  volatile int* abort = reinterpret_cast<volatile int*>(s_full + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -181,7 +193,7 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
     tma_prefetch_map(&tmV);
     tma_prefetch_map(&tmDO);
     mbar_init(qd_full, 1);
-    mbar_init(qd_empty, 1);
+    mbar_init(qd_empty, 8);  // the staging copy is in TMEM
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
@@ -190,13 +202,13 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
       mbar_init(v_full + s, 1);
       mbar_init(v_empty + s, 1);
     }
-    for (int e = 0; e < 2; ++e) {
-      mbar_init(s_full + e, 1);
-      mbar_init(s_read + e, 8);
-      mbar_init(ds_full + e, 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(ds_full + b, 8);
     }
     mbar_init(dq_done, 1);
     mbar_init(dq_free, 8);
+    mbar_init(qa_full, 8);
     *abort = 0;
     fence_mbar_init();
   }
@@ -221,18 +233,18 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
           const Unit x = decode(p, u);
           int n_list = 0;
           const int32_t* kv = unit_keys(p, x.bh, x.tile, n_list);
-          const int n_steps = n_list * p.S;
+          const int n_steps = n_list * p.KS;
           if (n_steps == 0) continue;  // no keys: the elementwise warps write dQ = 0
           if (is_k) {
             ok = mbar_wait(qd_empty, (uc & 1) ^ 1, abort, 110);
             if (!ok) break;
             const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
             const int t0 = qt * p.tt + x.sub * p.tcs;
-            mbar_arrive_expect_tx(qd_full, 2 * kTileBytes);
+            mbar_arrive_expect_tx(qd_full, 2 * kQTileBytes);
             tma_load_5d(smem + kOffQ, &tmQ, qd_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
-            tma_load_5d(smem + kOffQ + kHalfBytes, &tmQ, qd_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
+            tma_load_5d(smem + kOffQ + kQHalfBytes, &tmQ, qd_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
             tma_load_5d(smem + kOffDO, &tmDO, qd_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
-            tma_load_5d(smem + kOffDO + kHalfBytes, &tmDO, qd_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
+            tma_load_5d(smem + kOffDO + kQHalfBytes, &tmDO, qd_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
           }
           ++uc;
           const int n_st = is_k ? kKStages : kVStages;
@@ -240,69 +252,60 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
             const int st = ld % n_st;
             ok = mbar_wait((is_k ? k_empty : v_empty) + st, ((ld / n_st) & 1) ^ 1, abort, is_k ? 111 : 112);
             if (!ok) break;
-            const int kt = min(max(kv[j / p.S], 0), p.n_tiles - 1), ks = j % p.S;
-            const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.tcs;
+            const int kt = min(max(kv[j / p.KS], 0), p.n_tiles - 1), ks = j % p.KS;
+            const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.kcs;
             const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
             uint64_t* full = (is_k ? k_full : v_full) + st;
-            uint8_t* dst = smem + (is_k ? kOffK : kOffV) + st * kTileBytes;
-            mbar_arrive_expect_tx(full, kTileBytes);
+            uint8_t* dst = smem + (is_k ? kOffK : kOffV) + st * kKTileBytes;
+            mbar_arrive_expect_tx(full, kKTileBytes);
             tma_load_5d(dst, is_k ? &tmK : &tmV, full, 0, w0, h0, t0, x.bh);
-            tma_load_5d(dst + kHalfBytes, is_k ? &tmK : &tmV, full, 64, w0, h0, t0, x.bh);
+            tma_load_5d(dst + kKHalfBytes, is_k ? &tmK : &tmV, full, 64, w0, h0, t0, x.bh);
           }
         }
       }
     } else if (warp == kMmaWarp) {
       // ------------------------------------------------------------------ MMA issuer (whole warp)
-      const uint64_t dQd = smem_desc_sw128(sbase + kOffQ, 16, 1024);
-      const uint64_t dDO = smem_desc_sw128(sbase + kOffDO, 16, 1024);
-      const uint64_t dKk = smem_desc_sw128(sbase + kOffK, 16, 1024);          // K stage 0, K-major
-      const uint64_t dKm = smem_desc_sw128(sbase + kOffK, kHalfBytes, 1024);  // K stage 0, MN-major
-      const uint64_t dVk = smem_desc_sw128(sbase + kOffV, 16, 1024);          // V stage 0, K-major
+      const uint64_t dKk = smem_desc_sw128(sbase + kOffK, 16, 1024);           // K stage 0, K-major
+      const uint64_t dKm = smem_desc_sw128(sbase + kOffK, kKHalfBytes, 1024);  // K stage 0, MN-major
+      const uint64_t dVk = smem_desc_sw128(sbase + kOffV, 16, 1024);           // V stage 0, K-major
       int ks = 0, kd = 0, vs = 0;  // K stages taken by the score and by the dQ products, V stages
       int uc = 0, g = 0;           // units with keys, steps before the current unit
-      int rc0 = 0, rc1 = 0;        // phases of s_read[0 / 1] consumed (ds_full alike)
       bool ok = true;
-      // S and dP of one step into the region of parity e; the V stage is released when they are done
-      auto issue_step = [&](int e) -> bool {
-        if (!warp_wait(k_full + ks % kKStages, (ks / kKStages) & 1, abort, 121)) return false;
-        if (!warp_wait(v_full + vs % kVStages, (vs / kVStages) & 1, abort, 122)) return false;
-        tc_fence_after();
-        issue_qk(tmem + col_s(e), dQd, desc_add(dKk, (ks % kKStages) * kTileBytes));
-        issue_qk(tmem + kColB, dDO, desc_add(dVk, (vs % kVStages) * kTileBytes));
-        mma_commit_warp(s_full + e);
-        mma_commit_warp(v_empty + vs % kVStages);
-        ++ks;
-        ++vs;
-        return true;
-      };
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         int n_list = 0;
         const Unit x = decode(p, u);
         unit_keys(p, x.bh, x.tile, n_list);
-        const int n_steps = n_list * p.S;
+        const int n_steps = n_list * p.KS;
         if (n_steps == 0) continue;
-        ok = warp_wait(qd_full, uc & 1, abort, 120);
-        if (ok) ok = issue_step(g & 1);
+        ok = warp_wait(qa_full, uc & 1, abort, 120);
         if (!ok) break;
-        if (n_steps == 1) mma_commit_warp(qd_empty);
-        for (int t = 0; t < n_steps && ok; ++t) {
-          const int e = (g + t) & 1;
-          const int ph = (e == 0 ? rc0++ : rc1++) & 1;
-          ok = warp_wait(s_read + e, ph, abort, 123);
-          if (!ok) break;
-          if (t + 1 < n_steps) {
-            // the elementwise warps hold S(t) and dP(t): S(t+1) goes to the other region, dP(t+1) to B
-            ok = issue_step(e ^ 1);
+        tc_fence_after();
+        for (int t = 0; t <= n_steps && ok; ++t) {
+          if (t < n_steps) {
+            // S(t) and dP(t) into buffer (g + t) % 2; the V stage is released when they are done
+            const int b = (g + t) & 1;
+            ok = warp_wait(k_full + ks % kKStages, (ks / kKStages) & 1, abort, 121);
+            if (ok) ok = warp_wait(v_full + vs % kVStages, (vs / kVStages) & 1, abort, 122);
             if (!ok) break;
-            if (t + 2 == n_steps) mma_commit_warp(qd_empty);  // every product reading Q and dO issued
+            tc_fence_after();
+            issue_qk(tmem + kColS + 64 * b, tmem + kColQ, desc_add(dKk, (ks % kKStages) * kKTileBytes));
+            issue_qk(tmem + kColDP + 64 * b, tmem + kColDO, desc_add(dVk, (vs % kVStages) * kKTileBytes));
+            mma_commit_warp(s_full + b);
+            mma_commit_warp(v_empty + vs % kVStages);
+            ++ks;
+            ++vs;
           }
-          ok = warp_wait(ds_full + e, ph, abort, 124);
-          if (ok && t == 0) ok = warp_wait(dq_free, (uc & 1) ^ 1, abort, 125);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dq(tmem + kColDQ, tmem + col_s(e), desc_add(dKm, (kd % kKStages) * kTileBytes), t > 0);
-          mma_commit_warp(k_empty + kd % kKStages);
-          ++kd;
+          if (t >= 1) {
+            // dQ += dS(t-1) K(t-1), once dS(t-1) is written
+            const int b = (g + t - 1) & 1;
+            ok = warp_wait(ds_full + b, ((g + t - 1) >> 1) & 1, abort, 124);
+            if (ok && t == 1) ok = warp_wait(dq_free, (uc & 1) ^ 1, abort, 125);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dq(tmem + kColDQ, tmem + kColS + 64 * b, desc_add(dKm, (kd % kKStages) * kKTileBytes), t > 1);
+            mma_commit_warp(k_empty + kd % kKStages);
+            ++kd;
+          }
         }
         if (!ok) break;
         mma_commit_warp(dq_done);
@@ -313,66 +316,91 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
   } else {
     setmaxnreg_inc<kRegsElem>();
     // ------------------------------------------------------------------ elementwise (P, dS) and dQ out
-    // Every barrier is waited on at most one phase behind its completions: s_full alternates
-    // with the step parity and each phase needs the previous step's s_read; dq_done completes
-    // once per unit and the next completion needs this warpgroup's dq_free arrival.
-    const int i = warp >> 2;
-    const int r = tid & 127;
+    // s_full[b] and ds_full[b] complete once per step of buffer b; a step's s_full completion
+    // needs the products of the step two earlier, which need this warp's ds_full arrival for
+    // it, so a wait by parity is never more than one phase behind.  dq_done completes once per
+    // unit and the next completion needs this warpgroup's dq_free arrival.
+    const int h = warp >> 2;
+    const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float kLog2e = 1.4426950408889634f;
-    int sc0 = 0, sc1 = 0, g = 0, uc = 0;
+    int g = 0, uc = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit x = decode(p, u);
       int n_list = 0;
       unit_keys(p, x.bh, x.tile, n_list);
-      const int n_steps = n_list * p.S;
+      const int n_steps = n_list * p.KS;
       const int64_t row = static_cast<int64_t>(x.bh) * p.N + chunk_token(p, x.tile, x.sub, r);
-      uint4* dst = reinterpret_cast<uint4*>(p.dq + row * 128) + 8 * i;
+      uint4* dst = reinterpret_cast<uint4*>(p.dq + row * 128) + 8 * h;
       if (n_steps == 0) {  // no keys: no gradient
 #pragma unroll
         for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
         continue;
       }
       const float neg_lse2 = -p.lse[row] * kLog2e, dd = p.delta[row];
-      for (int t = 0; t < n_steps; ++t) {
-        const int e = (g + t) & 1;
-        ok = warp_wait(s_full + e, (e == 0 ? sc0++ : sc1++) & 1, abort, 130);
+      {
+        // the unit's row of Q (h = 0) or dO (h = 1) from the staging copy (128-byte swizzled
+        // 64-channel halves, 8-row groups of 1 KB) into TMEM as packed bf16 pairs.  The
+        // previous unit's products have all completed: this warp has seen its last scores.
+        ok = warp_wait(qd_full, uc & 1, abort, 132);
         if (!ok) break;
-        tc_fence_after();
-        uint32_t s[64], dp[64];
-        tmem_ld64_wait(tmem + col_s(e) + 64 * i + lane_off, s);
-        tmem_ld64_wait(tmem + kColB + 64 * i + lane_off, dp);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_read + e);  // dP(t+1) may now go into B
+        const uint32_t src_row = sbase + (h ? kOffDO : kOffQ) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float x0, x1;
-          ffma2(x0, x1, __uint_as_float(s[c]), __uint_as_float(s[c + 1]), p.scale_log2, p.scale_log2, neg_lse2,
-                neg_lse2);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          s[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - dd), p1 * (__uint_as_float(dp[c + 1]) - dd));
-        }
-        {
+        for (int half = 0; half < 2; ++half) {
           uint32_t w[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) w[c] = s[c];
-          tmem_st32(tmem + col_s(e) + 64 * i + lane_off, w);  // over this thread's own S columns
+          for (int c = 0; c < 8; ++c) {  // 16-byte chunk c of the 128-byte row of this half
+            uint32_t x0, x1, x2, x3;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                         : "r"(src_row + half * kQHalfBytes + ((c ^ (r & 7)) << 4)));
+            w[4 * c] = x0;
+            w[4 * c + 1] = x1;
+            w[4 * c + 2] = x2;
+            w[4 * c + 3] = x3;
+          }
+          tmem_st32(tmem + (h ? kColDO : kColQ) + 32 * half + lane_off, w);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(ds_full + e);
+        if (lane == 0) {
+          mbar_arrive(qa_full);
+          mbar_arrive(qd_empty);  // the staging copy may take the next unit's rows
+        }
+      }
+      for (int t = 0; t < n_steps; ++t) {
+        const int gt = g + t, b = gt & 1;
+        ok = warp_wait(s_full + b, (gt >> 1) & 1, abort, 130);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t s[32], dp[32];
+        tmem_ld32_wait(tmem + kColS + 64 * b + 32 * h + lane_off, s);
+        tmem_ld32_wait(tmem + kColDP + 64 * b + 32 * h + lane_off, dp);
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float x0, x1;
+          ffma2(x0, x1, __uint_as_float(s[c]), __uint_as_float(s[c + 1]), p.scale_log2, p.scale_log2, neg_lse2,
+                neg_lse2);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          w[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - dd), p1 * (__uint_as_float(dp[c + 1]) - dd));
+        }
+        tmem_st16(tmem + kColS + 64 * b + 32 * h + lane_off, w);  // over this thread's own score columns
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full + b);
       }
       if (!ok) break;
-      // epilogue: dQ = scale * accumulator, channels [64i, 64i + 64) of the row
+      // epilogue: dQ = scale * accumulator, channels [64h, 64h + 64) of the row
       ok = warp_wait(dq_done, uc & 1, abort, 131);
       if (!ok) break;
       tc_fence_after();
-      uint32_t a[32], b[32];
-      tmem_ld32_wait(tmem + kColDQ + 64 * i + lane_off, a);
-      tmem_ld32_wait(tmem + kColDQ + 64 * i + 32 + lane_off, b);
+      uint32_t a[32], c2[32];
+      tmem_ld32_wait(tmem + kColDQ + 64 * h + lane_off, a);
+      tmem_ld32_wait(tmem + kColDQ + 64 * h + 32 + lane_off, c2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
@@ -388,10 +416,10 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint4 v;
-        v.x = pack_bf16x2(__uint_as_float(b[8 * c + 0]) * p.scale, __uint_as_float(b[8 * c + 1]) * p.scale);
-        v.y = pack_bf16x2(__uint_as_float(b[8 * c + 2]) * p.scale, __uint_as_float(b[8 * c + 3]) * p.scale);
-        v.z = pack_bf16x2(__uint_as_float(b[8 * c + 4]) * p.scale, __uint_as_float(b[8 * c + 5]) * p.scale);
-        v.w = pack_bf16x2(__uint_as_float(b[8 * c + 6]) * p.scale, __uint_as_float(b[8 * c + 7]) * p.scale);
+        v.x = pack_bf16x2(__uint_as_float(c2[8 * c + 0]) * p.scale, __uint_as_float(c2[8 * c + 1]) * p.scale);
+        v.y = pack_bf16x2(__uint_as_float(c2[8 * c + 2]) * p.scale, __uint_as_float(c2[8 * c + 3]) * p.scale);
+        v.z = pack_bf16x2(__uint_as_float(c2[8 * c + 4]) * p.scale, __uint_as_float(c2[8 * c + 5]) * p.scale);
+        v.w = pack_bf16x2(__uint_as_float(c2[8 * c + 6]) * p.scale, __uint_as_float(c2[8 * c + 7]) * p.scale);
         dst[4 + c] = v;
       }
       g += n_steps;
