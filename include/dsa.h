@@ -205,10 +205,13 @@ dsa_status_t dsa_fwd_prefix(const dsa_problem_t* p, const void* q, const void* k
  * out_text, lse_text and the output gradients dout [B, heads, T, H, W, 128] and dout_text
  * [B, heads, L_text, 128] (bf16).  Writes dq, dk, dv (video, the layout of q) and dq_text,
  * dk_text, dv_text (the layout of q_text), bf16.  Video keys are reduced over their windows'
- * queries and every text query by the window backward kernel; text keys over every video
+ * queries and every text query by the key-major backward kernel; text keys over every video
  * and text query by the same kernel in a flat-key mode (query chunks cut into parts for
- * load balance, fp32 partial dK / dV summed at the end).  L_text = 0 is dsa_bwd (text
- * pointers may be NULL).  workspace: at least dsa_bwd_prefix_workspace_size(p, L_text)
+ * load balance); video queries' dQ over their windows' keys and every text key by the
+ * query-major kernel; text queries' dQ over every key by that kernel in a flat mode (key
+ * chunks cut into parts).  The parts' fp32 sums are added in part order and nothing is
+ * summed with atomics, so the gradients are identical from run to run.  L_text = 0 is dsa_bwd
+ * (text pointers may be NULL).  workspace: at least dsa_bwd_prefix_workspace_size(p, L_text)
  * bytes, 256-byte aligned.  bf16, d = 128. */
 size_t dsa_bwd_prefix_workspace_size(const dsa_problem_t* p, int32_t L_text);
 dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k, const void* v, const void* out,

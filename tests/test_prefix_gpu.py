@@ -186,3 +186,15 @@ def test_prefix_backward_720p_sampled():
                rows(grads[4], t_rows), rows(grads[5], t_rows))
         for g, r, name in zip(got, ref, ("dq", "dq_text", "dk", "dv", "dk_text", "dv_text")):
             assert_close(g, r, w.dtype, f"{name} of (batch, head) {h}")
+
+
+def test_prefix_backward_is_bit_identical_across_runs():
+    """No gradient of the text prefix is summed with atomics (parts are added in part order):
+    two runs of the backward give the same bits."""
+    w = Workload("prefix_repeat", 1, 2, 128, (8, 16, 24), (4, 8, 8), (3, 3, 3), (-2, 2), "bf16", 64)
+    inp = make_inputs(w)
+    txt = make_text_inputs(w, 150, seed=65)
+    first, _, _ = run_backward(w, inp, txt, 66)
+    again, _, _ = run_backward(w, inp, txt, 66)
+    for a, b, name in zip(first, again, ("dq", "dk", "dv", "dq_text", "dk_text", "dv_text")):
+        assert torch.equal(a, b), f"{name} differs between runs"

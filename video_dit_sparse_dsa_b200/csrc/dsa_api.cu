@@ -102,11 +102,10 @@ struct BwdWorkspace {
   int32_t* row_ptr;
   int32_t* q_tiles;
   float* delta;  // D = rowsum(dO * O), [BH, N]
-  float* dq_acc; // fp32 dq accumulator, [BH, N, d]
   size_t bytes;
 };
 
-BwdWorkspace bwd_workspace(const Geom& g, int d, void* base, bool with_dq_acc = false) {
+BwdWorkspace bwd_workspace(const Geom& g, void* base) {
   BwdWorkspace w;
   uint8_t* b = static_cast<uint8_t*>(base);
   size_t off = 0;
@@ -120,11 +119,6 @@ BwdWorkspace bwd_workspace(const Geom& g, int d, void* base, bool with_dq_acc = 
   off += round_up(sizeof(int32_t) * static_cast<size_t>(g.n_tiles) * g.Wt, kAlign);
   w.delta = reinterpret_cast<float*>(b + off);
   off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N), kAlign);
-  w.dq_acc = nullptr;
-  if (with_dq_acc) {
-    w.dq_acc = reinterpret_cast<float*>(b + off);
-    off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N) * d, kAlign);
-  }
   w.bytes = off;
   return w;
 }
@@ -139,7 +133,7 @@ struct ListBwdWorkspace {
   size_t bytes;
 };
 
-ListBwdWorkspace list_bwd_workspace(const Geom& g, int d, int nnz, int n_lists, void* base) {
+ListBwdWorkspace list_bwd_workspace(const Geom& g, int nnz, int n_lists, void* base) {
   ListBwdWorkspace w;
   uint8_t* b = static_cast<uint8_t*>(base);
   size_t off = 0;
@@ -152,7 +146,6 @@ ListBwdWorkspace list_bwd_workspace(const Geom& g, int d, int nnz, int n_lists, 
   w.delta = reinterpret_cast<float*>(b + off);
   off += round_up(sizeof(float) * static_cast<size_t>(g.BH * g.N), kAlign);
   w.bytes = off;
-  (void)d;
   return w;
 }
 
@@ -455,100 +448,6 @@ dsa_status_t launch_merge_parts(const void* o, const float* lse, int n_parts, in
   return launch_status();
 }
 
-// The backward after planning: D preprocess (and zeroing of the dQ accumulator), the
-// key-major kernel over the inverse CSR (row_ptr, q_tiles), and the dQ conversion.
-// Extra (text) query rows of a backward: flat q, dO [BH, L, 128] bf16, LSE and D copies
-// padded to [BH, Lp] fp32, and their fp32 dQ accumulator.
-struct ExtraQueries {
-  const void* q;
-  const void* dout;
-  const float* lse_pad;
-  const float* delta_pad;
-  float* dq_acc;
-  int L, Lp;
-};
-
-template <bool kFlatK, bool kExtra>
-dsa_status_t launch_bwd_kernel(const dsa::BwdBf16Params& bp, const CUtensorMap& tq, const CUtensorMap& tk,
-                               const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tlse,
-                               const CUtensorMap& tdel, const ExtraQueries* x, int64_t BH, cudaStream_t s) {
-  CUtensorMap tqx = tq, tdox = tdo, tlsex = tlse, tdx = tdel;
-  if (x != nullptr && x->L > 0) {
-    if (!make_flat_map(&tqx, x->q, BH, x->L, 64) || !make_flat_map(&tdox, x->dout, BH, x->L, 64) ||
-        !make_vec_map(&tlsex, x->lse_pad, BH, x->Lp) || !make_vec_map(&tdx, x->delta_pad, BH, x->Lp))
-      return DSA_ERR_CUDA;
-  }
-  auto kernel = dsa::bwd_bf16_kernel<kFlatK, kExtra>;
-  constexpr uint32_t smem = dsa::bwd::Layout<true>::kSmemBytes;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  int sms = 0;
-  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
-  kernel<<<grid, dsa::bwd::kThreads, smem, s>>>(tq, tk, tv, tdo, tlse, tdel, tqx, tdox, tlsex, tdx,
-                                                                 bp);
-  return launch_status();
-}
-
-dsa_status_t launch_bwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
-                        const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
-                        const int32_t* q_tiles, float* delta, float* dq_acc, void* dq, void* dk, void* dv,
-                        cudaStream_t s, int rp_head_stride = 0, const ExtraQueries* x = nullptr,
-                        bool convert_dq = true) {
-  dsa_status_t st;
-  const int64_t rows = g.BH * g.N;
-  dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta, dq_acc, rows);
-  st = launch_status();
-  if (st != DSA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo, tlse, tdel;
-  if (!make_token_map(&tq, q, p, g, 64) || !make_token_map(&tk, k, p, g, 128) ||
-      !make_token_map(&tv, v, p, g, 128) || !make_token_map(&tdo, dout, p, g, 64) ||
-      !make_row_map(&tlse, lse, p, g, 64) || !make_row_map(&tdel, delta, p, g, 64))
-    return DSA_ERR_CUDA;
-  dsa::BwdBf16Params bp;
-  bp.row_ptr = row_ptr;
-  bp.rp_head_stride = rp_head_stride;
-  bp.q_tiles = q_tiles;
-  bp.dq_acc = dq_acc;
-  bp.dk = static_cast<__nv_bfloat16*>(dk);
-  bp.dv = static_cast<__nv_bfloat16*>(dv);
-  bp.n_tiles = g.n_tiles;
-  bp.KU = g.tile_tokens / 128;
-  bp.QS = g.tile_tokens / 64;
-  bp.n_units = static_cast<int>(g.BH * g.n_tiles * bp.KU);
-  bp.G1 = g.G[1];
-  bp.G2 = g.G[2];
-  bp.tt = p->tile[0];
-  bp.th = p->tile[1];
-  bp.tw = p->tile[2];
-  bp.kcs = 128 / (p->tile[1] * p->tile[2]);
-  bp.qcs = 64 / (p->tile[1] * p->tile[2]);
-  bp.T = p->T;
-  bp.H = p->H;
-  bp.W = p->W;
-  bp.N = static_cast<int>(g.N);
-  bp.scale = p->scale;
-  bp.scale_log2 = p->scale * 1.4426950408889634f;
-  bp.Lxq = 0;
-  bp.dq_acc_x = nullptr;
-  bp.Lk = bp.Nq = 0;
-  bp.n_split = 1;
-  bp.dk_part = bp.dv_part = nullptr;
-  bp.part_stride = 0;
-  if (x != nullptr) {  // extra (text) queries after every key unit's own
-    bp.Lxq = x->L;
-    bp.dq_acc_x = x->dq_acc;
-  }
-  st = bp.Lxq > 0 ? launch_bwd_kernel<false, true>(bp, tq, tk, tv, tdo, tlse, tdel, x, g.BH, s)
-                  : launch_bwd_kernel<false, false>(bp, tq, tk, tv, tdo, tlse, tdel, x, g.BH, s);
-  if (st != DSA_OK || !convert_dq) return st;
-  const int64_t n8 = rows * p->d / 8;
-  dsa::bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
-      dq_acc, static_cast<__nv_bfloat16*>(dq), p->scale, n8);
-  return launch_status();
-}
-
 // Key tiles of each query tile as the forward takes them: the window plan's kv_tiles
 // (row_ptr null) or a caller's CSR (row_ptr, nnz entries, rp_head_stride 0 or nTiles + 1).
 struct FwdKeys {
@@ -556,6 +455,52 @@ struct FwdKeys {
   const int32_t* row_ptr;
   int nnz, rp_head_stride;
 };
+
+// Parameters of the dQ kernel for the problem's tile geometry (the window / list form).
+dsa::BwdDqParams dq_params(const dsa_problem_t* p, const Geom& g, const float* lse, const float* delta, void* dq) {
+  dsa::BwdDqParams dp;
+  std::memset(&dp, 0, sizeof(dp));
+  dp.lse = lse;
+  dp.delta = delta;
+  dp.dq = static_cast<__nv_bfloat16*>(dq);
+  dp.n_tiles = g.n_tiles;
+  dp.Wt = g.Wt;
+  dp.S = g.tile_tokens / 128;
+  dp.KS = g.tile_tokens / 64;
+  dp.n_units = static_cast<int>(g.BH * g.n_tiles * dp.S);
+  dp.G1 = g.G[1];
+  dp.G2 = g.G[2];
+  dp.tt = p->tile[0];
+  dp.th = p->tile[1];
+  dp.tw = p->tile[2];
+  dp.tcs = 128 / (p->tile[1] * p->tile[2]);
+  dp.kcs = 64 / (p->tile[1] * p->tile[2]);
+  dp.T = p->T;
+  dp.H = p->H;
+  dp.W = p->W;
+  dp.N = static_cast<int>(g.N);
+  dp.scale = p->scale;
+  dp.scale_log2 = p->scale * 1.4426950408889634f;
+  dp.n_split = 1;
+  return dp;
+}
+
+template <bool kFlat, bool kExtra>
+dsa_status_t launch_dq(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                       const CUtensorMap& tkx, const CUtensorMap& tvx, const dsa::BwdDqParams& dp, cudaStream_t s) {
+  auto kernel = dsa::bwd_dq_kernel<kFlat, kExtra>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::bdq::kSmemBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  // the kernel's setmaxnreg split needs exactly the registers it was compiled for at launch
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
+  if (fa.numRegs < dsa::bdq::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
+  int sms = 0;
+  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(dp.n_units < sms ? dp.n_units : sms);
+  kernel<<<grid, dsa::bdq::kThreads, dsa::bdq::kSmemBytes, s>>>(tq, tk, tv, tdo, tkx, tvx, dp);
+  return launch_status();
+}
 
 // The backward of the window and key-tile-list forms: D = rowsum(dO * O), the key-major
 // kernel for dK and dV over the inverse lists (row_ptr, q_tiles), and the query-major
@@ -566,7 +511,7 @@ dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q
                             void* dk, void* dv, cudaStream_t s) {
   const int64_t rows = g.BH * g.N;
   dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta, nullptr, rows);
+      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), delta, rows);
   dsa_status_t st = launch_status();
   if (st != DSA_OK) return st;
   CUtensorMap tq, tk, tv, tdo, tlse, tdel;
@@ -600,8 +545,8 @@ dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q
   bp.scale_log2 = p->scale * 1.4426950408889634f;
   bp.n_split = 1;
   {
-    auto kernel = dsa::bwd_bf16_kernel<false, false, false>;
-    constexpr uint32_t smem = dsa::bwd::Layout<false>::kSmemBytes;
+    auto kernel = dsa::bwd_bf16_kernel<false, false>;
+    constexpr uint32_t smem = dsa::bwd::kSmemBytes;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return DSA_ERR_CUDA;
     int sms = 0;
@@ -616,45 +561,12 @@ dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q
   if (!make_token_map(&tq2, q, p, g, 128) || !make_token_map(&tdo2, dout, p, g, 128) ||
       !make_token_map(&tk2, k, p, g, 64) || !make_token_map(&tv2, v, p, g, 64))
     return DSA_ERR_CUDA;
-  dsa::BwdDqParams dp;
-  std::memset(&dp, 0, sizeof(dp));
+  dsa::BwdDqParams dp = dq_params(p, g, lse, delta, dq);
   dp.kv_tiles = fk.kv;
   dp.row_ptr = fk.row_ptr;
   dp.rp_head_stride = fk.rp_head_stride;
   dp.nnz = fk.nnz;
-  dp.lse = lse;
-  dp.delta = delta;
-  dp.dq = static_cast<__nv_bfloat16*>(dq);
-  dp.n_tiles = g.n_tiles;
-  dp.Wt = g.Wt;
-  dp.S = g.tile_tokens / 128;
-  dp.KS = g.tile_tokens / 64;
-  dp.n_units = static_cast<int>(g.BH * g.n_tiles * dp.S);
-  dp.G1 = g.G[1];
-  dp.G2 = g.G[2];
-  dp.tt = p->tile[0];
-  dp.th = p->tile[1];
-  dp.tw = p->tile[2];
-  dp.tcs = 128 / (p->tile[1] * p->tile[2]);
-  dp.kcs = 64 / (p->tile[1] * p->tile[2]);
-  dp.T = p->T;
-  dp.H = p->H;
-  dp.W = p->W;
-  dp.N = static_cast<int>(g.N);
-  dp.scale = p->scale;
-  dp.scale_log2 = p->scale * 1.4426950408889634f;
-  auto kernel = dsa::bwd_dq_kernel;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::bdq::kSmemBytes) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  // the kernel's setmaxnreg split needs exactly the registers it was compiled for at launch
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
-  if (fa.numRegs < dsa::bdq::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
-  int sms = 0;
-  if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(dp.n_units < sms ? dp.n_units : sms);
-  kernel<<<grid, dsa::bdq::kThreads, dsa::bdq::kSmemBytes, s>>>(tq2, tk2, tv2, tdo2, dp);
-  return launch_status();
+  return launch_dq<false, false>(tq2, tk2, tv2, tdo2, tk2, tv2, dp, s);
 }
 
 }  // namespace
@@ -689,7 +601,7 @@ size_t dsa_workspace_size(const dsa_problem_t* p, int32_t kind) {
   Geom g;
   if (check_shape(p, &g) != DSA_OK) return 0;
   if (kind == DSA_WS_FWD) return fwd_workspace(g, nullptr).bytes;
-  if (kind == DSA_WS_BWD) return bwd_workspace(g, p->d, nullptr).bytes;
+  if (kind == DSA_WS_BWD) return bwd_workspace(g, nullptr).bytes;
   return 0;
 }
 
@@ -853,7 +765,7 @@ dsa_status_t dsa_bwd(const dsa_problem_t* p, const void* q, const void* k, const
   for (const void* ptr : ptrs)
     if (!aligned(ptr, 16)) return DSA_ERR_INVALID_ARG;
   if (!aligned(lse, 4) || !aligned(tile_offsets, 4)) return DSA_ERR_INVALID_ARG;
-  BwdWorkspace ws = bwd_workspace(g, p->d, workspace);
+  BwdWorkspace ws = bwd_workspace(g, workspace);
   if (workspace == nullptr || ws_bytes < ws.bytes || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_plan(g, tile_offsets, ws.starts, ws.kv_tiles, ws.row_ptr, ws.q_tiles, s);
@@ -866,7 +778,7 @@ size_t dsa_list_workspace_size(const dsa_problem_t* p, int32_t nnz, int32_t per_
   Geom g;
   if (check_shape(p, &g) != DSA_OK || nnz < 0) return 0;
   if (kind == DSA_WS_FWD) return 0;
-  if (kind == DSA_WS_BWD) return list_bwd_workspace(g, p->d, nnz, per_head ? static_cast<int>(g.BH) : 1, nullptr).bytes;
+  if (kind == DSA_WS_BWD) return list_bwd_workspace(g, nnz, per_head ? static_cast<int>(g.BH) : 1, nullptr).bytes;
   return 0;
 }
 
@@ -933,7 +845,7 @@ dsa_status_t dsa_bwd_list(const dsa_problem_t* p, const void* q, const void* k, 
   for (const void* ptr : ptrs)
     if (!aligned(ptr, 16)) return DSA_ERR_INVALID_ARG;
   if (!aligned(lse, 4)) return DSA_ERR_INVALID_ARG;
-  ListBwdWorkspace ws = list_bwd_workspace(g, p->d, nnz, n_lists, workspace);
+  ListBwdWorkspace ws = list_bwd_workspace(g, nnz, n_lists, workspace);
   if (workspace == nullptr || ws_bytes < ws.bytes || !aligned(workspace, kAlign)) return DSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_list_check(g, kv_row_ptr, kv_list, n_lists, nnz, s);
@@ -1095,24 +1007,36 @@ int prefix_bwd_split(const Geom& g, int32_t L_text) {
   return static_cast<int>(n < 1 ? 1 : n);
 }
 
+// Parts the text queries' dQ is cut into over the video keys: enough units for about four
+// waves of persistent CTAs, at most one part per 64-key chunk of the video.
+int prefix_dq_split(const Geom& g, int32_t L_text) {
+  const int64_t units = g.BH * ((static_cast<int64_t>(L_text) + 127) / 128);
+  const int64_t nk = (g.N + 63) / 64;
+  int64_t n = (4 * 148 + units - 1) / (units > 0 ? units : 1);
+  if (n > nk) n = nk;
+  if (n > 16) n = 16;
+  return static_cast<int>(n < 1 ? 1 : n);
+}
+
 struct PrefixBwdWorkspace {
   BwdWorkspace video;
   float* lse_pad;    // [BH, Lp] text LSE, zeros past L
   float* delta_pad;  // [BH, Lp] text D
-  float* dq_acc_x;   // [BH, L, 128] fp32
-  float* dk_part;    // [n_split][BH, L, 128] fp32
+  float* dk_part;    // [n_split][BH, L, 128] fp32: the text keys' dK, dV per part of the queries
   float* dv_part;
-  int Lp, n_split;
+  float* dq_part;    // [n_split_q][BH, L, 128] fp32: the text queries' dQ per part of the keys
+  int Lp, n_split, n_split_q;
   size_t bytes;
 };
 
 PrefixBwdWorkspace prefix_bwd_workspace(const Geom& g, int32_t L, void* base) {
   PrefixBwdWorkspace w;
-  w.video = bwd_workspace(g, 128, base, true);
+  w.video = bwd_workspace(g, base);
   uint8_t* b = static_cast<uint8_t*>(base);
   size_t off = w.video.bytes;
   w.Lp = (L + 63) / 64 * 64;
   w.n_split = prefix_bwd_split(g, L);
+  w.n_split_q = prefix_dq_split(g, L);
   const size_t rows = static_cast<size_t>(g.BH) * L, rows_p = static_cast<size_t>(g.BH) * w.Lp;
   auto take = [&](size_t bytes) {
     float* ptr = b ? reinterpret_cast<float*>(b + off) : nullptr;
@@ -1121,9 +1045,9 @@ PrefixBwdWorkspace prefix_bwd_workspace(const Geom& g, int32_t L, void* base) {
   };
   w.lse_pad = take(sizeof(float) * rows_p);
   w.delta_pad = take(sizeof(float) * rows_p);
-  w.dq_acc_x = take(sizeof(float) * rows * 128);
   w.dk_part = take(sizeof(float) * rows * 128 * w.n_split);
   w.dv_part = take(sizeof(float) * rows * 128 * w.n_split);
+  w.dq_part = take(sizeof(float) * rows * 128 * w.n_split_q);
   w.bytes = off;
   return w;
 }
@@ -1168,59 +1092,153 @@ dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k
   if (L_text == 0)
     return launch_bwd_det(p, g, q, k, v, out, lse, dout, wv.row_ptr, wv.q_tiles, 0,
                           FwdKeys{wv.kv_tiles, nullptr, 0, 0}, wv.delta, dq, dk, dv, s);
-  // text rows: D, padded LSE / D copies, zeroed dQ accumulator
+  // Every gradient is summed in one CTA in a fixed order (no atomics), as in dsa_bwd:
+  //   video keys (dK, dV): the key-major kernel over their windows' queries and every text query;
+  //   text keys: the same kernel in the flat-key mode over every video and text query, in parts
+  //     whose fp32 sums are added in part order;
+  //   video queries (dQ): the query-major kernel over their windows' keys and every text key;
+  //   text queries: the query-major kernel in the flat mode over every video key, in parts,
+  //     and every text key, the parts' fp32 sums added in part order.
+  const int64_t rows = g.BH * g.N;
+  dsa::bwd_preprocess<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), wv.delta, rows);
+  st = launch_status();
+  if (st != DSA_OK) return st;
   const int64_t prow = g.BH * ws.Lp;
   dsa::bwd_preprocess_flat<<<static_cast<unsigned>((prow * 16 + 255) / 256), 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(out_text), static_cast<const __nv_bfloat16*>(dout_text), lse_text,
-      ws.delta_pad, ws.lse_pad, ws.dq_acc_x, L_text, ws.Lp, g.BH);
+      ws.delta_pad, ws.lse_pad, L_text, ws.Lp, g.BH);
   st = launch_status();
   if (st != DSA_OK) return st;
-  const ExtraQueries xq{q_text, dout_text, ws.lse_pad, ws.delta_pad, ws.dq_acc_x, L_text, ws.Lp};
-  // video keys: their windows' query chunks, then every text query chunk (dK, dV final)
-  st = launch_bwd(p, g, q, k, v, out, lse, dout, wv.row_ptr, wv.q_tiles, wv.delta, wv.dq_acc, dq, dk, dv, s, 0, &xq,
-                  false);
-  if (st != DSA_OK) return st;
-  // text keys: every video query chunk (the video as flat rows), in parts, then every text
-  // query chunk; fp32 partial dK, dV per part
-  CUtensorMap tq, tk, tv, tdo, tlse, tdel;
-  if (!make_flat_map(&tq, q, g.BH, g.N, 64) || !make_flat_map(&tk, k_text, g.BH, L_text, 128) ||
-      !make_flat_map(&tv, v_text, g.BH, L_text, 128) || !make_flat_map(&tdo, dout, g.BH, g.N, 64) ||
-      !make_vec_map(&tlse, lse, g.BH, g.N) || !make_vec_map(&tdel, wv.delta, g.BH, g.N))
+  CUtensorMap tq, tk, tv, tdo, tlse, tdel, tqx, tdox, tlsex, tdx;
+  if (!make_token_map(&tq, q, p, g, 64) || !make_token_map(&tk, k, p, g, 128) ||
+      !make_token_map(&tv, v, p, g, 128) || !make_token_map(&tdo, dout, p, g, 64) ||
+      !make_row_map(&tlse, lse, p, g, 64) || !make_row_map(&tdel, wv.delta, p, g, 64) ||
+      !make_flat_map(&tqx, q_text, g.BH, L_text, 64) || !make_flat_map(&tdox, dout_text, g.BH, L_text, 64) ||
+      !make_vec_map(&tlsex, ws.lse_pad, g.BH, ws.Lp) || !make_vec_map(&tdx, ws.delta_pad, g.BH, ws.Lp))
     return DSA_ERR_CUDA;
+  // video keys
   dsa::BwdBf16Params bp;
   std::memset(&bp, 0, sizeof(bp));
-  bp.dq_acc = wv.dq_acc;
+  bp.row_ptr = wv.row_ptr;
+  bp.q_tiles = wv.q_tiles;
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.n_tiles = g.n_tiles;
+  bp.KU = g.tile_tokens / 128;
+  bp.QS = g.tile_tokens / 64;
+  bp.n_units = static_cast<int>(g.BH * g.n_tiles * bp.KU);
+  bp.G1 = g.G[1];
+  bp.G2 = g.G[2];
+  bp.tt = p->tile[0];
+  bp.th = p->tile[1];
+  bp.tw = p->tile[2];
+  bp.kcs = 128 / (p->tile[1] * p->tile[2]);
+  bp.qcs = 64 / (p->tile[1] * p->tile[2]);
+  bp.T = p->T;
+  bp.H = p->H;
+  bp.W = p->W;
   bp.N = static_cast<int>(g.N);
   bp.scale = p->scale;
   bp.scale_log2 = p->scale * 1.4426950408889634f;
   bp.Lxq = L_text;
-  bp.dq_acc_x = ws.dq_acc_x;
-  bp.Lk = L_text;
-  bp.Nq = static_cast<int>(g.N);
-  bp.n_split = ws.n_split;
-  bp.dk_part = ws.dk_part;
-  bp.dv_part = ws.dv_part;
-  bp.part_stride = g.BH * static_cast<int64_t>(L_text) * 128;
-  bp.n_units = static_cast<int>(g.BH * ((L_text + 127) / 128) * ws.n_split);
-  bp.tt = bp.th = bp.tw = 1;  // no tile geometry in the flat-key mode
-  bp.T = bp.H = bp.W = 1;
-  st = launch_bwd_kernel<true, true>(bp, tq, tk, tv, tdo, tlse, tdel, &xq, g.BH, s);
-  if (st != DSA_OK) return st;
-  // dQ of both token types, dK and dV of the text
-  const int64_t n8v = g.BH * g.N * 128 / 8, n8t = g.BH * static_cast<int64_t>(L_text) * 128 / 8;
-  dsa::bwd_dq_convert<<<static_cast<unsigned>((n8v + 255) / 256), 256, 0, s>>>(
-      wv.dq_acc, static_cast<__nv_bfloat16*>(dq), p->scale, n8v);
-  st = launch_status();
-  if (st != DSA_OK) return st;
-  dsa::bwd_dq_convert<<<static_cast<unsigned>((n8t + 255) / 256), 256, 0, s>>>(
-      ws.dq_acc_x, static_cast<__nv_bfloat16*>(dq_text), p->scale, n8t);
-  st = launch_status();
-  if (st != DSA_OK) return st;
-  const int64_t n4 = 2 * n8t;
-  dsa::bwd_kv_combine<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
-      ws.dk_part, ws.dv_part, ws.n_split, bp.part_stride, p->scale, n4, static_cast<__nv_bfloat16*>(dk_text),
-      static_cast<__nv_bfloat16*>(dv_text));
-  return launch_status();
+  bp.n_split = 1;
+  {
+    auto kernel = dsa::bwd_bf16_kernel<false, true>;
+    constexpr uint32_t smem = dsa::bwd::kSmemBytes;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    int sms = 0;
+    if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(bp.n_units < sms ? bp.n_units : sms);
+    kernel<<<grid, dsa::bwd::kThreads, smem, s>>>(tq, tk, tv, tdo, tlse, tdel, tqx, tdox, tlsex, tdx, bp);
+    st = launch_status();
+    if (st != DSA_OK) return st;
+  }
+  // text keys: every video query chunk (the video as flat rows), in parts, then every text
+  // query chunk; fp32 partial dK, dV per part
+  {
+    CUtensorMap fq, fk, fv, fdo, flse, fdel;
+    if (!make_flat_map(&fq, q, g.BH, g.N, 64) || !make_flat_map(&fk, k_text, g.BH, L_text, 128) ||
+        !make_flat_map(&fv, v_text, g.BH, L_text, 128) || !make_flat_map(&fdo, dout, g.BH, g.N, 64) ||
+        !make_vec_map(&flse, lse, g.BH, g.N) || !make_vec_map(&fdel, wv.delta, g.BH, g.N))
+      return DSA_ERR_CUDA;
+    dsa::BwdBf16Params fp;
+    std::memset(&fp, 0, sizeof(fp));
+    fp.N = static_cast<int>(g.N);
+    fp.scale = p->scale;
+    fp.scale_log2 = p->scale * 1.4426950408889634f;
+    fp.Lxq = L_text;
+    fp.Lk = L_text;
+    fp.Nq = static_cast<int>(g.N);
+    fp.n_split = ws.n_split;
+    fp.dk_part = ws.dk_part;
+    fp.dv_part = ws.dv_part;
+    fp.part_stride = g.BH * static_cast<int64_t>(L_text) * 128;
+    fp.n_units = static_cast<int>(g.BH * ((L_text + 127) / 128) * ws.n_split);
+    fp.tt = fp.th = fp.tw = 1;  // no tile geometry in the flat-key mode
+    fp.T = fp.H = fp.W = 1;
+    auto kernel = dsa::bwd_bf16_kernel<true, true>;
+    constexpr uint32_t smem = dsa::bwd::kSmemBytes;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    int sms = 0;
+    if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(fp.n_units < sms ? fp.n_units : sms);
+    kernel<<<grid, dsa::bwd::kThreads, smem, s>>>(fq, fk, fv, fdo, flse, fdel, tqx, tdox, tlsex, tdx, fp);
+    st = launch_status();
+    if (st != DSA_OK) return st;
+    const int64_t n4 = g.BH * static_cast<int64_t>(L_text) * 128 / 4;
+    dsa::bwd_kv_combine<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
+        ws.dk_part, ws.dv_part, ws.n_split, fp.part_stride, p->scale, n4, static_cast<__nv_bfloat16*>(dk_text),
+        static_cast<__nv_bfloat16*>(dv_text));
+    st = launch_status();
+    if (st != DSA_OK) return st;
+  }
+  // video queries: dQ over their windows' keys and every text key
+  {
+    CUtensorMap tq2, tdo2, tk2, tv2, tkx, tvx;
+    if (!make_token_map(&tq2, q, p, g, 128) || !make_token_map(&tdo2, dout, p, g, 128) ||
+        !make_token_map(&tk2, k, p, g, 64) || !make_token_map(&tv2, v, p, g, 64) ||
+        !make_flat_map(&tkx, k_text, g.BH, L_text, 64) || !make_flat_map(&tvx, v_text, g.BH, L_text, 64))
+      return DSA_ERR_CUDA;
+    dsa::BwdDqParams dp = dq_params(p, g, lse, wv.delta, dq);
+    dp.kv_tiles = wv.kv_tiles;
+    dp.Lx = L_text;
+    st = launch_dq<false, true>(tq2, tk2, tv2, tdo2, tkx, tvx, dp, s);
+    if (st != DSA_OK) return st;
+  }
+  // text queries: dQ over every video key (flat, in parts) and every text key (with part 0)
+  {
+    CUtensorMap fq, fdo, fk, fv, tkx, tvx;
+    if (!make_flat_map(&fq, q_text, g.BH, L_text, 128) || !make_flat_map(&fdo, dout_text, g.BH, L_text, 128) ||
+        !make_flat_map(&fk, k, g.BH, g.N, 64) || !make_flat_map(&fv, v, g.BH, g.N, 64) ||
+        !make_flat_map(&tkx, k_text, g.BH, L_text, 64) || !make_flat_map(&tvx, v_text, g.BH, L_text, 64))
+      return DSA_ERR_CUDA;
+    dsa::BwdDqParams dp;
+    std::memset(&dp, 0, sizeof(dp));
+    dp.lse = ws.lse_pad;
+    dp.delta = ws.delta_pad;
+    dp.ld_rows = ws.Lp;
+    dp.Lq = L_text;
+    dp.Lk = static_cast<int>(g.N);
+    dp.Lx = L_text;
+    dp.n_split = ws.n_split_q;
+    dp.dq_part = ws.dq_part;
+    dp.part_stride = g.BH * static_cast<int64_t>(L_text) * 128;
+    dp.n_units = static_cast<int>(g.BH * ((L_text + 127) / 128) * ws.n_split_q);
+    dp.scale = p->scale;
+    dp.scale_log2 = p->scale * 1.4426950408889634f;
+    dp.tt = dp.th = dp.tw = 1;
+    dp.T = dp.H = dp.W = 1;
+    dp.S = dp.KS = 1;
+    st = launch_dq<true, true>(fq, fk, fv, fdo, tkx, tvx, dp, s);
+    if (st != DSA_OK) return st;
+    const int64_t n8 = g.BH * static_cast<int64_t>(L_text) * 128 / 8;
+    dsa::dq_parts_combine<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
+        ws.dq_part, ws.n_split_q, dp.part_stride, n8, static_cast<__nv_bfloat16*>(dq_text));
+    return launch_status();
+  }
 }
 
 dsa_status_t dsa_selftest_wait(void* stream) {

@@ -8,14 +8,14 @@
 //   dK_m = scale sum_n dS_nm q_n,   dQ_n = scale sum_m dS_nm k_m,
 // where n runs over the query tokens whose window holds key m.
 //
-// Kernels:
-//   bwd_preprocess : D = rowsum(dO * O) (fp32), and zeroes the fp32 dQ accumulator of the
-//                    forms that reduce dQ with atomics (the text prefix);
-//   bwd_bf16_kernel: key-major and persistent (described above the kernel): dK and dV, and
-//                    with kDq also dQ, added with fp32 atomics into the accumulator;
-//   bwd_dq_convert : dQ = scale * accumulator, as bf16.
-// The window and key-tile-list backward take dQ from the query-major bwd_dq_kernel
-// (dsa_bwd_dq.cuh) instead: deterministic, with no accumulator.
+// Kernels here:
+//   bwd_preprocess      : D = rowsum(dO * O) (fp32);
+//   bwd_preprocess_flat : the same for flat (text) rows, with padded LSE and D copies;
+//   bwd_bf16_kernel     : key-major and persistent (described above the kernel): dK and dV,
+//                         each key row summed by one CTA in a fixed order;
+//   bwd_kv_combine      : the flat-key mode's per-part fp32 dK, dV summed in part order.
+// dQ comes from the query-major bwd_dq_kernel (dsa_bwd_dq.cuh).  No gradient is summed with
+// atomics, so the backward gives the same bits from run to run.
 #pragma once
 
 #include <stdint.h>
@@ -28,7 +28,6 @@ struct BwdBf16Params {
   const int32_t* row_ptr;  // inverse plan: [n_tiles + 1], or per (batch, head) [B*heads, n_tiles + 1]
   int rp_head_stride;      // 0 (one inverse map for every head) or n_tiles + 1
   const int32_t* q_tiles;  // [n_tiles * Wt]
-  float* dq_acc;           // [BH, N, 128] fp32, zeroed by bwd_preprocess
   __nv_bfloat16* dk;       // [BH, N, 128]
   __nv_bfloat16* dv;
   int n_tiles;
@@ -42,9 +41,8 @@ struct BwdBf16Params {
   int T, H, W, N;
   float scale, scale_log2;
   // extra (text) query rows after every unit's own query chunks: flat [B*heads, Lxq, 128] Q
-  // and dO, [B*heads, Lxq] LSE and D; their dQ goes to dq_acc_x [B*heads, Lxq, 128] fp32
+  // and dO, LSE and D padded to [B*heads, Lp] (Lp a multiple of 64)
   int Lxq;
-  float* dq_acc_x;
   // flat-key mode: the keys are Lk rows of a flat sequence and the main query rows Nq rows
   // of another, in 64-row chunks cut into n_split parts; part j writes fp32 dK, dV at
   // dk_part / dv_part + j * part_stride (the extra queries go with part 0)
@@ -65,39 +63,24 @@ constexpr uint32_t kQHalf = kQBytes / 2;
 constexpr uint32_t kStageBytes = 2 * kQBytes + 1024;  // Q, dO, LSE (at +0) and D (at +512) vectors
 constexpr uint32_t kOffK = 0, kOffV = kKBytes;
 constexpr uint32_t kOffStage = 2 * kKBytes;
-constexpr uint32_t kDSBytes = 128 * 64 * 2;
-// Shared-memory layout: K, V, the query-chunk ring, then (kDq only) two dS^T buffers of
-// 128 x 64 bf16 (the B operand of dQ^T), 64 int32 token offsets within a query chunk, the
-// barriers.  Without dQ the dS^T buffers' room gives the ring a fourth stage.
-template <bool kDq>
-struct Layout {
-  static constexpr int kStages = kDq ? 3 : 4;
-  static constexpr uint32_t kOffDS = kOffStage + kStages * kStageBytes;
-  static constexpr uint32_t kOffRel = kOffDS + (kDq ? 2 * kDSBytes : 0);
-  static constexpr uint32_t kOffBar = kOffRel + 256;
-  static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-};
-static_assert(Layout<true>::kSmemBytes <= 227 * 1024 && Layout<false>::kSmemBytes <= 227 * 1024,
-              "shared memory layout too large");
-constexpr uint32_t kTmemCols = 512;  // dV [0,128), dK [128,256), S^T buffers [256,384), dP^T / dQ^T [384,512)
+// Shared-memory layout: K, V, a 4-stage ring of query chunks (Q, dO, LSE, D), 64 int32 token
+// offsets within a query chunk, the barriers.
+constexpr int kStages = 4;
+constexpr uint32_t kOffRel = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kOffBar = kOffRel + 256;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory layout too large");
+constexpr uint32_t kTmemCols = 512;  // dV [0,128), dK [128,256), S^T buffers [256,384), dP^T buffers [384,512)
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, 0, 0);     // K Q^T and V dO^T
 constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 128, 0, 1);  // P^T dO, dS^T Q
-constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, 64, 1, 1);    // K^T dS^T
 // A byte offset added to a shared-memory descriptor's address field (16-byte units).
 __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
 // Columns (within a chunk's 64-column S^T buffer) of packed bf16 P^T and dS^T for queries
-// [16kk, 16kk + 16).  With kDq one thread per key row handles all 64 queries: P^T in columns
-// [0, 32), dS^T in [32, 64).  Without it two threads share a row, thread h taking queries
-// [32h, 32h + 32) and writing over its own score columns [32h, 32h + 32): P^T in the first
-// 16, dS^T in the next 16.
-template <bool kDq>
-__device__ __forceinline__ uint32_t pt_col(int kk) {
-  return kDq ? 8u * kk : 32u * (kk >> 1) + 8u * (kk & 1);
-}
-template <bool kDq>
-__device__ __forceinline__ uint32_t dst_col(int kk) {
-  return kDq ? 32u + 8u * kk : 32u * (kk >> 1) + 16u + 8u * (kk & 1);
-}
+// [16kk, 16kk + 16): two threads share a key row, thread h taking queries [32h, 32h + 32)
+// and writing over its own score columns [32h, 32h + 32), P^T in the first 16, dS^T in the
+// next 16.
+__device__ __forceinline__ uint32_t pt_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
+__device__ __forceinline__ uint32_t dst_col(int kk) { return 32u * (kk >> 1) + 16u + 8u * (kk & 1); }
 }  // namespace bwd
 
 // A work unit: (batch, head), key tile and its 128-key chunk (flat-key mode: the 128-row key
@@ -166,8 +149,7 @@ __device__ __forceinline__ int64_t chunk_row_token(int r, int t0, int h0, int w0
 
 __global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ dout,
-                                                      float* __restrict__ delta, float* __restrict__ dq_acc,
-                                                      int64_t rows) {
+                                                      float* __restrict__ delta, int64_t rows) {
   // 16 threads per 128-wide row, 8 elements (16 bytes) each
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 16;
   const int part = threadIdx.x % 16;
@@ -184,11 +166,6 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __res
       s = fmaf(x.x, y.x, s);
       s = fmaf(x.y, y.y, s);
     }
-    if (dq_acc != nullptr) {
-      float4* z = reinterpret_cast<float4*>(dq_acc + row * 128) + part * 2;
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
   }
 #pragma unroll
   for (int o2 = 8; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
@@ -197,13 +174,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const __nv_bfloat16* __res
 
 // bwd_preprocess for flat rows ([B*heads, L, 128]) whose LSE and D are read by 64-row TMA
 // boxes: D and a copy of the LSE go to [B*heads, Lp] arrays (Lp a multiple of 64, so every
-// box starts 16-byte aligned) with zeros past L; the fp32 dQ accumulator [B*heads, L, 128]
-// is zeroed.
+// box starts 16-byte aligned) with zeros past L.
 __global__ void __launch_bounds__(256) bwd_preprocess_flat(const __nv_bfloat16* __restrict__ o,
                                                            const __nv_bfloat16* __restrict__ dout,
                                                            const float* __restrict__ lse, float* __restrict__ delta_pad,
-                                                           float* __restrict__ lse_pad, float* __restrict__ dq_acc,
-                                                           int L, int Lp, int64_t BH) {
+                                                           float* __restrict__ lse_pad, int L, int Lp, int64_t BH) {
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 16;
   const int part = threadIdx.x % 16;
   const bool in = r < BH * Lp;
@@ -224,9 +199,6 @@ __global__ void __launch_bounds__(256) bwd_preprocess_flat(const __nv_bfloat16* 
       s = fmaf(x.x, y.x, s);
       s = fmaf(x.y, y.y, s);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + row * 128) + part * 2;
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int o2 = 8; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
@@ -234,20 +206,6 @@ __global__ void __launch_bounds__(256) bwd_preprocess_flat(const __nv_bfloat16* 
     delta_pad[r] = s;
     lse_pad[r] = live ? lse[row] : 0.f;
   }
-}
-
-__global__ void __launch_bounds__(256) bwd_dq_convert(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
-                                                      float scale, int64_t n8) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n8) return;
-  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-  const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
-  uint4 v;
-  v.x = pack_bf16x2(a.x * scale, a.y * scale);
-  v.y = pack_bf16x2(a.z * scale, a.w * scale);
-  v.z = pack_bf16x2(b.x * scale, b.y * scale);
-  v.w = pack_bf16x2(b.z * scale, b.w * scale);
-  reinterpret_cast<uint4*>(dq)[i] = v;
 }
 
 // dK = scale * sum of the parts' dK, dV = sum of their dV (fp32 parts of flat keys), bf16.
@@ -272,18 +230,16 @@ __global__ void __launch_bounds__(256) bwd_kv_combine(const float* __restrict__ 
 // per work unit.  The unit walks the 64-query chunks of every query tile whose window
 // holds its key tile (the CSR row of the inverse plan).  Roles:
 //   warp 8      TMA producer: K and V of the unit, then per query chunk Q, dO, LSE and D
-//               through a 3-stage ring;
+//               through a 4-stage ring;
 //   warp 9      MMA issuer, per chunk c (buffer b = c % 2):
 //                 S^T_b = K Q_c^T, dP^T_b = V dO_c^T                 (TMEM, 64 columns each)
 //                 dV += P^T dO_c, dK += dS^T Q_c (P^T and dS^T read from TMEM)
-//                 dQ^T_c = K^T dS^T into the dP^T_b columns
-//               so the scores of chunk c+1 are ready while chunk c's softmax runs;
-//   warps 0-3   one thread per key row: P^T = exp2(S^T * scale * log2 e - LSE_n * log2 e),
-//               dS^T = P^T (dP^T - D_n); P^T and dS^T go back into TMEM as bf16 (the dV and dK
-//               products read them there), dS^T also into smem (the B operand of dQ^T);
-//   warps 4-7   one thread per channel d: reads dQ^T_c and adds it to the fp32 dQ
-//               accumulator (a warp covers 32 consecutive channels of one query row); at
-//               the end of a unit, one thread per key row writes dV and scale * dK as bf16.
+//               so the scores of chunk c+1 are ready while chunk c's elementwise work runs;
+//   warps 0-7   two threads per key row (lane of warps w and w + 4), thread h taking queries
+//               [32h, 32h + 32) of every chunk: P^T = exp2(S^T * scale * log2 e - LSE_n *
+//               log2 e), dS^T = P^T (dP^T - D_n), both back into TMEM as bf16 over the
+//               thread's own score columns (the dV and dK products read them there); at the
+//               end of a unit warps 0-3 write dV and warps 4-7 scale * dK as bf16.
 // Barriers advance at most one phase ahead of their waiters (each refill of a buffer waits
 // for the previous consumer), so waiting by phase parity is unambiguous.
 //
@@ -291,7 +247,7 @@ __global__ void __launch_bounds__(256) bwd_kv_combine(const float* __restrict__ 
 // the end of either load as zeros and get P = dS = 0, and their gradients are not written.
 // kExtra: extra queries (p.Lxq of them, flat maps tmQx, tmDOx, tmLsex, tmDx) follow every
 // unit's own.
-template <bool kFlatK, bool kExtra, bool kDq = true>
+template <bool kFlatK, bool kExtra>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -300,27 +256,23 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
                     const __grid_constant__ CUtensorMap tmLsex, const __grid_constant__ CUtensorMap tmDx,
                     BwdBf16Params p) {
   using namespace bwd;
-  using L = Layout<kDq>;
-  constexpr int kStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw + pad;
-  int32_t* rel = reinterpret_cast<int32_t*>(smem + L::kOffRel);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  int32_t* rel = reinterpret_cast<int32_t*>(smem + kOffRel);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_free = bars + 1;
   uint64_t* ld_full = bars + 2;               // [kStages]
   uint64_t* ld_empty = bars + 2 + kStages;    // [kStages]
   uint64_t* s_full = bars + 2 + 2 * kStages;  // [2]
   uint64_t* p_full = s_full + 2;              // [2]
-  uint64_t* dq_full = s_full + 4;             // [2]
-  uint64_t* dq_free = s_full + 6;             // [2]
-  uint64_t* dkv_full = s_full + 8;
-  uint64_t* dkv_free = s_full + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
-  volatile int* abort = reinterpret_cast<volatile int*>(s_full + 11);
+  uint64_t* dkv_full = s_full + 4;
+  uint64_t* dkv_free = s_full + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 6);
+  volatile int* abort = reinterpret_cast<volatile int*>(s_full + 7);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -345,12 +297,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(p_full + b, kDq ? 4 : 8);  // the warps that write P^T and dS^T
-      mbar_init(dq_full + b, 1);
-      mbar_init(dq_free + b, 4);
+      mbar_init(p_full + b, 8);  // the warps that write P^T and dS^T
     }
     mbar_init(dkv_full, 1);
-    mbar_init(dkv_free, kDq ? 4 : 8);  // the warps that read dK and dV out
+    mbar_init(dkv_free, 8);  // the warps that read dK and dV out
     *abort = 0;
     fence_mbar_init();
   }
@@ -432,10 +382,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     {
       const uint64_t dK = smem_desc_sw128(sbase + kOffK, 16, 1024);            // K, K-major
       const uint64_t dV = smem_desc_sw128(sbase + kOffV, 16, 1024);            // V, K-major
-      const uint64_t dKt = smem_desc_sw128(sbase + kOffK, kKHalf, 1024);       // K^T, MN-major
       const uint64_t dQk = smem_desc_sw128(sbase + kOffStage, 16, 1024);       // stage 0 Q, K-major
       const uint64_t dQm = smem_desc_sw128(sbase + kOffStage, kQHalf, 1024);   // stage 0 Q, MN-major
-      const uint64_t dSm = smem_desc_sw128(sbase + L::kOffDS, kKHalf, 1024);      // dS^T buffer 0, MN-major
       int ld = 0, uc = 0, sc = 0, pc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -459,20 +407,13 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             tc_fence_after();
             const uint32_t so = ((ld0 + cc) % kStages) * kStageBytes;
             const uint64_t q_m = desc_add(dQm, so), do_m = desc_add(dQm, so + kQBytes);
-            const uint64_t ds_m = desc_add(dSm, b * kDSBytes);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
-              mma_ts_warp(tDV, tS + b * 64 + pt_col<kDq>(kk), desc_add(do_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
+              mma_ts_warp(tDV, tS + b * 64 + pt_col(kk), desc_add(do_m, kk * 2048), kIdescAcc, (cc > 0) || (kk > 0));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q (dS^T from TMEM, beside P^T)
-              mma_ts_warp(tDK, tS + b * 64 + dst_col<kDq>(kk), desc_add(q_m, kk * 2048), kIdescAcc,
+              mma_ts_warp(tDK, tS + b * 64 + dst_col(kk), desc_add(q_m, kk * 2048), kIdescAcc,
                           (cc > 0) || (kk > 0));
-            if constexpr (kDq) {
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
-                mma_ss_warp(tDP + b * 64, desc_add(dKt, kk * 2048), desc_add(ds_m, kk * 2048), kIdescDQ, kk > 0);
-              mma_commit_warp(dq_full + b);
-            }
             mma_commit_warp(ld_empty + (ld0 + cc) % kStages);
           }
           if (c < n) {
@@ -487,10 +428,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
               const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
               mma_ss_warp(tS + b * 64, desc_add(dK, ko), desc_add(q_k, qo), kIdescS, kk > 0);
             }
-            // dP^T overwrites the dQ^T of chunk sc - 2: wait until it has been read out
-            if (kDq && sc >= 2) ok = __all_sync(0xffffffffu, mbar_wait(dq_free + b, ((sc >> 1) - 1) & 1, abort, 62));
-            if (!ok) break;
-            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, qo = (kk >> 2) * kQHalf + (kk & 3) * 32;
@@ -506,7 +443,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         ++uc;
       }
     }
-  } else if (!kDq && warp < 8) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ P^T, dS^T and dK / dV out
     // Two threads per key row (lane of warps w and w + 4): thread h takes queries [32h, 32h + 32)
     // of every chunk.  At the end of a unit warps 0-3 write dV and warps 4-7 scale * dK.
@@ -619,183 +556,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             y.z = pack_bf16x2(__uint_as_float(a[8 * j + 4]) * sc_out, __uint_as_float(a[8 * j + 5]) * sc_out);
             y.w = pack_bf16x2(__uint_as_float(a[8 * j + 6]) * sc_out, __uint_as_float(a[8 * j + 7]) * sc_out);
             dst[g * 4 + j] = y;
-          }
-        }
-      }
-      if (n > 0) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dkv_free);
-        ++uc;
-      }
-    }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------------ P^T, dS^T (key rows)
-    const int m = tid;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    int cc = 0, ld = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const BwdUnit x = bwd_unit<kFlatK>(p, u);
-      const BwdChunks qc = bwd_chunks<kFlatK, kExtra>(p, x);
-      const int n = qc.nm + qc.nx;
-      // flat keys: this thread's key row may lie past the end (zeros, no gradient)
-      const bool k_ok = !kFlatK || 128 * x.kt + m < p.Lk;
-      for (int c = 0; c < n; ++c, ++cc, ++ld) {
-        const int nvq = bwd_qvalid<kFlatK, kExtra>(p, qc, c);
-        const bool masked = !k_ok || nvq < 64;  // P = dS = 0 for missing keys and queries
-        const int b = cc & 1;
-        ok = mbar_wait(s_full + b, (cc >> 1) & 1, abort, 70);
-        if (ok) ok = mbar_wait(ld_full + ld % kStages, (ld / kStages) & 1, abort, 71);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const float* lse = reinterpret_cast<const float*>(smem + kOffStage + (ld % kStages) * kStageBytes + 2 * kQBytes);
-        const float* dd = lse + 128;
-        uint32_t sr[64], dr[64];
-        tmem_ld64_wait(tS + lane_off + b * 64, sr);
-        tmem_ld64_wait(tDP + lane_off + b * 64, dr);
-        const uint32_t dsrow = sbase + L::kOffDS + b * kDSBytes + (m >> 3) * 1024 + (m & 7) * 128;
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {  // query columns 8g..8g+7 form one 16-byte chunk
-          uint32_t pk[4], dk2[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int n0 = 8 * g + 2 * e;
-            float p0 = ex2_approx(fmaf(__uint_as_float(sr[n0]), p.scale_log2, -lse[n0] * 1.4426950408889634f));
-            float p1 = ex2_approx(fmaf(__uint_as_float(sr[n0 + 1]), p.scale_log2, -lse[n0 + 1] * 1.4426950408889634f));
-            if (masked) {
-              if (!k_ok || n0 >= nvq) p0 = 0.f;
-              if (!k_ok || n0 + 1 >= nvq) p1 = 0.f;
-            }
-            pk[e] = pack_bf16x2(p0, p1);
-            dk2[e] = pack_bf16x2(p0 * (__uint_as_float(dr[n0]) - dd[n0]), p1 * (__uint_as_float(dr[n0 + 1]) - dd[n0 + 1]));
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sr[4 * g + e] = pk[e];  // packed P^T of columns 8g..8g+7
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dr[4 * g + e] = dk2[e];  // packed dS^T (dP^T of these columns is used)
-          if constexpr (kDq) st_shared_v4(dsrow + ((g ^ (m & 7)) << 4), dk2[0], dk2[1], dk2[2], dk2[3]);
-        }
-        {
-          uint32_t w[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] = sr[e];
-          tmem_st32(tS + lane_off + b * 64, w);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] = dr[e];
-          tmem_st32(tS + lane_off + b * 64 + 32, w);
-        }
-        if constexpr (kDq) fence_proxy_async_smem();
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + b);
-      }
-      if (!ok) break;
-    }
-  } else {
-    // ------------------------------------------------------------------ dQ out, dK/dV epilogue
-    const int t = tid - 128;  // channel d for dQ^T, key row for dK / dV
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    int cc = 0, uc = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const BwdUnit x = bwd_unit<kFlatK>(p, u);
-      const BwdChunks qc = bwd_chunks<kFlatK, kExtra>(p, x);
-      const int bh = x.bh, kt = x.kt, ku = x.ku, n = qc.nm + qc.nx;
-      const int64_t slice = static_cast<int64_t>(bh) * p.N;
-      for (int c = 0; c < (kDq ? n : 0); ++c, ++cc) {
-        const int b = cc & 1;
-        ok = mbar_wait(dq_full + b, (cc >> 1) & 1, abort, 80);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t r[64];
-        tmem_ld64_wait(tDP + lane_off + b * 64, r);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dq_free + b);
-        if ((kExtra && c >= qc.nm) || kFlatK) {  // flat query rows: consecutive, the last chunk maybe partial
-          const bool extra = c >= qc.nm;
-          const int nvq = bwd_qvalid<kFlatK, kExtra>(p, qc, c);
-          float* base = extra ? p.dq_acc_x + (static_cast<int64_t>(bh) * p.Lxq + 64 * (c - qc.nm)) * 128 + t
-                              : p.dq_acc + (static_cast<int64_t>(bh) * p.Nq + 64 * (qc.c0 + c)) * 128 + t;
-#pragma unroll
-          for (int nn = 0; nn < 64; ++nn)
-            if (nn < nvq) atomicAdd(base + static_cast<int64_t>(nn) * 128, __uint_as_float(r[nn]));
-        } else {
-          const int qi = p.q_tiles[qc.row0 + c / p.QS], qs = c % p.QS;
-          const int q_t0 = (qi / (p.G1 * p.G2)) * p.tt + qs * p.qcs;
-          const int q_h0 = ((qi / p.G2) % p.G1) * p.th, q_w0 = (qi % p.G2) * p.tw;
-          float* base = p.dq_acc + (slice + (static_cast<int64_t>(q_t0) * p.H + q_h0) * p.W + q_w0) * 128 + t;
-#pragma unroll
-          for (int nn = 0; nn < 64; ++nn) atomicAdd(base + static_cast<int64_t>(rel[nn]) * 128, __uint_as_float(r[nn]));
-        }
-      }
-      if (!ok) break;
-      // dV and scale * dK of the unit's 128 keys; zeros for a key tile no window holds.
-      // Flat keys: fp32 partial sums of this part (unscaled dK), rows past Lk not written.
-      int64_t ktok;
-      bool k_row_ok = true;
-      if constexpr (kFlatK) {
-        ktok = 128 * static_cast<int64_t>(kt) + t;
-        k_row_ok = ktok < p.Lk;
-        if (!k_row_ok) ktok = 0;
-      } else {
-        const int k_t0 = (kt / (p.G1 * p.G2)) * p.tt + ku * p.kcs;
-        const int k_h0 = ((kt / p.G2) % p.G1) * p.th, k_w0 = (kt % p.G2) * p.tw;
-        ktok = chunk_row_token(t, k_t0, k_h0, k_w0, p.th, p.tw, p.H, p.W);
-      }
-      uint4* dv_dst = reinterpret_cast<uint4*>(p.dv + (slice + ktok) * 128);
-      uint4* dk_dst = reinterpret_cast<uint4*>(p.dk + (slice + ktok) * 128);
-      float4* dvp = nullptr;
-      float4* dkp = nullptr;
-      if constexpr (kFlatK) {
-        const int64_t o = static_cast<int64_t>(x.part) * p.part_stride + (static_cast<int64_t>(bh) * p.Lk + ktok) * 128;
-        dvp = reinterpret_cast<float4*>(p.dv_part + o);
-        dkp = reinterpret_cast<float4*>(p.dk_part + o);
-      }
-      if (n > 0) {
-        ok = mbar_wait(dkv_full, uc & 1, abort, 81);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-      }
-#pragma unroll 1
-      for (int g = 0; g < 4; ++g) {
-        uint32_t a[32], bb[32];
-        if (n > 0) {
-          tmem_ld32_wait(tDV + lane_off + g * 32, a);
-          tmem_ld32_wait(tDK + lane_off + g * 32, bb);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) a[j] = bb[j] = 0u;
-        }
-        if constexpr (kFlatK) {
-          if (k_row_ok) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              dvp[g * 8 + j] = make_float4(__uint_as_float(a[4 * j]), __uint_as_float(a[4 * j + 1]),
-                                           __uint_as_float(a[4 * j + 2]), __uint_as_float(a[4 * j + 3]));
-              dkp[g * 8 + j] = make_float4(__uint_as_float(bb[4 * j]), __uint_as_float(bb[4 * j + 1]),
-                                           __uint_as_float(bb[4 * j + 2]), __uint_as_float(bb[4 * j + 3]));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 x, y;
-            x.x = pack_bf16x2(__uint_as_float(a[8 * j + 0]), __uint_as_float(a[8 * j + 1]));
-            x.y = pack_bf16x2(__uint_as_float(a[8 * j + 2]), __uint_as_float(a[8 * j + 3]));
-            x.z = pack_bf16x2(__uint_as_float(a[8 * j + 4]), __uint_as_float(a[8 * j + 5]));
-            x.w = pack_bf16x2(__uint_as_float(a[8 * j + 6]), __uint_as_float(a[8 * j + 7]));
-            y.x = pack_bf16x2(__uint_as_float(bb[8 * j + 0]) * p.scale, __uint_as_float(bb[8 * j + 1]) * p.scale);
-            y.y = pack_bf16x2(__uint_as_float(bb[8 * j + 2]) * p.scale, __uint_as_float(bb[8 * j + 3]) * p.scale);
-            y.z = pack_bf16x2(__uint_as_float(bb[8 * j + 4]) * p.scale, __uint_as_float(bb[8 * j + 5]) * p.scale);
-            y.w = pack_bf16x2(__uint_as_float(bb[8 * j + 6]) * p.scale, __uint_as_float(bb[8 * j + 7]) * p.scale);
-            dv_dst[g * 4 + j] = x;
-            dk_dst[g * 4 + j] = y;
           }
         }
       }

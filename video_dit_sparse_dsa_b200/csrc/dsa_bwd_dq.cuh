@@ -67,6 +67,16 @@ struct BwdDqParams {
   int kcs;                  // t-extent of a 64-token key chunk
   int T, H, W, N;
   float scale, scale_log2;
+  // extra (text) keys after every unit's own: Lx rows of flat [B*heads, Lx, 128] K and V
+  // (0: none); the tail of their last 64-row chunk is masked
+  int Lx;
+  // flat mode: the query rows are Lq rows of a flat [B*heads, Lq, 128] sequence (lse, delta
+  // [B*heads, Lq]) and the keys Lk rows of another, in 64-row chunks cut into n_split parts
+  // (the extra keys go with part 0); part j writes fp32 scale * dQ to dq_part + j * part_stride
+  int Lq, Lk, n_split;
+  float* dq_part;
+  int64_t part_stride;
+  int ld_rows;              // flat mode: rows per (batch, head) of lse and delta (>= Lq)
 };
 
 namespace bdq {
@@ -125,14 +135,58 @@ struct Unit {
   int bh, tile, sub;
 };
 
+// Window / list form: units run (batch*head, tile, chunk).  Flat form: (batch*head, part,
+// query chunk), so the query chunks that read the same keys are neighbours; tile = the query
+// chunk, sub = the part.
+template <bool kFlat>
 __device__ __forceinline__ Unit decode(const BwdDqParams& p, int u) {
   Unit x;
-  const int per_bh = p.S * p.n_tiles;
-  x.bh = u / per_bh;
-  const int rem = u % per_bh;
-  x.tile = rem / p.S;
-  x.sub = rem % p.S;
+  if constexpr (kFlat) {
+    const int nq = (p.Lq + 127) / 128, per_bh = nq * p.n_split;
+    x.bh = u / per_bh;
+    const int rem = u % per_bh;
+    x.sub = rem / nq;
+    x.tile = rem % nq;
+  } else {
+    const int per_bh = p.S * p.n_tiles;
+    x.bh = u / per_bh;
+    const int rem = u % per_bh;
+    x.tile = rem / p.S;
+    x.sub = rem % p.S;
+  }
   return x;
+}
+
+// The unit's 64-key chunks: nm main chunks from main chunk c0 (the listed tiles' chunks, or
+// rows of the flat key sequence), then nx chunks of the extra keys.
+struct Chunks {
+  int c0, nm, nx;
+};
+
+template <bool kFlat, bool kExtra>
+__device__ __forceinline__ Chunks unit_chunks(const BwdDqParams& p, const Unit& x, int n_list) {
+  Chunks k;
+  const int nx = kExtra ? (p.Lx + 63) / 64 : 0;
+  if constexpr (kFlat) {
+    const int n_main = (p.Lk + 63) / 64, per = (n_main + p.n_split - 1) / p.n_split;
+    k.c0 = x.sub * per;
+    k.nm = max(min(per, n_main - k.c0), 0);
+    k.nx = x.sub == 0 ? nx : 0;
+  } else {
+    k.c0 = 0;
+    k.nm = n_list * p.KS;
+    k.nx = nx;
+  }
+  return k;
+}
+
+// Keys present in local chunk j: the last chunk of a flat sequence and of the extra keys can
+// be partial.
+template <bool kFlat, bool kExtra>
+__device__ __forceinline__ int chunk_valid(const BwdDqParams& p, const Chunks& k, int j) {
+  if (!kFlat && !kExtra) return 64;
+  if (j < k.nm) return kFlat ? min(p.Lk - 64 * (k.c0 + j), 64) : 64;
+  return min(p.Lx - 64 * (j - k.nm), 64);
 }
 
 // Key tiles of query tile `tile` (window plan or the caller's list, every index clamped
@@ -157,9 +211,14 @@ __device__ __forceinline__ int64_t chunk_token(const BwdDqParams& p, int tile, i
 }
 }  // namespace bdq
 
+// kFlat: flat query rows over flat key rows in parts (rank-3 maps; rows past the end load as
+// zeros, keys past the end are masked, rows past the end are not written).  kExtra: the
+// extra keys (maps tmKx, tmVx) follow every unit's own.
+template <bool kFlat, bool kExtra>
 __global__ void __launch_bounds__(bdq::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdDqParams p) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmKx, const __grid_constant__ CUtensorMap tmVx, BwdDqParams p) {
   using namespace bdq;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -192,6 +251,10 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
     tma_prefetch_map(&tmDO);
+    if (kExtra && p.Lx > 0) {
+      tma_prefetch_map(&tmKx);
+      tma_prefetch_map(&tmVx);
+    }
     mbar_init(qd_full, 1);
     mbar_init(qd_empty, 8);  // the staging copy is in TMEM
     for (int s = 0; s < kKStages; ++s) {
@@ -230,21 +293,29 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
         int ld = 0, uc = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-          const Unit x = decode(p, u);
+          const Unit x = decode<kFlat>(p, u);
           int n_list = 0;
-          const int32_t* kv = unit_keys(p, x.bh, x.tile, n_list);
-          const int n_steps = n_list * p.KS;
+          const int32_t* kv = kFlat ? nullptr : unit_keys(p, x.bh, x.tile, n_list);
+          const Chunks ck = unit_chunks<kFlat, kExtra>(p, x, n_list);
+          const int n_steps = ck.nm + ck.nx;
           if (n_steps == 0) continue;  // no keys: the elementwise warps write dQ = 0
           if (is_k) {
             ok = mbar_wait(qd_empty, (uc & 1) ^ 1, abort, 110);
             if (!ok) break;
-            const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
-            const int t0 = qt * p.tt + x.sub * p.tcs;
             mbar_arrive_expect_tx(qd_full, 2 * kQTileBytes);
-            tma_load_5d(smem + kOffQ, &tmQ, qd_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
-            tma_load_5d(smem + kOffQ + kQHalfBytes, &tmQ, qd_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
-            tma_load_5d(smem + kOffDO, &tmDO, qd_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
-            tma_load_5d(smem + kOffDO + kQHalfBytes, &tmDO, qd_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
+            if constexpr (kFlat) {  // rows past Lq load as zeros
+              tma_load_3d(smem + kOffQ, &tmQ, qd_full, 0, 128 * x.tile, x.bh);
+              tma_load_3d(smem + kOffQ + kQHalfBytes, &tmQ, qd_full, 64, 128 * x.tile, x.bh);
+              tma_load_3d(smem + kOffDO, &tmDO, qd_full, 0, 128 * x.tile, x.bh);
+              tma_load_3d(smem + kOffDO + kQHalfBytes, &tmDO, qd_full, 64, 128 * x.tile, x.bh);
+            } else {
+              const int qt = x.tile / (p.G1 * p.G2), qh = (x.tile / p.G2) % p.G1, qw = x.tile % p.G2;
+              const int t0 = qt * p.tt + x.sub * p.tcs;
+              tma_load_5d(smem + kOffQ, &tmQ, qd_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
+              tma_load_5d(smem + kOffQ + kQHalfBytes, &tmQ, qd_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
+              tma_load_5d(smem + kOffDO, &tmDO, qd_full, 0, qw * p.tw, qh * p.th, t0, x.bh);
+              tma_load_5d(smem + kOffDO + kQHalfBytes, &tmDO, qd_full, 64, qw * p.tw, qh * p.th, t0, x.bh);
+            }
           }
           ++uc;
           const int n_st = is_k ? kKStages : kVStages;
@@ -252,14 +323,24 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
             const int st = ld % n_st;
             ok = mbar_wait((is_k ? k_empty : v_empty) + st, ((ld / n_st) & 1) ^ 1, abort, is_k ? 111 : 112);
             if (!ok) break;
-            const int kt = min(max(kv[j / p.KS], 0), p.n_tiles - 1), ks = j % p.KS;
-            const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.kcs;
-            const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
             uint64_t* full = (is_k ? k_full : v_full) + st;
             uint8_t* dst = smem + (is_k ? kOffK : kOffV) + st * kKTileBytes;
             mbar_arrive_expect_tx(full, kKTileBytes);
-            tma_load_5d(dst, is_k ? &tmK : &tmV, full, 0, w0, h0, t0, x.bh);
-            tma_load_5d(dst + kKHalfBytes, is_k ? &tmK : &tmV, full, 64, w0, h0, t0, x.bh);
+            if (kExtra && j >= ck.nm) {  // extra keys (rows past Lx load as zeros and are masked)
+              const CUtensorMap* m = is_k ? &tmKx : &tmVx;
+              tma_load_3d(dst, m, full, 0, 64 * (j - ck.nm), x.bh);
+              tma_load_3d(dst + kKHalfBytes, m, full, 64, 64 * (j - ck.nm), x.bh);
+            } else if (kFlat) {  // flat key rows (past Lk: zeros, masked)
+              const CUtensorMap* m = is_k ? &tmK : &tmV;
+              tma_load_3d(dst, m, full, 0, 64 * (ck.c0 + j), x.bh);
+              tma_load_3d(dst + kKHalfBytes, m, full, 64, 64 * (ck.c0 + j), x.bh);
+            } else {
+              const int kt = min(max(kv[j / p.KS], 0), p.n_tiles - 1), ks = j % p.KS;
+              const int t0 = (kt / (p.G1 * p.G2)) * p.tt + ks * p.kcs;
+              const int h0 = ((kt / p.G2) % p.G1) * p.th, w0 = (kt % p.G2) * p.tw;
+              tma_load_5d(dst, is_k ? &tmK : &tmV, full, 0, w0, h0, t0, x.bh);
+              tma_load_5d(dst + kKHalfBytes, is_k ? &tmK : &tmV, full, 64, w0, h0, t0, x.bh);
+            }
           }
         }
       }
@@ -273,9 +354,9 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         int n_list = 0;
-        const Unit x = decode(p, u);
-        unit_keys(p, x.bh, x.tile, n_list);
-        const int n_steps = n_list * p.KS;
+        const Unit x = decode<kFlat>(p, u);
+        if constexpr (!kFlat) unit_keys(p, x.bh, x.tile, n_list);
+        const int n_steps = unit_chunks<kFlat, kExtra>(p, x, n_list).nm + unit_chunks<kFlat, kExtra>(p, x, n_list).nx;
         if (n_steps == 0) continue;
         ok = warp_wait(qa_full, uc & 1, abort, 120);
         if (!ok) break;
@@ -327,18 +408,32 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
     int g = 0, uc = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit x = decode(p, u);
+      const Unit x = decode<kFlat>(p, u);
       int n_list = 0;
-      unit_keys(p, x.bh, x.tile, n_list);
-      const int n_steps = n_list * p.KS;
-      const int64_t row = static_cast<int64_t>(x.bh) * p.N + chunk_token(p, x.tile, x.sub, r);
+      if constexpr (!kFlat) unit_keys(p, x.bh, x.tile, n_list);
+      const Chunks ck = unit_chunks<kFlat, kExtra>(p, x, n_list);
+      const int n_steps = ck.nm + ck.nx;
+      // the row: a token of the tile (window / list form) or of the flat query sequence (rows
+      // past Lq of the last chunk have no gradient; their Q and dO load as zeros)
+      const int64_t qrow = kFlat ? 128 * static_cast<int64_t>(x.tile) + r : chunk_token(p, x.tile, x.sub, r);
+      const bool row_ok = !kFlat || qrow < p.Lq;
+      const int64_t row = static_cast<int64_t>(x.bh) * (kFlat ? p.Lq : p.N) + (row_ok ? qrow : 0);
       uint4* dst = reinterpret_cast<uint4*>(p.dq + row * 128) + 8 * h;
+      float4* dstp = kFlat ? reinterpret_cast<float4*>(p.dq_part + x.sub * p.part_stride + row * 128) + 16 * h : nullptr;
       if (n_steps == 0) {  // no keys: no gradient
+        if (row_ok) {
+          if constexpr (kFlat) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+            for (int c = 0; c < 16; ++c) dstp[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
         continue;
       }
-      const float neg_lse2 = -p.lse[row] * kLog2e, dd = p.delta[row];
+      const int64_t lrow = kFlat ? static_cast<int64_t>(x.bh) * p.ld_rows + qrow : row;
+      const float neg_lse2 = row_ok ? -p.lse[lrow] * kLog2e : 0.f, dd = row_ok ? p.delta[lrow] : 0.f;
       {
         // the unit's row of Q (h = 0) or dO (h = 1) from the staging copy (128-byte swizzled
         // 64-channel halves, 8-row groups of 1 KB) into TMEM as packed bf16 pairs.  The
@@ -378,13 +473,20 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
         uint32_t s[32], dp[32];
         tmem_ld32_wait(tmem + kColS + 64 * b + 32 * h + lane_off, s);
         tmem_ld32_wait(tmem + kColDP + 64 * b + 32 * h + lane_off, dp);
+        // keys of this thread's 32 columns present in the chunk (a flat sequence's or the extra
+        // keys' last chunk may be partial): the others get P = dS = 0
+        const int nv = chunk_valid<kFlat, kExtra>(p, ck, t) - 32 * h;
         uint32_t w[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           float x0, x1;
           ffma2(x0, x1, __uint_as_float(s[c]), __uint_as_float(s[c + 1]), p.scale_log2, p.scale_log2, neg_lse2,
                 neg_lse2);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (kFlat || kExtra) {
+            if (c >= nv) p0 = 0.f;
+            if (c + 1 >= nv) p1 = 0.f;
+          }
           w[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - dd), p1 * (__uint_as_float(dp[c + 1]) - dd));
         }
         tmem_st16(tmem + kColS + 64 * b + 32 * h + lane_off, w);  // over this thread's own score columns
@@ -404,23 +506,36 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
+      if constexpr (kFlat) {  // this part's fp32 share of scale * dQ
+        if (row_ok) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 v;
-        v.x = pack_bf16x2(__uint_as_float(a[8 * c + 0]) * p.scale, __uint_as_float(a[8 * c + 1]) * p.scale);
-        v.y = pack_bf16x2(__uint_as_float(a[8 * c + 2]) * p.scale, __uint_as_float(a[8 * c + 3]) * p.scale);
-        v.z = pack_bf16x2(__uint_as_float(a[8 * c + 4]) * p.scale, __uint_as_float(a[8 * c + 5]) * p.scale);
-        v.w = pack_bf16x2(__uint_as_float(a[8 * c + 6]) * p.scale, __uint_as_float(a[8 * c + 7]) * p.scale);
-        dst[c] = v;
-      }
+          for (int c = 0; c < 8; ++c)
+            dstp[c] = make_float4(__uint_as_float(a[4 * c]) * p.scale, __uint_as_float(a[4 * c + 1]) * p.scale,
+                                  __uint_as_float(a[4 * c + 2]) * p.scale, __uint_as_float(a[4 * c + 3]) * p.scale);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 v;
-        v.x = pack_bf16x2(__uint_as_float(c2[8 * c + 0]) * p.scale, __uint_as_float(c2[8 * c + 1]) * p.scale);
-        v.y = pack_bf16x2(__uint_as_float(c2[8 * c + 2]) * p.scale, __uint_as_float(c2[8 * c + 3]) * p.scale);
-        v.z = pack_bf16x2(__uint_as_float(c2[8 * c + 4]) * p.scale, __uint_as_float(c2[8 * c + 5]) * p.scale);
-        v.w = pack_bf16x2(__uint_as_float(c2[8 * c + 6]) * p.scale, __uint_as_float(c2[8 * c + 7]) * p.scale);
-        dst[4 + c] = v;
+          for (int c = 0; c < 8; ++c)
+            dstp[8 + c] = make_float4(__uint_as_float(c2[4 * c]) * p.scale, __uint_as_float(c2[4 * c + 1]) * p.scale,
+                                      __uint_as_float(c2[4 * c + 2]) * p.scale, __uint_as_float(c2[4 * c + 3]) * p.scale);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(a[8 * c + 0]) * p.scale, __uint_as_float(a[8 * c + 1]) * p.scale);
+          v.y = pack_bf16x2(__uint_as_float(a[8 * c + 2]) * p.scale, __uint_as_float(a[8 * c + 3]) * p.scale);
+          v.z = pack_bf16x2(__uint_as_float(a[8 * c + 4]) * p.scale, __uint_as_float(a[8 * c + 5]) * p.scale);
+          v.w = pack_bf16x2(__uint_as_float(a[8 * c + 6]) * p.scale, __uint_as_float(a[8 * c + 7]) * p.scale);
+          dst[c] = v;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(c2[8 * c + 0]) * p.scale, __uint_as_float(c2[8 * c + 1]) * p.scale);
+          v.y = pack_bf16x2(__uint_as_float(c2[8 * c + 2]) * p.scale, __uint_as_float(c2[8 * c + 3]) * p.scale);
+          v.z = pack_bf16x2(__uint_as_float(c2[8 * c + 4]) * p.scale, __uint_as_float(c2[8 * c + 5]) * p.scale);
+          v.w = pack_bf16x2(__uint_as_float(c2[8 * c + 6]) * p.scale, __uint_as_float(c2[8 * c + 7]) * p.scale);
+          dst[4 + c] = v;
+        }
       }
       g += n_steps;
       ++uc;
@@ -433,6 +548,27 @@ __global__ void __launch_bounds__(bdq::kThreads, 1)
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// dQ = the sum of the parts' fp32 shares (in part order), as bf16: n8 groups of 8 channels.
+__global__ void __launch_bounds__(256) dq_parts_combine(const float* __restrict__ part, int n_parts,
+                                                        int64_t part_stride, int64_t n8,
+                                                        __nv_bfloat16* __restrict__ dq) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+  for (int j = 0; j < n_parts; ++j) {
+    const float4 x = reinterpret_cast<const float4*>(part + j * part_stride)[2 * i];
+    const float4 y = reinterpret_cast<const float4*>(part + j * part_stride)[2 * i + 1];
+    a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+    b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+  }
+  uint4 v;
+  v.x = pack_bf16x2(a.x, a.y);
+  v.y = pack_bf16x2(a.z, a.w);
+  v.z = pack_bf16x2(b.x, b.y);
+  v.w = pack_bf16x2(b.z, b.w);
+  reinterpret_cast<uint4*>(dq)[i] = v;
 }
 
 }  // namespace dsa
