@@ -463,8 +463,7 @@ def run_lstsq_workload(dsa, device, steps: int, warmup: int, m: int = 300 * 300,
 
     def read(s=stream):
         with torch.cuda.stream(s):
-            torch.sum(S, out=acc)
-            acc.add_(M.sum())
+            acc.copy_(S.sum() + M.sum())
 
     with torch.cuda.stream(side):
         read(side)
