@@ -54,7 +54,7 @@ def peaks():
 # single-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the full-size
 # launch.  The figure holds only for the kernel sources it was taken on, identified by a
 # hash of them; with any other sources the line reports null.
-FWD_TRAFFIC = {"bf16_720p": (3.54e9, "cafcb10850cbd1e3")}
+FWD_TRAFFIC = {"bf16_720p": (3.30e9, "c25f5712cf06440d")}
 FWD_SOURCES = ("dsa_fwd_bf16.cuh", "sm100.cuh")
 
 
@@ -650,9 +650,14 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the per-workload table")
     ap.add_argument("--extra-only", choices=["text_prefix", "lists", "dense_map", "lstsq"],
                     help="run one entry of the per-workload table on the workload alone and print it (profiling)")
+    ap.add_argument("--batch", type=int, help="run the workload with this batch size instead (profiling captures)")
+    ap.add_argument("--heads", type=int, help="run the workload with this many heads instead (profiling captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
+    if args.batch or args.heads:  # a reduced copy of the workload, named for what it is
+        w = w.replace(B=args.batch or w.B, heads=args.heads or w.heads)
+        w = w.replace(name=f"{args.workload}_B{w.B}_h{w.heads}")
     if args.impl == "reference":
         reference_arm(args, w)
         return
