@@ -232,7 +232,7 @@ dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k
  * tile.  Lists as dsa_fwd_list.  map: device fp32 [B * heads, nTiles, nTiles], overwritten.
  * The scores are recomputed on the tensor cores; one CTA sums each row of the map (all
  * chunks of query tile i) in fp32 in a fixed order, so the map is the same from run to run.
- * A row of the lists may hold at most 8192 entries here (a longer row is recorded as
+ * A row of the lists may hold at most 1024 entries here (a longer row is recorded as
  * DSA_ERR_DEVICE, site 48, and its map row left zero).  bf16, d = 128. */
 dsa_status_t dsa_block_map(const dsa_problem_t* p, const void* q, const void* k, const float* lse,
                            const int32_t* kv_row_ptr, const int32_t* kv_list, int32_t nnz, int32_t per_head, float* map,

@@ -120,10 +120,10 @@ constexpr uint32_t kPolyMask = 0x88u;
 // the block-map pass's share of 2^x on the FMA pipe (the forward's: a larger share was
 // slower, the polynomial's issue slots cost more than the MUFU time they free)
 constexpr uint32_t kPolyMaskMap = 0x88u;
-// list positions of a query tile's row the block-map pass keeps totals for (the V ring's
-// shared memory, which the pass does not use)
-constexpr int kMapCap = 8192;
-static_assert(8 * kMapCap <= kVStages * kTileBytes, "map totals must fit in the V ring");
+// list positions of a query tile's row the block-map pass keeps totals for, one total per
+// position and softmax warp (the V ring's shared memory, which the pass does not use)
+constexpr int kMapCap = 1024;
+static_assert(4 * 8 * kMapCap + 4 * kMapCap <= kVStages * kTileBytes, "map totals must fit in the V ring");
 
 // TMEM columns of the scores and of P for a step of parity e.
 __device__ __forceinline__ uint32_t col_s(int e) { return e ? 128u : 0u; }
@@ -637,18 +637,19 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       // ---------------------------------------------------------------- block attention mass
       // One CTA owns every chunk of a query tile (next_unit), so the tile's row of the map is
       // summed here in a fixed order and written once: per step each warp sums its 32 rows x
-      // 128 keys, the warps' sums meet in shared memory and one thread adds them, in warp
-      // order, to the list position's total; at the tile's end the totals of each listed key
-      // tile (in list order, so a tile listed twice counts twice) are written to the map.
-      // Every map warp takes every named barrier, even after a failed wait, so none waits
-      // for a warp that has left.
+      // 128 keys and adds the sum to its own total for the list position (only that warp
+      // writes that total, in step order); at the tile's end the eight warps' totals of each
+      // position are added in warp order, and those of every position listing a key tile (in
+      // list order, so a tile listed twice counts twice) are written to the map.  The named
+      // barriers are taken by every map warp, even after a failed wait, so none waits for a
+      // warp that has left.
       const int i = warp >> 2;
       const int r = tid & 127;
       const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
       const float inv_rows = 1.f / static_cast<float>(p.S * 128);
-      float* acc = reinterpret_cast<float*>(smem + kOffV);                 // [kMapCap] per list position
-      int32_t* kvs = reinterpret_cast<int32_t*>(smem + kOffV + 4 * kMapCap);  // [kMapCap] the row's key tiles
-      float* stage = xbuf;                                                   // [2][8] warp sums of a step
+      float* acc = reinterpret_cast<float*>(smem + kOffV);                        // [8][kMapCap]
+      int32_t* kvs = reinterpret_cast<int32_t*>(smem + kOffV + 4 * 8 * kMapCap);  // [kMapCap]
+      float* my_acc = acc + warp * kMapCap;
       int sc0 = 0, sc1 = 0, g = 0;
       bool ok = true;
       Unit x;
@@ -660,10 +661,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (x.sub == 0) {  // a new query tile: its totals start at zero
           named_bar_sync(5, 256);  // the previous tile's row has been written
           if (fits) {
-            for (int e = tid; e < n_list; e += 256) {
-              acc[e] = 0.f;
-              kvs[e] = min(max(kv[e], 0), p.n_tiles - 1);
-            }
+            for (int e = tid; e < 8 * n_list; e += 256) acc[(e / n_list) * kMapCap + e % n_list] = 0.f;
+            for (int e = tid; e < n_list; e += 256) kvs[e] = min(max(kv[e], 0), p.n_tiles - 1);
           } else if (tid == 0) {
             device_report(DSA_DEV_BOUNDS, 48);  // a list row longer than the map pass takes
           }
@@ -674,59 +673,47 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         for (int t = 0; t < n_steps; ++t) {
           const int e = (g + t) & 1;
           if (ok) ok = warp_wait(s_full + e, (e == 0 ? sc0++ : sc1++) & 1, abort, 49);
+          if (!ok) continue;
+          tc_fence_after();
           const bool full = 2 * t + 1 < n_chunks;
-          float sum = 0.f;
-          if (ok) {
-            tc_fence_after();
-            uint32_t sv[128];
-            if (full) {
-              tmem_ld128_wait(tmem + col_s(e) + 128 * i + lane_off, sv);
-            } else {
-              uint32_t (&half)[64] = *reinterpret_cast<uint32_t(*)[64]>(sv);
-              tmem_ld64_wait(tmem + col_s(e) + 64 * i + lane_off, half);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_read + e);  // the scores' columns may be overwritten
-            const int nc = full ? 128 : 64;
-            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t sv[128];
+          if (full) {
+            tmem_ld128_wait(tmem + col_s(e) + 128 * i + lane_off, sv);
+          } else {
+            uint32_t (&half)[64] = *reinterpret_cast<uint32_t(*)[64]>(sv);
+            tmem_ld64_wait(tmem + col_s(e) + 64 * i + lane_off, half);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_read + e);  // the scores' columns may be overwritten
+          const int nc = full ? 128 : 64;
+          float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 128; c += 2) {
-              if (c < nc) {
-                float x0, x1;
-                ffma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), p.scale_log2, p.scale_log2,
-                      neg_lse, neg_lse);
-                float p0, p1;
-                if ((kPolyMaskMap >> (c >> 4)) & 1u) {  // a share of 2^x on the FMA pipe
-                  exp2_poly2(x0, x1, p0, p1);
-                } else {
-                  p0 = ex2_approx(x0);
-                  p1 = ex2_approx(x1);
-                }
-                fadd2(sa[(c >> 1) & 3], sb[(c >> 1) & 3], sa[(c >> 1) & 3], sb[(c >> 1) & 3], p0, p1);
+          for (int c = 0; c < 128; c += 2) {
+            if (c < nc) {
+              float x0, x1;
+              ffma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), p.scale_log2, p.scale_log2, neg_lse,
+                    neg_lse);
+              float p0, p1;
+              if ((kPolyMaskMap >> (c >> 4)) & 1u) {  // a share of 2^x on the FMA pipe
+                exp2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
               }
+              fadd2(sa[(c >> 1) & 3], sb[(c >> 1) & 3], sa[(c >> 1) & 3], sb[(c >> 1) & 3], p0, p1);
             }
-            sum = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
+          }
+          float sum = ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-          }
-          if (lane == 0) stage[8 * e + warp] = sum;
-          named_bar_sync(5, 256);
-          if (tid == 0 && fits) {
-            // warpgroup i summed chunk 2t + i of a full step, or half i of the single chunk 2t
-            const float* st = stage + 8 * e;
-            const float s0 = (st[0] + st[1]) + (st[2] + st[3]), s1 = (st[4] + st[5]) + (st[6] + st[7]);
-            if (full) {
-              acc[(2 * t) / p.S] += s0;
-              acc[(2 * t + 1) / p.S] += s1;
-            } else {
-              acc[(2 * t) / p.S] += s0 + s1;
-            }
-          }
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          // this warp's keys: chunk 2t + i of a full step, or half i of the single chunk 2t
+          const int c = full ? 2 * t + i : 2 * t;
+          if (lane == 0 && fits) my_acc[c / p.S] += sum;
         }
         g += n_steps;
         if (x.sub == p.S - 1) {
-          named_bar_sync(5, 256);  // the tile's totals are complete
+          named_bar_sync(5, 256);  // every warp's totals of the tile are complete
           float* mrow = p.bmap + (static_cast<int64_t>(x.bh) * p.n_tiles + x.tile) * p.n_tiles;
           if (fits) {
             for (int e = tid; e < n_list; e += 256) {
@@ -735,8 +722,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
               for (int f = 0; f < e && first; ++f) first = kvs[f] != kt;
               if (!first) continue;  // counted with the tile's first occurrence
               float s = 0.f;
-              for (int f = e; f < n_list; ++f)
-                if (kvs[f] == kt) s += acc[f];
+              for (int f = e; f < n_list; ++f) {
+                if (kvs[f] != kt) continue;
+                float tf = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) tf += acc[w * kMapCap + f];
+                s += tf;
+              }
               mrow[kt] = s * inv_rows;
             }
           }
