@@ -14,6 +14,7 @@
 #include "dsa_device_status.cuh"
 #include "dsa_fwd_bf16.cuh"
 #include "dsa_fwd_f32.cuh"
+#include "dsa_fwd_pair.cuh"
 #include "dsa_lists.cuh"
 #include "dsa_lstsq.cuh"
 #include "dsa_plan.cuh"
@@ -307,6 +308,44 @@ dsa_status_t launch_plan(const Geom& g, const int32_t* offsets, int32_t* starts,
   return launch_status();
 }
 
+// Clusters of two the CTA-pair forward can keep resident on the current device (one CTA
+// per SM), looked up once per device and kernel; 0 if none fits.  Also checks, as for the
+// single-CTA kernel, that the kernel got the registers its setmaxnreg split needs.
+constexpr int kPairMaxDevices = 128;
+
+dsa_status_t pair_cluster_count(void (*kernel)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                                               dsa::FwdBf16Params),
+                                int sms, int* clusters) {
+  static int cache[2][kPairMaxDevices] = {};
+  const int which = kernel == dsa::fwd_pair_kernel<true> ? 1 : 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::fwdp::kSmemBytes) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
+  if (fa.numRegs < dsa::fwd::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
+  if (dev >= 0 && dev < kPairMaxDevices && cache[which][dev] > 0) {
+    *clusters = cache[which][dev];
+    return DSA_OK;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(sms >= 2 ? sms / 2 * 2 : 2), 1, 1);
+  cfg.blockDim = dim3(dsa::fwdp::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = dsa::fwdp::kSmemBytes;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  if (n > sms / 2) n = sms / 2;
+  if (n > 0 && dev >= 0 && dev < kPairMaxDevices) cache[which][dev] = n;
+  *clusters = n;
+  return DSA_OK;
+}
+
 // kv_tiles: the plan's [n_tiles, Wt] key tiles (row_ptr null) or a caller's key-tile list
 // with its CSR offsets row_ptr [n_tiles + 1] and nnz entries (bf16 only).
 dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, const void* k, const void* v,
@@ -382,6 +421,21 @@ dsa_status_t launch_fwd(const dsa_problem_t* p, const Geom& g, const void* q, co
   const bool map_mode = bmap != nullptr;
   int sms = 0;
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
+  if (!map_mode && row_ptr == nullptr && bp.S % 2 == 0) {
+    // the window form with an even number of 128-row chunks per tile: one product per pair
+    // of SMs over two chunks of a tile (which share its window)
+    auto pk = bp.Lx > 0 ? dsa::fwd_pair_kernel<true> : dsa::fwd_pair_kernel<false>;
+    int clusters = 0;
+    const dsa_status_t st = pair_cluster_count(pk, sms, &clusters);
+    if (st != DSA_OK) return st;
+    if (clusters > 0) {
+      const int pairs = bp.n_units / 2;
+      const unsigned grid = static_cast<unsigned>(2 * (clusters < pairs ? clusters : pairs));
+      pk<<<grid, dsa::fwdp::kThreads, dsa::fwdp::kSmemBytes, s>>>(tq, tk, tv, tkx, tvx, bp);
+      return launch_status();
+    }
+    // no cluster of two fits on this device: the single-CTA kernel below
+  }
   auto kernel = map_mode ? dsa::fwd_bf16_kernel<dsa::fwd::kModeMap>
                          : (bp.Lx > 0 ? dsa::fwd_bf16_kernel<dsa::fwd::kModeFwdX> : dsa::fwd_bf16_kernel<dsa::fwd::kModeFwd>);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::fwd::kSmemBytes) != cudaSuccess)

@@ -284,14 +284,15 @@ __device__ __forceinline__ float pair_exchange(float* xbuf, int& xe, int i, int 
 // The softmax of one step for this thread's NC score columns at tS (NC = 128: a full step,
 // NC = 64: a half step): agrees on the row max with the partner thread, writes packed bf16
 // P (NC/2 columns) at tP, updates m_used and l, and returns whether the reference max
-// moved; it arrives on `loaded` as soon as its scores are in registers.  Columns from
+// moved; it arrives on the mbarrier at `loaded` (a shared::cta address, or with kCluster a
+// shared::cluster one, possibly the peer CTA's) as soon as its scores are in registers.  Columns from
 // nvalid on hold no key (the tail of a flat key sequence) and get probability 0 (alpha: the factor the old O and l take).  With !ok (an earlier wait failed; TMEM
 // stays allocated, so the load is harmless) the thread still takes part in the exchange,
 // so its partner never waits for it, and does nothing else.  The load is unconditional: a
 // load under `ok` with the exchange between it and the use makes the compiler keep far
 // more registers live.
-template <int NC>
-__device__ __forceinline__ bool softmax_step(bool ok, uint32_t tS, uint32_t tP, uint64_t* loaded, float scale_log2,
+template <int NC, bool kCluster = false>
+__device__ __forceinline__ bool softmax_step(bool ok, uint32_t tS, uint32_t tP, uint32_t loaded, float scale_log2,
                                              float& m_used, float& l, float& alpha, float* xbuf, int& xe, int i,
                                              int r, int bar_id, int nvalid = NC) {
   uint32_t s[NC];
@@ -307,7 +308,12 @@ __device__ __forceinline__ bool softmax_step(bool ok, uint32_t tS, uint32_t tP, 
   if (ok) {  // the scores are in registers: their TMEM columns may be overwritten
     tc_fence_before();
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(loaded);
+    if ((threadIdx.x & 31) == 0) {
+      if constexpr (kCluster)
+        mbar_arrive_cluster(loaded);
+      else
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(loaded) : "memory");
+    }
   }
   // row max: 8 independent chains over columns e, e + 8, ..., e + NC - 8
   float mxs[8];
@@ -788,10 +794,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
                                 : min(max(chunk_valid<kFlat, kExtra>(p, ck, 2 * t) - 64 * i, 0), 64);
         if (full)
           need = softmax_step<128>(ok, tmem + col_s(e) + 128 * i + lane_off, tmem + col_p(e) + 64 * i + lane_off,
-                                   s_read + e, p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id, nvalid);
+                                   smem_u32(s_read + e), p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id, nvalid);
         else
           need = softmax_step<64>(ok, tmem + col_s(e) + 64 * i + lane_off, tmem + col_p(e) + 32 * i + lane_off,
-                                  s_read + e, p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id, nvalid);
+                                  smem_u32(s_read + e), p.scale_log2, m_used, l, alpha, xbuf, xe, i, r, bar_id, nvalid);
         if (ok && t > 0 && __any_sync(0xffffffffu, need)) {
           // O holds sum P V up to step t-1 with the old reference max: rescale this
           // warpgroup's channels of it
