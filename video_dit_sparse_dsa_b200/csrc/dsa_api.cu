@@ -520,7 +520,7 @@ dsa::BwdDqParams dq_params(const dsa_problem_t* p, const Geom& g, const float* l
   dp.n_tiles = g.n_tiles;
   dp.Wt = g.Wt;
   dp.S = g.tile_tokens / 128;
-  dp.KS = g.tile_tokens / 64;
+  dp.KS = g.tile_tokens / 128;
   dp.n_units = static_cast<int>(g.BH * g.n_tiles * dp.S);
   dp.G1 = g.G[1];
   dp.G2 = g.G[2];
@@ -528,7 +528,7 @@ dsa::BwdDqParams dq_params(const dsa_problem_t* p, const Geom& g, const float* l
   dp.th = p->tile[1];
   dp.tw = p->tile[2];
   dp.tcs = 128 / (p->tile[1] * p->tile[2]);
-  dp.kcs = 64 / (p->tile[1] * p->tile[2]);
+  dp.kcs = 128 / (p->tile[1] * p->tile[2]);
   dp.T = p->T;
   dp.H = p->H;
   dp.W = p->W;
@@ -540,8 +540,8 @@ dsa::BwdDqParams dq_params(const dsa_problem_t* p, const Geom& g, const float* l
 }
 
 template <bool kFlat, bool kExtra>
-dsa_status_t launch_dq(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const CUtensorMap& tkx, const CUtensorMap& tvx, const dsa::BwdDqParams& dp, cudaStream_t s) {
+dsa_status_t launch_dq(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tkx, const CUtensorMap& tvx,
+                       const dsa::BwdDqParams& dp, cudaStream_t s) {
   auto kernel = dsa::bwd_dq_kernel<kFlat, kExtra>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::bdq::kSmemBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
@@ -552,7 +552,7 @@ dsa_status_t launch_dq(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   int sms = 0;
   if (sm_count(&sms) != DSA_OK) return DSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(dp.n_units < sms ? dp.n_units : sms);
-  kernel<<<grid, dsa::bdq::kThreads, dsa::bdq::kSmemBytes, s>>>(tq, tk, tv, tdo, tkx, tvx, dp);
+  kernel<<<grid, dsa::bdq::kThreads, dsa::bdq::kSmemBytes, s>>>(tk, tv, tkx, tvx, dp);
   return launch_status();
 }
 
@@ -610,17 +610,16 @@ dsa_status_t launch_bwd_det(const dsa_problem_t* p, const Geom& g, const void* q
     st = launch_status();
     if (st != DSA_OK) return st;
   }
-  // dQ: 128-row query chunks over the forward's key lists, 64 keys per step
-  CUtensorMap tq2, tdo2, tk2, tv2;
-  if (!make_token_map(&tq2, q, p, g, 128) || !make_token_map(&tdo2, dout, p, g, 128) ||
-      !make_token_map(&tk2, k, p, g, 64) || !make_token_map(&tv2, v, p, g, 64))
-    return DSA_ERR_CUDA;
+  // dQ: 128-row query chunks over the forward's key lists, 128 keys per step (the K and V
+  // maps of 128-token boxes serve both kernels)
   dsa::BwdDqParams dp = dq_params(p, g, lse, delta, dq);
+  dp.q = static_cast<const __nv_bfloat16*>(q);
+  dp.dout = static_cast<const __nv_bfloat16*>(dout);
   dp.kv_tiles = fk.kv;
   dp.row_ptr = fk.row_ptr;
   dp.rp_head_stride = fk.rp_head_stride;
   dp.nnz = fk.nnz;
-  return launch_dq<false, false>(tq2, tk2, tv2, tdo2, tk2, tv2, dp, s);
+  return launch_dq<false, false>(tk, tv, tk, tv, dp, s);
 }
 
 }  // namespace
@@ -1065,7 +1064,7 @@ int prefix_bwd_split(const Geom& g, int32_t L_text) {
 // waves of persistent CTAs, at most one part per 64-key chunk of the video.
 int prefix_dq_split(const Geom& g, int32_t L_text) {
   const int64_t units = g.BH * ((static_cast<int64_t>(L_text) + 127) / 128);
-  const int64_t nk = (g.N + 63) / 64;
+  const int64_t nk = (g.N + 127) / 128;
   int64_t n = (4 * 148 + units - 1) / (units > 0 ? units : 1);
   if (n > nk) n = nk;
   if (n > 16) n = 16;
@@ -1251,26 +1250,28 @@ dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k
   }
   // video queries: dQ over their windows' keys and every text key
   {
-    CUtensorMap tq2, tdo2, tk2, tv2, tkx, tvx;
-    if (!make_token_map(&tq2, q, p, g, 128) || !make_token_map(&tdo2, dout, p, g, 128) ||
-        !make_token_map(&tk2, k, p, g, 64) || !make_token_map(&tv2, v, p, g, 64) ||
-        !make_flat_map(&tkx, k_text, g.BH, L_text, 64) || !make_flat_map(&tvx, v_text, g.BH, L_text, 64))
+    CUtensorMap tk2, tv2, tkx, tvx;
+    if (!make_token_map(&tk2, k, p, g, 128) || !make_token_map(&tv2, v, p, g, 128) ||
+        !make_flat_map(&tkx, k_text, g.BH, L_text, 128) || !make_flat_map(&tvx, v_text, g.BH, L_text, 128))
       return DSA_ERR_CUDA;
     dsa::BwdDqParams dp = dq_params(p, g, lse, wv.delta, dq);
+    dp.q = static_cast<const __nv_bfloat16*>(q);
+    dp.dout = static_cast<const __nv_bfloat16*>(dout);
     dp.kv_tiles = wv.kv_tiles;
     dp.Lx = L_text;
-    st = launch_dq<false, true>(tq2, tk2, tv2, tdo2, tkx, tvx, dp, s);
+    st = launch_dq<false, true>(tk2, tv2, tkx, tvx, dp, s);
     if (st != DSA_OK) return st;
   }
   // text queries: dQ over every video key (flat, in parts) and every text key (with part 0)
   {
-    CUtensorMap fq, fdo, fk, fv, tkx, tvx;
-    if (!make_flat_map(&fq, q_text, g.BH, L_text, 128) || !make_flat_map(&fdo, dout_text, g.BH, L_text, 128) ||
-        !make_flat_map(&fk, k, g.BH, g.N, 64) || !make_flat_map(&fv, v, g.BH, g.N, 64) ||
-        !make_flat_map(&tkx, k_text, g.BH, L_text, 64) || !make_flat_map(&tvx, v_text, g.BH, L_text, 64))
+    CUtensorMap fk, fv, tkx, tvx;
+    if (!make_flat_map(&fk, k, g.BH, g.N, 128) || !make_flat_map(&fv, v, g.BH, g.N, 128) ||
+        !make_flat_map(&tkx, k_text, g.BH, L_text, 128) || !make_flat_map(&tvx, v_text, g.BH, L_text, 128))
       return DSA_ERR_CUDA;
     dsa::BwdDqParams dp;
     std::memset(&dp, 0, sizeof(dp));
+    dp.q = static_cast<const __nv_bfloat16*>(q_text);
+    dp.dout = static_cast<const __nv_bfloat16*>(dout_text);
     dp.lse = ws.lse_pad;
     dp.delta = ws.delta_pad;
     dp.ld_rows = ws.Lp;
@@ -1286,7 +1287,7 @@ dsa_status_t dsa_bwd_prefix(const dsa_problem_t* p, const void* q, const void* k
     dp.tt = dp.th = dp.tw = 1;
     dp.T = dp.H = dp.W = 1;
     dp.S = dp.KS = 1;
-    st = launch_dq<true, true>(fq, fk, fv, fdo, tkx, tvx, dp, s);
+    st = launch_dq<true, true>(fk, fv, tkx, tvx, dp, s);
     if (st != DSA_OK) return st;
     const int64_t n8 = g.BH * static_cast<int64_t>(L_text) * 128 / 8;
     dsa::dq_parts_combine<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
