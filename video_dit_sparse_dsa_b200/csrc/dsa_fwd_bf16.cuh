@@ -117,9 +117,13 @@ constexpr float kRescaleThreshold = 8.0f;                        // log2 units
 // taken from the FMA-pipe polynomial instead of the MUFU unit, which takes 16 per clock per
 // SM and would otherwise bound the softmax
 constexpr uint32_t kPolyMask = 0x88u;
-// the block-map pass's share of 2^x on the FMA pipe (the forward's: a larger share was
-// slower, the polynomial's issue slots cost more than the MUFU time they free)
-constexpr uint32_t kPolyMaskMap = 0x88u;
+// the block-map pass's share of 2^x on the FMA pipe: column pairs (bit e of the 8 pairs of
+// every 16-column group) 1, 4 and 7, spread through each group so that the two softmax warps
+// of a sub-partition keep the MUFU unit and the FMA pipe busy side by side (measured on the
+// dense 16x32x32 map: 3/8 spread 2.04-2.12 ms; 2/8 spread 2.09; 4/8 2.24; 5/8 2.23-2.31;
+// 2/8 as whole groups 2.16; the pass has no bf16 pack, so it takes a larger share than the
+// forward)
+constexpr uint32_t kPolyMaskMap = 0x92u;
 // list positions of a query tile's row the block-map pass keeps totals for, one total per
 // position and softmax warp (the V ring's shared memory, which the pass does not use)
 constexpr int kMapCap = 1024;
@@ -701,7 +705,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
               ffma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), p.scale_log2, p.scale_log2, neg_lse,
                     neg_lse);
               float p0, p1;
-              if ((kPolyMaskMap >> (c >> 4)) & 1u) {  // a share of 2^x on the FMA pipe
+              if ((kPolyMaskMap >> ((c >> 1) & 7)) & 1u) {  // a share of 2^x on the FMA pipe
                 exp2_poly2(x0, x1, p0, p1);
               } else {
                 p0 = ex2_approx(x0);
