@@ -40,8 +40,8 @@
  * that ran out, an index outside its buffer) is recorded in a device status word that
  * dsa_device_status() reads.
  *
- * Supported: bf16 with d = 128 on the tensor-core path, where 64-token key chunks and
- * 128-token query chunks of a tile must be whole (h, w) planes (th*tw divides 64 and
+ * Supported: bf16 with d = 128 on the tensor-core path, where a tile's 128-token chunks and
+ * the backward's 64-token query chunks must be whole (h, w) planes (th*tw divides 64 and
  * 128/(th*tw) divides tt), and for the backward tw a multiple of 4;
  * fp32 with d in {64, 128} on the exact-fp32 path (any tile shape).  Pointers of the bf16
  * path must be 16-byte aligned.
@@ -102,7 +102,9 @@ dsa_status_t dsa_plan(const dsa_problem_t* p, const int32_t* tile_offsets, int32
 
 /* Forward: plans the windows of tile_offsets, then writes out (dtype of p) and lse (fp32).
  * workspace: device memory of at least dsa_workspace_size(p, DSA_WS_FWD) bytes, 256-byte
- * aligned; its contents on entry do not matter. */
+ * aligned; its contents on entry do not matter.  bf16 tiles of an even number of 128-token
+ * chunks run on clusters of two CTAs (one product per pair of SMs over two chunks of a
+ * tile), other tiles on one CTA per chunk; every row's arithmetic is the same in both. */
 dsa_status_t dsa_fwd(const dsa_problem_t* p, const void* q, const void* k, const void* v,
                      const int32_t* tile_offsets, void* out, float* lse, void* workspace, size_t ws_bytes,
                      void* stream);

@@ -18,7 +18,10 @@
 // 2t + r of the step), and the P.V product takes the 128 channels as N, 64 from each CTA
 // (CTA r loads channel half r of every V chunk).  Each CTA so loads 64 KB per step for its
 // 128 rows instead of 128 KB, and its shared memory carries 160 KB per step instead of
-// 288 KB.  (Tiles of an odd number of chunks run on the single-CTA kernel.)
+// 288 KB.  (Tiles of an odd number of chunks run on the single-CTA kernel.)  Measured, the
+// L2-to-SM bytes and the MMA operand reads halve as designed while the tensor pipe stays at
+// the single-CTA kernel's occupancy: the softmax warps' latency chain sets the step, and the
+// pair gains a few percent.
 //
 // Roles (per CTA, 12 warps as in the single-CTA kernel): warp 8 loads Q (its own chunk) and
 // its K halves, warp 10 its V halves, warps 0-7 run the softmax of its own 128 rows; the
