@@ -79,8 +79,18 @@ def test_list_backward_against_oracle(w):
         assert_close(got.float().cpu().numpy(), ref, "bf16", name)
 
 
-def test_window_plan_as_lists_is_bit_exact():
-    w = Workload("list_plan", 1, 2, 128, (12, 16, 24), (6, 8, 8), (3, 1, 3), (-1, 1), "bf16", 43)
+# The window form of tiles with an even number of 128-token chunks runs on the CTA-pair
+# kernel, the list form always on the single-CTA kernel: with the plan's windows as lists
+# the two must agree bit for bit (same products in the same order, same softmax).
+PLAN_AS_LISTS = [
+    Workload("list_plan_s3", 1, 2, 128, (12, 16, 24), (6, 8, 8), (3, 1, 3), (-1, 1), "bf16", 43),  # single vs single
+    Workload("list_plan_s2", 2, 2, 128, (12, 16, 24), (4, 8, 8), (3, 3, 3), (-2, 2), "bf16", 44),  # pair vs single
+    Workload("list_plan_s4", 1, 3, 128, (16, 16, 24), (8, 8, 8), (1, 3, 3), (-1, 1), "bf16", 45),  # 2 pairs per tile
+]
+
+
+@pytest.mark.parametrize("w", PLAN_AS_LISTS, ids=lambda w: w.name)
+def test_window_plan_as_lists_is_bit_exact(w):
     inp = make_inputs(w)
     geo = oracle.Geometry.of(w)
     q, k, v, off = inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.offsets.cuda()
