@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -309,14 +310,15 @@ dsa_status_t launch_plan(const Geom& g, const int32_t* offsets, int32_t* starts,
 }
 
 // Clusters of two the CTA-pair forward can keep resident on the current device (one CTA
-// per SM), looked up once per device and kernel; 0 if none fits.  Also checks, as for the
-// single-CTA kernel, that the kernel got the registers its setmaxnreg split needs.
+// per SM), looked up once per device and kernel (atomically cached: host threads may call
+// concurrently); 0 if none fits.  Also checks, as for the single-CTA kernel, that the
+// kernel got the registers its setmaxnreg split needs.
 constexpr int kPairMaxDevices = 128;
 
 dsa_status_t pair_cluster_count(void (*kernel)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
                                                dsa::FwdBf16Params),
                                 int sms, int* clusters) {
-  static int cache[2][kPairMaxDevices] = {};
+  static std::atomic<int> cache[2][kPairMaxDevices] = {};
   const int which = kernel == dsa::fwd_pair_kernel<true> ? 1 : 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
@@ -326,9 +328,12 @@ dsa_status_t pair_cluster_count(void (*kernel)(CUtensorMap, CUtensorMap, CUtenso
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return DSA_ERR_CUDA;
   if (fa.numRegs < dsa::fwd::kRegsAtLaunch) return DSA_ERR_UNSUPPORTED;
-  if (dev >= 0 && dev < kPairMaxDevices && cache[which][dev] > 0) {
-    *clusters = cache[which][dev];
-    return DSA_OK;
+  if (dev >= 0 && dev < kPairMaxDevices) {
+    const int c = cache[which][dev].load(std::memory_order_relaxed);
+    if (c > 0) {
+      *clusters = c;
+      return DSA_OK;
+    }
   }
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
@@ -341,7 +346,7 @@ dsa_status_t pair_cluster_count(void (*kernel)(CUtensorMap, CUtensorMap, CUtenso
     n = 0;
   }
   if (n > sms / 2) n = sms / 2;
-  if (n > 0 && dev >= 0 && dev < kPairMaxDevices) cache[which][dev] = n;
+  if (n > 0 && dev >= 0 && dev < kPairMaxDevices) cache[which][dev].store(n, std::memory_order_relaxed);
   *clusters = n;
   return DSA_OK;
 }
